@@ -1,0 +1,321 @@
+#!/usr/bin/env python
+"""Benchmark of the AWQ per-layer activation-aware scale search on B200.
+
+One step = one complete search of one synthetic layer (statistic, 20 candidate scale
+vectors, QDQ + fold-back of every candidate, the reference GEMM, 20 candidate GEMMs
+with the fused squared-error epilogue, argmin, packing) through the library's C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Under torchrun each rank searches its own layer (a different seed) on its own GPU:
+independent problems, no data-path collective, weak scaling. Rank 0 prints one JSON
+line. ``--impl reference`` times the CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from workloads import WORKLOADS, LayerSpec, generate, as_f32_numpy  # noqa: E402
+
+METRIC = "AWQ search candidate-GEMM TFLOP/s & layers/s; % of BF16 tensor peak"
+DEFAULT_WORKLOAD = "llama7b_attn_proj_4096x4096x4096"
+FLUSH_BYTES = 256 << 20   # > 126 MB L2
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=None, help="steps of the host-buffer run (default: --steps)")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------- helpers
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int, period_ms: int = 50):
+        self.proc = None
+        self.file = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", str(period_ms), "-i", ident], stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.seek(0)
+        rows = [r for r in csv.reader(io.StringIO(self.file.read())) if len(r) >= 9]
+        self.file.close()
+        os.unlink(self.file.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_oracle_sample(spec: LayerSpec, target_s: float):
+    """Time the oracle as it stands on a column slice of the layer (full X)."""
+    import oracle as O
+    X, W = generate(spec)
+    X32, W32 = as_f32_numpy(X), as_f32_numpy(W)
+
+    def run(ncols):
+        t0 = time.perf_counter()
+        O.search(X32, W32[:, :ncols], group=spec.group, n_grid=spec.n_grid)
+        return time.perf_counter() - t0
+
+    n = min(spec.N, 64)
+    t = run(n)
+    while t < target_s / 3 and n < spec.N:
+        n = min(spec.N, n * 4)
+        t = run(n)
+    flops = 2.0 * spec.M * spec.K * n * spec.n_grid
+    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{n} of {spec.N} output columns with the full {spec.M}x{spec.K} X "
+                      f"({t:.1f} s, numpy fp64 oracle)",
+            "seconds": t, "columns": n}
+
+
+# ----------------------------------------------------------------------------- arms
+def run_reference(args, rank, world):
+    spec = WORKLOADS[args.workload]
+    if rank != 0:
+        return 0
+    import oracle as O
+    X, W = generate(spec)
+    X32, W32 = as_f32_numpy(X), as_f32_numpy(W)
+    # size the per-step sample so warm-up + steps end within a few minutes
+    per_step_s = max(1.0, 150.0 / max(1, args.steps + args.warmup))
+    n = min(spec.N, 64)
+    t0 = time.perf_counter()
+    O.search(X32, W32[:, :n], group=spec.group, n_grid=spec.n_grid)
+    t = time.perf_counter() - t0
+    while t < per_step_s / 3 and n < spec.N:
+        n = min(spec.N, n * 4)
+        t0 = time.perf_counter()
+        O.search(X32, W32[:, :n], group=spec.group, n_grid=spec.n_grid)
+        t = time.perf_counter() - t0
+    for _ in range(args.warmup):
+        O.search(X32, W32[:, :n], group=spec.group, n_grid=spec.n_grid)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        O.search(X32, W32[:, :n], group=spec.group, n_grid=spec.n_grid)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    flops = 2.0 * spec.M * spec.K * n * spec.n_grid
+    value = flops * args.steps / total / 1e12
+    sample = f"{n} of {spec.N} output columns with the full {spec.M}x{spec.K} X per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": spec.name, "M": spec.M, "K": spec.K, "N": spec.N, "group": spec.group,
+                   "n_grid": spec.n_grid, "sample_columns": n},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, rank, world, local):
+    import post_quantization_column_b200 as awq
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    base = WORKLOADS[args.workload]
+    spec = LayerSpec(**{**base.as_dict(), "seed": base.seed + rank})
+    X, W = generate(spec)
+    Xd, Wd = X.to(dev), W.to(dev)
+    stream = torch.cuda.Stream(dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    awq.profile_enable(True)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier(device_ids=[local])
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            awq.search(Xd, Wd, spec.group, spec.n_grid, stream=stream)
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        gemm_ms, qdq_ms, stat_ms, pack_ms = [], [], [], []
+        barrier()
+        torch.cuda.synchronize(dev)
+        clocks = ClockSampler(local)
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            out = awq.search(Xd, Wd, spec.group, spec.n_grid, stream=stream)
+            ends[i].record(stream)
+            prof = awq.profile_last()
+            gemm_ms.append(prof["gemm_loss"])
+            qdq_ms.append(prof["qdq"])
+            stat_ms.append(prof["statistic"])
+            pack_ms.append(prof["pack"])
+        torch.cuda.synchronize(dev)
+        barrier()
+        clock_info = clocks.stop()
+        launches = awq.last_launch_count() * args.steps
+        step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+        total_ms = float(sum(step_ms))
+
+        # end to end through the host-buffer entry point: H2D of X and W + search + D2H of the artifact
+        e2e_steps = args.e2e_steps or max(3, min(args.steps, 20))
+        Xh, Wh = X.pin_memory(), W.pin_memory()
+        outs = (torch.empty(spec.K, dtype=torch.float32, pin_memory=True),
+                torch.empty(spec.K, spec.N // 8, dtype=torch.int32, pin_memory=True),
+                torch.empty(spec.K // spec.group, spec.N, dtype=torch.float16, pin_memory=True),
+                torch.empty(spec.K // spec.group, spec.N, dtype=torch.float16, pin_memory=True),
+                torch.empty(spec.n_grid, dtype=torch.float32, pin_memory=True))
+        awq.search_host(Xh, Wh, spec.group, spec.n_grid, stream=stream, out=outs, device=dev)
+        e_s = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+        e_e = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+        barrier()
+        torch.cuda.synchronize(dev)
+        for i in range(e2e_steps):
+            flush.zero_()
+            e_s[i].record(stream)
+            awq.search_host(Xh, Wh, spec.group, spec.n_grid, stream=stream, out=outs, device=dev)
+            e_e[i].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e2e_ms = float(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)))
+
+    times = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms = times.tolist()
+
+    flops = spec.candidate_flops
+    value = world * args.steps * flops / (total_ms / 1e3) / 1e12
+    layers_per_s = world * args.steps / (total_ms / 1e3)
+    e2e_value = world * e2e_steps * flops / (e2e_ms / 1e3) / 1e12
+    peaks, peak_kind = measured_peaks()
+    gemm_avg = statistics.mean(gemm_ms)
+    achieved = flops / (gemm_avg / 1e3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    h2d = X.numel() * X.element_size() + W.numel() * W.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+    qdq_bytes = (W.element_size() + 2 * (spec.n_grid + 1)) * spec.K * spec.N
+    stat_bytes = X.numel() * X.element_size() + 4 * spec.K
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": spec.name, "M": spec.M, "K": spec.K, "N": spec.N, "group": spec.group,
+                   "n_grid": spec.n_grid, "input_dtype": spec.dtype, "parallelism": f"independent layers x{world}",
+                   "l2": "flushed between steps (256 MiB device write outside the timed events)"},
+        "layers_per_s": layers_per_s,
+        "roofline": {"bound": "tensor", "kernel": "loss_gemm_kernel (candidate GEMMs + fused squared error)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_kind} bf16_tflops (burst)", "traffic": None,
+                     "ms_per_launch": gemm_avg},
+        "other_kernels": {
+            "qdq": {"ms": statistics.mean(qdq_ms),
+                    "GB/s": qdq_bytes / (statistics.mean(qdq_ms) / 1e3) / 1e9,
+                    "hbm_frac": qdq_bytes / (statistics.mean(qdq_ms) / 1e3) / 1e9 / float(peaks["hbm_gbs"])},
+            "statistic": {"ms": statistics.mean(stat_ms),
+                          "GB/s": stat_bytes / (statistics.mean(stat_ms) / 1e3) / 1e9},
+            "pack": {"ms": statistics.mean(pack_ms)},
+        },
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms / e2e_steps, "steps": e2e_steps},
+        "gpu_launches": launches,
+        "clocks": clock_info,
+        "chosen_alpha_index": out.best,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_sample(spec, args.cpu_seconds)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,149 @@
+/*
+ * awq_search.h — C ABI of libawqsearch.so: AWQ's activation-aware per-layer scale
+ * search on one NVIDIA B200 (sm_100a).
+ *
+ * The operation (cited by page title and section):
+ *   [AWQ-P1] "AWQ：为什么 4-bit 权重量化要先观察 Activation" — §1 statistic,
+ *            §3-§4 scale family, 20-point grid and forward-output loss,
+ *            §7 asymmetric 4-bit zero-point quantizer, orientation and packing,
+ *            §8 bits-per-weight budget.
+ *   [AWQ-P2] "AWQ salient weight / GGUF compilation" — §二 scale formula.
+ *   [QUANT-P4] "model-quantization / 05 core modules" — §5.3 int4 codes packed
+ *            eight per int32 with separate scale tensors.
+ *
+ * For one linear layer with calibration activations X (M x K, row-major, K
+ * contiguous) and weights W (K x N, row-major, N contiguous — the paper's
+ * orientation: K input channels, N output channels; AWQ-P1 §1, §7):
+ *   1. a_j = mean_m |X[m,j]|                       (fp64 sum, one rounding to fp32)
+ *   2. for alpha_i = i/n_grid, i = 0..n_grid-1:
+ *        raw_ij = max(a_j^alpha_i, 1e-4);  s_ij = raw_ij / sqrt(max_j raw_ij * min_j raw_ij)
+ *   3. W' = diag(s_i) W, group-wise along K (`group` rows of one column):
+ *        step = (max - min)/15 (1 for an all-equal group); z = clamp(rint(-min/step), 0, 15);
+ *        q = clamp(rint(W'/step) + z, 0, 15)       (rint = round half to even)
+ *   4. W_hat_i = diag(s_i)^-1 ((q - z) * step)     (fp32, then bf16 for the GEMM)
+ *   5. L_i = ||X_b W_b - X_b W_hat_i,b||_F^2 / (M N)  (bf16 operands, fp32 accumulation,
+ *        fp64 cross-tile sum; the reference output X_b W_b is computed once)
+ *   6. i* = first argmin of the fp32 losses; emit s_i*, the codes, steps and zeros.
+ *
+ * Artifact layout (AWQ-P1 §7-§8, QUANT-P4 §5.3):
+ *   out_scales [K]        fp32   s_i* (the activation is divided by it, W' multiplied)
+ *   out_codes  [K][N/8]   int32  nibble i (bits 4i..4i+3) of word [k][w] = code of column 8w+i
+ *   out_steps  [K/group][N] fp16 step of each (group, column), in the scaled domain
+ *   out_zeros  [K/group][N] fp16 zero point (an integer 0..15)
+ *   out_losses [n_grid]   fp32   L_i (optional, may be NULL)
+ *   Dequantized weight: W[k][n] ~= step[g][n] * (q[k][n] - zero[g][n]) / s[k], g = k/group.
+ *   4 bits + 32/group bits per weight: 4.25 at group 128 (AWQ-P1 §8).
+ *
+ * Preconditions (AWQ-P1 §7 shape contract, plus this library's): M, K, N > 0;
+ * group in {32, 64, 128}, K % group == 0; N % 8 == 0; 1 <= n_grid <= 64;
+ * device pointers 16-byte aligned; K, N < 2^31, M < 2^31.
+ *
+ * Ownership: every pointer is owned by the caller; the library neither keeps nor
+ * frees it. Device work space (candidate weights, the reference output, partial
+ * sums) comes from a library-owned stream-ordered memory pool on the current
+ * device, is allocated on `stream` and returned to the pool before the call
+ * returns (the pool keeps its memory for later calls; awq_release_cached frees it).
+ *
+ * Streams: all device work is enqueued on `stream` (NULL = the legacy default
+ * stream); the call then synchronizes `stream`, so the status reflects errors the
+ * kernels detected (non-finite input, a wait that ran out). Outputs are valid only
+ * when the status is AWQ_OK. The library is not reentrant across host threads
+ * that share a device (one call at a time per process is the tested use).
+ *
+ * Errors: every entry point returns an awq_status; awq_status_string names it and
+ * awq_last_error_message gives the detail of the last failure on this thread.
+ */
+#ifndef AWQ_SEARCH_H_
+#define AWQ_SEARCH_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream. */
+typedef struct CUstream_st* awq_stream_t;
+
+typedef enum awq_status {
+  AWQ_OK = 0,
+  AWQ_ERR_INVALID_ARG = 1,        /* NULL or misaligned pointer, bad n_grid/group/dtype */
+  AWQ_ERR_SHAPE = 2,              /* M, K, N out of range; K % group; N % 8 */
+  AWQ_ERR_NONFINITE = 3,          /* NaN or Inf in X or W (AWQ-P1 §2: finite reals only) */
+  AWQ_ERR_OOM = 4,                /* device work space could not be allocated */
+  AWQ_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed */
+  AWQ_ERR_TIMEOUT = 6,            /* a bounded wait inside a kernel ran out */
+  AWQ_ERR_UNSUPPORTED_DEVICE = 7  /* the current device is not sm_100 */
+} awq_status;
+
+enum { AWQ_DTYPE_BF16 = 0, AWQ_DTYPE_F32 = 1 };
+
+/* The search on bf16 X [M][K] and bf16 W [K][N] (device pointers). */
+int awq_search(const void* X, const void* W, int64_t M, int64_t K, int64_t N,
+               int group, int n_grid, float* out_scales, int32_t* out_codes,
+               void* out_steps, void* out_zeros, float* out_losses,
+               awq_stream_t stream);
+
+/* The same search on fp32 X and W (device pointers). The statistic, scales and
+ * QDQ read the fp32 values; the loss GEMM takes them rounded to bf16. */
+int awq_search_f32(const float* X, const float* W, int64_t M, int64_t K, int64_t N,
+                   int group, int n_grid, float* out_scales, int32_t* out_codes,
+                   void* out_steps, void* out_zeros, float* out_losses,
+                   awq_stream_t stream);
+
+/* Full form: `in_dtype` is AWQ_DTYPE_BF16 or AWQ_DTYPE_F32 for both X and W.
+ * `out_tile_sq_err` (may be NULL) receives the fp64 squared-error partial sums the
+ * loss GEMM produced: [n_grid][tiles_m][tiles_n], tile (tm, tn) covering rows
+ * tm*tile_m .. and columns tn*tile_n .. (awq_tile_shape); L_i equals the sum of row i
+ * divided by M*N. `tile_sq_err_len` is its capacity in elements. */
+int awq_search_ex(const void* X, const void* W, int in_dtype, int64_t M, int64_t K,
+                  int64_t N, int group, int n_grid, float* out_scales,
+                  int32_t* out_codes, void* out_steps, void* out_zeros,
+                  float* out_losses, double* out_tile_sq_err, int64_t tile_sq_err_len,
+                  awq_stream_t stream);
+
+/* End-to-end form with HOST buffers: copies X and W to the device on `stream`,
+ * runs awq_search_ex, copies the outputs back (out_losses may be NULL). Pinned
+ * host memory makes the copies asynchronous; pageable memory also works. */
+int awq_search_host(const void* X_host, const void* W_host, int in_dtype, int64_t M,
+                    int64_t K, int64_t N, int group, int n_grid, float* out_scales_host,
+                    int32_t* out_codes_host, void* out_steps_host, void* out_zeros_host,
+                    float* out_losses_host, awq_stream_t stream);
+
+/* Output tile of the loss GEMM (rows of X, columns of W). */
+void awq_tile_shape(int* tile_m, int* tile_n);
+
+/* Work space bytes one call needs for these sizes (0 on bad arguments). */
+int64_t awq_workspace_bytes(int in_dtype, int64_t M, int64_t K, int64_t N, int group,
+                            int n_grid);
+
+/* Return the memory cached by the library's pool on the current device. */
+int awq_release_cached(void);
+
+const char* awq_status_string(int status);
+/* Detail of the last failure on the calling thread (empty when none). */
+const char* awq_last_error_message(void);
+
+/* Per-phase device timing of the next calls: CUDA events recorded on `stream`
+ * between the kernels of each call. awq_profile_last writes up to `n` phase
+ * times (ms) of the last call and returns the number of phases. */
+int awq_profile_enable(int on);
+int awq_profile_last(float* ms, int n);
+const char* awq_profile_phase_name(int phase);
+/* Kernel launches the last call made (all of them this library's own kernels). */
+int awq_last_launch_count(void);
+
+/* Testing hook for the bounded waits: mode 1 makes the loss GEMM's producer skip
+ * one stage's loads and arrive, so its consumer's wait runs out and the call
+ * returns AWQ_ERR_TIMEOUT; `timeout_ns` bounds every wait (0 = the default 2 s).
+ * Mode 0 restores normal operation. */
+int awq_debug_set_fault(int mode, int64_t timeout_ns);
+
+int awq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AWQ_SEARCH_H_ */

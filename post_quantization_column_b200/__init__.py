@@ -1,0 +1,238 @@
+"""AWQ activation-aware per-layer scale search on NVIDIA B200 (sm_100a).
+
+Python binding of ``libawqsearch.so`` (C ABI in ``include/awq_search.h``). This module
+only marshals arguments: torch provides device memory and the stream, and every step
+of the search runs in the library's CUDA kernels. There is no CPU fallback: if the
+library is missing or cannot load, every call raises.
+
+    import torch, post_quantization_column_b200 as awq
+    out = awq.search(X, W, group=128, n_grid=20)   # X: (M, K) bf16/fp32 CUDA, W: (K, N)
+    out.scales, out.codes, out.steps, out.zeros, out.losses, out.best
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from dataclasses import dataclass
+
+import torch
+
+__all__ = [
+    "AwqError", "SearchOutput", "search", "search_host", "library", "library_path", "header_path",
+    "tile_shape", "workspace_bytes", "release_cached", "profile_enable", "profile_last",
+    "last_launch_count", "debug_set_fault", "status_string", "exported_functions",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libawqsearch.so")
+_HEADER = os.path.join(os.path.dirname(_PKG), "include", "awq_search.h")
+
+DTYPE_BF16, DTYPE_F32 = 0, 1
+_STATUS = {0: "AWQ_OK", 1: "AWQ_ERR_INVALID_ARG", 2: "AWQ_ERR_SHAPE", 3: "AWQ_ERR_NONFINITE",
+           4: "AWQ_ERR_OOM", 5: "AWQ_ERR_CUDA", 6: "AWQ_ERR_TIMEOUT", 7: "AWQ_ERR_UNSUPPORTED_DEVICE"}
+
+_lib = None
+
+
+class AwqError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def header_path() -> str:
+    return _HEADER
+
+
+def library() -> ctypes.CDLL:
+    """Load libawqsearch.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                           "`python -m post_quantization_column_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i64, i32, f32p, f64p = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p
+    lib.awq_search.argtypes = [vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp]
+    lib.awq_search_f32.argtypes = [vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp]
+    lib.awq_search_ex.argtypes = [vp, vp, i32, i64, i64, i64, i32, i32, vp, vp, vp, vp, f32p, f64p, i64, vp]
+    lib.awq_search_host.argtypes = [vp, vp, i32, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp]
+    for name in ("awq_search", "awq_search_f32", "awq_search_ex", "awq_search_host", "awq_release_cached",
+                 "awq_profile_enable", "awq_profile_last", "awq_last_launch_count", "awq_debug_set_fault",
+                 "awq_version"):
+        getattr(lib, name).restype = ctypes.c_int
+    lib.awq_tile_shape.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
+    lib.awq_tile_shape.restype = None
+    lib.awq_workspace_bytes.argtypes = [i32, i64, i64, i64, i32, i32]
+    lib.awq_workspace_bytes.restype = ctypes.c_int64
+    lib.awq_status_string.argtypes = [i32]
+    lib.awq_status_string.restype = ctypes.c_char_p
+    lib.awq_last_error_message.argtypes = []
+    lib.awq_last_error_message.restype = ctypes.c_char_p
+    lib.awq_profile_enable.argtypes = [i32]
+    lib.awq_profile_last.argtypes = [ctypes.POINTER(ctypes.c_float), i32]
+    lib.awq_profile_phase_name.argtypes = [i32]
+    lib.awq_profile_phase_name.restype = ctypes.c_char_p
+    lib.awq_debug_set_fault.argtypes = [i32, i64]
+    _lib = lib
+    return lib
+
+
+def exported_functions() -> list[str]:
+    """Function names `include/awq_search.h` declares."""
+    with open(_HEADER) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(awq_[a-z0-9_]+)\s*\(", text)))
+
+
+def status_string(status: int) -> str:
+    return library().awq_status_string(status).decode()
+
+
+def _check(status: int):
+    if status != 0:
+        msg = library().awq_last_error_message().decode()
+        raise AwqError(status, msg)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream_handle(stream, device) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def tile_shape() -> tuple[int, int]:
+    m, n = ctypes.c_int(), ctypes.c_int()
+    library().awq_tile_shape(ctypes.byref(m), ctypes.byref(n))
+    return m.value, n.value
+
+
+def workspace_bytes(M: int, K: int, N: int, group: int = 128, n_grid: int = 20, dtype=torch.bfloat16) -> int:
+    return int(library().awq_workspace_bytes(DTYPE_BF16 if dtype == torch.bfloat16 else DTYPE_F32,
+                                             M, K, N, group, n_grid))
+
+
+def release_cached() -> None:
+    _check(library().awq_release_cached())
+
+
+def profile_enable(on: bool = True) -> None:
+    library().awq_profile_enable(1 if on else 0)
+
+
+def profile_last() -> dict:
+    lib = library()
+    buf = (ctypes.c_float * 16)()
+    n = lib.awq_profile_last(buf, 16)
+    return {lib.awq_profile_phase_name(i).decode(): float(buf[i]) for i in range(n)}
+
+
+def last_launch_count() -> int:
+    return int(library().awq_last_launch_count())
+
+
+def debug_set_fault(mode: int, timeout_ns: int = 0) -> None:
+    _check(library().awq_debug_set_fault(mode, timeout_ns))
+
+
+@dataclass
+class SearchOutput:
+    scales: torch.Tensor        # (K,) fp32: the chosen s
+    codes: torch.Tensor         # (K, N/8) int32: eight 4-bit codes per word along N
+    steps: torch.Tensor         # (K/group, N) fp16
+    zeros: torch.Tensor         # (K/group, N) fp16
+    losses: torch.Tensor        # (n_grid,) fp32
+    tile_sq_err: torch.Tensor | None = None  # (n_grid, tiles_m, tiles_n) fp64
+
+    @property
+    def best(self) -> int:
+        """Index of the chosen alpha = first minimum of the losses."""
+        vals = self.losses.detach().cpu().tolist()
+        b = 0
+        for i, v in enumerate(vals):
+            if v < vals[b]:
+                b = i
+        return b
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return DTYPE_BF16
+    if t.dtype == torch.float32:
+        return DTYPE_F32
+    raise TypeError(f"X and W must be bfloat16 or float32, got {t.dtype}")
+
+
+def _alloc_outputs(K, N, group, n_grid, device, pin=False):
+    kw = dict(device=device) if not pin else dict(pin_memory=True)
+    return (torch.empty(K, dtype=torch.float32, **kw),
+            torch.empty(K, N // 8, dtype=torch.int32, **kw),
+            torch.empty(K // group, N, dtype=torch.float16, **kw),
+            torch.empty(K // group, N, dtype=torch.float16, **kw),
+            torch.empty(n_grid, dtype=torch.float32, **kw))
+
+
+def search(X: torch.Tensor, W: torch.Tensor, group: int = 128, n_grid: int = 20, *,
+           stream: torch.cuda.Stream | None = None, tile_sq_err: bool = False) -> SearchOutput:
+    """Run the search on device tensors X (M, K) and W (K, N) of the same dtype."""
+    if X.dim() != 2 or W.dim() != 2 or X.shape[1] != W.shape[0]:
+        raise ValueError("X must be (M, K) and W must be (K, N)")
+    if X.dtype != W.dtype:
+        raise TypeError("X and W must share a dtype")
+    if not (X.is_cuda and W.is_cuda):
+        raise ValueError("search() takes CUDA tensors; use search_host() for host tensors")
+    lib = library()
+    X = X.contiguous()
+    W = W.contiguous()
+    M, K = X.shape
+    N = W.shape[1]
+    if group <= 0 or K % group or N % 8:
+        raise ValueError("group must divide K and N must be a multiple of 8")
+    scales, codes, steps, zeros, losses = _alloc_outputs(K, N, group, n_grid, X.device)
+    tiles = None
+    if tile_sq_err:
+        tm, tn = tile_shape()
+        tiles = torch.empty(n_grid, -(-M // tm), -(-N // tn), dtype=torch.float64, device=X.device)
+    st = lib.awq_search_ex(_ptr(X), _ptr(W), _dtype_code(X), M, K, N, group, n_grid, _ptr(scales), _ptr(codes),
+                           _ptr(steps), _ptr(zeros), _ptr(losses), _ptr(tiles),
+                           tiles.numel() if tiles is not None else 0, _stream_handle(stream, X.device))
+    _check(st)
+    return SearchOutput(scales, codes, steps, zeros, losses, tiles)
+
+
+def search_host(X: torch.Tensor, W: torch.Tensor, group: int = 128, n_grid: int = 20, *,
+                stream: torch.cuda.Stream | None = None, out: tuple | None = None,
+                device: int | torch.device | None = None) -> SearchOutput:
+    """End-to-end form: host tensors in (pinned for asynchronous copies), host tensors out.
+
+    The library copies X and W to the device, runs the search and copies the artifact
+    back, all on `stream` (default: the current stream of `device`).
+    """
+    if X.is_cuda or W.is_cuda:
+        raise ValueError("search_host() takes host tensors")
+    if X.dtype != W.dtype:
+        raise TypeError("X and W must share a dtype")
+    lib = library()
+    X = X.contiguous()
+    W = W.contiguous()
+    M, K = X.shape
+    N = W.shape[1]
+    if out is None:
+        out = _alloc_outputs(K, N, group, n_grid, None, pin=True)
+    scales, codes, steps, zeros, losses = out
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    st = lib.awq_search_host(_ptr(X), _ptr(W), _dtype_code(X), M, K, N, group, n_grid, _ptr(scales), _ptr(codes),
+                             _ptr(steps), _ptr(zeros), _ptr(losses), _stream_handle(stream, dev))
+    _check(st)
+    return SearchOutput(scales, codes, steps, zeros, losses)

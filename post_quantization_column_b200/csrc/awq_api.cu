@@ -1,0 +1,482 @@
+// awq_api.cu — the C ABI of libawqsearch.so (declared in include/awq_search.h).
+//
+// Validates the call, carves the device work space from a library-owned
+// stream-ordered memory pool, enqueues the search kernels on the caller's stream in
+// the order of "AWQ：为什么 4-bit 权重量化要先观察 Activation" §4 (statistic -> scales ->
+// QDQ of every candidate -> loss GEMM -> argmin) and §7 (artifact), synchronizes the
+// stream and turns the kernels' device status word into an awq_status.
+#include "../../include/awq_search.h"
+#include "awq_device.cuh"
+#include "awq_kernels.h"
+
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <unordered_map>
+
+namespace {
+
+using namespace awq;
+
+constexpr int kVersion = 1;
+constexpr int kMaxGrid = 64;
+constexpr uint64_t kDefaultTimeoutNs = 2000ull * 1000 * 1000;
+
+enum Phase { kPhStatistic, kPhScales, kPhConvert, kPhQdq, kPhGemmY, kPhGemmLoss, kPhReduce, kPhPack, kNumPhases };
+const char* kPhaseNames[kNumPhases] = {"statistic", "scales", "to_bf16", "qdq",
+                                       "gemm_reference", "gemm_loss", "loss_reduce", "pack"};
+
+thread_local std::string t_last_error;
+std::mutex g_mu;
+std::unordered_map<int, cudaMemPool_t> g_pools;
+bool g_profile = false;
+float g_phase_ms[kNumPhases] = {0};
+int g_last_launches = 0;
+int g_fault_mode = 0;
+uint64_t g_timeout_ns = kDefaultTimeoutNs;
+
+int set_error(int status, const std::string& msg) {
+  t_last_error = msg;
+  return status;
+}
+
+int cuda_error(cudaError_t e, const char* where) {
+  return set_error(AWQ_ERR_CUDA, std::string(where) + ": " + cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
+
+int get_pool(int dev, cudaMemPool_t* out) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  auto it = g_pools.find(dev);
+  if (it != g_pools.end()) {
+    *out = it->second;
+    return AWQ_OK;
+  }
+  cudaMemPoolProps props;
+  std::memset(&props, 0, sizeof(props));
+  props.allocType = cudaMemAllocationTypePinned;
+  props.handleTypes = cudaMemHandleTypeNone;
+  props.location.type = cudaMemLocationTypeDevice;
+  props.location.id = dev;
+  cudaMemPool_t pool;
+  cudaError_t e = cudaMemPoolCreate(&pool, &props);
+  if (e != cudaSuccess) return cuda_error(e, "cudaMemPoolCreate");
+  uint64_t keep = UINT64_MAX;  // keep freed blocks for the next call
+  e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+  if (e != cudaSuccess) return cuda_error(e, "cudaMemPoolSetAttribute");
+  g_pools[dev] = pool;
+  *out = pool;
+  return AWQ_OK;
+}
+
+struct Layout {
+  size_t err, a, stat_partial, S, best, losses, Xb, Wt, Y, loss_partial, total;
+  int row_chunks;
+  int64_t tiles;
+};
+
+Layout plan(int in_dtype, int64_t M, int64_t K, int64_t N, int n_grid, int num_sms) {
+  Layout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += align_up(bytes);
+    return at;
+  };
+  L.row_chunks = statistic_row_chunks(M, K, in_dtype, num_sms);
+  const int64_t tiles_m = ceil_div(M, kTileM), tiles_n = ceil_div(N, kTileN);
+  L.tiles = tiles_m * tiles_n;
+  L.err = take(16);
+  L.a = take(static_cast<size_t>(K) * 4);
+  L.stat_partial = take(static_cast<size_t>(L.row_chunks) * K * 8);
+  L.S = take(static_cast<size_t>(n_grid) * K * 4);
+  L.best = take(16);
+  L.losses = take(static_cast<size_t>(n_grid) * 4);
+  L.Xb = in_dtype == AWQ_DTYPE_F32 ? take(static_cast<size_t>(M) * K * 2) : 0;
+  L.Wt = take(static_cast<size_t>(n_grid + 1) * N * K * 2);
+  L.Y = take(static_cast<size_t>(L.tiles) * kTileM * kTileN * 4);
+  L.loss_partial = take(static_cast<size_t>(n_grid) * L.tiles * 8);
+  L.total = off;
+  return L;
+}
+
+int validate(const void* X, const void* W, int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid,
+             const void* out_scales, const void* out_codes, const void* out_steps, const void* out_zeros,
+             bool device_ptrs) {
+  if (!X || !W || !out_scales || !out_codes || !out_steps || !out_zeros)
+    return set_error(AWQ_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (in_dtype != AWQ_DTYPE_BF16 && in_dtype != AWQ_DTYPE_F32)
+    return set_error(AWQ_ERR_INVALID_ARG, "in_dtype must be AWQ_DTYPE_BF16 or AWQ_DTYPE_F32");
+  if (group != 32 && group != 64 && group != 128)
+    return set_error(AWQ_ERR_INVALID_ARG, "group must be 32, 64 or 128");
+  if (n_grid < 1 || n_grid > kMaxGrid) return set_error(AWQ_ERR_INVALID_ARG, "n_grid must be in 1..64");
+  if (M <= 0 || K <= 0 || N <= 0) return set_error(AWQ_ERR_SHAPE, "M, K and N must be positive");
+  if (M >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) || N >= (int64_t(1) << 31))
+    return set_error(AWQ_ERR_SHAPE, "M, K and N must be below 2^31");
+  if (K % group) return set_error(AWQ_ERR_SHAPE, "group must divide K");
+  if (K / group > 65535) return set_error(AWQ_ERR_SHAPE, "K / group must not exceed 65535");
+  if (N % 8) return set_error(AWQ_ERR_SHAPE, "N must be a multiple of 8 (eight codes per int32)");
+  if (device_ptrs && (!aligned16(X) || !aligned16(W) || !aligned16(out_scales) || !aligned16(out_codes) ||
+                      !aligned16(out_steps) || !aligned16(out_zeros)))
+    return set_error(AWQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  return AWQ_OK;
+}
+
+// Makes the device of `s` (or, for the legacy default stream, the device that owns
+// `ptr`) current for this library's runtime, so calls from any host thread and any
+// device work without a separate device-selection call.
+void bind_device(cudaStream_t s, const void* ptr) {
+  int dev = -1;
+  if (s != nullptr && cudaStreamGetDevice(s, &dev) != cudaSuccess) {
+    cudaGetLastError();
+    dev = -1;
+  }
+  if (dev < 0 && ptr != nullptr) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, ptr) == cudaSuccess && at.type == cudaMemoryTypeDevice)
+      dev = at.device;
+    else
+      cudaGetLastError();
+  }
+  if (dev >= 0) cudaSetDevice(dev);
+}
+
+bool is_device_memory(const void* p) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+}
+
+int check_device(int* dev, int* num_sms) {
+  cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return cuda_error(e, "cudaGetDevice");
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, *dev);
+  cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, *dev);
+  if (major != 10 || minor != 0)
+    return set_error(AWQ_ERR_UNSUPPORTED_DEVICE,
+                     "this library is built for sm_100a (B200); device is sm_" + std::to_string(major * 10 + minor));
+  return AWQ_OK;
+}
+
+struct Events {
+  cudaEvent_t ev[kNumPhases + 1];
+  bool on = false;
+  cudaStream_t s;
+  void create(bool enable, cudaStream_t stream) {
+    on = enable;
+    s = stream;
+    if (!on) return;
+    for (auto& e : ev) cudaEventCreate(&e);
+  }
+  void mark(int i) {
+    if (on) cudaEventRecord(ev[i], s);
+  }
+  void collect() {
+    if (!on) return;
+    for (int i = 0; i < kNumPhases; ++i) cudaEventElapsedTime(&g_phase_ms[i], ev[i], ev[i + 1]);
+    for (auto& e : ev) cudaEventDestroy(e);
+    on = false;
+  }
+  ~Events() {
+    if (on)
+      for (auto& e : ev) cudaEventDestroy(e);
+  }
+};
+
+int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid,
+                  float* out_scales, int32_t* out_codes, void* out_steps, void* out_zeros, float* out_losses,
+                  double* out_tile_sq_err, int64_t tile_sq_err_len, cudaStream_t s) {
+  int st = validate(X, W, in_dtype, M, K, N, group, n_grid, out_scales, out_codes, out_steps, out_zeros, true);
+  if (st != AWQ_OK) return st;
+  if (out_losses && !aligned16(out_losses)) {
+    // losses are written as plain floats; 4-byte alignment is enough
+    if (reinterpret_cast<uintptr_t>(out_losses) & 3u) return set_error(AWQ_ERR_INVALID_ARG, "out_losses misaligned");
+  }
+  bind_device(s, X);
+  int dev = 0, num_sms = 0;
+  st = check_device(&dev, &num_sms);
+  if (st != AWQ_OK) return st;
+  if (!is_device_memory(X) || !is_device_memory(W) || !is_device_memory(out_scales) ||
+      !is_device_memory(out_codes) || !is_device_memory(out_steps) || !is_device_memory(out_zeros) ||
+      (out_losses && !is_device_memory(out_losses)) || (out_tile_sq_err && !is_device_memory(out_tile_sq_err)))
+    return set_error(AWQ_ERR_INVALID_ARG, "inputs and outputs must be device memory (use awq_search_host for host buffers)");
+  const Layout L = plan(in_dtype, M, K, N, n_grid, num_sms);
+  if (out_tile_sq_err && tile_sq_err_len < static_cast<int64_t>(n_grid) * L.tiles)
+    return set_error(AWQ_ERR_INVALID_ARG, "out_tile_sq_err holds fewer than n_grid * tiles values");
+
+  cudaMemPool_t pool;
+  st = get_pool(dev, &pool);
+  if (st != AWQ_OK) return st;
+  void* ws = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, L.total, pool, s);
+  if (e != cudaSuccess || !ws) {
+    cudaGetLastError();
+    return set_error(AWQ_ERR_OOM, "work space of " + std::to_string(L.total) + " bytes: " + cudaGetErrorString(e));
+  }
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int* err = reinterpret_cast<int*>(base + L.err);
+  float* a = reinterpret_cast<float*>(base + L.a);
+  double* stat_partial = reinterpret_cast<double*>(base + L.stat_partial);
+  float* S = reinterpret_cast<float*>(base + L.S);
+  int* best = reinterpret_cast<int*>(base + L.best);
+  float* losses = reinterpret_cast<float*>(base + L.losses);
+  __nv_bfloat16* Wt = reinterpret_cast<__nv_bfloat16*>(base + L.Wt);
+  float* Y = reinterpret_cast<float*>(base + L.Y);
+  double* loss_partial = reinterpret_cast<double*>(base + L.loss_partial);
+  const __nv_bfloat16* Xb = in_dtype == AWQ_DTYPE_F32 ? reinterpret_cast<__nv_bfloat16*>(base + L.Xb)
+                                                      : static_cast<const __nv_bfloat16*>(X);
+
+  int launches = 0;
+  Events ev;
+  ev.create(g_profile, s);
+  const char* where = "";
+  int status = AWQ_OK;
+  do {
+    if ((e = cudaMemsetAsync(err, 0, 16, s)) != cudaSuccess) { where = "cudaMemsetAsync"; break; }
+    ev.mark(kPhStatistic);
+    if ((e = launch_statistic(X, in_dtype, M, K, L.row_chunks, stat_partial, a, err, s, &launches)) != cudaSuccess) {
+      where = "statistic kernel";
+      break;
+    }
+    ev.mark(kPhScales);
+    if ((e = launch_scales(a, K, n_grid, S, s, &launches)) != cudaSuccess) { where = "scales kernel"; break; }
+    ev.mark(kPhConvert);
+    if (in_dtype == AWQ_DTYPE_F32) {
+      if ((e = launch_to_bf16(static_cast<const float*>(X), M * K, const_cast<__nv_bfloat16*>(Xb), s, &launches)) !=
+          cudaSuccess) {
+        where = "bf16 operand kernel";
+        break;
+      }
+    }
+    ev.mark(kPhQdq);
+    if ((e = launch_qdq(W, in_dtype, K, N, group, n_grid, S, Wt, err, s, &launches)) != cudaSuccess) {
+      where = "qdq kernel";
+      break;
+    }
+    LossGemmArgs ga;
+    ga.Xb = Xb;
+    ga.Wt = Wt;
+    ga.M = M;
+    ga.K = K;
+    ga.N = N;
+    ga.n_grid = n_grid;
+    ga.Y = Y;
+    ga.partial = loss_partial;
+    ga.err = err;
+    ga.timeout_ns = g_timeout_ns;
+    ga.fault_mode = g_fault_mode;
+    ga.num_sms = num_sms;
+    CUtensorMap mapA, mapB;
+    const char* why = "";
+    if ((e = make_operand_maps(ga, &mapA, &mapB, &why)) != cudaSuccess) {
+      status = set_error(AWQ_ERR_CUDA, std::string("TMA descriptor: ") + why);
+      break;
+    }
+    ev.mark(kPhGemmY);
+    if ((e = launch_loss_gemm(ga, mapA, mapB, 0, s, &launches)) != cudaSuccess) { where = "reference GEMM"; break; }
+    ev.mark(kPhGemmLoss);
+    if ((e = launch_loss_gemm(ga, mapA, mapB, 1, s, &launches)) != cudaSuccess) { where = "loss GEMM"; break; }
+    ev.mark(kPhReduce);
+    if ((e = launch_loss_reduce(loss_partial, L.tiles, n_grid, M, N, losses, best, s, &launches)) != cudaSuccess) {
+      where = "loss reduction kernel";
+      break;
+    }
+    ev.mark(kPhPack);
+    if ((e = launch_pack(W, in_dtype, K, N, group, S, best, out_codes, static_cast<__half*>(out_steps),
+                         static_cast<__half*>(out_zeros), out_scales, s, &launches)) != cudaSuccess) {
+      where = "pack kernel";
+      break;
+    }
+    ev.mark(kNumPhases);
+    if (out_losses &&
+        (e = cudaMemcpyAsync(out_losses, losses, static_cast<size_t>(n_grid) * 4, cudaMemcpyDeviceToDevice, s)) !=
+            cudaSuccess) {
+      where = "copy of the losses";
+      break;
+    }
+    if (out_tile_sq_err &&
+        (e = cudaMemcpyAsync(out_tile_sq_err, loss_partial, static_cast<size_t>(n_grid) * L.tiles * 8,
+                             cudaMemcpyDeviceToDevice, s)) != cudaSuccess) {
+      where = "copy of the tile partials";
+      break;
+    }
+  } while (false);
+
+  int h_err = 0;
+  if (status == AWQ_OK && e == cudaSuccess) {
+    e = cudaMemcpyAsync(&h_err, err, sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) where = "status read-back";
+  }
+  if (status == AWQ_OK && e != cudaSuccess) status = cuda_error(e, where);
+  cudaFreeAsync(ws, s);
+  cudaError_t se = cudaStreamSynchronize(s);
+  if (status == AWQ_OK && se != cudaSuccess) status = cuda_error(se, "stream synchronize");
+  if (status == AWQ_OK) {
+    ev.collect();
+    g_last_launches = launches;
+    if (h_err & kErrTimeout)
+      status = set_error(AWQ_ERR_TIMEOUT, "a bounded wait in the loss GEMM ran out");
+    else if (h_err & (kErrNonfiniteX | kErrNonfiniteW))
+      status = set_error(AWQ_ERR_NONFINITE, (h_err & kErrNonfiniteX) ? "non-finite value in X" : "non-finite value in W");
+    else if (h_err)
+      status = set_error(AWQ_ERR_CUDA, "device status word " + std::to_string(h_err));
+  }
+  return status;
+}
+
+}  // namespace
+
+extern "C" {
+
+int awq_search_ex(const void* X, const void* W, int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid,
+                  float* out_scales, int32_t* out_codes, void* out_steps, void* out_zeros, float* out_losses,
+                  double* out_tile_sq_err, int64_t tile_sq_err_len, awq_stream_t stream) {
+  t_last_error.clear();
+  return search_device(X, W, in_dtype, M, K, N, group, n_grid, out_scales, out_codes, out_steps, out_zeros,
+                       out_losses, out_tile_sq_err, tile_sq_err_len, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int awq_search(const void* X, const void* W, int64_t M, int64_t K, int64_t N, int group, int n_grid,
+               float* out_scales, int32_t* out_codes, void* out_steps, void* out_zeros, float* out_losses,
+               awq_stream_t stream) {
+  return awq_search_ex(X, W, AWQ_DTYPE_BF16, M, K, N, group, n_grid, out_scales, out_codes, out_steps, out_zeros,
+                       out_losses, nullptr, 0, stream);
+}
+
+int awq_search_f32(const float* X, const float* W, int64_t M, int64_t K, int64_t N, int group, int n_grid,
+                   float* out_scales, int32_t* out_codes, void* out_steps, void* out_zeros, float* out_losses,
+                   awq_stream_t stream) {
+  return awq_search_ex(X, W, AWQ_DTYPE_F32, M, K, N, group, n_grid, out_scales, out_codes, out_steps, out_zeros,
+                       out_losses, nullptr, 0, stream);
+}
+
+int awq_search_host(const void* X_host, const void* W_host, int in_dtype, int64_t M, int64_t K, int64_t N, int group,
+                    int n_grid, float* out_scales_host, int32_t* out_codes_host, void* out_steps_host,
+                    void* out_zeros_host, float* out_losses_host, awq_stream_t stream) {
+  t_last_error.clear();
+  int st = validate(X_host, W_host, in_dtype, M, K, N, group, n_grid, out_scales_host, out_codes_host,
+                    out_steps_host, out_zeros_host, false);
+  if (st != AWQ_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  bind_device(s, nullptr);
+  int dev = 0, num_sms = 0;
+  st = check_device(&dev, &num_sms);
+  if (st != AWQ_OK) return st;
+  cudaMemPool_t pool;
+  st = get_pool(dev, &pool);
+  if (st != AWQ_OK) return st;
+  const size_t eb = in_dtype == AWQ_DTYPE_BF16 ? 2 : 4;
+  const size_t G = static_cast<size_t>(K / group);
+  const size_t bx = static_cast<size_t>(M) * K * eb, bw = static_cast<size_t>(K) * N * eb;
+  const size_t bs = static_cast<size_t>(K) * 4, bc = static_cast<size_t>(K) * (N / 8) * 4;
+  const size_t bst = G * N * 2, bl = static_cast<size_t>(n_grid) * 4;
+  size_t off[7], total = 0;
+  const size_t sizes[7] = {bx, bw, bs, bc, bst, bst, bl};
+  for (int i = 0; i < 7; ++i) {
+    off[i] = total;
+    total += align_up(sizes[i]);
+  }
+  void* buf = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(&buf, total, pool, s);
+  if (e != cudaSuccess || !buf) {
+    cudaGetLastError();
+    return set_error(AWQ_ERR_OOM, "device buffers for the host call");
+  }
+  uint8_t* b = static_cast<uint8_t*>(buf);
+  int status = AWQ_OK;
+  if ((e = cudaMemcpyAsync(b + off[0], X_host, bx, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(b + off[1], W_host, bw, cudaMemcpyHostToDevice, s)) != cudaSuccess) {
+    status = cuda_error(e, "host-to-device copy");
+  }
+  if (status == AWQ_OK)
+    status = search_device(b + off[0], b + off[1], in_dtype, M, K, N, group, n_grid, reinterpret_cast<float*>(b + off[2]),
+                           reinterpret_cast<int32_t*>(b + off[3]), b + off[4], b + off[5],
+                           reinterpret_cast<float*>(b + off[6]), nullptr, 0, s);
+  if (status == AWQ_OK) {
+    if ((e = cudaMemcpyAsync(out_scales_host, b + off[2], bs, cudaMemcpyDeviceToHost, s)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(out_codes_host, b + off[3], bc, cudaMemcpyDeviceToHost, s)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(out_steps_host, b + off[4], bst, cudaMemcpyDeviceToHost, s)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(out_zeros_host, b + off[5], bst, cudaMemcpyDeviceToHost, s)) != cudaSuccess ||
+        (out_losses_host &&
+         (e = cudaMemcpyAsync(out_losses_host, b + off[6], bl, cudaMemcpyDeviceToHost, s)) != cudaSuccess))
+      status = cuda_error(e, "device-to-host copy");
+  }
+  cudaFreeAsync(buf, s);
+  cudaError_t se = cudaStreamSynchronize(s);
+  if (status == AWQ_OK && se != cudaSuccess) status = cuda_error(se, "stream synchronize");
+  return status;
+}
+
+void awq_tile_shape(int* tile_m, int* tile_n) {
+  if (tile_m) *tile_m = kTileM;
+  if (tile_n) *tile_n = kTileN;
+}
+
+int64_t awq_workspace_bytes(int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid) {
+  static int dummy;
+  if (validate(&dummy, &dummy, in_dtype, M, K, N, group, n_grid, &dummy, &dummy, &dummy, &dummy, false) != AWQ_OK)
+    return 0;
+  return static_cast<int64_t>(plan(in_dtype, M, K, N, n_grid, 148).total);
+}
+
+int awq_release_cached(void) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return set_error(AWQ_ERR_CUDA, "cudaGetDevice");
+  std::lock_guard<std::mutex> lock(g_mu);
+  auto it = g_pools.find(dev);
+  if (it == g_pools.end()) return AWQ_OK;
+  cudaError_t e = cudaMemPoolTrimTo(it->second, 0);
+  return e == cudaSuccess ? AWQ_OK : cuda_error(e, "cudaMemPoolTrimTo");
+}
+
+const char* awq_status_string(int status) {
+  switch (status) {
+    case AWQ_OK: return "AWQ_OK";
+    case AWQ_ERR_INVALID_ARG: return "AWQ_ERR_INVALID_ARG";
+    case AWQ_ERR_SHAPE: return "AWQ_ERR_SHAPE";
+    case AWQ_ERR_NONFINITE: return "AWQ_ERR_NONFINITE";
+    case AWQ_ERR_OOM: return "AWQ_ERR_OOM";
+    case AWQ_ERR_CUDA: return "AWQ_ERR_CUDA";
+    case AWQ_ERR_TIMEOUT: return "AWQ_ERR_TIMEOUT";
+    case AWQ_ERR_UNSUPPORTED_DEVICE: return "AWQ_ERR_UNSUPPORTED_DEVICE";
+    default: return "AWQ_ERR_UNKNOWN";
+  }
+}
+
+const char* awq_last_error_message(void) { return t_last_error.c_str(); }
+
+int awq_profile_enable(int on) {
+  g_profile = on != 0;
+  return AWQ_OK;
+}
+
+int awq_profile_last(float* ms, int n) {
+  for (int i = 0; i < n && i < kNumPhases; ++i) ms[i] = g_phase_ms[i];
+  return kNumPhases;
+}
+
+const char* awq_profile_phase_name(int phase) {
+  return (phase >= 0 && phase < kNumPhases) ? kPhaseNames[phase] : "";
+}
+
+int awq_last_launch_count(void) { return g_last_launches; }
+
+int awq_debug_set_fault(int mode, int64_t timeout_ns) {
+  if (mode != 0 && mode != 1) return set_error(AWQ_ERR_INVALID_ARG, "fault mode must be 0 or 1");
+  g_fault_mode = mode;
+  g_timeout_ns = timeout_ns > 0 ? static_cast<uint64_t>(timeout_ns) : kDefaultTimeoutNs;
+  return AWQ_OK;
+}
+
+int awq_version(void) { return kVersion; }
+
+}  // extern "C"

@@ -1,0 +1,68 @@
+// awq_kernels.h — host-side launchers of the search kernels (internal to libawqsearch).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace awq {
+
+// Loss GEMM tile: BM rows of X by BN columns of W per output tile.
+constexpr int kTileM = 128;
+constexpr int kTileN = 256;
+constexpr int kTileK = 64;
+
+// ---- statistic (AWQ-P1 §1) -------------------------------------------------------
+// Number of row chunks the first pass splits M into for a K of this size.
+int statistic_row_chunks(int64_t M, int64_t K, int in_dtype, int num_sms);
+cudaError_t launch_statistic(const void* X, int in_dtype, int64_t M, int64_t K, int row_chunks,
+                             double* partial, float* a, int* err, cudaStream_t s, int* launches);
+
+// ---- candidate scales (AWQ-P1 §3-§4) ---------------------------------------------
+cudaError_t launch_scales(const float* a, int64_t K, int n_grid, float* S, cudaStream_t s,
+                          int* launches);
+
+// ---- fp32 -> bf16 operand copy (fp32 layers only) --------------------------------
+cudaError_t launch_to_bf16(const float* x, int64_t n, __nv_bfloat16* out, cudaStream_t s,
+                           int* launches);
+
+// ---- scale + QDQ + fold-back of every candidate (AWQ-P1 §4, §7) -------------------
+// Writes Wt[0] = bf16(W)^T and Wt[1 + i] = bf16(W_hat_i)^T, each N x K (K contiguous).
+cudaError_t launch_qdq(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid,
+                       const float* S, __nv_bfloat16* Wt, int* err, cudaStream_t s, int* launches);
+
+// ---- artifact of the chosen candidate (AWQ-P1 §7; QUANT-P4 §5.3) ------------------
+cudaError_t launch_pack(const void* W, int in_dtype, int64_t K, int64_t N, int group, const float* S,
+                        const int* best, int32_t* codes, __half* steps, __half* zeros,
+                        float* out_scales, cudaStream_t s, int* launches);
+
+// ---- loss GEMM (AWQ-P1 §4) ---------------------------------------------------------
+struct LossGemmArgs {
+  const __nv_bfloat16* Xb;   // [M][K]
+  const __nv_bfloat16* Wt;   // [n_grid + 1][N][K]
+  int64_t M, K, N;
+  int n_grid;
+  float* Y;                  // tiled reference output, tiles_m * tiles_n * BM * BN floats
+  double* partial;           // [n_grid][tiles_m * tiles_n]
+  int* err;
+  uint64_t timeout_ns;
+  int fault_mode;
+  int num_sms;
+};
+// Builds the TMA descriptors (driver entry point) for the two operands.
+cudaError_t make_operand_maps(const LossGemmArgs& a, CUtensorMap* mapA, CUtensorMap* mapB,
+                              const char** why);
+// mode 0: Y = X_b W_b into the tiled buffer; mode 1: per-tile sum of (X_b W_hat_i - Y)^2.
+cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, const CUtensorMap& mapB,
+                             int mode, cudaStream_t s, int* launches);
+
+// Sum the tile partials in a fixed order, divide by M*N, round to fp32, take the
+// first argmin (AWQ-P1 §3).
+cudaError_t launch_loss_reduce(const double* partial, int64_t tiles, int n_grid, int64_t M, int64_t N,
+                               float* losses, int* best, cudaStream_t s, int* launches);
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace awq

@@ -1,0 +1,394 @@
+// k_loss_gemm.cu — the candidate forward and its loss ("AWQ：为什么 4-bit 权重量化要先观察
+// Activation" §4: every candidate is scored by the mean squared difference between the
+// original output and the candidate output, the difference cast to FP32).
+//
+// One persistent kernel, two modes:
+//   mode 0: Y = X_b W_b, written once to HBM in a tile-major layout;
+//   mode 1: for every (candidate i, output tile): acc = X_b W_hat_i,b on the tensor
+//           cores, and the epilogue adds (acc - Y)^2 over the tile and writes one fp64
+//           partial sum. The candidate output Y_hat is never written to HBM.
+//
+// Blackwell structure (sm_100a): 128 x 256 output tiles, K in 64-element (128-byte)
+// slices; a 4-stage TMA -> shared-memory ring (128-byte swizzle, no multicast); one
+// elected thread issues tcgen05.mma (M=128, N=256, K=16, bf16 -> fp32) into one of
+// two 256-column tensor-memory accumulators, so the epilogue of tile t overlaps the
+// main loop of tile t+1; four epilogue warps read the accumulator with tcgen05.ld
+// (warp w % 4 owns TMEM lanes 32(w%4)..+31 = tile rows). Warp roles: 0 TMA producer,
+// 1 MMA issuer, 2 TMEM allocator, 4-7 epilogue. Units (candidate, tile) are walked in
+// a grouped raster (group_m row tiles at a time) so the X row block and the W_hat
+// column block of neighbouring CTAs stay in L2.
+//
+// Every wait is bounded (global timer); a wait that runs out sets the call's
+// timeout bit, raises a CTA-wide abort flag, the producer waits for its own copies in
+// flight, the MMA thread waits for its issued MMAs, and tensor memory is freed.
+#include "awq_device.cuh"
+#include "awq_kernels.h"
+
+#include <cudaTypedefs.h>
+
+namespace awq {
+namespace {
+
+constexpr int BM = kTileM, BN = kTileN, BK = kTileK;
+constexpr int kStages = 4;
+constexpr int kABytes = BM * BK * 2;  // 16 KB
+constexpr int kBBytes = BN * BK * 2;  // 32 KB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kTmemCols = 2 * BN;     // two fp32 accumulators of 256 columns
+constexpr int kThreads = 256;
+constexpr int kEpiThreads = 128;
+constexpr int kBarrierBytes = 256;
+constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;  // + alignment slack
+constexpr int kGroupM = 16;
+constexpr uint64_t kDrainNs = 200ull * 1000 * 1000;  // bound on the waits of the abort path
+
+struct GemmParams {
+  int mode;
+  int n_grid;
+  int tiles_m, tiles_n;
+  int nk;
+  float* Y;
+  double* partial;
+  int* err;
+  uint64_t timeout_ns;
+  int fault_mode;
+};
+
+__device__ __forceinline__ void unit_coords(int64_t u, const GemmParams& p, int& c, int& mt, int& nt) {
+  const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
+  c = static_cast<int>(u / tiles);
+  const int64_t t = u - static_cast<int64_t>(c) * tiles;
+  const int64_t group_size = static_cast<int64_t>(kGroupM) * p.tiles_n;
+  const int64_t gi = t / group_size;
+  const int first_m = static_cast<int>(gi * kGroupM);
+  const int gm = min(kGroupM, p.tiles_m - first_m);
+  const int64_t r = t - gi * group_size;
+  mt = first_m + static_cast<int>(r % gm);
+  nt = static_cast<int>(r / gm);
+}
+
+__device__ __forceinline__ int named_barrier_or(uint32_t id, uint32_t nthreads, int pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %3, 0;\n\t"
+      "bar.red.or.pred p, %1, %2, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(id), "r"(nthreads), "r"(pred)
+      : "memory");
+  return static_cast<int>(r);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    loss_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                     const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kStages * kABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* full = bars;                    // [kStages] TMA landed
+  uint64_t* empty = bars + kStages;         // [kStages] MMAs done reading the stage
+  uint64_t* tfull = bars + 2 * kStages;     // [2] accumulator ready
+  uint64_t* tempty = bars + 2 * kStages + 2;  // [2] accumulator drained by the epilogue
+  uint64_t* drain = bars + 2 * kStages + 4;   // [1] abort path: all issued MMAs done
+  double* red = reinterpret_cast<double*>(bars + 2 * kStages + 5);  // [2][4]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 13);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull + a, 1);
+      mbar_init(tempty + a, kEpiThreads);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&mapA);
+    tma_prefetch_desc(&mapB);
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
+  const int64_t n_units = (p.mode == 0 ? 1 : p.n_grid) * tiles;
+  const uint64_t budget = p.timeout_ns;
+
+  auto fail = [&]() {
+    *abort_flag = 1;
+    atomicOr(p.err, kErrTimeout);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, last_parity = 0;  // per-stage bits
+      bool ok = true;
+      for (int64_t u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        int c, mt, nt;
+        unit_coords(u, p, c, mt, nt);
+        const int slot = p.mode == 0 ? 0 : c + 1;
+        for (int kb = 0; kb < p.nk; ++kb) {
+          if (!mbar_wait_bounded(empty + stage, phase ^ 1u, abort_flag, budget)) {
+            ok = false;
+            break;
+          }
+          const bool skip = p.fault_mode == 1 && p.mode == 1 && u == blockIdx.x && kb == 0;
+          if (!skip) {
+            mbar_arrive_expect_tx(full + stage, kStageBytes);
+            tma_load_2d(&mapA, full + stage, sA + stage * kABytes, kb * BK, mt * BM);
+            tma_load_3d(&mapB, full + stage, sB + stage * kBBytes, kb * BK, nt * BN, slot);
+            issued |= 1u << stage;
+            last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          }
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        fail();
+        // let the copies this thread started land before the CTA goes away
+        for (int s = 0; s < kStages; ++s)
+          if (issued & (1u << s)) mbar_wait_bounded(full + s, (last_parity >> s) & 1u, nullptr, kDrainNs);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int local = 0;
+      for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t acc_parity = (local >> 1) & 1;
+        if (!mbar_wait_bounded(tempty + acc, acc_parity ^ 1u, abort_flag, budget)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < p.nk; ++kb) {
+          if (!mbar_wait_bounded(full + stage, phase, abort_flag, budget)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t adesc = smem_desc_k_sw128(smem_u32(sA + stage * kABytes));
+          const uint64_t bdesc = smem_desc_k_sw128(smem_u32(sB + stage * kBBytes));
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)  // K = 16 per MMA: advance 32 bytes = 2 descriptor units
+            umma_bf16_f32(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          umma_commit(empty + stage);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(tfull + acc);
+      }
+      if (!ok) {
+        fail();
+        umma_commit(drain);
+        mbar_wait_bounded(drain, 0, nullptr, kDrainNs);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------- epilogue
+    const int ew = warp - 4;  // == warp % 4: TMEM lanes 32*ew .. 32*ew+31
+    const int row = ew * 32 + lane;
+    int local = 0;
+    for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, ++local) {
+      int c, mt, nt;
+      unit_coords(u, p, c, mt, nt);
+      const int acc = local & 1;
+      const uint32_t acc_parity = (local >> 1) & 1;
+      const bool ok = mbar_wait_bounded(tfull + acc, acc_parity, abort_flag, budget);
+      if (named_barrier_or(1, kEpiThreads, !ok)) {
+        if (!ok) fail();
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const int64_t tile = static_cast<int64_t>(mt) * p.tiles_n + nt;
+      float4* ytile = reinterpret_cast<float4*>(p.Y + tile * (BM * BN));
+      float sq = 0.0f;
+#pragma unroll 1
+      for (int j0 = 0; j0 < BN; j0 += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(j0), v);
+        tmem_ld_wait();
+        float4* yrow = ytile + (j0 / 4) * BM + row;  // tile layout [BN/4][BM][4]
+        if (p.mode == 0) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            yrow[q * BM] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                       __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 y = __ldg(yrow + q * BM);
+            const float d0 = __uint_as_float(v[4 * q]) - y.x;
+            const float d1 = __uint_as_float(v[4 * q + 1]) - y.y;
+            const float d2 = __uint_as_float(v[4 * q + 2]) - y.z;
+            const float d3 = __uint_as_float(v[4 * q + 3]) - y.w;
+            sq = fmaf(d0, d0, sq);
+            sq = fmaf(d1, d1, sq);
+            sq = fmaf(d2, d2, sq);
+            sq = fmaf(d3, d3, sq);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tempty + acc);
+      if (p.mode == 1) {
+        double ds = static_cast<double>(sq);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
+        if (lane == 0) red[acc * 4 + ew] = ds;
+        named_barrier_sync(2, kEpiThreads);
+        if (ew == 0 && lane == 0)
+          p.partial[static_cast<int64_t>(c) * tiles + tile] =
+              ((red[acc * 4 + 0] + red[acc * 4 + 1]) + red[acc * 4 + 2]) + red[acc * 4 + 3];
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem_base, kTmemCols);
+}
+
+// ---------------------------------------------------------------------------------
+// Loss reduction and argmin: one block, fixed summation order.
+// ---------------------------------------------------------------------------------
+constexpr int kReduceThreads = 256;
+
+__global__ void __launch_bounds__(kReduceThreads)
+    loss_reduce_kernel(const double* __restrict__ partial, int64_t tiles, int n_grid, int64_t M, int64_t N,
+                       float* __restrict__ losses, int* __restrict__ best) {
+  __shared__ double buf[kReduceThreads];
+  __shared__ float lf[64];
+  for (int c = 0; c < n_grid; ++c) {
+    double s = 0.0;
+    for (int64_t t = threadIdx.x; t < tiles; t += kReduceThreads) s += partial[static_cast<int64_t>(c) * tiles + t];
+    buf[threadIdx.x] = s;
+    __syncthreads();
+    for (int w = kReduceThreads / 2; w > 0; w >>= 1) {
+      if (threadIdx.x < w) buf[threadIdx.x] += buf[threadIdx.x + w];
+      __syncthreads();
+    }
+    if (threadIdx.x == 0) lf[c] = __double2float_rn(buf[0] / (static_cast<double>(M) * static_cast<double>(N)));
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    int b = 0;
+    for (int c = 1; c < n_grid; ++c)
+      if (lf[c] < lf[b]) b = c;  // keeps the first minimum
+    *best = b;
+    for (int c = 0; c < n_grid; ++c) losses[c] = lf[c];
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+}  // namespace
+
+cudaError_t make_operand_maps(const LossGemmArgs& a, CUtensorMap* mapA, CUtensorMap* mapB, const char** why) {
+  auto fn = encode_fn();
+  if (!fn) {
+    *why = "cuTensorMapEncodeTiled unavailable";
+    return cudaErrorNotSupported;
+  }
+  // A = X_b [M][K]: dims (K, M), box (64, 128), 128-byte swizzle
+  const cuuint64_t dimsA[2] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(a.M)};
+  const cuuint64_t strideA[1] = {static_cast<cuuint64_t>(a.K) * 2};
+  const cuuint32_t boxA[2] = {BK, BM};
+  const cuuint32_t ones[3] = {1, 1, 1};
+  CUresult r = fn(mapA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16*>(a.Xb), dimsA, strideA, boxA,
+                  ones, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    *why = "tensor map of X";
+    return cudaErrorInvalidValue;
+  }
+  // B = W_hat^T slots [n_grid+1][N][K]: dims (K, N, slots), box (64, 256, 1)
+  const cuuint64_t dimsB[3] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(a.N),
+                               static_cast<cuuint64_t>(a.n_grid + 1)};
+  const cuuint64_t strideB[2] = {static_cast<cuuint64_t>(a.K) * 2, static_cast<cuuint64_t>(a.K) * a.N * 2};
+  const cuuint32_t boxB[3] = {BK, BN, 1};
+  r = fn(mapB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16*>(a.Wt), dimsB, strideB, boxB, ones,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    *why = "tensor map of the candidate weights";
+    return cudaErrorInvalidValue;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, const CUtensorMap& mapB, int mode,
+                             cudaStream_t s, int* launches) {
+  cudaError_t e = cudaFuncSetAttribute(loss_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  GemmParams p;
+  p.mode = mode;
+  p.n_grid = a.n_grid;
+  p.tiles_m = static_cast<int>(ceil_div(a.M, BM));
+  p.tiles_n = static_cast<int>(ceil_div(a.N, BN));
+  p.nk = static_cast<int>(ceil_div(a.K, BK));
+  p.Y = a.Y;
+  p.partial = a.partial;
+  p.err = a.err;
+  p.timeout_ns = a.timeout_ns;
+  p.fault_mode = a.fault_mode;
+  const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
+  const int64_t units = (mode == 0 ? 1 : a.n_grid) * tiles;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(units, a.num_sms));
+  loss_gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(mapA, mapB, p);
+  *launches += 1;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_loss_reduce(const double* partial, int64_t tiles, int n_grid, int64_t M, int64_t N, float* losses,
+                               int* best, cudaStream_t s, int* launches) {
+  loss_reduce_kernel<<<1, kReduceThreads, 0, s>>>(partial, tiles, n_grid, M, N, losses, best);
+  *launches += 1;
+  return cudaGetLastError();
+}
+
+}  // namespace awq

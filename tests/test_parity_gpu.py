@@ -1,0 +1,136 @@
+"""CUDA search vs the CPU oracle, element by element (B200 only).
+
+Small layers use the complete oracle; they span several 128 x 256 output tiles,
+ragged row/column tails, ragged K blocks (group 32 with K not a multiple of 64),
+every group size and a few grid sizes.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import post_quantization_column_b200 as awq
+from tests import parity as P
+from workloads import WORKLOADS, custom_spec, generate, as_f32_numpy
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.init()
+
+
+def test_single_linear_layer_fp32():
+    spec = WORKLOADS["single_linear_128x256x256_f32"]
+    X, W = generate(spec)
+    P.full_parity(X, W, spec.group, spec.n_grid)
+
+
+@pytest.mark.parametrize("M,K,N,group,n_grid,law,dtype", [
+    (300, 384, 520, 128, 20, "normal", "bf16"),      # ragged M and N tails, 3 x 3 tiles
+    (200, 160, 264, 32, 20, "normal", "bf16"),       # group 32, K = 2.5 K-blocks
+    (129, 320, 776, 64, 7, "abs_normal", "bf16"),    # group 64, one extra row, odd grid
+    (64, 256, 256, 128, 1, "normal", "bf16"),        # a single candidate
+    (260, 512, 1032, 128, 20, "abs_normal", "f32"),  # fp32 inputs, ragged tails
+    (1, 128, 8, 128, 20, "normal", "bf16"),          # one token, one packed word
+])
+def test_small_layers(M, K, N, group, n_grid, law, dtype):
+    spec = custom_spec(M, K, N, dtype=dtype, law=law, group=group, n_grid=n_grid, seed=M + K + N,
+                       sigma=1.0 if law == "abs_normal" else 0.5,
+                       outlier_mult=50.0 if law == "abs_normal" else 20.0)
+    X, W = generate(spec)
+    P.full_parity(X, W, group, n_grid)
+
+
+def test_weights_on_the_grid_give_zero_loss():
+    # every (group, column) spans all 16 levels with step 1/16 and zero 7: alpha = 0
+    # reproduces W exactly (AWQ-P1 §7 reconstruction), so L_0 = 0 and alpha 0 wins
+    rng = np.random.default_rng(1)
+    K, N, group = 256, 512, 128
+    q = rng.integers(0, 16, size=(K, N))
+    q[0::group] = 0
+    q[1::group] = 15
+    W = torch.from_numpy(((q - 7) / 16.0).astype(np.float32)).to(torch.bfloat16)
+    X = torch.randn(192, K).to(torch.bfloat16)
+    gpu = P.run_gpu(X, W, group, 20)
+    assert gpu["losses"][0] == 0.0 and gpu["best"] == 0
+    assert np.array_equal(O.unpack_codes(gpu["codes"], N), q)
+
+
+def test_constant_groups_take_step_one():
+    # all-equal groups (AWQ-P1 §7's positive lower bound; step 1 here). With a single
+    # candidate alpha = 0 the scales are all 1, so every group of W' stays constant.
+    K, N, group = 128, 16, 128
+    W = torch.full((K, N), 0.25).to(torch.bfloat16)
+    W[:, 8:] = -3.0
+    X = torch.randn(8, K).to(torch.bfloat16)
+    gpu = P.run_gpu(X, W, group, 1)
+    orc = O.search(as_f32_numpy(X), as_f32_numpy(W), group=group, n_grid=1)
+    assert np.all(gpu["steps"] == 1.0)
+    assert gpu["zeros"][0, :8].tolist() == [0.0] * 8 and gpu["zeros"][0, 8:].tolist() == [3.0] * 8
+    P.check_artifact(gpu, as_f32_numpy(W), orc.S, group)
+
+
+def test_results_are_deterministic():
+    spec = custom_spec(256, 512, 768, seed=5)
+    X, W = generate(spec)
+    a = awq.search(X.cuda(), W.cuda(), tile_sq_err=True)
+    b = awq.search(X.cuda(), W.cuda(), tile_sq_err=True)
+    for name in ("scales", "codes", "steps", "zeros", "losses", "tile_sq_err"):
+        assert torch.equal(getattr(a, name), getattr(b, name)), name
+
+
+def test_host_entry_point_matches_device_entry_point():
+    spec = custom_spec(256, 384, 520, seed=9)
+    X, W = generate(spec)
+    d = awq.search(X.cuda(), W.cuda())
+    h = awq.search_host(X.pin_memory(), W.pin_memory())
+    for name in ("scales", "codes", "steps", "zeros", "losses"):
+        assert torch.equal(getattr(d, name).cpu(), getattr(h, name)), name
+
+
+def test_nonfinite_inputs_are_rejected():
+    spec = custom_spec(64, 128, 64, seed=3)
+    X, W = generate(spec)
+    Xn = X.clone()
+    Xn[5, 7] = float("nan")
+    with pytest.raises(awq.AwqError) as e:
+        awq.search(Xn.cuda(), W.cuda())
+    assert e.value.status == 3
+    Wn = W.clone()
+    Wn[3, 2] = float("inf")
+    with pytest.raises(awq.AwqError) as e:
+        awq.search(X.cuda(), Wn.cuda())
+    assert e.value.status == 3
+    # the context stays usable
+    awq.search(X.cuda(), W.cuda())
+
+
+def test_host_pointer_is_rejected_by_the_device_entry_point():
+    import ctypes
+    lib = awq.library()
+    X = torch.zeros(16, 128, dtype=torch.bfloat16)   # host memory
+    W = torch.zeros(128, 64, dtype=torch.bfloat16, device="cuda")
+    outs = [torch.empty(n, device="cuda", dtype=torch.float32) for n in (128, 128 * 8, 64, 64)]
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    st = lib.awq_search(p(X), p(W), 16, 128, 64, 128, 20, p(outs[0]), p(outs[1]), p(outs[2]), p(outs[3]),
+                        ctypes.c_void_p(0), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 1
+
+
+def test_launch_count_and_profile():
+    spec = custom_spec(256, 256, 512, seed=2)
+    X, W = generate(spec)
+    awq.profile_enable(True)
+    try:
+        awq.search(X.cuda(), W.cuda())
+        prof = awq.profile_last()
+    finally:
+        awq.profile_enable(False)
+    # statistic (2) + scales + qdq + reference GEMM + loss GEMM + reduce + pack
+    assert awq.last_launch_count() == 8
+    assert set(prof) >= {"statistic", "scales", "qdq", "gemm_reference", "gemm_loss", "loss_reduce", "pack"}
+    assert all(v >= 0 for v in prof.values()) and prof["gemm_loss"] > 0
