@@ -153,7 +153,8 @@ def asym_qdq(Wp, group: int):
     mx = Wg.max(axis=1)
     step = ((mx - mn).astype(dt) / dt(Q_MAX)).astype(dt)
     step = np.where((mx == mn) | (step == 0), dt(1), step).astype(dt)
-    zero = np.clip(np.rint((-mn / step).astype(dt)), 0, Q_MAX).astype(dt)
+    # the zero point is an integer in 0..15: adding +0 turns a rounded -0 into 0
+    zero = (np.clip(np.rint((-mn / step).astype(dt)), 0, Q_MAX).astype(dt) + dt(0)).astype(dt)
     q = np.clip(np.rint((Wg / step[:, None, :]).astype(dt)) + zero[:, None, :], 0, Q_MAX).astype(dt)
     rec = ((q - zero[:, None, :]) * step[:, None, :]).astype(dt)
     K, N = Wp.shape

@@ -39,6 +39,7 @@ __device__ __forceinline__ QdqParams qdq_params(float mn, float mx) {
   if (mx == mn || step == 0.0f) step = 1.0f;  // all-equal group (or underflow): step 1
   float z = rintf(__fdiv_rn(-mn, step));
   z = fminf(fmaxf(z, 0.0f), 15.0f);
+  z = __fadd_rn(z, 0.0f);  // the zero point is an integer: rint(-0.25) = -0 becomes +0
   p.step = step;
   p.zero = z;
   return p;

@@ -98,6 +98,10 @@ def test_asym_hand_derived_cases():
     assert step.item() == 1.0 and zero.item() == 3 and q.ravel().tolist() == [0, 0]
     q, step, zero, rec = O.asym_qdq(np.array([[2.0], [2.0]], dtype=np.float32), 2)
     assert step.item() == 1.0 and zero.item() == 0 and q.ravel().tolist() == [2, 2]
+    # the zero point is an integer: -min/step = -0.25 rounds to -0, stored as +0
+    q, step, zero, rec = O.asym_qdq(np.array([[0.25], [0.25]], dtype=np.float32), 2)
+    assert zero.item() == 0 and not np.signbit(zero).any()
+    assert not np.signbit(zero.astype(np.float16)).any()
 
 
 @pytest.mark.parametrize("gsize", [2, 3, 4])
