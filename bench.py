@@ -67,6 +67,26 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu record, if it still matches the source."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "roofline_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("kernel") != kernel or rec.get("workload") != workload:
+        return None
+    for rel, digest in rec.get("sources_sha256", {}).items():
+        full = os.path.join(ROOT, rel)
+        if not os.path.exists(full):
+            return None
+        with open(full, "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != digest:
+                return None
+    return float(rec["dram_bytes_per_launch"])
+
+
 def cpu_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -283,7 +303,9 @@ def run_ours(args, rank, world, local):
         "layers_per_s": layers_per_s,
         "roofline": {"bound": "tensor", "kernel": "loss_gemm_kernel (candidate GEMMs + fused squared error)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "peak_source": f"{peak_kind} bf16_tflops (burst)", "traffic": None,
+                     "peak_source": f"{peak_kind} bf16_tflops (burst)",
+                     "traffic": recorded_traffic("loss_gemm_kernel", spec.name),
+                     "traffic_unit": "DRAM bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
                      "ms_per_launch": gemm_avg},
         "other_kernels": {
             "qdq": {"ms": statistics.mean(qdq_ms),
