@@ -142,6 +142,31 @@ int awq_debug_set_fault(int mode, int64_t timeout_ns);
 
 int awq_version(void);
 
+/* ---- Searching without allocating -------------------------------------------
+ * No counterpart in the paper or the pages: this is a deployment variant of
+ * awq_search_ex for callers that cannot call cudaMalloc — e.g. a plugin whose host
+ * framework owns all device memory, a process whose memory budget was fixed at
+ * start-up, or a loop that must not risk an allocation's synchronisation or
+ * failure. Same arguments, same kernels and same results as awq_search_ex (without
+ * the tile partials), but the work space comes from one array of
+ * AWQ_NOALLOC_SCRATCH_BYTES compiled into the library, which every GPU that loads
+ * the library holds until the process exits; nothing is allocated or freed.
+ * Layers whose work space (awq_workspace_bytes) exceeds the array are rejected with
+ * AWQ_ERR_SHAPE and a message giving both sizes — a 1024 x 1024 x 1024 bf16 layer
+ * with 20 candidates fits, the Llama-shaped layers do not.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call before
+ * any stream capture. All calls share the array and it keeps the last call's
+ * contents (the status word is cleared at the start of each call, everything else
+ * is overwritten before it is read): calls that overlap on the GPU — on different
+ * streams or from different host threads on one device — race on it and must be
+ * serialised by the caller. */
+#define AWQ_NOALLOC_SCRATCH_BYTES (64ll << 20)
+int awq_search_noalloc(const void* X, const void* W, int in_dtype, int64_t M, int64_t K,
+                       int64_t N, int group, int n_grid, float* out_scales,
+                       int32_t* out_codes, void* out_steps, void* out_zeros,
+                       float* out_losses, awq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -335,6 +335,10 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
 
 }  // namespace
 
+namespace awq {
+void record_error_message(const char* msg) { t_last_error = msg; }
+}  // namespace awq
+
 extern "C" {
 
 int awq_search_ex(const void* X, const void* W, int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid,

@@ -65,4 +65,7 @@ cudaError_t launch_loss_reduce(const double* partial, int64_t tiles, int n_grid,
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Sets the text awq_last_error_message returns on the calling thread.
+void record_error_message(const char* msg);
+
 }  // namespace awq
