@@ -111,6 +111,20 @@ int awq_search_host(const void* X_host, const void* W_host, int in_dtype, int64_
                     int32_t* out_codes_host, void* out_steps_host, void* out_zeros_host,
                     float* out_losses_host, awq_stream_t stream);
 
+/* ---- The steps one at a time (same kernels as awq_search; device pointers) ----
+ * Step 1 (AWQ-P1 §1): out_a[K] = mean_m |X[m,j]| (fp64 sum, one rounding to fp32).
+ * Returns AWQ_ERR_NONFINITE if X holds NaN or Inf. */
+int awq_activation_statistic(const void* X, int in_dtype, int64_t M, int64_t K,
+                             float* out_a, awq_stream_t stream);
+/* Step 2 (AWQ-P1 §3-§4): out_S[n_grid][K], row i the scales of alpha_i = i/n_grid. */
+int awq_candidate_scales(const float* a, int64_t K, int n_grid, float* out_S,
+                         awq_stream_t stream);
+/* Steps 3-4 (AWQ-P1 §4, §7): from W [K][N] and S [n_grid][K], the operands the loss
+ * GEMM reads: out_wt [n_grid + 1][N][K] bf16, K contiguous; slot 0 = bf16(W)^T,
+ * slot 1 + i = bf16(diag(s_i)^-1 Q(diag(s_i) W))^T. */
+int awq_qdq_candidates(const void* W, int in_dtype, int64_t K, int64_t N, int group,
+                       int n_grid, const float* S, void* out_wt, awq_stream_t stream);
+
 /* Output tile of the loss GEMM (rows of X, columns of W). */
 void awq_tile_shape(int* tile_m, int* tile_n);
 

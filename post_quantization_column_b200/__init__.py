@@ -22,6 +22,7 @@ __all__ = [
     "AwqError", "SearchOutput", "search", "search_host", "library", "library_path", "header_path",
     "tile_shape", "workspace_bytes", "release_cached", "profile_enable", "profile_last",
     "last_launch_count", "debug_set_fault", "status_string", "exported_functions",
+    "activation_statistic", "candidate_scales", "qdq_candidates",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -80,6 +81,11 @@ def library() -> ctypes.CDLL:
     lib.awq_profile_phase_name.argtypes = [i32]
     lib.awq_profile_phase_name.restype = ctypes.c_char_p
     lib.awq_debug_set_fault.argtypes = [i32, i64]
+    lib.awq_activation_statistic.argtypes = [vp, i32, i64, i64, vp, vp]
+    lib.awq_candidate_scales.argtypes = [vp, i64, i32, vp, vp]
+    lib.awq_qdq_candidates.argtypes = [vp, i32, i64, i64, i32, i32, vp, vp, vp]
+    for name in ("awq_activation_statistic", "awq_candidate_scales", "awq_qdq_candidates"):
+        getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -209,6 +215,36 @@ def search(X: torch.Tensor, W: torch.Tensor, group: int = 128, n_grid: int = 20,
                            tiles.numel() if tiles is not None else 0, _stream_handle(stream, X.device))
     _check(st)
     return SearchOutput(scales, codes, steps, zeros, losses, tiles)
+
+
+def activation_statistic(X: torch.Tensor, *, stream=None) -> torch.Tensor:
+    """Step 1 alone: a_j = mean_m |X[m, j]| (fp32, shape (K,))."""
+    M, K = X.shape
+    X = X.contiguous()
+    a = torch.empty(K, dtype=torch.float32, device=X.device)
+    _check(library().awq_activation_statistic(_ptr(X), _dtype_code(X), M, K, _ptr(a),
+                                              _stream_handle(stream, X.device)))
+    return a
+
+
+def candidate_scales(a: torch.Tensor, n_grid: int = 20, *, stream=None) -> torch.Tensor:
+    """Step 2 alone: the (n_grid, K) candidate scale vectors."""
+    a = a.contiguous()
+    S = torch.empty(n_grid, a.numel(), dtype=torch.float32, device=a.device)
+    _check(library().awq_candidate_scales(_ptr(a), a.numel(), n_grid, _ptr(S), _stream_handle(stream, a.device)))
+    return S
+
+
+def qdq_candidates(W: torch.Tensor, S: torch.Tensor, group: int = 128, *, stream=None) -> torch.Tensor:
+    """Steps 3-4 alone: (n_grid + 1, N, K) bf16 operands; slot 0 is bf16(W)^T."""
+    K, N = W.shape
+    W = W.contiguous()
+    S = S.contiguous()
+    n_grid = S.shape[0]
+    out = torch.empty(n_grid + 1, N, K, dtype=torch.bfloat16, device=W.device)
+    _check(library().awq_qdq_candidates(_ptr(W), _dtype_code(W), K, N, group, n_grid, _ptr(S), _ptr(out),
+                                        _stream_handle(stream, W.device)))
+    return out
 
 
 def search_host(X: torch.Tensor, W: torch.Tensor, group: int = 128, n_grid: int = 20, *,

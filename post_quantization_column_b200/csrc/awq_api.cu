@@ -286,12 +286,12 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
     ev.mark(kPhGemmLoss);
     if ((e = launch_loss_gemm(ga, mapA, mapB, 1, s, &launches)) != cudaSuccess) { where = "loss GEMM"; break; }
     ev.mark(kPhReduce);
-    if ((e = launch_loss_reduce(loss_partial, L.tiles, n_grid, M, N, losses, best, s, &launches)) != cudaSuccess) {
+    if ((e = launch_loss_reduce(loss_partial, L.tiles, n_grid, M, N, losses, s, &launches)) != cudaSuccess) {
       where = "loss reduction kernel";
       break;
     }
     ev.mark(kPhPack);
-    if ((e = launch_pack(W, in_dtype, K, N, group, S, best, out_codes, static_cast<__half*>(out_steps),
+    if ((e = launch_pack(W, in_dtype, K, N, group, n_grid, S, losses, best, out_codes, static_cast<__half*>(out_steps),
                          static_cast<__half*>(out_zeros), out_scales, s, &launches)) != cudaSuccess) {
       where = "pack kernel";
       break;
@@ -418,6 +418,102 @@ int awq_search_host(const void* X_host, const void* W_host, int in_dtype, int64_
   cudaError_t se = cudaStreamSynchronize(s);
   if (status == AWQ_OK && se != cudaSuccess) status = cuda_error(se, "stream synchronize");
   return status;
+}
+
+// ---- the steps one at a time (same kernels as the search) --------------------------
+int awq_activation_statistic(const void* X, int in_dtype, int64_t M, int64_t K, float* out_a, awq_stream_t stream) {
+  t_last_error.clear();
+  static int dummy;
+  int st = validate(X, &dummy, in_dtype, M, K, 8, 32, 1, out_a, &dummy, &dummy, &dummy, false);
+  if (st != AWQ_OK) return st;
+  if (!aligned16(X) || (reinterpret_cast<uintptr_t>(out_a) & 3u))
+    return set_error(AWQ_ERR_INVALID_ARG, "X must be 16-byte aligned and out_a 4-byte aligned");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  bind_device(s, X);
+  int dev = 0, num_sms = 0;
+  if ((st = check_device(&dev, &num_sms)) != AWQ_OK) return st;
+  if (!is_device_memory(X) || !is_device_memory(out_a))
+    return set_error(AWQ_ERR_INVALID_ARG, "X and out_a must be device memory");
+  cudaMemPool_t pool;
+  if ((st = get_pool(dev, &pool)) != AWQ_OK) return st;
+  const int R = statistic_row_chunks(M, K, in_dtype, num_sms);
+  const size_t bytes = 256 + align_up(static_cast<size_t>(R) * K * 8);
+  void* ws = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, bytes, pool, s);
+  if (e != cudaSuccess || !ws) {
+    cudaGetLastError();
+    return set_error(AWQ_ERR_OOM, "statistic work space");
+  }
+  int* err = static_cast<int*>(ws);
+  double* partial = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + 256);
+  int launches = 0, h_err = 0;
+  if ((e = cudaMemsetAsync(err, 0, 16, s)) == cudaSuccess &&
+      (e = launch_statistic(X, in_dtype, M, K, R, partial, out_a, err, s, &launches)) == cudaSuccess)
+    e = cudaMemcpyAsync(&h_err, err, sizeof(int), cudaMemcpyDeviceToHost, s);
+  cudaFreeAsync(ws, s);
+  cudaError_t se = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_error(e, "statistic");
+  if (se != cudaSuccess) return cuda_error(se, "stream synchronize");
+  g_last_launches = launches;
+  if (h_err & kErrNonfiniteX) return set_error(AWQ_ERR_NONFINITE, "non-finite value in X");
+  return AWQ_OK;
+}
+
+int awq_candidate_scales(const float* a, int64_t K, int n_grid, float* out_S, awq_stream_t stream) {
+  t_last_error.clear();
+  if (!a || !out_S) return set_error(AWQ_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (K <= 0 || K >= (int64_t(1) << 31)) return set_error(AWQ_ERR_SHAPE, "K must be in 1 .. 2^31-1");
+  if (n_grid < 1 || n_grid > kMaxGrid) return set_error(AWQ_ERR_INVALID_ARG, "n_grid must be in 1..64");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  bind_device(s, a);
+  int dev = 0, num_sms = 0, st;
+  if ((st = check_device(&dev, &num_sms)) != AWQ_OK) return st;
+  if (!is_device_memory(a) || !is_device_memory(out_S))
+    return set_error(AWQ_ERR_INVALID_ARG, "a and out_S must be device memory");
+  int launches = 0;
+  cudaError_t e = launch_scales(a, K, n_grid, out_S, s, &launches);
+  cudaError_t se = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_error(e, "scales");
+  if (se != cudaSuccess) return cuda_error(se, "stream synchronize");
+  g_last_launches = launches;
+  return AWQ_OK;
+}
+
+int awq_qdq_candidates(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid, const float* S,
+                       void* out_wt, awq_stream_t stream) {
+  t_last_error.clear();
+  static int dummy;
+  int st = validate(&dummy, W, in_dtype, 1, K, N, group, n_grid, S, out_wt, &dummy, &dummy, false);
+  if (st != AWQ_OK) return st;
+  if (!aligned16(W) || !aligned16(out_wt) || (reinterpret_cast<uintptr_t>(S) & 3u))
+    return set_error(AWQ_ERR_INVALID_ARG, "W and out_wt must be 16-byte aligned, S 4-byte aligned");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  bind_device(s, W);
+  int dev = 0, num_sms = 0;
+  if ((st = check_device(&dev, &num_sms)) != AWQ_OK) return st;
+  if (!is_device_memory(W) || !is_device_memory(S) || !is_device_memory(out_wt))
+    return set_error(AWQ_ERR_INVALID_ARG, "W, S and out_wt must be device memory");
+  cudaMemPool_t pool;
+  if ((st = get_pool(dev, &pool)) != AWQ_OK) return st;
+  void* ws = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, 256, pool, s);
+  if (e != cudaSuccess || !ws) {
+    cudaGetLastError();
+    return set_error(AWQ_ERR_OOM, "status word");
+  }
+  int* err = static_cast<int*>(ws);
+  int launches = 0, h_err = 0;
+  if ((e = cudaMemsetAsync(err, 0, 16, s)) == cudaSuccess &&
+      (e = launch_qdq(W, in_dtype, K, N, group, n_grid, S, static_cast<__nv_bfloat16*>(out_wt), err, s,
+                      &launches)) == cudaSuccess)
+    e = cudaMemcpyAsync(&h_err, err, sizeof(int), cudaMemcpyDeviceToHost, s);
+  cudaFreeAsync(ws, s);
+  cudaError_t se = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_error(e, "qdq");
+  if (se != cudaSuccess) return cuda_error(se, "stream synchronize");
+  g_last_launches = launches;
+  if (h_err & kErrNonfiniteW) return set_error(AWQ_ERR_NONFINITE, "non-finite value in W");
+  return AWQ_OK;
 }
 
 void awq_tile_shape(int* tile_m, int* tile_n) {

@@ -34,8 +34,10 @@ cudaError_t launch_qdq(const void* W, int in_dtype, int64_t K, int64_t N, int gr
                        const float* S, __nv_bfloat16* Wt, int* err, cudaStream_t s, int* launches);
 
 // ---- artifact of the chosen candidate (AWQ-P1 §7; QUANT-P4 §5.3) ------------------
-cudaError_t launch_pack(const void* W, int in_dtype, int64_t K, int64_t N, int group, const float* S,
-                        const int* best, int32_t* codes, __half* steps, __half* zeros,
+// The chosen candidate is the first minimum of `losses` (AWQ-P1 §3); its index is
+// also written to *best.
+cudaError_t launch_pack(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid, const float* S,
+                        const float* losses, int* best, int32_t* codes, __half* steps, __half* zeros,
                         float* out_scales, cudaStream_t s, int* launches);
 
 // ---- loss GEMM (AWQ-P1 §4) ---------------------------------------------------------
@@ -58,10 +60,9 @@ cudaError_t make_operand_maps(const LossGemmArgs& a, CUtensorMap* mapA, CUtensor
 cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, const CUtensorMap& mapB,
                              int mode, cudaStream_t s, int* launches);
 
-// Sum the tile partials in a fixed order, divide by M*N, round to fp32, take the
-// first argmin (AWQ-P1 §3).
+// Sum the tile partials of each candidate in a fixed order, divide by M*N, round to fp32.
 cudaError_t launch_loss_reduce(const double* partial, int64_t tiles, int n_grid, int64_t M, int64_t N,
-                               float* losses, int* best, cudaStream_t s, int* launches);
+                               float* losses, cudaStream_t s, int* launches);
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 

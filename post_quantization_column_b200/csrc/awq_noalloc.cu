@@ -187,11 +187,11 @@ extern "C" int awq_search_noalloc(const void* X, const void* W, int in_dtype, in
     if ((e = make_operand_maps(ga, &mapA, &mapB, &why)) != cudaSuccess) { where = why; break; }
     if ((e = launch_loss_gemm(ga, mapA, mapB, 0, s, &launches)) != cudaSuccess) { where = "reference GEMM"; break; }
     if ((e = launch_loss_gemm(ga, mapA, mapB, 1, s, &launches)) != cudaSuccess) { where = "loss GEMM"; break; }
-    if ((e = launch_loss_reduce(loss_partial, tiles, n_grid, M, N, losses, best, s, &launches)) != cudaSuccess) {
+    if ((e = launch_loss_reduce(loss_partial, tiles, n_grid, M, N, losses, s, &launches)) != cudaSuccess) {
       where = "loss reduction kernel";
       break;
     }
-    if ((e = launch_pack(W, in_dtype, K, N, group, S, best, out_codes, static_cast<__half*>(out_steps),
+    if ((e = launch_pack(W, in_dtype, K, N, group, n_grid, S, losses, best, out_codes, static_cast<__half*>(out_steps),
                          static_cast<__half*>(out_zeros), out_scales, s, &launches)) != cudaSuccess) {
       where = "pack kernel";
       break;

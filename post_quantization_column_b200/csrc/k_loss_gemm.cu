@@ -284,34 +284,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------------
-// Loss reduction and argmin: one block, fixed summation order.
+// Loss reduction: one block per candidate, fixed summation order (strided per-thread
+// sums, then a tree), divided by M*N and rounded once to fp32. The first argmin is
+// taken by the pack kernel from these fp32 values.
 // ---------------------------------------------------------------------------------
 constexpr int kReduceThreads = 256;
 
 __global__ void __launch_bounds__(kReduceThreads)
-    loss_reduce_kernel(const double* __restrict__ partial, int64_t tiles, int n_grid, int64_t M, int64_t N,
-                       float* __restrict__ losses, int* __restrict__ best) {
+    loss_reduce_kernel(const double* __restrict__ partial, int64_t tiles, int64_t M, int64_t N,
+                       float* __restrict__ losses) {
   __shared__ double buf[kReduceThreads];
-  __shared__ float lf[64];
-  for (int c = 0; c < n_grid; ++c) {
-    double s = 0.0;
-    for (int64_t t = threadIdx.x; t < tiles; t += kReduceThreads) s += partial[static_cast<int64_t>(c) * tiles + t];
-    buf[threadIdx.x] = s;
-    __syncthreads();
-    for (int w = kReduceThreads / 2; w > 0; w >>= 1) {
-      if (threadIdx.x < w) buf[threadIdx.x] += buf[threadIdx.x + w];
-      __syncthreads();
-    }
-    if (threadIdx.x == 0) lf[c] = __double2float_rn(buf[0] / (static_cast<double>(M) * static_cast<double>(N)));
+  const int c = blockIdx.x;
+  const double* row = partial + static_cast<int64_t>(c) * tiles;
+  double s = 0.0;
+  for (int64_t t = threadIdx.x; t < tiles; t += kReduceThreads) s += row[t];
+  buf[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = kReduceThreads / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) buf[threadIdx.x] += buf[threadIdx.x + w];
     __syncthreads();
   }
-  if (threadIdx.x == 0) {
-    int b = 0;
-    for (int c = 1; c < n_grid; ++c)
-      if (lf[c] < lf[b]) b = c;  // keeps the first minimum
-    *best = b;
-    for (int c = 0; c < n_grid; ++c) losses[c] = lf[c];
-  }
+  if (threadIdx.x == 0)
+    losses[c] = __double2float_rn(buf[0] / (static_cast<double>(M) * static_cast<double>(N)));
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -385,8 +379,8 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
 }
 
 cudaError_t launch_loss_reduce(const double* partial, int64_t tiles, int n_grid, int64_t M, int64_t N, float* losses,
-                               int* best, cudaStream_t s, int* launches) {
-  loss_reduce_kernel<<<1, kReduceThreads, 0, s>>>(partial, tiles, n_grid, M, N, losses, best);
+                               cudaStream_t s, int* launches) {
+  loss_reduce_kernel<<<n_grid, kReduceThreads, 0, s>>>(partial, tiles, M, N, losses);
   *launches += 1;
   return cudaGetLastError();
 }
