@@ -232,7 +232,8 @@ def run_ours(args, rank, world, local):
             awq.search(Xd, Wd, spec.group, spec.n_grid, stream=stream)
         starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
         ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        gemm_ms, qdq_ms, stat_ms, pack_ms = [], [], [], []
+        gemm_ms, qdq_ms, stat_ms, pack_ms, phase_sums = [], [], [], [], []
+        phase_tot = {}
         barrier()
         torch.cuda.synchronize(dev)
         clocks = ClockSampler(local)
@@ -242,6 +243,9 @@ def run_ours(args, rank, world, local):
             out = awq.search(Xd, Wd, spec.group, spec.n_grid, stream=stream)
             ends[i].record(stream)
             prof = awq.profile_last()
+            for k, v in prof.items():
+                phase_tot[k] = phase_tot.get(k, 0.0) + v
+            phase_sums.append(sum(prof.values()))
             gemm_ms.append(prof["gemm_loss"])
             qdq_ms.append(prof["qdq"])
             stat_ms.append(prof["statistic"])
@@ -315,6 +319,8 @@ def run_ours(args, rank, world, local):
                           "GB/s": stat_bytes / (statistics.mean(stat_ms) / 1e3) / 1e9},
             "pack": {"ms": statistics.mean(pack_ms)},
         },
+        "phases_ms": {k: v / args.steps for k, v in phase_tot.items()},
+        "host_gap_ms": total_ms / args.steps - statistics.mean(phase_sums),
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms / e2e_steps, "steps": e2e_steps},
         "gpu_launches": launches,

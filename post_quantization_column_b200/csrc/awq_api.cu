@@ -167,30 +167,51 @@ int check_device(int* dev, int* num_sms) {
   return AWQ_OK;
 }
 
+// Phase events, created once per device and reused by every profiled call.
 struct Events {
-  cudaEvent_t ev[kNumPhases + 1];
-  bool on = false;
-  cudaStream_t s;
+  static cudaEvent_t cache[64][kNumPhases + 1];
+  static bool made[64];
+  cudaEvent_t* ev = nullptr;
+  cudaStream_t s = nullptr;
   void create(bool enable, cudaStream_t stream) {
-    on = enable;
     s = stream;
-    if (!on) return;
-    for (auto& e : ev) cudaEventCreate(&e);
+    if (!enable) return;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return;
+    if (!made[dev]) {
+      for (auto& e : cache[dev])
+        if (cudaEventCreate(&e) != cudaSuccess) return;
+      made[dev] = true;
+    }
+    ev = cache[dev];
   }
   void mark(int i) {
-    if (on) cudaEventRecord(ev[i], s);
+    if (ev) cudaEventRecord(ev[i], s);
   }
   void collect() {
-    if (!on) return;
+    if (!ev) return;
     for (int i = 0; i < kNumPhases; ++i) cudaEventElapsedTime(&g_phase_ms[i], ev[i], ev[i + 1]);
-    for (auto& e : ev) cudaEventDestroy(e);
-    on = false;
-  }
-  ~Events() {
-    if (on)
-      for (auto& e : ev) cudaEventDestroy(e);
   }
 };
+cudaEvent_t Events::cache[64][kNumPhases + 1];
+bool Events::made[64] = {false};
+
+// A pinned host word per device for the kernels' status, so reading it back is one
+// asynchronous copy followed by the stream synchronisation the call does anyway.
+int* pinned_status_word(int dev) {
+  static int* words[64] = {nullptr};
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!words[dev]) {
+    void* p = nullptr;
+    if (cudaHostAlloc(&p, 64, cudaHostAllocPortable) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    words[dev] = static_cast<int*>(p);
+  }
+  return words[dev];
+}
 
 int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid,
                   float* out_scales, int32_t* out_codes, void* out_steps, void* out_zeros, float* out_losses,
@@ -312,14 +333,17 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
   } while (false);
 
   int h_err = 0;
+  int* pinned = pinned_status_word(dev);
+  int* status_dst = pinned ? pinned : &h_err;
   if (status == AWQ_OK && e == cudaSuccess) {
-    e = cudaMemcpyAsync(&h_err, err, sizeof(int), cudaMemcpyDeviceToHost, s);
+    e = cudaMemcpyAsync(status_dst, err, sizeof(int), cudaMemcpyDeviceToHost, s);
     if (e != cudaSuccess) where = "status read-back";
   }
   if (status == AWQ_OK && e != cudaSuccess) status = cuda_error(e, where);
   cudaFreeAsync(ws, s);
   cudaError_t se = cudaStreamSynchronize(s);
   if (status == AWQ_OK && se != cudaSuccess) status = cuda_error(se, "stream synchronize");
+  if (pinned) h_err = *pinned;
   if (status == AWQ_OK) {
     ev.collect();
     g_last_launches = launches;

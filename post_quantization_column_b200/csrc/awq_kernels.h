@@ -66,6 +66,20 @@ cudaError_t launch_loss_reduce(const double* partial, int64_t tiles, int n_grid,
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Raise a kernel's dynamic shared-memory limit to `bytes` once per device (the first
+// launch on each device pays for the attribute call, later launches skip it).
+template <typename Kernel>
+cudaError_t set_smem_limit_once(Kernel kernel, int bytes, unsigned long long* done_mask) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (__atomic_load_n(done_mask, __ATOMIC_ACQUIRE) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) __atomic_fetch_or(done_mask, bit, __ATOMIC_ACQ_REL);
+  return e;
+}
+
 // Sets the text awq_last_error_message returns on the calling thread.
 void record_error_message(const char* msg);
 

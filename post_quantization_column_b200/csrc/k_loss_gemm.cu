@@ -357,7 +357,8 @@ cudaError_t make_operand_maps(const LossGemmArgs& a, CUtensorMap* mapA, CUtensor
 
 cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, const CUtensorMap& mapB, int mode,
                              cudaStream_t s, int* launches) {
-  cudaError_t e = cudaFuncSetAttribute(loss_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  static unsigned long long attr_done = 0;
+  cudaError_t e = set_smem_limit_once(loss_gemm_kernel, kSmemBytes, &attr_done);
   if (e != cudaSuccess) return e;
   GemmParams p;
   p.mode = mode;

@@ -135,6 +135,41 @@ __device__ __forceinline__ void column_params(const float (&mn)[2], const float 
   }
 }
 
+// Skewed index of row r in a per-candidate row of scales (one padding float every 16
+// rows), so the 8 row-lanes of a warp, 16 rows apart, read 8 different banks.
+template <int G>
+__device__ __forceinline__ int skew(int r) { return r + (r >> 4); }
+template <int G>
+__host__ __device__ constexpr int skewed_pitch() { return G + G / 16; }
+
+// Whether every scaled weight of a column rounds inside [lo, hi] without clamping:
+// t = w' * (1/step) is monotone in w', so its extremes are mn/mx times the reciprocal,
+// and a margin of 2^-15 covers the difference to the exact quotient.
+__device__ __forceinline__ bool clamp_free(float mn, float mx, const ColumnQdq& c) {
+  const float lo = -c.p.zero, hi = 15.0f - c.p.zero;
+  return !c.exact && __fmul_rn(mn, c.recip) >= lo - kNearHalf && __fmul_rn(mx, c.recip) <= hi + kNearHalf;
+}
+
+// Codes, reconstruction and fold-back of CH consecutive rows of one column. Returns
+// whether any element needs the exact divisions (near a rounding boundary).
+template <int CH, bool kClamp>
+__device__ __forceinline__ bool fold_back_run(const float* s, const float* w, const float* rs, const ColumnQdq& c,
+                                              float (&out)[CH]) {
+  const float lo = -c.p.zero, hi = 15.0f - c.p.zero;
+  bool need = false;
+#pragma unroll
+  for (int i = 0; i < CH; ++i) {
+    float t = __fmul_rn(__fmul_rn(s[i], w[i]), c.recip);
+    if (kClamp) t = fminf(fmaxf(t, lo), hi);
+    const float qz = round_small(t);  // q - z, an integer in [-z, 15 - z]
+    need |= fabsf(__fsub_rn(t, qz)) >= kNearHalf;
+    const float v = __fmul_rn(__fmul_rn(qz, c.p.step), rs[i]);
+    need |= near_bf16_midpoint(v);
+    out[i] = v;
+  }
+  return need;
+}
+
 template <typename T, int G>
 __global__ void __launch_bounds__(kQdqThreads, 2)
     qdq_kernel(const T* __restrict__ W, int64_t K, int64_t N, int n_grid, const float* __restrict__ S,
@@ -142,10 +177,11 @@ __global__ void __launch_bounds__(kQdqThreads, 2)
   constexpr int RPL = G / 8;
   constexpr int CH = RPL < 8 ? RPL : 8;  // rows per store run
   constexpr int PITCH = G + 1;
+  constexpr int SP = skewed_pitch<G>();
   extern __shared__ float smem[];
   float* sWT = smem;                        // [64][PITCH]
-  float* sS = smem + kQdqCols * PITCH;      // [n_grid][G] scales
-  float* sR = sS + n_grid * G;              // [n_grid][G] correctly rounded 1/s
+  float* sS = smem + kQdqCols * PITCH;      // [n_grid][SP] scales, skewed
+  float* sR = sS + n_grid * SP;             // [n_grid][SP] correctly rounded 1/s, skewed
 
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kQdqCols;
   const int64_t k0 = static_cast<int64_t>(blockIdx.y) * G;
@@ -155,8 +191,8 @@ __global__ void __launch_bounds__(kQdqThreads, 2)
   for (int idx = threadIdx.x; idx < n_grid * G; idx += kQdqThreads) {
     const int c = idx / G, r = idx % G;
     const float s = S[static_cast<int64_t>(c) * K + k0 + r];
-    sS[idx] = s;
-    sR[idx] = __frcp_rn(s);
+    sS[c * SP + skew<G>(r)] = s;
+    sR[c * SP + skew<G>(r)] = __frcp_rn(s);
   }
   __syncthreads();
 
@@ -180,12 +216,14 @@ __global__ void __launch_bounds__(kQdqThreads, 2)
 
   for (int c = 0; c < n_grid; ++c) {
     float s[RPL];
-    const float* rs = sR + c * G + row0;  // reciprocals, read from shared memory where used
+    // the row reciprocals stay in shared memory (16 rows = 16 + 1 floats, conflict-free)
+    const float* rs = sR + c * SP + skew<G>(row0);
     bool rows_exact = false;
 #pragma unroll
     for (int i = 0; i < RPL; ++i) {
-      s[i] = sS[c * G + row0 + i];
-      rows_exact |= !(fabsf(rs[i]) <= kHugeRecip && fabsf(rs[i]) >= kTinyStep);
+      s[i] = sS[c * SP + skew<G>(row0 + i)];
+      const float r = rs[skew<G>(row0 + i) - skew<G>(row0)];
+      rows_exact |= !(fabsf(r) <= kHugeRecip && fabsf(r) >= kTinyStep);
     }
     // pass 1: the group range of each column of W' = s * W
     float mn[2], mx[2];
@@ -203,26 +241,23 @@ __global__ void __launch_bounds__(kQdqThreads, 2)
     column_range_reduce(mn, mx);
     ColumnQdq cq[2];
     column_params(mn, mx, cq);
+    const bool no_clamp =
+        __all_sync(0xffffffffu, clamp_free(mn[0], mx[0], cq[0]) && clamp_free(mn[1], mx[1], cq[1]));
 
     // pass 2: codes, reconstruction and fold-back, in runs of CH rows of one column
     __nv_bfloat16* slot = Wt + static_cast<int64_t>(c + 1) * N * K;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-      const float lo = -cq[j].p.zero, hi = 15.0f - cq[j].p.zero;
 #pragma unroll
       for (int h = 0; h < RPL; h += CH) {
         float out[CH];
         bool need = rows_exact || cq[j].exact;
-#pragma unroll
-        for (int i = 0; i < CH; ++i) {
-          const float t = __fmul_rn(__fmul_rn(s[h + i], w[j][h + i]), cq[j].recip);
-          const float tc = fminf(fmaxf(t, lo), hi);
-          const float qz = round_small(tc);  // q - z, an integer in [-z, 15 - z]
-          need |= fabsf(__fsub_rn(tc, qz)) >= kNearHalf;
-          const float v = __fmul_rn(__fmul_rn(qz, cq[j].p.step), rs[h + i]);
-          need |= near_bf16_midpoint(v);
-          out[i] = v;
-        }
+        // rows h .. h+CH-1 of this lane never cross a skew pad (CH divides 16)
+        const float* rsh = rs + skew<G>(row0 + h) - skew<G>(row0);
+        if (no_clamp)
+          need |= fold_back_run<CH, false>(s + h, w[j] + h, rsh, cq[j], out);
+        else
+          need |= fold_back_run<CH, true>(s + h, w[j] + h, rsh, cq[j], out);
         if (__any_sync(0xffffffffu, need) && need) {
 #pragma unroll
           for (int i = 0; i < CH; ++i)
@@ -234,7 +269,6 @@ __global__ void __launch_bounds__(kQdqThreads, 2)
   }
 }
 
-constexpr int kMaxGridPack = 64;
 
 template <typename T, int G>
 __global__ void __launch_bounds__(kQdqThreads)
@@ -342,9 +376,11 @@ template <typename T, int G>
 cudaError_t launch_qdq_t(const T* W, int64_t K, int64_t N, int n_grid, const float* S, __nv_bfloat16* Wt,
                          int* err, cudaStream_t s) {
   const size_t smem =
-      (static_cast<size_t>(kQdqCols) * (G + 1) + 2 * static_cast<size_t>(n_grid) * G) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(qdq_kernel<T, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+      (static_cast<size_t>(kQdqCols) * (G + 1) + 2 * static_cast<size_t>(n_grid) * skewed_pitch<G>()) * sizeof(float);
+  // the limit is raised once, to what the largest grid (64 candidates) needs
+  const int smem_max = (kQdqCols * (G + 1) + 2 * 64 * skewed_pitch<G>()) * static_cast<int>(sizeof(float));
+  static unsigned long long attr_done = 0;
+  cudaError_t e = set_smem_limit_once(qdq_kernel<T, G>, smem_max, &attr_done);
   if (e != cudaSuccess) return e;
   dim3 grid(static_cast<unsigned>(ceil_div(N, kQdqCols)), static_cast<unsigned>(K / G));
   qdq_kernel<T, G><<<grid, kQdqThreads, smem, s>>>(W, K, N, n_grid, S, Wt, err);
