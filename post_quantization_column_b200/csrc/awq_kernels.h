@@ -64,7 +64,7 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
 cudaError_t launch_loss_reduce(const double* partial, int64_t tiles, int n_grid, int64_t M, int64_t N,
                                float* losses, cudaStream_t s, int* launches);
 
-inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+__host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Raise a kernel's dynamic shared-memory limit to `bytes` once per device (the first
 // launch on each device pays for the attribute call, later launches skip it).

@@ -258,15 +258,53 @@ __global__ void __launch_bounds__(Tile<G>::kThreads, Tile<G>::kBlocksPerSm)
   }
 }
 
+// Register-staged tile loads for the persistent pack kernel: each thread holds its
+// share of the next G x 64 tile (16-byte vectors) while the current tile is computed.
 template <typename T, int G>
-__global__ void __launch_bounds__(Tile<G>::kThreads)
+struct TileLoad {
+  static constexpr int VEC = 16 / sizeof(T);
+  static constexpr int VPR = kQdqCols / VEC;
+  static constexpr int kPerThread = G * VPR / Tile<G>::kThreads;  // 2 (bf16) or 4 (fp32)
+  uint4 v[kPerThread];
+
+  __device__ __forceinline__ void load(const T* __restrict__ W, int64_t N, int64_t k0, int64_t n0) {
+#pragma unroll
+    for (int it = 0; it < kPerThread; ++it) {
+      const int idx = threadIdx.x + it * Tile<G>::kThreads;
+      const int r = idx / VPR, vv = idx % VPR;
+      const int64_t col = n0 + static_cast<int64_t>(vv) * VEC;
+      v[it] = col < N ? __ldcs(reinterpret_cast<const uint4*>(W + (k0 + r) * N + col)) : make_uint4(0, 0, 0, 0);
+    }
+  }
+  __device__ __forceinline__ void store(float* sWT) const {
+#pragma unroll
+    for (int it = 0; it < kPerThread; ++it) {
+      const int idx = threadIdx.x + it * Tile<G>::kThreads;
+      const int r = idx / VPR, vv = idx % VPR;
+      const T* e = reinterpret_cast<const T*>(&v[it]);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) sWT[(vv * VEC + i) * Tile<G>::kPitch + r] = to_f32<T>(e[i]);
+    }
+  }
+};
+
+// Persistent: each CTA walks tiles blockIdx.x, + gridDim.x, ... (column tiles of one
+// group are adjacent), loading the next tile into registers while it quantizes the
+// current one, so HBM reads overlap the arithmetic.
+template <typename T, int G>
+__global__ void __launch_bounds__(Tile<G>::kThreads, Tile<G>::kBlocksPerSm)
     pack_kernel(const T* __restrict__ W, int64_t K, int64_t N, int n_grid, const float* __restrict__ S,
                 const float* __restrict__ losses, int* __restrict__ best_out, int32_t* __restrict__ codes,
                 __half* __restrict__ steps, __half* __restrict__ zeros, float* __restrict__ out_scales) {
   using L = Tile<G>;
   __shared__ float sWT[kQdqCols * L::kPitch];
   __shared__ __align__(16) uint8_t sQ[G][kQdqCols];
+  __shared__ float sScale[G];
   __shared__ int sBest;
+
+  const int64_t tiles_n = ceil_div(N, kQdqCols);
+  const int64_t tiles = tiles_n * (K / G);
+  const int64_t words = N / 8;
 
   // the chosen candidate: first minimum of the fp32 losses
   if (threadIdx.x == 0) {
@@ -274,87 +312,96 @@ __global__ void __launch_bounds__(Tile<G>::kThreads)
     for (int c = 1; c < n_grid; ++c)
       if (losses[c] < losses[b]) b = c;
     sBest = b;
-    if (blockIdx.x == 0 && blockIdx.y == 0) *best_out = b;
+    if (blockIdx.x == 0) *best_out = b;
   }
-  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kQdqCols;
-  const int64_t k0 = static_cast<int64_t>(blockIdx.y) * G;
-  stage_tile<T, G>(W, N, k0, n0, sWT);
-  __syncthreads();
-  const int c = sBest;
-  const float* srow = S + static_cast<int64_t>(c) * K + k0;
-  if (blockIdx.x == 0)
-    for (int r = threadIdx.x; r < G; r += L::kThreads) out_scales[k0 + r] = srow[r];
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int rl = lane % L::RL, cg = lane / L::RL;
   const int col0 = warp * L::kColsPerWarp + cg * 2;
   const int row0 = rl * kRowsPerLane;
-  float s[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) s[i] = srow[row0 + i];
-  float wp[2][8];
-  float mn[2], mx[2];
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    mn[j] = INFINITY;
-    mx[j] = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      wp[j][i] = __fmul_rn(s[i], sWT[(col0 + j) * L::kPitch + row0 + i]);
-      mn[j] = fminf(mn[j], wp[j][i]);
-      mx[j] = fmaxf(mx[j], wp[j][i]);
-    }
-  }
-  ColumnQdq cq[2];
-  column_qdq<L::RL>(mn, mx, cq);
 
-  float q[2][8];
-  bool need = cq[0].exact || cq[1].exact;
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const float lo = -cq[j].p.zero, hi = 15.0f - cq[j].p.zero;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float tc = fminf(fmaxf(__fmul_rn(wp[j][i], cq[j].recip), lo), hi);
-      const float qz = round_small(tc);
-      need |= fabsf(__fsub_rn(tc, qz)) >= kNearHalf;
-      q[j][i] = __fadd_rn(qz, cq[j].p.zero);
+  TileLoad<T, G> next;
+  int64_t t = blockIdx.x;
+  if (t < tiles) next.load(W, N, (t / tiles_n) * G, (t % tiles_n) * kQdqCols);
+  __syncthreads();
+  const float* Sbest = S + static_cast<int64_t>(sBest) * K;
+
+  for (; t < tiles; t += gridDim.x) {
+    const int64_t k0 = (t / tiles_n) * G, n0 = (t % tiles_n) * kQdqCols;
+    next.store(sWT);
+    for (int r = threadIdx.x; r < G; r += L::kThreads) {
+      const float sv = Sbest[k0 + r];
+      sScale[r] = sv;
+      if (n0 == 0) out_scales[k0 + r] = sv;
     }
-  }
-  if (__any_sync(0xffffffffu, need) && need) {
+    __syncthreads();
+    const int64_t tn = t + gridDim.x;
+    if (tn < tiles) next.load(W, N, (tn / tiles_n) * G, (tn % tiles_n) * kQdqCols);
+
+    float wp[2][8];
+    float mn[2], mx[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      mn[j] = INFINITY;
+      mx[j] = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        wp[j][i] = __fmul_rn(sScale[row0 + i], sWT[(col0 + j) * L::kPitch + row0 + i]);
+        mn[j] = fminf(mn[j], wp[j][i]);
+        mx[j] = fmaxf(mx[j], wp[j][i]);
+      }
+    }
+    ColumnQdq cq[2];
+    column_qdq<L::RL>(mn, mx, cq);
+
+    float q[2][8];
+    bool need = cq[0].exact || cq[1].exact;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const float lo = -cq[j].p.zero, hi = 15.0f - cq[j].p.zero;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float tc = fminf(fmaxf(__fmul_rn(wp[j][i], cq[j].recip), lo), hi);
+        const float qz = round_small(tc);
+        need |= fabsf(__fsub_rn(tc, qz)) >= kNearHalf;
+        q[j][i] = __fadd_rn(qz, cq[j].p.zero);
+      }
+    }
+    if (__any_sync(0xffffffffu, need) && need) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[j][i] = qdq_code(wp[j][i], cq[j].p);
+    }
 #pragma unroll
     for (int j = 0; j < 2; ++j)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) q[j][i] = qdq_code(wp[j][i], cq[j].p);
-  }
-#pragma unroll
-  for (int j = 0; j < 2; ++j)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) sQ[row0 + i][col0 + j] = static_cast<uint8_t>(q[j][i]);
+      for (int i = 0; i < 8; ++i) sQ[row0 + i][col0 + j] = static_cast<uint8_t>(q[j][i]);
 
-  const int64_t n = n0 + col0;
-  if (rl == 0 && n < N) {
-    const int64_t g = blockIdx.y;
-    *reinterpret_cast<__half2*>(steps + g * N + n) = __halves2half2(__float2half_rn(cq[0].p.step),
-                                                                    __float2half_rn(cq[1].p.step));
-    *reinterpret_cast<__half2*>(zeros + g * N + n) = __halves2half2(__float2half_rn(cq[0].p.zero),
-                                                                    __float2half_rn(cq[1].p.zero));
-  }
-  __syncthreads();
-  // eight codes (one 8-byte run of a tile row) -> one int32, nibble i = column 8w + i
-  const int64_t words = N / 8;
-  for (int idx = threadIdx.x; idx < G * (kQdqCols / 8); idx += L::kThreads) {
-    const int r = idx / (kQdqCols / 8), wd = idx % (kQdqCols / 8);
-    const int64_t word = n0 / 8 + wd;
-    if (word >= words) continue;
-    const uint2 b = *reinterpret_cast<const uint2*>(&sQ[r][wd * 8]);
-    uint32_t packed = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      packed |= ((b.x >> (8 * i)) & 0xFu) << (4 * i);
-      packed |= ((b.y >> (8 * i)) & 0xFu) << (4 * (i + 4));
+    const int64_t n = n0 + col0;
+    if (rl == 0 && n < N) {
+      const int64_t g = k0 / G;
+      *reinterpret_cast<__half2*>(steps + g * N + n) = __halves2half2(__float2half_rn(cq[0].p.step),
+                                                                      __float2half_rn(cq[1].p.step));
+      *reinterpret_cast<__half2*>(zeros + g * N + n) = __halves2half2(__float2half_rn(cq[0].p.zero),
+                                                                      __float2half_rn(cq[1].p.zero));
     }
-    codes[(k0 + r) * words + word] = static_cast<int32_t>(packed);
+    __syncthreads();
+    // eight codes (one 8-byte run of a tile row) -> one int32, nibble i = column 8w + i
+    for (int idx = threadIdx.x; idx < G * (kQdqCols / 8); idx += L::kThreads) {
+      const int r = idx / (kQdqCols / 8), wd = idx % (kQdqCols / 8);
+      const int64_t word = n0 / 8 + wd;
+      if (word >= words) continue;
+      const uint2 b = *reinterpret_cast<const uint2*>(&sQ[r][wd * 8]);
+      uint32_t packed = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        packed |= ((b.x >> (8 * i)) & 0xFu) << (4 * i);
+        packed |= ((b.y >> (8 * i)) & 0xFu) << (4 * (i + 4));
+      }
+      codes[(k0 + r) * words + word] = static_cast<int32_t>(packed);
+    }
+    __syncthreads();  // sWT, sQ and sScale are rewritten by the next tile
   }
 }
 
@@ -378,7 +425,12 @@ template <typename T, int G>
 cudaError_t launch_pack_t(const T* W, int64_t K, int64_t N, int n_grid, const float* S, const float* losses,
                           int* best, int32_t* codes, __half* steps, __half* zeros, float* out_scales,
                           cudaStream_t s) {
-  dim3 grid(static_cast<unsigned>(ceil_div(N, kQdqCols)), static_cast<unsigned>(K / G));
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t tiles = ceil_div(N, kQdqCols) * (K / G);
+  const int64_t per_sm = Tile<G>::kBlocksPerSm;  // resident CTAs per SM at <= 64 registers
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, per_sm * sms));
   pack_kernel<T, G><<<grid, Tile<G>::kThreads, 0, s>>>(W, K, N, n_grid, S, losses, best, codes, steps, zeros,
                                                        out_scales);
   return cudaGetLastError();

@@ -3,78 +3,100 @@
 // candidate scale family (same AWQ page, §3 code and §4) and the fp32 -> bf16 operand
 // copy for fp32 layers.
 //
-// The statistic is one coalesced pass over X: each thread owns a 16-byte column
-// vector and walks rows, accumulating |x| in fp64; a second tiny pass adds the
-// per-chunk partial sums in a fixed order and rounds once to fp32. HBM-bound: M*K*b
-// bytes read.
+// Both reductions run as one launch of 8-CTA thread-block clusters and combine their
+// partial results through distributed shared memory in a fixed order, so they need no
+// global scratch and no second pass:
+//  * statistic: a cluster owns 256 columns; its 8 CTAs split the rows, each thread
+//    walks rows with 16-byte column vectors (coalesced, fp64 accumulation), the CTA
+//    sums its 8 row-threads, and CTA rank 0 sums the 8 CTAs' partials, divides by M
+//    once in fp64 and rounds once to fp32. HBM-bound: one read of X.
+//  * scales: a cluster owns one candidate alpha_i; its 8 CTAs split K, exchange their
+//    max/min of raw = max(a^alpha, 1e-4) and each normalises its share by
+//    sqrt(max * min) — fp64 throughout, one rounding to fp32.
 #include "awq_device.cuh"
 #include "awq_kernels.h"
+
+#include <cooperative_groups.h>
+
+namespace cg = cooperative_groups;
 
 namespace awq {
 namespace {
 
-constexpr int kStatCols = 64;  // column vectors per block
-constexpr int kStatRows = 4;   // row lanes per block
+constexpr int kCluster = 8;       // CTAs per cluster (portable size)
+constexpr int kStatVecs = 32;     // 16-byte column vectors per CTA
+constexpr int kStatRows = 8;      // row-threads per column vector
+constexpr int kStatThreads = kStatVecs * kStatRows;
 
 template <typename T>
-__global__ void __launch_bounds__(kStatCols * kStatRows)
-    statistic_partial_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t rows_per_chunk,
-                             double* __restrict__ partial) {
+__global__ void __cluster_dims__(1, kCluster, 1) __launch_bounds__(kStatThreads)
+    statistic_kernel(const T* __restrict__ X, int64_t M, int64_t K, float* __restrict__ a, int* err) {
   constexpr int VEC = 16 / sizeof(T);
-  const int tx = threadIdx.x % kStatCols;
-  const int ty = threadIdx.x / kStatCols;
-  const int64_t c0 = (static_cast<int64_t>(blockIdx.x) * kStatCols + tx) * VEC;
-  const int64_t r_begin = static_cast<int64_t>(blockIdx.y) * rows_per_chunk;
-  const int64_t r_end = min(M, r_begin + rows_per_chunk);
+  constexpr int kCols = kStatVecs * VEC;  // columns per cluster
+  __shared__ double red[kStatRows][kStatVecs][VEC];
+  __shared__ double part[kCols];          // this CTA's column sums, read by rank 0
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int tx = threadIdx.x % kStatVecs, ty = threadIdx.x / kStatVecs;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kCols + static_cast<int64_t>(tx) * VEC;
 
   double acc[VEC];
 #pragma unroll
   for (int i = 0; i < VEC; ++i) acc[i] = 0.0;
-  if (c0 < K) {
+  if (c0 < K) {  // K % 32 == 0, so a vector lies wholly inside or outside
     const T* base = X + c0;
+    const int64_t stride = static_cast<int64_t>(kStatRows) * kCluster;
 #pragma unroll 4
-    for (int64_t r = r_begin + ty; r < r_end; r += kStatRows) {
+    for (int64_t r = static_cast<int64_t>(rank) * kStatRows + ty; r < M; r += stride) {
       const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(base + r * K));
       const T* e = reinterpret_cast<const T*>(&raw);
 #pragma unroll
       for (int i = 0; i < VEC; ++i) acc[i] += fabs(static_cast<double>(to_f32<T>(e[i])));
     }
   }
-  __shared__ double red[kStatRows][kStatCols][VEC];
 #pragma unroll
   for (int i = 0; i < VEC; ++i) red[ty][tx][i] = acc[i];
   __syncthreads();
-  if (ty == 0 && c0 < K) {
+  if (ty == 0) {
 #pragma unroll
     for (int i = 0; i < VEC; ++i) {
       double s = red[0][tx][i];
 #pragma unroll
       for (int r = 1; r < kStatRows; ++r) s += red[r][tx][i];
-      partial[static_cast<int64_t>(blockIdx.y) * K + c0 + i] = s;
+      part[tx * VEC + i] = s;
     }
   }
+  cluster.sync();
+  if (rank == 0) {
+    for (int j = threadIdx.x; j < kCols; j += kStatThreads) {
+      const int64_t col = static_cast<int64_t>(blockIdx.x) * kCols + j;
+      if (col >= K) continue;
+      double s = 0.0;
+      for (int q = 0; q < kCluster; ++q) s += cluster.map_shared_rank(part, q)[j];
+      if (!isfinite(s)) atomicOr(err, kErrNonfiniteX);  // NaN/Inf anywhere in the column
+      a[col] = __double2float_rn(s / static_cast<double>(M));
+    }
+  }
+  cluster.sync();  // keep every CTA's partials alive until rank 0 has read them
 }
 
-__global__ void statistic_final_kernel(const double* __restrict__ partial, int row_chunks, int64_t K,
-                                       int64_t M, float* __restrict__ a, int* err) {
-  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (j >= K) return;
-  double s = 0.0;
-  for (int r = 0; r < row_chunks; ++r) s += partial[static_cast<int64_t>(r) * K + j];
-  if (!isfinite(s)) atomicOr(err, kErrNonfiniteX);  // NaN/Inf anywhere in the column
-  a[j] = __double2float_rn(s / static_cast<double>(M));
-}
+constexpr int kScaleThreads = 256;
 
-// One block per candidate i: alpha = i / n_grid; raw_j = max(a_j^alpha, 1e-4);
-// s_j = raw_j / sqrt(max raw * min raw), in fp64, one rounding to fp32.
-constexpr int kScaleThreads = 1024;
-
-__global__ void __launch_bounds__(kScaleThreads)
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kScaleThreads)
     scales_kernel(const float* __restrict__ a, int64_t K, int n_grid, float* __restrict__ S) {
-  const int i = blockIdx.x;
+  __shared__ double smx[kScaleThreads / 32], smn[kScaleThreads / 32];
+  __shared__ double cta_range[2];  // this CTA's max and min of raw, read by the cluster
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int i = blockIdx.y;  // candidate
   const double alpha = static_cast<double>(i) / static_cast<double>(n_grid);
+  const int64_t share = ceil_div(K, kCluster);
+  const int64_t j0 = rank * share, j1 = min(K, j0 + share);
+
   double mx = 0.0, mn = INFINITY;
-  for (int64_t j = threadIdx.x; j < K; j += blockDim.x) {
+  for (int64_t j = j0 + threadIdx.x; j < j1; j += kScaleThreads) {
     const double raw = fmax(pow(static_cast<double>(a[j]), alpha), kClampMin);
     mx = fmax(mx, raw);
     mn = fmin(mn, raw);
@@ -84,30 +106,30 @@ __global__ void __launch_bounds__(kScaleThreads)
     mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, o));
   }
-  __shared__ double smx[kScaleThreads / 32], smn[kScaleThreads / 32];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (lane == 0) {
     smx[warp] = mx;
     smn[warp] = mn;
   }
   __syncthreads();
-  if (warp == 0) {
-    const int nw = blockDim.x / 32;
-    mx = lane < nw ? smx[lane] : 0.0;
-    mn = lane < nw ? smn[lane] : INFINITY;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < kScaleThreads / 32; ++w) {
+      mx = fmax(mx, smx[w]);
+      mn = fmin(mn, smn[w]);
     }
-    if (lane == 0) {
-      smx[0] = mx;
-      smn[0] = mn;
-    }
+    cta_range[0] = mx;
+    cta_range[1] = mn;
   }
-  __syncthreads();
-  const double normaliser = sqrt(__dmul_rn(smx[0], smn[0]));
-  for (int64_t j = threadIdx.x; j < K; j += blockDim.x) {
+  cluster.sync();
+  double gmx = 0.0, gmn = INFINITY;
+  for (int q = 0; q < kCluster; ++q) {
+    const double* r = cluster.map_shared_rank(cta_range, q);
+    gmx = fmax(gmx, r[0]);
+    gmn = fmin(gmn, r[1]);
+  }
+  cluster.sync();  // every CTA has read every range before any CTA exits
+  const double normaliser = sqrt(__dmul_rn(gmx, gmn));
+  for (int64_t j = j0 + threadIdx.x; j < j1; j += kScaleThreads) {
     const double raw = fmax(pow(static_cast<double>(a[j]), alpha), kClampMin);
     S[static_cast<int64_t>(i) * K + j] = __double2float_rn(__ddiv_rn(raw, normaliser));
   }
@@ -128,38 +150,23 @@ __global__ void to_bf16_kernel(const float4* __restrict__ x, int64_t n4, uint2* 
 
 }  // namespace
 
-int statistic_row_chunks(int64_t M, int64_t K, int in_dtype, int num_sms) {
-  const int vec = in_dtype == 0 ? 8 : 4;
-  const int64_t col_blocks = ceil_div(K, static_cast<int64_t>(kStatCols) * vec);
-  int64_t want = ceil_div(static_cast<int64_t>(num_sms) * 4, col_blocks);
-  // at least 16 rows per chunk, at most 65535 chunks
-  want = std::min<int64_t>(want, std::max<int64_t>(1, M / 16));
-  want = std::min<int64_t>(want, 65535);
-  return static_cast<int>(std::max<int64_t>(1, want));
-}
+int statistic_row_chunks(int64_t, int64_t, int, int) { return 1; }
 
-cudaError_t launch_statistic(const void* X, int in_dtype, int64_t M, int64_t K, int row_chunks,
-                             double* partial, float* a, int* err, cudaStream_t s, int* launches) {
+cudaError_t launch_statistic(const void* X, int in_dtype, int64_t M, int64_t K, int /*row_chunks*/,
+                             double* /*partial*/, float* a, int* err, cudaStream_t s, int* launches) {
   const int vec = in_dtype == 0 ? 8 : 4;
-  const int64_t rows_per_chunk = ceil_div(M, row_chunks);
-  dim3 grid(static_cast<unsigned>(ceil_div(K, static_cast<int64_t>(kStatCols) * vec)),
-            static_cast<unsigned>(row_chunks));
+  dim3 grid(static_cast<unsigned>(ceil_div(K, static_cast<int64_t>(kStatVecs) * vec)), kCluster);
   if (in_dtype == 0)
-    statistic_partial_kernel<__nv_bfloat16><<<grid, kStatCols * kStatRows, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(X), M, K, rows_per_chunk, partial);
+    statistic_kernel<__nv_bfloat16><<<grid, kStatThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(X), M, K, a,
+                                                                   err);
   else
-    statistic_partial_kernel<float><<<grid, kStatCols * kStatRows, 0, s>>>(static_cast<const float*>(X), M, K,
-                                                                           rows_per_chunk, partial);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  statistic_final_kernel<<<static_cast<unsigned>(ceil_div(K, 256)), 256, 0, s>>>(partial, row_chunks, K, M, a,
-                                                                                 err);
-  *launches += 2;
+    statistic_kernel<float><<<grid, kStatThreads, 0, s>>>(static_cast<const float*>(X), M, K, a, err);
+  *launches += 1;
   return cudaGetLastError();
 }
 
 cudaError_t launch_scales(const float* a, int64_t K, int n_grid, float* S, cudaStream_t s, int* launches) {
-  scales_kernel<<<n_grid, kScaleThreads, 0, s>>>(a, K, n_grid, S);
+  scales_kernel<<<dim3(kCluster, n_grid), kScaleThreads, 0, s>>>(a, K, n_grid, S);
   *launches += 1;
   return cudaGetLastError();
 }

@@ -130,7 +130,7 @@ def test_launch_count_and_profile():
         prof = awq.profile_last()
     finally:
         awq.profile_enable(False)
-    # statistic (2) + scales + qdq + reference GEMM + loss GEMM + reduce + pack
-    assert awq.last_launch_count() == 8
+    # statistic + scales + qdq + reference GEMM + loss GEMM + reduce + pack
+    assert awq.last_launch_count() == 7
     assert set(prof) >= {"statistic", "scales", "qdq", "gemm_reference", "gemm_loss", "loss_reduce", "pack"}
     assert all(v >= 0 for v in prof.values()) and prof["gemm_loss"] > 0
