@@ -298,7 +298,7 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
     ga.num_sms = num_sms;
     CUtensorMap mapA, mapB;
     const char* why = "";
-    if ((e = make_operand_maps(ga, &mapA, &mapB, &why)) != cudaSuccess) {
+    if ((e = make_operand_maps(ga, &mapA, &mapB, &why, operand_b_box_rows())) != cudaSuccess) {
       status = set_error(AWQ_ERR_CUDA, std::string("TMA descriptor: ") + why);
       break;
     }

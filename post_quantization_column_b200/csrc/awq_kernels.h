@@ -53,9 +53,15 @@ struct LossGemmArgs {
   int fault_mode;
   int num_sms;
 };
+// Which loss GEMM runs: 2 = the two-SM (cta_group::2) kernel, 1 = the one-SM kernel
+// (AWQ_GEMM_VARIANT=1 in the environment selects the latter).
+int gemm_variant();
+// Rows of the W_hat box one CTA loads: the full 256-column tile, or half of it when a
+// CTA pair shares the tile.
+inline int operand_b_box_rows() { return gemm_variant() == 2 ? kTileN / 2 : kTileN; }
 // Builds the TMA descriptors (driver entry point) for the two operands.
 cudaError_t make_operand_maps(const LossGemmArgs& a, CUtensorMap* mapA, CUtensorMap* mapB,
-                              const char** why);
+                              const char** why, int b_box_rows);
 // mode 0: Y = X_b W_b into the tiled buffer; mode 1: per-tile sum of (X_b W_hat_i - Y)^2.
 cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, const CUtensorMap& mapB,
                              int mode, cudaStream_t s, int* launches);

@@ -184,7 +184,7 @@ extern "C" int awq_search_noalloc(const void* X, const void* W, int in_dtype, in
     ga.num_sms = num_sms;
     CUtensorMap mapA, mapB;
     const char* why = "";
-    if ((e = make_operand_maps(ga, &mapA, &mapB, &why)) != cudaSuccess) { where = why; break; }
+    if ((e = make_operand_maps(ga, &mapA, &mapB, &why, operand_b_box_rows())) != cudaSuccess) { where = why; break; }
     if ((e = launch_loss_gemm(ga, mapA, mapB, 0, s, &launches)) != cudaSuccess) { where = "reference GEMM"; break; }
     if ((e = launch_loss_gemm(ga, mapA, mapB, 1, s, &launches)) != cudaSuccess) { where = "loss GEMM"; break; }
     if ((e = launch_loss_reduce(loss_partial, tiles, n_grid, M, N, losses, s, &launches)) != cudaSuccess) {

@@ -25,6 +25,7 @@
 #include "awq_kernels.h"
 
 #include <cudaTypedefs.h>
+#include <cstdlib>
 
 namespace awq {
 namespace {
@@ -308,6 +309,278 @@ __global__ void __launch_bounds__(kReduceThreads)
     losses[c] = __double2float_rn(buf[0] / (static_cast<double>(M) * static_cast<double>(N)));
 }
 
+// ---------------------------------------------------------------------------------
+// Two-SM variant. A cluster of 2 CTAs (one TPC) computes 256 x 256 output tiles with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16): each CTA loads its own 128 rows
+// of X and 128 of the tile's 256 columns of W_hat (rows of the K-major operand), the
+// even CTA issues the MMA over both CTAs' shared memory, and each CTA's tensor memory
+// holds its 128 rows of the accumulator. A stage is 32 KB per CTA (16 KB of X, 16 KB of
+// W_hat) instead of 48 KB, so 6 stages fit and each SM moves a third less operand data
+// per flop. The even CTA owns the stage-full barriers (both CTAs' TMA loads count their
+// bytes there) and the accumulator-empty barriers (both CTAs' epilogue warps arrive);
+// the MMA's commits are multicast to both CTAs' stage-empty and accumulator-full
+// barriers. Output sub-tiles, the Y layout and the partial sums are the 128 x 256 ones
+// of the one-SM kernel.
+// ---------------------------------------------------------------------------------
+constexpr int kPairStages = 6;
+constexpr int kPairBBytes = (BN / 2) * BK * 2;         // 16 KB
+constexpr int kPairStageBytes = kABytes + kPairBBytes;  // 32 KB
+constexpr int kPairSmemBytes = kPairStages * kPairStageBytes + kBarrierBytes + 1024;
+constexpr int kGroupPairs = 8;                          // grouped raster: 8 pair rows
+constexpr uint64_t kInFlightNs = 1000ull * 1000;        // abort path: let issued copies land
+
+struct PairParams {
+  int mode;
+  int n_grid;
+  int tiles_m, tiles_n, pairs_m;
+  int nk;
+  float* Y;
+  double* partial;
+  int* err;
+  uint64_t timeout_ns;
+  int fault_mode;
+};
+
+__device__ __forceinline__ void pair_unit_coords(int64_t u, const PairParams& p, int& c, int& pm, int& nt) {
+  const int64_t ptiles = static_cast<int64_t>(p.pairs_m) * p.tiles_n;
+  c = static_cast<int>(u / ptiles);
+  const int64_t t = u - static_cast<int64_t>(c) * ptiles;
+  const int64_t group_size = static_cast<int64_t>(kGroupPairs) * p.tiles_n;
+  const int64_t gi = t / group_size;
+  const int first = static_cast<int>(gi * kGroupPairs);
+  const int gm = min(kGroupPairs, p.pairs_m - first);
+  const int64_t r = t - gi * group_size;
+  pm = first + static_cast<int>(r % gm);
+  nt = static_cast<int>(r / gm);
+}
+
+__device__ __forceinline__ void spin_ns(uint64_t ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (global_timer_ns() - t0 < ns) {
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    loss_gemm_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                          const PairParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kPairStages * kABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPairStages * kPairStageBytes);
+  uint64_t* full = bars;                          // [kPairStages] in rank 0: both CTAs' loads landed
+  uint64_t* empty = bars + kPairStages;           // [kPairStages] each CTA: the pair's MMAs read the stage
+  uint64_t* tfull = bars + 2 * kPairStages;       // [2] each CTA: accumulator ready
+  uint64_t* tempty = bars + 2 * kPairStages + 2;  // [2] in rank 0: both CTAs' epilogues drained it
+  uint64_t* drain = bars + 2 * kPairStages + 4;   // [1] rank 0, abort path
+  double* red = reinterpret_cast<double*>(bars + 2 * kPairStages + 5);  // [2][4]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kPairStages + 13);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int64_t cid = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(full + s, 2);  // rank 0's expect_tx arrival + rank 1's arrival
+      mbar_init(empty + s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull + a, 1);
+      mbar_init(tempty + a, 8);  // one arrival per epilogue warp of both CTAs
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&mapA);
+    tma_prefetch_desc(&mapB);
+  }
+  if (warp == 2) {
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA arrival
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
+  const int64_t n_units = (p.mode == 0 ? 1 : p.n_grid) * static_cast<int64_t>(p.pairs_m) * p.tiles_n;
+  const uint64_t budget = p.timeout_ns;
+  const uint32_t full0 = mapa_shared(smem_u32(full), 0);      // rank 0's full[0]
+  const uint32_t tempty0 = mapa_shared(smem_u32(tempty), 0);  // rank 0's tempty[0]
+
+  auto fail = [&]() {
+    *abort_flag = 1;
+    atomicOr(p.err, kErrTimeout);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true, issued_any = false;
+      for (int64_t u = cid; u < n_units && ok; u += nclusters) {
+        int c, pm, nt;
+        pair_unit_coords(u, p, c, pm, nt);
+        const int slot = p.mode == 0 ? 0 : c + 1;
+        const int mt = 2 * pm + static_cast<int>(rank);
+        for (int kb = 0; kb < p.nk; ++kb) {
+          if (!mbar_wait_bounded(empty + stage, phase ^ 1u, abort_flag, budget)) {
+            ok = false;
+            break;
+          }
+          const bool skip = p.fault_mode == 1 && p.mode == 1 && leader && u == cid && kb == 0;
+          if (!skip) {
+            const uint32_t fbar = full0 + 8u * static_cast<uint32_t>(stage);
+            if (leader)
+              mbar_arrive_expect_tx(full + stage, 2 * kPairStageBytes);
+            else
+              mbar_arrive_cluster(fbar);
+            tma_load_2d_pair(&mapA, fbar, sA + stage * kABytes, kb * BK, mt * BM);
+            tma_load_3d_pair(&mapB, fbar, sB + stage * kPairBBytes, kb * BK, nt * BN + static_cast<int>(rank) * (BN / 2),
+                             slot);
+            issued_any = true;
+          }
+          if (++stage == kPairStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        fail();
+        if (issued_any) spin_ns(kInFlightNs);  // copies already issued land within microseconds
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer (rank 0)
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int local = 0;
+      for (int64_t u = cid; u < n_units; u += nclusters, ++local) {
+        const int acc = local & 1;
+        const uint32_t acc_parity = (local >> 1) & 1;
+        if (!mbar_wait_bounded(tempty + acc, acc_parity ^ 1u, abort_flag, budget)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < p.nk; ++kb) {
+          if (!mbar_wait_bounded(full + stage, phase, abort_flag, budget)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t adesc = smem_desc_k_sw128(smem_u32(sA + stage * kABytes));
+          const uint64_t bdesc = smem_desc_k_sw128(smem_u32(sB + stage * kPairBBytes));
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_bf16_f32_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          umma_commit_pair(empty + stage, 0x3);
+          if (++stage == kPairStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair(tfull + acc, 0x3);
+      }
+      if (!ok) {
+        fail();
+        umma_commit_pair(drain, 0x1);
+        mbar_wait_bounded(drain, 0, nullptr, kDrainNs);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------- epilogue (both CTAs)
+    const int ew = warp - 4;  // TMEM lanes 32*ew .. 32*ew+31 = rows of this CTA's half
+    const int row = ew * 32 + lane;
+    int local = 0;
+    for (int64_t u = cid; u < n_units; u += nclusters, ++local) {
+      int c, pm, nt;
+      pair_unit_coords(u, p, c, pm, nt);
+      const int mt = 2 * pm + static_cast<int>(rank);
+      const bool valid = mt < p.tiles_m;  // an odd tile count leaves rank 1 of the last pair row empty
+      const int acc = local & 1;
+      const uint32_t acc_parity = (local >> 1) & 1;
+      const bool ok = mbar_wait_bounded(tfull + acc, acc_parity, abort_flag, budget);
+      if (named_barrier_or(1, kEpiThreads, !ok)) {
+        if (!ok) fail();
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const int64_t tile = static_cast<int64_t>(valid ? mt : 0) * p.tiles_n + nt;
+      float4* ytile = reinterpret_cast<float4*>(p.Y + tile * (BM * BN));
+      float sq = 0.0f;
+#pragma unroll 1
+      for (int j0 = 0; j0 < BN; j0 += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(j0), v);
+        tmem_ld_wait();
+        if (!valid) continue;
+        float4* yrow = ytile + (j0 / 4) * BM + row;  // tile layout [BN/4][BM][4]
+        if (p.mode == 0) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            yrow[q * BM] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                       __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 y = __ldg(yrow + q * BM);
+            const float d0 = __uint_as_float(v[4 * q]) - y.x;
+            const float d1 = __uint_as_float(v[4 * q + 1]) - y.y;
+            const float d2 = __uint_as_float(v[4 * q + 2]) - y.z;
+            const float d3 = __uint_as_float(v[4 * q + 3]) - y.w;
+            sq = fmaf(d0, d0, sq);
+            sq = fmaf(d1, d1, sq);
+            sq = fmaf(d2, d2, sq);
+            sq = fmaf(d3, d3, sq);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(tempty + acc);
+        else
+          mbar_arrive_cluster(tempty0 + 8u * static_cast<uint32_t>(acc));
+      }
+      if (p.mode == 1) {
+        double ds = static_cast<double>(sq);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
+        if (lane == 0) red[acc * 4 + ew] = ds;
+        named_barrier_sync(2, kEpiThreads);
+        if (ew == 0 && lane == 0 && valid)
+          p.partial[static_cast<int64_t>(c) * tiles + tile] =
+              ((red[acc * 4 + 0] + red[acc * 4 + 1]) + red[acc * 4 + 2]) + red[acc * 4 + 3];
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  cluster_sync_all();  // neither CTA leaves while the other may still touch its barriers or operands
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc_pair(tmem_base, kTmemCols);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
@@ -322,7 +595,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 }  // namespace
 
-cudaError_t make_operand_maps(const LossGemmArgs& a, CUtensorMap* mapA, CUtensorMap* mapB, const char** why) {
+cudaError_t make_operand_maps(const LossGemmArgs& a, CUtensorMap* mapA, CUtensorMap* mapB, const char** why,
+                              int b_box_rows) {
   auto fn = encode_fn();
   if (!fn) {
     *why = "cuTensorMapEncodeTiled unavailable";
@@ -344,7 +618,7 @@ cudaError_t make_operand_maps(const LossGemmArgs& a, CUtensorMap* mapA, CUtensor
   const cuuint64_t dimsB[3] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(a.N),
                                static_cast<cuuint64_t>(a.n_grid + 1)};
   const cuuint64_t strideB[2] = {static_cast<cuuint64_t>(a.K) * 2, static_cast<cuuint64_t>(a.K) * a.N * 2};
-  const cuuint32_t boxB[3] = {BK, BN, 1};
+  const cuuint32_t boxB[3] = {BK, static_cast<cuuint32_t>(b_box_rows), 1};
   r = fn(mapB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16*>(a.Wt), dimsB, strideB, boxB, ones,
          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -355,16 +629,63 @@ cudaError_t make_operand_maps(const LossGemmArgs& a, CUtensorMap* mapA, CUtensor
   return cudaSuccess;
 }
 
+int gemm_variant() {
+  const char* v = getenv("AWQ_GEMM_VARIANT");
+  return (v && v[0] == '1') ? 1 : 2;
+}
+
 cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, const CUtensorMap& mapB, int mode,
                              cudaStream_t s, int* launches) {
+  const int tiles_m = static_cast<int>(ceil_div(a.M, BM));
+  const int tiles_n = static_cast<int>(ceil_div(a.N, BN));
+  if (gemm_variant() == 2) {
+    static unsigned long long attr_done = 0;
+    cudaError_t e = set_smem_limit_once(loss_gemm_pair_kernel, kPairSmemBytes, &attr_done);
+    if (e != cudaSuccess) return e;
+    PairParams p;
+    p.mode = mode;
+    p.n_grid = a.n_grid;
+    p.tiles_m = tiles_m;
+    p.tiles_n = tiles_n;
+    p.pairs_m = (tiles_m + 1) / 2;
+    p.nk = static_cast<int>(ceil_div(a.K, BK));
+    p.Y = a.Y;
+    p.partial = a.partial;
+    p.err = a.err;
+    p.timeout_ns = a.timeout_ns;
+    p.fault_mode = a.fault_mode;
+    const int64_t units = (mode == 0 ? 1 : a.n_grid) * static_cast<int64_t>(p.pairs_m) * tiles_n;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kPairSmemBytes;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int max_clusters = a.num_sms / 2;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * max_clusters));
+    int active = 0;
+    if (cudaOccupancyMaxActiveClusters(&active, loss_gemm_pair_kernel, &cfg) == cudaSuccess && active > 0)
+      max_clusters = std::min(max_clusters, active);
+    else
+      cudaGetLastError();
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * std::min<int64_t>(units, max_clusters)));
+    e = cudaLaunchKernelEx(&cfg, loss_gemm_pair_kernel, mapA, mapB, p);
+    *launches += 1;
+    return e != cudaSuccess ? e : cudaGetLastError();
+  }
   static unsigned long long attr_done = 0;
   cudaError_t e = set_smem_limit_once(loss_gemm_kernel, kSmemBytes, &attr_done);
   if (e != cudaSuccess) return e;
   GemmParams p;
   p.mode = mode;
   p.n_grid = a.n_grid;
-  p.tiles_m = static_cast<int>(ceil_div(a.M, BM));
-  p.tiles_n = static_cast<int>(ceil_div(a.N, BN));
+  p.tiles_m = tiles_m;
+  p.tiles_n = tiles_n;
   p.nk = static_cast<int>(ceil_div(a.K, BK));
   p.Y = a.Y;
   p.partial = a.partial;

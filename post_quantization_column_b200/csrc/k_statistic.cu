@@ -6,10 +6,11 @@
 // Both reductions run as one launch of 8-CTA thread-block clusters and combine their
 // partial results through distributed shared memory in a fixed order, so they need no
 // global scratch and no second pass:
-//  * statistic: a cluster owns 256 columns; its 8 CTAs split the rows, each thread
-//    walks rows with 16-byte column vectors (coalesced, fp64 accumulation), the CTA
-//    sums its 8 row-threads, and CTA rank 0 sums the 8 CTAs' partials, divides by M
-//    once in fp64 and rounds once to fp32. HBM-bound: one read of X.
+//  * statistic: a cluster owns 64 columns (bf16; 32 for fp32); its 8 CTAs split the
+//    rows, each thread walks rows with 16-byte column vectors (a warp reads 128-byte
+//    row segments; fp64 accumulation), the CTA sums its 32 row-threads, and CTA rank 0
+//    sums the 8 CTAs' partials, divides by M once in fp64 and rounds once to fp32.
+//    HBM-bound: one read of X, with enough CTAs (8 per 64 columns) to keep HBM busy.
 //  * scales: a cluster owns one candidate alpha_i; its 8 CTAs split K, exchange their
 //    max/min of raw = max(a^alpha, 1e-4) and each normalises its share by
 //    sqrt(max * min) — fp64 throughout, one rounding to fp32.
@@ -24,8 +25,8 @@ namespace awq {
 namespace {
 
 constexpr int kCluster = 8;       // CTAs per cluster (portable size)
-constexpr int kStatVecs = 32;     // 16-byte column vectors per CTA
-constexpr int kStatRows = 8;      // row-threads per column vector
+constexpr int kStatVecs = 8;      // 16-byte column vectors per CTA (a warp reads 128-byte row segments)
+constexpr int kStatRows = 32;     // row-threads per column vector
 constexpr int kStatThreads = kStatVecs * kStatRows;
 
 template <typename T>

@@ -45,6 +45,18 @@ def test_small_layers(M, K, N, group, n_grid, law, dtype):
     P.full_parity(X, W, group, n_grid)
 
 
+@pytest.mark.parametrize("variant", ["1", "2"])
+@pytest.mark.parametrize("M,K,N,group,dtype", [(300, 384, 520, 128, "bf16"), (129, 320, 776, 64, "f32"),
+                                               (520, 256, 264, 32, "bf16")])
+def test_both_gemm_variants(M, K, N, group, dtype, variant, monkeypatch):
+    # the one-SM (128 x 256 tiles) and two-SM (256 x 256 tiles, cta_group::2) loss
+    # GEMMs, including odd row-tile counts that leave half of the last pair empty
+    monkeypatch.setenv("AWQ_GEMM_VARIANT", variant)
+    spec = custom_spec(M, K, N, dtype=dtype, group=group, seed=M * 7 + N)
+    X, W = generate(spec)
+    P.full_parity(X, W, group, 20)
+
+
 def test_weights_on_the_grid_give_zero_loss():
     # every (group, column) spans all 16 levels with step 1/16 and zero 7: alpha = 0
     # reproduces W exactly (AWQ-P1 §7 reconstruction), so L_0 = 0 and alpha 0 wins
