@@ -133,10 +133,12 @@ class ClockSampler:
             return None
         sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
         smax = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        watts = [float(r[3]) for r in rows if r[3].strip().replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows),
+                "power_w_median": statistics.median(watts) if watts else None}
 
 
 def cpu_oracle_sample(spec: LayerSpec, target_s: float):
@@ -305,7 +307,9 @@ def run_ours(args, rank, world, local):
                    "n_grid": spec.n_grid, "input_dtype": spec.dtype, "parallelism": f"independent layers x{world}",
                    "l2": "flushed between steps (256 MiB device write outside the timed events)"},
         "layers_per_s": layers_per_s,
-        "roofline": {"bound": "tensor", "kernel": "loss_gemm_kernel (candidate GEMMs + fused squared error)",
+        "roofline": {"bound": "tensor",
+                     "kernel": ("loss_gemm_pair_kernel" if os.environ.get("AWQ_GEMM_VARIANT", "1").startswith("2")
+                                else "loss_gemm_kernel") + " (candidate GEMMs + fused squared error)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} bf16_tflops (burst)",
                      "traffic": recorded_traffic("loss_gemm_kernel", spec.name),

@@ -247,8 +247,12 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t local_addr, uint32_t ra
   return r;
 }
 
+// Arrive on a barrier of another CTA of the cluster. The default (CTA-scope) release is
+// enough here: the peer's operand bytes reach the barrier through the TMA's own
+// transaction count, and tensor-memory reads are ordered by tcgen05 fences, so no
+// cluster-wide fence (which would stall every stage) is needed.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 __device__ __forceinline__ void cluster_sync_all() {

@@ -53,8 +53,8 @@ struct LossGemmArgs {
   int fault_mode;
   int num_sms;
 };
-// Which loss GEMM runs: 2 = the two-SM (cta_group::2) kernel, 1 = the one-SM kernel
-// (AWQ_GEMM_VARIANT=1 in the environment selects the latter).
+// Which loss GEMM runs: 1 = the one-SM kernel (default), 2 = the two-SM
+// (cta_group::2) kernel, selected with AWQ_GEMM_VARIANT=2 in the environment.
 int gemm_variant();
 // Rows of the W_hat box one CTA loads: the full 256-column tile, or half of it when a
 // CTA pair shares the tile.

@@ -26,6 +26,7 @@
 
 #include <cudaTypedefs.h>
 #include <cstdlib>
+#include <cstdio>
 
 namespace awq {
 namespace {
@@ -629,9 +630,12 @@ cudaError_t make_operand_maps(const LossGemmArgs& a, CUtensorMap* mapA, CUtensor
   return cudaSuccess;
 }
 
+// The one-SM kernel is the default: under the B200's 1 kW power cap it sustains a
+// higher clock than the pair kernel on long searches (70B-shaped layer: 1276 vs 1090
+// TFLOP/s at 1260 vs 930 MHz), while the pair kernel is ahead only on short ones.
 int gemm_variant() {
   const char* v = getenv("AWQ_GEMM_VARIANT");
-  return (v && v[0] == '1') ? 1 : 2;
+  return (v && v[0] == '2') ? 2 : 1;
 }
 
 cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, const CUtensorMap& mapB, int mode,
@@ -674,6 +678,9 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
     else
       cudaGetLastError();
     cfg.gridDim = dim3(static_cast<unsigned>(2 * std::min<int64_t>(units, max_clusters)));
+    if (getenv("AWQ_DEBUG_LAUNCH"))
+      fprintf(stderr, "loss_gemm_pair_kernel: mode %d, %d clusters (occupancy query %d), %lld units\n", mode,
+              cfg.gridDim.x / 2, active, static_cast<long long>(units));
     e = cudaLaunchKernelEx(&cfg, loss_gemm_pair_kernel, mapA, mapB, p);
     *launches += 1;
     return e != cudaSuccess ? e : cudaGetLastError();
