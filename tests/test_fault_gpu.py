@@ -1,0 +1,37 @@
+"""Failure detection: a bounded wait in the loss GEMM runs out (B200 only).
+
+The fault hook makes the loss GEMM's producer skip one stage's loads and its arrive,
+so the MMA thread waits on a barrier nothing will complete. Every wait in the kernel
+is bounded (here 50 ms): the waiting thread raises the CTA's abort flag, the other
+roles stop at their next wait, copies and MMAs already issued are allowed to land,
+tensor memory is freed, and the call returns AWQ_ERR_TIMEOUT. No trap, no fault,
+no hang; the context stays usable and the next search is exact again.
+"""
+import pytest
+import torch
+
+import post_quantization_column_b200 as awq
+from workloads import custom_spec, generate
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("variant", ["1", "2"])
+def test_wait_that_runs_out_returns_timeout_and_the_context_survives(variant, monkeypatch):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    monkeypatch.setenv("AWQ_GEMM_VARIANT", variant)
+    spec = custom_spec(520, 512, 776, seed=31)
+    X, W = (t.cuda() for t in generate(spec))
+    ref = awq.search(X, W)
+    awq.debug_set_fault(1, 50_000_000)
+    try:
+        with pytest.raises(awq.AwqError) as err:
+            awq.search(X, W)
+        assert err.value.status == 6  # AWQ_ERR_TIMEOUT
+        assert "wait" in str(err.value)
+    finally:
+        awq.debug_set_fault(0)
+    again = awq.search(X, W)
+    for name in ("scales", "codes", "steps", "zeros", "losses"):
+        assert torch.equal(getattr(again, name), getattr(ref, name)), name
