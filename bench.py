@@ -164,6 +164,25 @@ def cpu_oracle_sample(spec: LayerSpec, target_s: float):
             "seconds": t, "columns": n}
 
 
+def rank_spec(base: LayerSpec, rank: int) -> LayerSpec:
+    """The layer rank `rank` searches: the workload's shape with its own seed."""
+    return LayerSpec(**{**base.as_dict(), "seed": base.seed + rank})
+
+
+def max_over_ranks(values, device) -> list:
+    """Element-wise maximum over all ranks (the slowest rank's device times)."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def weak_scaling_tflops(world: int, steps: int, flops_per_step: float, total_ms: float) -> float:
+    """All ranks' candidate-GEMM work divided by the slowest rank's time."""
+    return world * steps * flops_per_step / (total_ms / 1e3) / 1e12
+
+
 # ----------------------------------------------------------------------------- arms
 def run_reference(args, rank, world):
     spec = WORKLOADS[args.workload]
@@ -216,8 +235,7 @@ def run_ours(args, rank, world, local):
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    base = WORKLOADS[args.workload]
-    spec = LayerSpec(**{**base.as_dict(), "seed": base.seed + rank})
+    spec = rank_spec(WORKLOADS[args.workload], rank)
     X, W = generate(spec)
     Xd, Wd = X.to(dev), W.to(dev)
     stream = torch.cuda.Stream(dev)
@@ -281,16 +299,12 @@ def run_ours(args, rank, world, local):
         barrier()
         e2e_ms = float(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)))
 
-    times = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        import torch.distributed as dist
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms = times.tolist()
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
 
     flops = spec.candidate_flops
-    value = world * args.steps * flops / (total_ms / 1e3) / 1e12
+    value = weak_scaling_tflops(world, args.steps, flops, total_ms)
     layers_per_s = world * args.steps / (total_ms / 1e3)
-    e2e_value = world * e2e_steps * flops / (e2e_ms / 1e3) / 1e12
+    e2e_value = weak_scaling_tflops(world, e2e_steps, flops, e2e_ms)
     peaks, peak_kind = measured_peaks()
     gemm_avg = statistics.mean(gemm_ms)
     achieved = flops / (gemm_avg / 1e3) / 1e12
