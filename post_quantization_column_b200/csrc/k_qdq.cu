@@ -61,10 +61,13 @@ __device__ __forceinline__ float round_small(float x) {
   return __fsub_rn(__fadd_rn(x, kRoundMagic), kRoundMagic);
 }
 
-// True when bf16 rounding of fp32 values within 8 ulps of v could differ.
+// True when bf16 rounding of fp32 values within 8 ulps of v could differ, i.e. when
+// the low 16 bits of v lie within 8 of 0x8000. Multiplying by 2^16 moves those bits
+// to the top (a multiply-add, off the integer-compare pipe the rest of the kernel
+// loads), so one unsigned compare decides: ((u - 0x7FF8) mod 2^16) << 16 <= 16 << 16.
 __device__ __forceinline__ bool near_bf16_midpoint(float v) {
-  const uint32_t u = __float_as_uint(v);
-  return ((u - 0x7FF8u) & 0xFFFFu) <= 16u;
+  const uint32_t x = __float_as_uint(v) * 65536u + 0x80080000u;  // 0x80080000 = -(0x7FF8 << 16) mod 2^32
+  return x <= 0x00100000u;
 }
 
 __device__ __forceinline__ void store_bf16x8(__nv_bfloat16* dst, const float (&v)[8]) {
