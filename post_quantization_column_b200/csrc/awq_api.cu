@@ -213,9 +213,44 @@ int* pinned_status_word(int dev) {
   return words[dev];
 }
 
+// Per-device copy stream and events for awq_search_host, created on first use.
+struct CopyLane {
+  static constexpr int kChunks = 8;
+  cudaStream_t stream = nullptr;
+  cudaEvent_t alloc_done = nullptr, x_ready = nullptr, copies_done = nullptr;
+  cudaEvent_t w_ready[kChunks] = {};
+};
+
+CopyLane* copy_lane(int dev) {
+  static CopyLane lanes[64];
+  static bool made[64] = {false};
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mu);
+  CopyLane& L = lanes[dev];
+  if (!made[dev]) {
+    if (cudaStreamCreateWithFlags(&L.stream, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    bool ok = cudaEventCreateWithFlags(&L.alloc_done, cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventCreateWithFlags(&L.x_ready, cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventCreateWithFlags(&L.copies_done, cudaEventDisableTiming) == cudaSuccess;
+    for (auto& ev : L.w_ready) ok = ok && cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) return nullptr;
+    made[dev] = true;
+  }
+  return &L;
+}
+
+// Inputs that are still arriving from the host: the search waits for X before the
+// statistic and for each chunk of W's row groups before quantizing those groups.
+struct HostFeed {
+  cudaEvent_t x_ready = nullptr;
+  const cudaEvent_t* w_ready = nullptr;  // one event per chunk
+  int chunks = 0;
+  int64_t groups_per_chunk = 0;
+};
+
 int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid,
                   float* out_scales, int32_t* out_codes, void* out_steps, void* out_zeros, float* out_losses,
-                  double* out_tile_sq_err, int64_t tile_sq_err_len, cudaStream_t s) {
+                  double* out_tile_sq_err, int64_t tile_sq_err_len, cudaStream_t s, const HostFeed* feed = nullptr) {
   int st = validate(X, W, in_dtype, M, K, N, group, n_grid, out_scales, out_codes, out_steps, out_zeros, true);
   if (st != AWQ_OK) return st;
   if (out_losses && !aligned16(out_losses)) {
@@ -263,6 +298,7 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
   int status = AWQ_OK;
   do {
     if ((e = cudaMemsetAsync(err, 0, 16, s)) != cudaSuccess) { where = "cudaMemsetAsync"; break; }
+    if (feed && (e = cudaStreamWaitEvent(s, feed->x_ready, 0)) != cudaSuccess) { where = "waiting for X"; break; }
     ev.mark(kPhStatistic);
     if ((e = launch_statistic(X, in_dtype, M, K, L.row_chunks, stat_partial, a, err, s, &launches)) != cudaSuccess) {
       where = "statistic kernel";
@@ -279,7 +315,20 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
       }
     }
     ev.mark(kPhQdq);
-    if ((e = launch_qdq(W, in_dtype, K, N, group, n_grid, S, Wt, err, s, &launches)) != cudaSuccess) {
+    if (feed) {
+      // quantize each chunk of row groups as soon as it has arrived
+      const int64_t groups = K / group;
+      for (int c = 0; c < feed->chunks && e == cudaSuccess; ++c) {
+        const int64_t g0 = c * feed->groups_per_chunk;
+        const int64_t gn = std::min(feed->groups_per_chunk, groups - g0);
+        if (gn <= 0) break;
+        if ((e = cudaStreamWaitEvent(s, feed->w_ready[c], 0)) == cudaSuccess)
+          e = launch_qdq_groups(W, in_dtype, K, N, group, n_grid, S, Wt, err, g0, gn, s, &launches);
+      }
+    } else {
+      e = launch_qdq(W, in_dtype, K, N, group, n_grid, S, Wt, err, s, &launches);
+    }
+    if (e != cudaSuccess) {
       where = "qdq kernel";
       break;
     }
@@ -402,6 +451,8 @@ int awq_search_host(const void* X_host, const void* W_host, int in_dtype, int64_
   cudaMemPool_t pool;
   st = get_pool(dev, &pool);
   if (st != AWQ_OK) return st;
+  CopyLane* lane = copy_lane(dev);
+  if (!lane) return set_error(AWQ_ERR_CUDA, "could not create the host-copy stream");
   const size_t eb = in_dtype == AWQ_DTYPE_BF16 ? 2 : 4;
   const size_t G = static_cast<size_t>(K / group);
   const size_t bx = static_cast<size_t>(M) * K * eb, bw = static_cast<size_t>(K) * N * eb;
@@ -421,14 +472,35 @@ int awq_search_host(const void* X_host, const void* W_host, int in_dtype, int64_
   }
   uint8_t* b = static_cast<uint8_t*>(buf);
   int status = AWQ_OK;
-  if ((e = cudaMemcpyAsync(b + off[0], X_host, bx, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(b + off[1], W_host, bw, cudaMemcpyHostToDevice, s)) != cudaSuccess) {
-    status = cuda_error(e, "host-to-device copy");
-  }
+  // X first, then W in chunks of whole row groups, on the copy stream; the search on
+  // `s` starts on X while W is still arriving and quantizes each chunk as it lands.
+  HostFeed feed;
+  feed.chunks = static_cast<int>(std::min<size_t>(CopyLane::kChunks, G));
+  feed.groups_per_chunk = static_cast<int64_t>((G + feed.chunks - 1) / feed.chunks);
+  feed.x_ready = lane->x_ready;
+  feed.w_ready = lane->w_ready;
+  const size_t chunk_bytes = static_cast<size_t>(feed.groups_per_chunk) * group * N * eb;
+  do {
+    if ((e = cudaEventRecord(lane->alloc_done, s)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(lane->stream, lane->alloc_done, 0)) != cudaSuccess)
+      break;
+    if ((e = cudaMemcpyAsync(b + off[0], X_host, bx, cudaMemcpyHostToDevice, lane->stream)) != cudaSuccess ||
+        (e = cudaEventRecord(lane->x_ready, lane->stream)) != cudaSuccess)
+      break;
+    for (int c = 0; c < feed.chunks && e == cudaSuccess; ++c) {
+      const size_t at = static_cast<size_t>(c) * chunk_bytes;
+      const size_t n = std::min(chunk_bytes, bw - std::min(bw, at));
+      if (n > 0)
+        e = cudaMemcpyAsync(b + off[1] + at, static_cast<const uint8_t*>(W_host) + at, n, cudaMemcpyHostToDevice,
+                            lane->stream);
+      if (e == cudaSuccess) e = cudaEventRecord(lane->w_ready[c], lane->stream);
+    }
+  } while (false);
+  if (e != cudaSuccess) status = cuda_error(e, "host-to-device copy");
   if (status == AWQ_OK)
     status = search_device(b + off[0], b + off[1], in_dtype, M, K, N, group, n_grid, reinterpret_cast<float*>(b + off[2]),
                            reinterpret_cast<int32_t*>(b + off[3]), b + off[4], b + off[5],
-                           reinterpret_cast<float*>(b + off[6]), nullptr, 0, s);
+                           reinterpret_cast<float*>(b + off[6]), nullptr, 0, s, &feed);
   if (status == AWQ_OK) {
     if ((e = cudaMemcpyAsync(out_scales_host, b + off[2], bs, cudaMemcpyDeviceToHost, s)) != cudaSuccess ||
         (e = cudaMemcpyAsync(out_codes_host, b + off[3], bc, cudaMemcpyDeviceToHost, s)) != cudaSuccess ||
@@ -438,6 +510,9 @@ int awq_search_host(const void* X_host, const void* W_host, int in_dtype, int64_
          (e = cudaMemcpyAsync(out_losses_host, b + off[6], bl, cudaMemcpyDeviceToHost, s)) != cudaSuccess))
       status = cuda_error(e, "device-to-host copy");
   }
+  // the copy stream must be done with the buffers before they return to the pool
+  cudaEventRecord(lane->copies_done, lane->stream);
+  cudaStreamWaitEvent(s, lane->copies_done, 0);
   cudaFreeAsync(buf, s);
   cudaError_t se = cudaStreamSynchronize(s);
   if (status == AWQ_OK && se != cudaSuccess) status = cuda_error(se, "stream synchronize");

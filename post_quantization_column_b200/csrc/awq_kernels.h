@@ -32,6 +32,10 @@ cudaError_t launch_to_bf16(const float* x, int64_t n, __nv_bfloat16* out, cudaSt
 // Writes Wt[0] = bf16(W)^T and Wt[1 + i] = bf16(W_hat_i)^T, each N x K (K contiguous).
 cudaError_t launch_qdq(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid,
                        const float* S, __nv_bfloat16* Wt, int* err, cudaStream_t s, int* launches);
+// The same for the groups group0 .. group0 + groups - 1 only (rows group0*group ..).
+cudaError_t launch_qdq_groups(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid,
+                              const float* S, __nv_bfloat16* Wt, int* err, int64_t group0, int64_t groups,
+                              cudaStream_t s, int* launches);
 
 // ---- artifact of the chosen candidate (AWQ-P1 §7; QUANT-P4 §5.3) ------------------
 // The chosen candidate is the first minimum of `losses` (AWQ-P1 §3); its index is

@@ -175,7 +175,7 @@ __device__ __forceinline__ bool fold_back_8(const float (&s)[8], const float (&w
 template <typename T, int G>
 __global__ void __launch_bounds__(Tile<G>::kThreads, Tile<G>::kBlocksPerSm)
     qdq_kernel(const T* __restrict__ W, int64_t K, int64_t N, int n_grid, const float* __restrict__ S,
-               __nv_bfloat16* __restrict__ Wt, int* err) {
+               __nv_bfloat16* __restrict__ Wt, int* err, int64_t group0) {
   using L = Tile<G>;
   extern __shared__ float smem[];
   float* sWT = smem;                                 // [64][kPitch]
@@ -183,7 +183,7 @@ __global__ void __launch_bounds__(Tile<G>::kThreads, Tile<G>::kBlocksPerSm)
   float* sR = sS + n_grid * L::kSkewPitch;           // [n_grid][kSkewPitch] correctly rounded 1/s
 
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kQdqCols;
-  const int64_t k0 = static_cast<int64_t>(blockIdx.y) * G;
+  const int64_t k0 = (group0 + static_cast<int64_t>(blockIdx.y)) * G;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
   if (stage_tile<T, G>(W, N, k0, n0, sWT)) atomicOr(err, kErrNonfiniteW);
@@ -410,7 +410,7 @@ __global__ void __launch_bounds__(Tile<G>::kThreads, Tile<G>::kBlocksPerSm)
 
 template <typename T, int G>
 cudaError_t launch_qdq_t(const T* W, int64_t K, int64_t N, int n_grid, const float* S, __nv_bfloat16* Wt,
-                         int* err, cudaStream_t s) {
+                         int* err, int64_t group0, int64_t groups, cudaStream_t s) {
   using L = Tile<G>;
   const size_t smem = (static_cast<size_t>(kQdqCols) * L::kPitch + 2 * static_cast<size_t>(n_grid) * L::kSkewPitch) *
                       sizeof(float);
@@ -419,8 +419,8 @@ cudaError_t launch_qdq_t(const T* W, int64_t K, int64_t N, int n_grid, const flo
   static unsigned long long attr_done = 0;
   cudaError_t e = set_smem_limit_once(qdq_kernel<T, G>, smem_max, &attr_done);
   if (e != cudaSuccess) return e;
-  dim3 grid(static_cast<unsigned>(ceil_div(N, kQdqCols)), static_cast<unsigned>(K / G));
-  qdq_kernel<T, G><<<grid, L::kThreads, smem, s>>>(W, K, N, n_grid, S, Wt, err);
+  dim3 grid(static_cast<unsigned>(ceil_div(N, kQdqCols)), static_cast<unsigned>(groups));
+  qdq_kernel<T, G><<<grid, L::kThreads, smem, s>>>(W, K, N, n_grid, S, Wt, err, group0);
   return cudaGetLastError();
 }
 
@@ -441,23 +441,29 @@ cudaError_t launch_pack_t(const T* W, int64_t K, int64_t N, int n_grid, const fl
 
 }  // namespace
 
-cudaError_t launch_qdq(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid, const float* S,
-                       __nv_bfloat16* Wt, int* err, cudaStream_t s, int* launches) {
+cudaError_t launch_qdq_groups(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid,
+                              const float* S, __nv_bfloat16* Wt, int* err, int64_t group0, int64_t groups,
+                              cudaStream_t s, int* launches) {
   *launches += 1;
   if (in_dtype == 0) {
     const auto* w = static_cast<const __nv_bfloat16*>(W);
     switch (group) {
-      case 32: return launch_qdq_t<__nv_bfloat16, 32>(w, K, N, n_grid, S, Wt, err, s);
-      case 64: return launch_qdq_t<__nv_bfloat16, 64>(w, K, N, n_grid, S, Wt, err, s);
-      default: return launch_qdq_t<__nv_bfloat16, 128>(w, K, N, n_grid, S, Wt, err, s);
+      case 32: return launch_qdq_t<__nv_bfloat16, 32>(w, K, N, n_grid, S, Wt, err, group0, groups, s);
+      case 64: return launch_qdq_t<__nv_bfloat16, 64>(w, K, N, n_grid, S, Wt, err, group0, groups, s);
+      default: return launch_qdq_t<__nv_bfloat16, 128>(w, K, N, n_grid, S, Wt, err, group0, groups, s);
     }
   }
   const auto* w = static_cast<const float*>(W);
   switch (group) {
-    case 32: return launch_qdq_t<float, 32>(w, K, N, n_grid, S, Wt, err, s);
-    case 64: return launch_qdq_t<float, 64>(w, K, N, n_grid, S, Wt, err, s);
-    default: return launch_qdq_t<float, 128>(w, K, N, n_grid, S, Wt, err, s);
+    case 32: return launch_qdq_t<float, 32>(w, K, N, n_grid, S, Wt, err, group0, groups, s);
+    case 64: return launch_qdq_t<float, 64>(w, K, N, n_grid, S, Wt, err, group0, groups, s);
+    default: return launch_qdq_t<float, 128>(w, K, N, n_grid, S, Wt, err, group0, groups, s);
   }
+}
+
+cudaError_t launch_qdq(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid, const float* S,
+                       __nv_bfloat16* Wt, int* err, cudaStream_t s, int* launches) {
+  return launch_qdq_groups(W, in_dtype, K, N, group, n_grid, S, Wt, err, 0, K / group, s, launches);
 }
 
 cudaError_t launch_pack(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid, const float* S,
