@@ -154,6 +154,37 @@ int awq_last_launch_count(void);
  * Mode 0 restores normal operation. */
 int awq_debug_set_fault(int mode, int64_t timeout_ns);
 
+/* ---- Clipping search after the scaling ----------------------------------------
+ * [AWQ-P1] §5: after the channel scaling, a few large weights can still stretch a
+ * group's range; clipping trades them for a finer step. For each input group g and
+ * output column n of the scaled layer W' = fl32(s W) (the layer once the scales are
+ * folded in, AWQ-P1 §6; `scales` [K] fp32, typically awq_search's out_scales):
+ *   c_i = fl32(absmax_g,n * fl32(1 - i/20)),  i = 0 .. n_shrink-1  (10 in the page: 1 .. 0.55)
+ *   delta_i = Q(clamp(W'_g[:, n], -c_i, c_i)) - W'_g[:, n]   (Q = the quantizer of step 3)
+ *   e_i = mean over sampled tokens t of (sum_{k in g} X'[t,k] delta_i[k])^2,  X' = fl32(X / s)
+ *   i* = first argmin of e_i (fp64); the output is the clipped group's artifact.
+ * Sampled tokens: rows 0, d, 2d, ... of X with d = max(1, M / max_tokens), at most
+ * max_tokens of them (awq_clip_token_count). The products run in fp64 as
+ * delta^T (X'_g^T X'_g) delta / T.
+ * Outputs (device memory):
+ *   out_max_val [K/group][N] fp32   c_i* (the clamp applied before quantizing)
+ *   out_best    [K/group][N] int32  i* (may be NULL)
+ *   out_errors  [n_shrink][K/group][N] fp64  e_i (may be NULL)
+ *   out_codes, out_steps, out_zeros: the artifact of Q(clamp(W', c_i*)), same layout as
+ *   awq_search (dequantized W ~= step * (q - zero) / s).
+ * Preconditions as awq_search (group 32/64/128, K % group == 0, N % 8 == 0; X and W
+ * 16-byte aligned); 1 <= n_shrink <= 20; max_tokens >= 1; scales positive and finite
+ * (AWQ_ERR_INVALID_ARG otherwise). Work space: (K/group) * group^2 * 8 bytes from the
+ * library's pool. Synchronizes `stream`. Skipping layers (the page leaves query/key
+ * projections unclipped) is the caller's decision. */
+int awq_clip_search(const void* X, const void* W, int in_dtype, const float* scales,
+                    int64_t M, int64_t K, int64_t N, int group, int n_shrink,
+                    int64_t max_tokens, float* out_max_val, int32_t* out_best,
+                    double* out_errors, int32_t* out_codes, void* out_steps,
+                    void* out_zeros, awq_stream_t stream);
+/* Number of tokens the clipping search samples from M rows (0 on bad arguments). */
+int64_t awq_clip_token_count(int64_t M, int64_t max_tokens);
+
 int awq_version(void);
 
 /* ---- Searching without allocating -------------------------------------------

@@ -22,7 +22,8 @@ __all__ = [
     "AwqError", "SearchOutput", "search", "search_host", "library", "library_path", "header_path",
     "tile_shape", "workspace_bytes", "release_cached", "profile_enable", "profile_last",
     "last_launch_count", "debug_set_fault", "status_string", "exported_functions",
-    "activation_statistic", "candidate_scales", "qdq_candidates",
+    "activation_statistic", "candidate_scales", "qdq_candidates", "ClipOutput", "clip_search",
+    "clip_token_count",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -84,7 +85,10 @@ def library() -> ctypes.CDLL:
     lib.awq_activation_statistic.argtypes = [vp, i32, i64, i64, vp, vp]
     lib.awq_candidate_scales.argtypes = [vp, i64, i32, vp, vp]
     lib.awq_qdq_candidates.argtypes = [vp, i32, i64, i64, i32, i32, vp, vp, vp]
-    for name in ("awq_activation_statistic", "awq_candidate_scales", "awq_qdq_candidates"):
+    lib.awq_clip_search.argtypes = [vp, vp, i32, vp, i64, i64, i64, i32, i32, i64, vp, vp, vp, vp, vp, vp, vp]
+    lib.awq_clip_token_count.argtypes = [i64, i64]
+    lib.awq_clip_token_count.restype = ctypes.c_int64
+    for name in ("awq_activation_statistic", "awq_candidate_scales", "awq_qdq_candidates", "awq_clip_search"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -272,3 +276,53 @@ def search_host(X: torch.Tensor, W: torch.Tensor, group: int = 128, n_grid: int 
                              _ptr(steps), _ptr(zeros), _ptr(losses), _stream_handle(stream, dev))
     _check(st)
     return SearchOutput(scales, codes, steps, zeros, losses)
+
+
+@dataclass
+class ClipOutput:
+    max_val: torch.Tensor              # (K/group, N) fp32: the chosen clamp threshold
+    best: torch.Tensor                 # (K/group, N) int32: index of the chosen shrink factor
+    codes: torch.Tensor                # (K, N/8) int32: the clipped group's codes
+    steps: torch.Tensor                # (K/group, N) fp16
+    zeros: torch.Tensor                # (K/group, N) fp16
+    errors: torch.Tensor | None = None  # (n_shrink, K/group, N) fp64
+
+
+def clip_token_count(M: int, max_tokens: int = 512) -> int:
+    """Number of rows of X the clipping search samples."""
+    return int(library().awq_clip_token_count(M, max_tokens))
+
+
+def clip_search(X: torch.Tensor, W: torch.Tensor, scales: torch.Tensor, group: int = 128, n_shrink: int = 10,
+                max_tokens: int = 512, *, errors: bool = False,
+                stream: torch.cuda.Stream | None = None) -> ClipOutput:
+    """Clipping search after the scaling on device tensors X (M, K), W (K, N) and the
+    chosen scales (K,) fp32: per (group, column) threshold, its index, and the artifact
+    of the clipped, scaled weights."""
+    if X.dim() != 2 or W.dim() != 2 or X.shape[1] != W.shape[0] or scales.shape != (X.shape[1],):
+        raise ValueError("X must be (M, K), W (K, N) and scales (K,)")
+    if X.dtype != W.dtype:
+        raise TypeError("X and W must share a dtype")
+    if scales.dtype != torch.float32:
+        raise TypeError("scales must be float32")
+    if not (X.is_cuda and W.is_cuda and scales.is_cuda):
+        raise ValueError("clip_search() takes CUDA tensors")
+    lib = library()
+    X, W, scales = X.contiguous(), W.contiguous(), scales.contiguous()
+    M, K = X.shape
+    N = W.shape[1]
+    if group <= 0 or K % group or N % 8:
+        raise ValueError("group must divide K and N must be a multiple of 8")
+    dev = X.device
+    G = K // group
+    max_val = torch.empty(G, N, dtype=torch.float32, device=dev)
+    best = torch.empty(G, N, dtype=torch.int32, device=dev)
+    codes = torch.empty(K, N // 8, dtype=torch.int32, device=dev)
+    steps = torch.empty(G, N, dtype=torch.float16, device=dev)
+    zeros = torch.empty(G, N, dtype=torch.float16, device=dev)
+    errs = torch.empty(n_shrink, G, N, dtype=torch.float64, device=dev) if errors else None
+    st = lib.awq_clip_search(_ptr(X), _ptr(W), _dtype_code(X), _ptr(scales), M, K, N, group, n_shrink, max_tokens,
+                             _ptr(max_val), _ptr(best), _ptr(errs), _ptr(codes), _ptr(steps), _ptr(zeros),
+                             _stream_handle(stream, dev))
+    _check(st)
+    return ClipOutput(max_val, best, codes, steps, zeros, errs)

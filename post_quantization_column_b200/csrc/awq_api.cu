@@ -21,6 +21,7 @@ using namespace awq;
 
 constexpr int kVersion = 1;
 constexpr int kMaxGrid = 64;
+constexpr int kMaxShrink = 20;  // factor 1 - i/20 stays positive for i < 20
 constexpr uint64_t kDefaultTimeoutNs = 2000ull * 1000 * 1000;
 
 enum Phase { kPhStatistic, kPhScales, kPhConvert, kPhQdq, kPhGemmY, kPhGemmLoss, kPhReduce, kPhPack, kNumPhases };
@@ -613,6 +614,81 @@ int awq_qdq_candidates(const void* W, int in_dtype, int64_t K, int64_t N, int gr
   g_last_launches = launches;
   if (h_err & kErrNonfiniteW) return set_error(AWQ_ERR_NONFINITE, "non-finite value in W");
   return AWQ_OK;
+}
+
+// ---- clipping search after the scaling ---------------------------------------------
+int awq_clip_search(const void* X, const void* W, int in_dtype, const float* scales, int64_t M, int64_t K, int64_t N,
+                    int group, int n_shrink, int64_t max_tokens, float* out_max_val, int32_t* out_best,
+                    double* out_errors, int32_t* out_codes, void* out_steps, void* out_zeros, awq_stream_t stream) {
+  t_last_error.clear();
+  int st = validate(X, W, in_dtype, M, K, N, group, 1, out_max_val, out_codes, out_steps, out_zeros, false);
+  if (st != AWQ_OK) return st;
+  if (!scales) return set_error(AWQ_ERR_INVALID_ARG, "scales is NULL");
+  if (n_shrink < 1 || n_shrink > kMaxShrink) return set_error(AWQ_ERR_INVALID_ARG, "n_shrink must be in 1..20");
+  if (max_tokens < 1) return set_error(AWQ_ERR_INVALID_ARG, "max_tokens must be positive");
+  if (!aligned16(X) || !aligned16(W) || (reinterpret_cast<uintptr_t>(scales) & 3u) ||
+      (reinterpret_cast<uintptr_t>(out_max_val) & 3u) || (reinterpret_cast<uintptr_t>(out_best) & 3u) ||
+      (reinterpret_cast<uintptr_t>(out_errors) & 7u) || (reinterpret_cast<uintptr_t>(out_codes) & 3u) ||
+      (reinterpret_cast<uintptr_t>(out_steps) & 1u) || (reinterpret_cast<uintptr_t>(out_zeros) & 1u))
+    return set_error(AWQ_ERR_INVALID_ARG, "X and W must be 16-byte aligned, the other pointers aligned to their type");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  bind_device(s, X);
+  int dev = 0, num_sms = 0;
+  if ((st = check_device(&dev, &num_sms)) != AWQ_OK) return st;
+  if (!is_device_memory(X) || !is_device_memory(W) || !is_device_memory(scales) || !is_device_memory(out_max_val) ||
+      !is_device_memory(out_codes) || !is_device_memory(out_steps) || !is_device_memory(out_zeros) ||
+      (out_best && !is_device_memory(out_best)) || (out_errors && !is_device_memory(out_errors)))
+    return set_error(AWQ_ERR_INVALID_ARG, "inputs and outputs must be device memory");
+  cudaMemPool_t pool;
+  if ((st = get_pool(dev, &pool)) != AWQ_OK) return st;
+  const size_t h_bytes = static_cast<size_t>(K / group) * group * group * sizeof(double);
+  void* ws = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, 256 + align_up(h_bytes), pool, s);
+  if (e != cudaSuccess || !ws) {
+    cudaGetLastError();
+    return set_error(AWQ_ERR_OOM, "clipping work space of " + std::to_string(256 + h_bytes) + " bytes");
+  }
+  ClipArgs a;
+  a.X = X;
+  a.W = W;
+  a.in_dtype = in_dtype;
+  a.s = scales;
+  a.M = M;
+  a.K = K;
+  a.N = N;
+  a.group = group;
+  a.n_shrink = n_shrink;
+  a.max_tokens = max_tokens;
+  a.tokens = static_cast<int>(clip_token_count(M, max_tokens));
+  a.err = static_cast<int*>(ws);
+  a.H = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + 256);
+  a.max_val = out_max_val;
+  a.best = out_best;
+  a.errors = out_errors;
+  a.codes = out_codes;
+  a.steps = static_cast<__half*>(out_steps);
+  a.zeros = static_cast<__half*>(out_zeros);
+  int launches = 0, h_err = 0;
+  int* pinned = pinned_status_word(dev);
+  int* status_dst = pinned ? pinned : &h_err;
+  if ((e = cudaMemsetAsync(a.err, 0, 16, s)) == cudaSuccess && (e = launch_clip(a, s, &launches)) == cudaSuccess)
+    e = cudaMemcpyAsync(status_dst, a.err, sizeof(int), cudaMemcpyDeviceToHost, s);
+  cudaFreeAsync(ws, s);
+  cudaError_t se = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_error(e, "clipping search");
+  if (se != cudaSuccess) return cuda_error(se, "stream synchronize");
+  if (pinned) h_err = *pinned;
+  g_last_launches = launches;
+  if (h_err & kErrBadScale) return set_error(AWQ_ERR_INVALID_ARG, "a scale is not a positive finite number");
+  if (h_err & kErrNonfiniteX) return set_error(AWQ_ERR_NONFINITE, "non-finite value in X / s");
+  if (h_err & kErrNonfiniteW) return set_error(AWQ_ERR_NONFINITE, "non-finite value in W");
+  if (h_err) return set_error(AWQ_ERR_CUDA, "device status word " + std::to_string(h_err));
+  return AWQ_OK;
+}
+
+int64_t awq_clip_token_count(int64_t M, int64_t max_tokens) {
+  if (M <= 0 || max_tokens <= 0) return 0;
+  return clip_token_count(M, max_tokens);
 }
 
 void awq_tile_shape(int* tile_m, int* tile_n) {

@@ -17,6 +17,7 @@ enum : int {
   kErrNonfiniteW = 2,
   kErrTimeout = 4,
   kErrBounds = 8,
+  kErrBadScale = 16,  // a scale that is not a positive finite number
 };
 
 constexpr int kQMax = 15;            // 4-bit unsigned codes (AWQ-P1 §7)

@@ -74,6 +74,31 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
 cudaError_t launch_loss_reduce(const double* partial, int64_t tiles, int n_grid, int64_t M, int64_t N,
                                float* losses, cudaStream_t s, int* launches);
 
+// ---- clipping search after the scaling (AWQ-P1 §5) ---------------------------------
+struct ClipArgs {
+  const void* X;       // [M][K], in_dtype
+  const void* W;       // [K][N], in_dtype
+  int in_dtype;
+  const float* s;      // [K] the chosen scales
+  int64_t M, K, N;
+  int group, n_shrink;
+  int64_t max_tokens;  // sampled tokens: every clip_token_stride-th row, at most max_tokens
+  int tokens;          // clip_token_count(M, max_tokens)
+  double* H;           // work space: [K / group][group][group]
+  float* max_val;      // [K / group][N]
+  int32_t* best;       // [K / group][N] or nullptr
+  double* errors;      // [n_shrink][K / group][N] or nullptr
+  int32_t* codes;      // [K][N / 8]
+  __half* steps;       // [K / group][N]
+  __half* zeros;       // [K / group][N]
+  int* err;
+};
+int64_t clip_token_stride(int64_t M, int64_t max_tokens);
+int64_t clip_token_count(int64_t M, int64_t max_tokens);
+// Gram matrices of the sampled scaled activations, then the per-(group, column) search
+// and the clipped artifact: two launches.
+cudaError_t launch_clip(const ClipArgs& a, cudaStream_t s, int* launches);
+
 __host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Raise a kernel's dynamic shared-memory limit to `bytes` once per device (the first

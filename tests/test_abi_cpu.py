@@ -77,3 +77,28 @@ def test_product_package_does_not_import_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(root, f), encoding="utf-8").read()
                 assert "import oracle" not in text and "from oracle" not in text, f
+
+
+def test_clip_token_sampling_matches_the_oracle_reading(lib):
+    # the token count is host logic; the oracle's strided sample is the reading it follows
+    import oracle.awq_clip as C
+    for M in (1, 7, 511, 512, 513, 1023, 1024, 1500, 4096, 16384, 16385):
+        for T in (1, 64, 512):
+            assert awq.clip_token_count(M, T) == len(C.sample_tokens(M, T)), (M, T)
+    assert lib.awq_clip_token_count(0, 512) == 0 and lib.awq_clip_token_count(16, 0) == 0
+
+
+def test_clip_search_validation_happens_on_the_host(lib):
+    null = ctypes.c_void_p(0)
+    buf = ctypes.create_string_buffer(64)
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    args = lambda **kw: [kw.get("X", p), p, 0, kw.get("s", p), 16, 128, 64, kw.get("group", 128),
+                         kw.get("n_shrink", 10), kw.get("tokens", 512), p, null, null, p, p, p, null]
+    assert lib.awq_clip_search(*args(X=null)) == 1
+    assert lib.awq_clip_search(*args(s=null)) == 1
+    assert lib.awq_clip_search(*args(n_shrink=0)) == 1
+    assert lib.awq_clip_search(*args(n_shrink=21)) == 1
+    assert lib.awq_clip_search(*args(tokens=0)) == 1
+    assert lib.awq_clip_search(*args(group=48)) == 1
+    assert b"n_shrink" in lib.awq_last_error_message() or b"max_tokens" in lib.awq_last_error_message() \
+        or b"group" in lib.awq_last_error_message()
