@@ -11,17 +11,17 @@
 //     delta_i = Q(clamp(W'_g[:, n], c_i)) - W'_g[:, n],  H_g = X'_g^T X'_g.
 // The first minimum wins; its threshold, codes, steps and zeros are written out.
 //
-// gram_kernel: H_g for every group, fp64 (products of two fp32 values are exact in
-// fp64; the token sum runs in token order, so H is bit-symmetric). Small: T * G^2 per
-// group.
+// gram_kernel: H_g for every group in fp64 on the tensor cores (the products of two
+// fp32 values are exact in fp64; only the token sums round). Small: T * G^2 per group.
 //
-// clip_kernel: one CTA per (group, 64 output columns). It stages H_g (G x G fp64) in
-// shared memory once, keeps its share of W' in registers, and for each threshold builds
-// the G x 64 matrix of deltas in shared memory, then forms Q = H_g Delta with a
-// register-tiled fp64 product (each thread 8 rows x 4 columns for G = 128) and the
-// column sums of Delta .* Q. The work is n_shrink * G^2 fp64 FMAs per (group, column):
-// the kernel is bound by the fp64 pipe, not by memory (H_g comes from L2, W is read
-// once).
+// clip_kernel: one CTA per (group, 64 output columns). It stages the lower block
+// triangle of H_g in shared memory once, keeps its share of W' in registers, and for
+// each threshold builds the G x 64 matrix of deltas in shared memory (double-buffered,
+// so building one threshold overlaps the products of the previous one), then evaluates
+// every column's delta^T H_g delta from one block triangle of H_g (32-row blocks,
+// G (G + 32) / 2 products per (threshold, column)) with fp64 tensor-core MMAs, 16 warps
+// sharing the work evenly. The kernel is bound by the fp64 tensor pipe, not by memory
+// (H_g comes from L2, W is read once).
 #include "awq_device.cuh"
 #include "awq_kernels.h"
 
@@ -30,64 +30,107 @@ namespace {
 
 constexpr int kShrinkGrid = 20;    // factor_i = 1 - i / 20
 constexpr int kClipCols = 64;      // output columns per CTA
-constexpr int kClipThreads = 256;  // 16 row-blocks x 16 column-lanes
-constexpr int kGramThreads = 256;  // 16 x 16
+constexpr int kClipThreads = 512;  // 16 warps
+constexpr int kGramThreads = 256;  // 8 warps
 constexpr int kGramChunk = 32;     // tokens staged per pass
 
+// ---- fp64 tensor-core helpers ------------------------------------------------------------
+// D (8x8) += A (8x4, row-major) * B (4x8) in fp64 on the tensor cores. Lane (g, t) =
+// (lane / 4, lane % 4) holds A[g][t], B[t][g] and D[g][2t], D[g][2t + 1].
+__device__ __forceinline__ void mma_f64(double (&d)[2], double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+               : "+d"(d[0]), "+d"(d[1])
+               : "d"(a), "d"(b));
+}
+
 // ---- Gram matrices -------------------------------------------------------------------
-// CTA (g, tile): a TB x TB tile of H_g, TB = min(G, 64). Thread (ty, tx) owns rows
-// r0 + ty + 16 a and columns c0 + tx + 16 b (a, b < TB / 16).
+// CTA (g, tile): a TB x TB tile of H_g, TB = min(G, 64), rows r0.., columns c0... The
+// sampled tokens are staged 32 at a time as fp64 X' values (rows part and columns part,
+// row pitch TB + 4 so the fragment loads hit 32 banks); each of the 8 warps owns a
+// (TB/2) x (TB/4) sub-tile and accumulates it with fp64 MMAs over 4 tokens per step.
 template <typename T, int G>
 __global__ void __launch_bounds__(kGramThreads) gram_kernel(const T* __restrict__ X, int64_t K, int64_t stride,
                                                             int tokens, const float* __restrict__ s,
                                                             double* __restrict__ H, int* err) {
   constexpr int TB = G < 64 ? G : 64;
-  constexpr int R = TB / 16;
   constexpr int TILES = G / TB;
-  __shared__ double xa[kGramChunk][TB];
-  __shared__ double xb[kGramChunk][TB];
+  constexpr int PX = TB + 4;
+  constexpr int WR = TB / 2, WC = TB / 4;  // warp sub-tile: 2 x 4 warps
+  constexpr int MI = WR / 8, MJ = WC / 8;  // 8x8 MMA tiles per warp (4x2 for TB 64, 2x1 for TB 32)
+  __shared__ __align__(16) double xa[kGramChunk][PX];
+  __shared__ __align__(16) double xb[kGramChunk][PX];
 
   const int64_t g = blockIdx.x;
   const int r0 = (blockIdx.y / TILES) * TB, c0 = (blockIdx.y % TILES) * TB;
-  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
   const int64_t col0 = g * G;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int wr = warp / 4, wc = warp % 4;
 
-  double acc[R][R];
+  double acc[MI][MJ][2];
 #pragma unroll
-  for (int a = 0; a < R; ++a)
+  for (int a = 0; a < MI; ++a)
 #pragma unroll
-    for (int b = 0; b < R; ++b) acc[a][b] = 0.0;
+    for (int b = 0; b < MJ; ++b) acc[a][b][0] = acc[a][b][1] = 0.0;
 
+  // the tile's scales, once
+  __shared__ float ss[2][TB];
   bool bad_x = false, bad_s = false;
+  for (int i = threadIdx.x; i < 2 * TB; i += kGramThreads) {
+    const float sc = s[col0 + (i < TB ? r0 + i : c0 + i - TB)];
+    bad_s |= !(sc > 0.0f) || !isfinite(sc);
+    ss[i / TB][i % TB] = sc;
+  }
+
+  // 16-byte vectors of the sampled rows: NV per thread per chunk, prefetched into
+  // registers one chunk ahead of the products
+  constexpr int VEC = 16 / sizeof(T);
+  constexpr int VPR = TB / VEC;  // vectors per row of one half
+  constexpr int NV = 2 * kGramChunk * VPR / kGramThreads;
+  static_assert(NV * kGramThreads == 2 * kGramChunk * VPR, "staging vectors must split evenly");
+  uint4 pre[NV];
+  auto fetch = [&](int t0) {
+#pragma unroll
+    for (int q = 0; q < NV; ++q) {
+      const int idx = threadIdx.x + q * kGramThreads;
+      const int half = idx / (kGramChunk * VPR), rem = idx % (kGramChunk * VPR);
+      const int t = rem / VPR, v = rem % VPR;
+      pre[q] = make_uint4(0, 0, 0, 0);  // tokens past the end contribute zero
+      if (t0 + t < tokens)
+        pre[q] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<int64_t>(t0 + t) * stride * K + col0 +
+                                                      (half ? c0 : r0) + v * VEC));
+    }
+  };
+  fetch(0);
+  __syncthreads();  // ss is visible
   for (int t0 = 0; t0 < tokens; t0 += kGramChunk) {
-    for (int idx = threadIdx.x; idx < 2 * kGramChunk * TB; idx += kGramThreads) {
-      const int half = idx / (kGramChunk * TB);
-      const int rem = idx % (kGramChunk * TB);
-      const int t = rem / TB, c = rem % TB;
-      const int64_t col = col0 + (half ? c0 : r0) + c;
-      double v = 0.0;
-      if (t0 + t < tokens) {
-        const float x = to_f32<T>(X[static_cast<int64_t>(t0 + t) * stride * K + col]);
-        const float sc = s[col];
-        bad_s |= !(sc > 0.0f) || !isfinite(sc);
-        const float xs = __fdiv_rn(x, sc);  // X' = fl32(X / s)
+#pragma unroll
+    for (int q = 0; q < NV; ++q) {
+      const int idx = threadIdx.x + q * kGramThreads;
+      const int half = idx / (kGramChunk * VPR), rem = idx % (kGramChunk * VPR);
+      const int t = rem / VPR, v = rem % VPR;
+      const T* e = reinterpret_cast<const T*>(&pre[q]);
+      double* dst = (half ? xb[t] : xa[t]) + v * VEC;
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) {
+        const float xs = __fdiv_rn(to_f32<T>(e[i]), ss[half][v * VEC + i]);  // X' = fl32(X / s)
         bad_x |= !isfinite(xs);
-        v = static_cast<double>(xs);
+        dst[i] = static_cast<double>(xs);
       }
-      (half ? xb : xa)[t][c] = v;
     }
     __syncthreads();
-#pragma unroll 4
-    for (int t = 0; t < kGramChunk; ++t) {
-      double ra[R], rb[R];
+    if (t0 + kGramChunk < tokens) fetch(t0 + kGramChunk);
+#pragma unroll 2
+    for (int k4 = 0; k4 < kGramChunk; k4 += 4) {
+      double av[MI], bv[MJ];
 #pragma unroll
-      for (int a = 0; a < R; ++a) ra[a] = xa[t][ty + 16 * a];
+      for (int a = 0; a < MI; ++a) av[a] = xa[k4 + tq][wr * WR + 8 * a + gq];  // A[k][t] = X'[t][k]
 #pragma unroll
-      for (int b = 0; b < R; ++b) rb[b] = xb[t][tx + 16 * b];
+      for (int b = 0; b < MJ; ++b) bv[b] = xb[k4 + tq][wc * WC + 8 * b + gq];  // B[t][l] = X'[t][l]
 #pragma unroll
-      for (int a = 0; a < R; ++a)
+      for (int a = 0; a < MI; ++a)
 #pragma unroll
-        for (int b = 0; b < R; ++b) acc[a][b] = __fma_rn(ra[a], rb[b], acc[a][b]);
+        for (int b = 0; b < MJ; ++b) mma_f64(acc[a][b], av[a], bv[b]);
     }
     __syncthreads();
   }
@@ -95,28 +138,69 @@ __global__ void __launch_bounds__(kGramThreads) gram_kernel(const T* __restrict_
   if (bad_s) atomicOr(err, kErrBadScale);
   double* Hg = H + g * G * G;
 #pragma unroll
-  for (int a = 0; a < R; ++a)
+  for (int a = 0; a < MI; ++a)
 #pragma unroll
-    for (int b = 0; b < R; ++b) Hg[(r0 + ty + 16 * a) * G + c0 + tx + 16 * b] = acc[a][b];
+    for (int b = 0; b < MJ; ++b) {
+      const int row = r0 + wr * WR + 8 * a + gq, col = c0 + wc * WC + 8 * b + 2 * tq;
+      *reinterpret_cast<double2*>(Hg + row * G + col) = make_double2(acc[a][b][0], acc[a][b][1]);
+    }
 }
 
 // ---- clipping search -------------------------------------------------------------------
+// Shared-memory layout (G = 128: 80 KB of H, 2 x 64 KB of deltas):
+//  * H_g, the lower block triangle only: the 32 x 32 blocks (c, b), c >= b, of the
+//    stored H[l][k], block (c, b) at index c (c + 1) / 2 + b, row-major inside;
+//  * two buffers of the G x 64 deltas (one threshold is built while the previous one
+//    is multiplied).
+// Both swizzle the column index with the row: column x of row y sits at x ^ f(y & 3),
+// f(0..3) = 0, 8, 4, 12, so the MMA fragment loads (rows l = 4 s + t for lane t), the
+// 16-byte loads of the fold (rows 8 i + g) and the delta stores touch distinct banks
+// without padding.
 template <int G>
 struct ClipTile {
-  static constexpr int RM = G / 16;                 // rows per thread in the product
-  static constexpr int EPT = G * kClipCols / kClipThreads;  // W' elements per thread (G / 4)
-  static constexpr int kRowStep = kClipThreads / kClipCols; // 4
-  static constexpr size_t kSmemH = sizeof(double) * G * G;
-  static constexpr size_t kSmemD = sizeof(double) * G * kClipCols;
-  static constexpr size_t kSmemRed = sizeof(double) * 16 * kClipCols;
-  static constexpr size_t kSmem = kSmemH + kSmemD + kSmemRed;
+  static constexpr int EPT = G * kClipCols / kClipThreads;   // W' elements per thread (G / 8)
+  static constexpr int kRowStep = kClipThreads / kClipCols;  // 8
+  static constexpr int kSliceCols = 16;                      // columns of one warp's tile
+  static constexpr int NB = G / 32;                          // 32-row blocks
+  static constexpr int kBlocksH = NB * (NB + 1) / 2;         // stored blocks of H
+  static constexpr int kSteps = 8 * kBlocksH;                // k-steps of 4 per column slice
+  static constexpr int kWarps = kClipThreads / 32;
+  static constexpr int kWarpsPerSlice = kWarps / (kClipCols / kSliceCols);
+  static constexpr int kStepsPerWarp = kSteps / kWarpsPerSlice;
+  static_assert(kSteps % kWarpsPerSlice == 0, "k-steps must split evenly over the warps of a slice");
+  static_assert(kStepsPerWarp % 2 == 0, "runs start and end on even steps");
+  static_assert(kSliceCols == 16, "the product is written for two 8-column MMA tiles per warp");
+  static constexpr size_t kSmemH = sizeof(double) * kBlocksH * 32 * 32;
+  static constexpr size_t kSmemD = sizeof(double) * G * kClipCols;  // one buffer
+  static constexpr size_t kSmemRed = sizeof(double) * 2 * kWarps * kSliceCols;
+  static constexpr size_t kSmem = kSmemH + 2 * kSmemD + kSmemRed;
 };
+
+__device__ __forceinline__ int swz(int row, int col) { return col ^ (((row & 1) << 3) | ((row & 2) << 1)); }
+
+// H[l][k] (l in block c >= k's block b) in the triangular layout
+__device__ __forceinline__ int h_index(int l, int k) {
+  const int c = l >> 5, b = k >> 5, lr = l & 31, kr = k & 31;
+  return ((c * (c + 1) / 2 + b) * 32 + lr) * 32 + swz(lr, kr);
+}
+
+__device__ __forceinline__ int d_index(int row, int col) { return row * kClipCols + swz(row, col); }
 
 __device__ __forceinline__ float shrink_factor(int i) {
   return __double2float_rn(__dsub_rn(1.0, __ddiv_rn(static_cast<double>(i), static_cast<double>(kShrinkGrid))));
 }
 
 __device__ __forceinline__ float clamp_to(float w, float c) { return fminf(fmaxf(w, -c), c); }
+
+__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+constexpr float kRoundMagic = 12582912.0f;            // 1.5 * 2^23: (x + m) - m = rint(x) for |x| < 2^22
+constexpr float kNearHalf = 0.5f - 1.0f / 32768.0f;   // |t - rint(t)| at or above this: exact division
+constexpr float kTinyStep = 7.888609052210118e-31f;   // 2^-100
+constexpr float kHugeRecip = 1.2676506002282294e30f;  // 2^100
 
 template <typename T, int G>
 __global__ void __launch_bounds__(kClipThreads, 1)
@@ -125,25 +209,34 @@ __global__ void __launch_bounds__(kClipThreads, 1)
                 double* __restrict__ errors, int32_t* __restrict__ codes, __half* __restrict__ steps,
                 __half* __restrict__ zeros, int* err) {
   using CT = ClipTile<G>;
+  constexpr int MJ = CT::kSliceCols / 8;  // 8-column MMA tiles per warp
   extern __shared__ __align__(16) uint8_t smem[];
-  double* sH = reinterpret_cast<double*>(smem);                           // [G][G]
-  double* sD = reinterpret_cast<double*>(smem + CT::kSmemH);              // [G][64]
-  double* sRed = reinterpret_cast<double*>(smem + CT::kSmemH + CT::kSmemD);  // [16][64]
-  __shared__ float sAbs[4][kClipCols], sMin[4][kClipCols], sMax[4][kClipCols];
+  double* sH = reinterpret_cast<double*>(smem);                                  // triangular H_g
+  double* sD = reinterpret_cast<double*>(smem + CT::kSmemH);                     // [2][G][64] deltas
+  double* sRed = reinterpret_cast<double*>(smem + CT::kSmemH + 2 * CT::kSmemD);  // [2][warp][kSliceCols]
+  __shared__ float sAbs[CT::kRowStep][kClipCols], sMin[CT::kRowStep][kClipCols], sMax[CT::kRowStep][kClipCols];
   __shared__ int sBest[kClipCols];
+  __shared__ float sF[kShrinkGrid];  // the shrink factors
 
   const int64_t g = blockIdx.y;
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kClipCols;
   const int64_t G_total = gridDim.y;
 
-  // H_g -> shared memory (16-byte vectors; it was written by the previous launch)
+  // the lower block triangle of H_g -> shared memory, asynchronously (it overlaps the
+  // load of W below); 16-byte pieces: block q, row lr, column pair kp
   {
-    const double2* src = reinterpret_cast<const double2*>(H + g * G * G);
-    double2* dst = reinterpret_cast<double2*>(sH);
-    for (int i = threadIdx.x; i < G * G / 2; i += kClipThreads) dst[i] = src[i];
+    const double* src = H + g * G * G;
+    for (int i = threadIdx.x; i < CT::kBlocksH * 32 * 16; i += kClipThreads) {
+      const int q = i / 512, rem = i % 512, lr = rem / 16, kp = rem % 16;
+      int c = 0;
+      while ((c + 1) * (c + 2) / 2 <= q) ++c;
+      const int b = q - c * (c + 1) / 2;
+      const int l = 32 * c + lr, k = 32 * b + 2 * kp;
+      cp_async_16(sH + h_index(l, k), src + l * G + k);
+    }
   }
 
-  // this thread's share of W': column n, rows k = r + 4 j
+  // this thread's share of W': column n, rows k = r + kRowStep j
   const int n = threadIdx.x % kClipCols, r = threadIdx.x / kClipCols;
   const bool col_ok = n0 + n < N;
   float wp[CT::EPT];
@@ -163,84 +256,215 @@ __global__ void __launch_bounds__(kClipThreads, 1)
     mx = fmaxf(mx, wp[j]);
   }
   if (bad) atomicOr(err, kErrNonfiniteW);
+  if (threadIdx.x < n_shrink) sF[threadIdx.x] = shrink_factor(threadIdx.x);
   sAbs[r][n] = amax;
   sMin[r][n] = mn;
   sMax[r][n] = mx;
+  cp_async_wait_all();
   __syncthreads();
-  amax = fmaxf(fmaxf(sAbs[0][n], sAbs[1][n]), fmaxf(sAbs[2][n], sAbs[3][n]));
-  mn = fminf(fminf(sMin[0][n], sMin[1][n]), fminf(sMin[2][n], sMin[3][n]));
-  mx = fmaxf(fmaxf(sMax[0][n], sMax[1][n]), fmaxf(sMax[2][n], sMax[3][n]));
+  amax = sAbs[0][n];
+  mn = sMin[0][n];
+  mx = sMax[0][n];
+#pragma unroll
+  for (int q = 1; q < CT::kRowStep; ++q) {
+    amax = fmaxf(amax, sAbs[q][n]);
+    mn = fminf(mn, sMin[q][n]);
+    mx = fmaxf(mx, sMax[q][n]);
+  }
 
-  // product layout: thread (tr, tc) owns rows RM*tr .. RM*tr+RM-1, columns tc + 16 c
-  const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
+  // Product. H_g is symmetric, so with 32-row blocks b, c:
+  //   delta^T H delta = sum_b delta_b^T (2 sum_{c > b} H_bc delta_c + H_bb delta_b),
+  // the upper block triangle only, read as H[l][k] from the stored lower one. For one
+  // 16-column slice these items, taken b-major (the weight-2 blocks c > b first, then
+  // the diagonal one) in k-steps of 4 values of l, form kSteps steps; each of the
+  // slice's warps takes an equal contiguous run of them and computes a 32 x 16 tile of
+  // Q_b = sum_c H_bc Delta_c with fp64 tensor-core MMAs, doubling Q_b when it reaches
+  // the diagonal block and folding Delta_b .* Q_b into its column sums when its row
+  // block changes.
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int slice = warp / CT::kWarpsPerSlice;
+  const int colw = slice * CT::kSliceCols;  // first column of the slice
+  int b_start = 0, ks_start = (warp % CT::kWarpsPerSlice) * CT::kStepsPerWarp;
+  while (ks_start >= 8 * (CT::NB - b_start)) {
+    ks_start -= 8 * (CT::NB - b_start);
+    ++b_start;
+  }
+  const int j_start = ks_start / 8;
+  ks_start %= 8;
+
+  // lanes 0..3 of every warp keep the running first minimum of column 4 warp + lane
+  const int my_col = warp * 4 + lane;
   double best_e = 0.0;
   int best_i = 0;
   const double tokens_d = static_cast<double>(tokens);
 
-  for (int i = 0; i < n_shrink; ++i) {
-    // clamp -> QDQ -> delta. Clamping is monotone, so the clamped group's min and max
-    // are the clamped min and max.
-    const float c = __fmul_rn(amax, shrink_factor(i));
-    const QdqParams p = qdq_params(clamp_to(mn, c), clamp_to(mx, c));
+  // One barrier per threshold: in step it, the deltas of threshold it are built into
+  // buffer it % 2 while the products of threshold it - 1 run on the other buffer and
+  // the column sums of threshold it - 2 are reduced. Odd warps multiply first and
+  // build second, even warps the other way round, so the ALU work of one half of the
+  // warps overlaps the tensor-core work of the other half.
+  auto build = [&](int it) {
+    if (it < n_shrink) {
+      // clamp -> QDQ -> delta. Clamping is monotone, so the clamped group's min and
+      // max are the clamped min and max. Codes use a correctly rounded reciprocal of
+      // the step; a quotient within 2^-15 of a half-integer takes the exact division.
+      double* dbuf = sD + (it & 1) * G * kClipCols;
+      const float c = __fmul_rn(amax, sF[it]);
+      const QdqParams p = qdq_params(clamp_to(mn, c), clamp_to(mx, c));
+      const float recip = __frcp_rn(p.step);
+      const bool col_exact = !(p.step >= kTinyStep && recip <= kHugeRecip);
+      const float lo = -p.zero, hi = 15.0f - p.zero;
 #pragma unroll
-    for (int j = 0; j < CT::EPT; ++j) {
-      const float q = qdq_code(clamp_to(wp[j], c), p);
-      const float rec = __fmul_rn(__fsub_rn(q, p.zero), p.step);
-      sD[(r + CT::kRowStep * j) * kClipCols + n] = __dsub_rn(static_cast<double>(rec), static_cast<double>(wp[j]));
-    }
-    __syncthreads();
-
-    double acc[CT::RM][4];
-#pragma unroll
-    for (int a = 0; a < CT::RM; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
-#pragma unroll 2
-    for (int l = 0; l < G; ++l) {
-      double ha[CT::RM], db[4];
-      const double2* hrow = reinterpret_cast<const double2*>(sH + l * G + CT::RM * tr);  // H symmetric: H[k][l] = H[l][k]
-#pragma unroll
-      for (int a = 0; a < CT::RM / 2; ++a) {
-        const double2 v = hrow[a];
-        ha[2 * a] = v.x;
-        ha[2 * a + 1] = v.y;
+      for (int j = 0; j < CT::EPT; ++j) {
+        const float wc = clamp_to(wp[j], c);
+        const float tv = fminf(fmaxf(__fmul_rn(wc, recip), lo), hi);
+        float qz = __fsub_rn(__fadd_rn(tv, kRoundMagic), kRoundMagic);  // q - z
+        if (col_exact || fabsf(__fsub_rn(tv, qz)) >= kNearHalf) qz = __fsub_rn(qdq_code(wc, p), p.zero);
+        const float rec = __fmul_rn(qz, p.step);
+        dbuf[d_index(r + CT::kRowStep * j, n)] = __dsub_rn(static_cast<double>(rec), static_cast<double>(wp[j]));
       }
-#pragma unroll
-      for (int b = 0; b < 4; ++b) db[b] = sD[l * kClipCols + tc + 16 * b];
-#pragma unroll
-      for (int a = 0; a < CT::RM; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = __fma_rn(ha[a], db[b], acc[a][b]);
     }
+  };
+  auto product = [&](int it) {
+    if (it >= 1 && it <= n_shrink) {
+      const double* dbuf = sD + ((it - 1) & 1) * G * kClipCols;
+      double ep[MJ][2];  // column sums of this lane: columns colw + 8 jt + 2 tq + {0, 1}
+      double acc[4][MJ][2];
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      double pe = 0.0;
+      for (int jt = 0; jt < MJ; ++jt) {
+        ep[jt][0] = ep[jt][1] = 0.0;
 #pragma unroll
-      for (int a = 0; a < CT::RM; ++a) pe = __fma_rn(sD[(CT::RM * tr + a) * kClipCols + tc + 16 * b], acc[a][b], pe);
-      sRed[tr * kClipCols + tc + 16 * b] = pe;
+        for (int i4 = 0; i4 < 4; ++i4) acc[i4][jt][0] = acc[i4][jt][1] = 0.0;
+      }
+      auto fold = [&](int blk) {  // ep += Delta_blk .* Q_blk, then clear Q
+#pragma unroll
+        for (int i4 = 0; i4 < 4; ++i4) {
+          const int row = 32 * blk + 8 * i4 + gq;
+#pragma unroll
+          for (int jt = 0; jt < MJ; ++jt) {
+            const double2 dv = *reinterpret_cast<const double2*>(dbuf + d_index(row, colw + 8 * jt + 2 * tq));
+            ep[jt][0] = __fma_rn(dv.x, acc[i4][jt][0], ep[jt][0]);
+            ep[jt][1] = __fma_rn(dv.y, acc[i4][jt][1], ep[jt][1]);
+            acc[i4][jt][0] = acc[i4][jt][1] = 0.0;
+          }
+        }
+      };
+      auto double_q = [&]() {  // exact: the weight-2 sums
+#pragma unroll
+        for (int i4 = 0; i4 < 4; ++i4)
+#pragma unroll
+          for (int jt = 0; jt < MJ; ++jt) {
+            acc[i4][jt][0] = __dadd_rn(acc[i4][jt][0], acc[i4][jt][0]);
+            acc[i4][jt][1] = __dadd_rn(acc[i4][jt][1], acc[i4][jt][1]);
+          }
+      };
+      // The run, as segments of one item each: row block b, column block cb, steps
+      // ks0 .. ks0 + cnt - 1. Inside a segment every load is a fixed offset from one of
+      // four per-lane pointers: with x = tq & 1 the swizzle maps the fragment columns
+      // 8 m + gq of row 4 s + tq to 8 (m ^ x) + (gq ^ 4 (tq >> 1)), so pointers pa0 / pa1
+      // (pd0 / pd1) serve the even / odd MMA rows (columns) and each step moves them by
+      // 4 rows. Runs start and end on even steps, so the inner loop takes two steps.
+      const int x = tq & 1;
+      const int lane_off = gq ^ (4 * (tq >> 1));
+      int b = b_start, j = j_start, ks = ks_start, remaining = CT::kStepsPerWarp;
+      bool on_diag = false;
+      while (remaining > 0) {
+        const int n_off = CT::NB - 1 - b;  // weight-2 blocks right of the diagonal
+        const int cb = j < n_off ? b + 1 + j : b;
+        const int cnt = min(8 - ks, remaining);
+        on_diag = cb == b;
+        if (on_diag && ks == 0) double_q();  // entering the diagonal block
+        const double* hrow = sH + ((cb * (cb + 1) / 2 + b) * 32 + 4 * ks + tq) * 32 + lane_off;
+        const double* pa0 = hrow + 8 * x;
+        const double* pa1 = hrow + 8 * (1 - x);
+        const double* drow = dbuf + (32 * cb + 4 * ks + tq) * kClipCols + colw + lane_off;
+        const double* pd0 = drow + 8 * x;
+        const double* pd1 = drow + 8 * (1 - x);
+#pragma unroll 1
+        for (int u = 0; u < cnt; u += 2) {
+#pragma unroll
+          for (int v = 0; v < 2; ++v) {
+            const int oa = (u + v) * 128, od = (u + v) * 4 * kClipCols;
+            const double a0 = pa0[oa], a1 = pa1[oa], a2 = pa0[oa + 16], a3 = pa1[oa + 16];
+            const double b0 = pd0[od], b1 = pd1[od];
+            mma_f64(acc[0][0], a0, b0);
+            mma_f64(acc[0][1], a0, b1);
+            mma_f64(acc[1][0], a1, b0);
+            mma_f64(acc[1][1], a1, b1);
+            mma_f64(acc[2][0], a2, b0);
+            mma_f64(acc[2][1], a2, b1);
+            mma_f64(acc[3][0], a3, b0);
+            mma_f64(acc[3][1], a3, b1);
+          }
+        }
+        remaining -= cnt;
+        ks += cnt;
+        if (ks == 8) {
+          ks = 0;
+          if (++j == CT::NB - b) {
+            fold(b);
+            ++b;
+            j = 0;
+          }
+        }
+      }
+      if (b < CT::NB) {  // the run ended inside row block b (a no-op after a clean block end)
+        if (!on_diag) double_q();  // it never reached the diagonal block
+        fold(b);
+      }
+      // combine the 8 lanes (gq) that hold partial sums of the same columns
+#pragma unroll
+      for (int jt = 0; jt < MJ; ++jt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          double v = ep[jt][h];
+          v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, 4));
+          v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, 8));
+          v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, 16));
+          ep[jt][h] = v;
+        }
+      if (gq == 0) {
+        double* red = sRed + ((it - 1) & 1) * CT::kWarps * CT::kSliceCols + warp * CT::kSliceCols;
+#pragma unroll
+        for (int jt = 0; jt < MJ; ++jt) {
+          red[8 * jt + 2 * tq] = ep[jt][0];
+          red[8 * jt + 2 * tq + 1] = ep[jt][1];
+        }
+      }
     }
-    __syncthreads();
-    if (threadIdx.x < kClipCols) {
+  };
+  for (int it = 0; it < n_shrink + 2; ++it) {
+    if (warp & 1) {
+      product(it);
+      build(it);
+    } else {
+      build(it);
+      product(it);
+    }
+    if (it >= 2 && lane < 4) {
+      const int i = it - 2;
+      const double* red = sRed + (i & 1) * CT::kWarps * CT::kSliceCols;
+      const int w0 = (my_col / CT::kSliceCols) * CT::kWarpsPerSlice;
       double e = 0.0;
 #pragma unroll
-      for (int q = 0; q < 16; ++q) e = __dadd_rn(e, sRed[q * kClipCols + threadIdx.x]);
+      for (int q = 0; q < CT::kWarpsPerSlice; ++q) e = __dadd_rn(e, red[(w0 + q) * CT::kSliceCols + my_col % CT::kSliceCols]);
       e = __ddiv_rn(e, tokens_d);  // the mean over the sampled tokens
-      if (errors && col_ok) errors[(static_cast<int64_t>(i) * G_total + g) * N + n0 + threadIdx.x] = e;
+      if (errors && n0 + my_col < N) errors[(static_cast<int64_t>(i) * G_total + g) * N + n0 + my_col] = e;
       if (i == 0 || e < best_e) {  // first minimum
         best_e = e;
         best_i = i;
       }
     }
-    // the next candidate overwrites sD only after this barrier-separated phase; sRed
-    // is rewritten after the next candidate's first barrier
+    __syncthreads();
   }
-  if (threadIdx.x < kClipCols) sBest[threadIdx.x] = best_i;
+  if (lane < 4) sBest[my_col] = best_i;
   __syncthreads();
 
   // artifact of the chosen threshold: codes through shared memory, packed eight per
   // int32 along N; steps and zeros as fp16
   const int bi = sBest[n];
-  const float c = __fmul_rn(amax, shrink_factor(bi));
+  const float c = __fmul_rn(amax, sF[bi]);
   const QdqParams p = qdq_params(clamp_to(mn, c), clamp_to(mx, c));
   uint8_t* sQ = reinterpret_cast<uint8_t*>(sD);  // [G][64] codes
 #pragma unroll
@@ -260,7 +484,7 @@ __global__ void __launch_bounds__(kClipThreads, 1)
     if (n0 + 8 * w >= N) continue;  // N % 8 == 0: a word lies wholly inside or outside
     uint32_t word = 0;
 #pragma unroll
-    for (int b = 0; b < 8; ++b) word |= static_cast<uint32_t>(sQ[k * kClipCols + 8 * w + b]) << (4 * b);
+    for (int bb = 0; bb < 8; ++bb) word |= static_cast<uint32_t>(sQ[k * kClipCols + 8 * w + bb]) << (4 * bb);
     codes[(g * G + k) * words + n0 / 8 + w] = static_cast<int32_t>(word);
   }
 }
