@@ -47,6 +47,7 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=None, help="steps of the host-buffer run (default: --steps)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clip", action="store_true", help="skip the clipping-search measurement")
     return ap.parse_args(argv)
 
 
@@ -162,6 +163,71 @@ def cpu_oracle_sample(spec: LayerSpec, target_s: float):
             "sample": f"{n} of {spec.N} output columns with the full {spec.M}x{spec.K} X "
                       f"({t:.1f} s, numpy fp64 oracle)",
             "seconds": t, "columns": n}
+
+
+def clip_fmas(spec: LayerSpec, n_shrink: int) -> float:
+    """Multiply-adds the clipping search needs: for every (threshold, group, column) the
+    distinct products of the symmetric quadratic form delta^T H delta, g (g + 1) / 2."""
+    g = spec.group
+    return float(n_shrink) * (spec.K // g) * spec.N * g * (g + 1) / 2
+
+
+def measure_clip(awq, spec: LayerSpec, Xd, Wd, scales, stream, flush, steps: int, n_shrink: int = 10):
+    """Device time of the clipping search (Gram matrices + search + clipped artifact) on
+    the same resident layer, with the fp64 tensor-core roofline of its search kernel."""
+    for _ in range(2):
+        awq.clip_search(Xd, Wd, scales, spec.group, n_shrink, stream=stream)
+    s_ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    gram, search = [], []
+    for i in range(steps):
+        flush.zero_()
+        s_ev[i].record(stream)
+        awq.clip_search(Xd, Wd, scales, spec.group, n_shrink, stream=stream)
+        e_ev[i].record(stream)
+        p = awq.clip_profile_last()
+        gram.append(p["gram"])
+        search.append(p["clip_search"])
+    torch.cuda.synchronize()
+    call_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(s_ev, e_ev))
+    peak = awq.fp64_mma_peak(stream=stream)
+    flops = 2.0 * clip_fmas(spec, n_shrink)
+    ms = statistics.mean(search)
+    achieved = flops / (ms / 1e3) / 1e12
+    return {
+        "n_shrink": n_shrink, "tokens": awq.clip_token_count(spec.M), "steps": steps,
+        "ms_per_call": call_ms, "gram_ms": statistics.mean(gram), "search_ms": ms,
+        "layers_per_s": 1e3 / call_ms, "gpu_launches_per_call": awq.last_launch_count(),
+        "roofline": {"bound": "tensor", "kernel": "clip_kernel (fp64 MMA quadratic forms + clipped artifact)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": "fp64 tensor-core MMA throughput measured in this run (awq_fp64_mma_peak)",
+                     "work": "2 * n_shrink * groups * N * g (g + 1) / 2 flops (distinct products of the "
+                             "symmetric quadratic forms)",
+                     "traffic": None},
+    }
+
+
+def cpu_clip_sample(spec: LayerSpec, target_s: float, n_shrink: int = 10):
+    """The clipping oracle as it stands on a column slice (full X, same scales reading)."""
+    import oracle as O
+    import oracle.awq_clip as C
+    X, W = generate(spec)
+    X32, W32 = as_f32_numpy(X), as_f32_numpy(W)
+    s = O.candidate_scales(O.activation_statistic(X32), spec.n_grid)[spec.n_grid // 2]
+
+    def run(ncols):
+        t0 = time.perf_counter()
+        C.clip_search(X32, W32[:, :ncols], s, spec.group, n_shrink)
+        return time.perf_counter() - t0
+
+    n = min(spec.N, 64)
+    t = run(n)
+    while t < target_s / 3 and n < spec.N:
+        n = min(spec.N, n * 4)
+        t = run(n)
+    sub = LayerSpec(**{**spec.as_dict(), "N": n})
+    return {"value": 2.0 * clip_fmas(sub, n_shrink) / t / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(),
+            "kind": "oracle", "sample": f"{n} of {spec.N} output columns ({t:.1f} s, numpy fp64 oracle)"}
 
 
 def rank_spec(base: LayerSpec, rank: int) -> LayerSpec:
@@ -299,6 +365,10 @@ def run_ours(args, rank, world, local):
         barrier()
         e2e_ms = float(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)))
 
+        # the next row of the pipeline: clipping search with the chosen scales
+        clip = None if args.no_clip else measure_clip(awq, spec, Xd, Wd, out.scales, stream, flush,
+                                                      max(3, min(args.steps, 10)))
+
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
 
     flops = spec.candidate_flops
@@ -345,8 +415,12 @@ def run_ours(args, rank, world, local):
         "clocks": clock_info,
         "chosen_alpha_index": out.best,
     }
+    if clip is not None:
+        line["clip_search"] = clip
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(spec, args.cpu_seconds)
+        if clip is not None:
+            clip["cpu_baseline"] = cpu_clip_sample(spec, min(args.cpu_seconds, 10.0))
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

@@ -184,6 +184,15 @@ int awq_clip_search(const void* X, const void* W, int in_dtype, const float* sca
                     void* out_zeros, awq_stream_t stream);
 /* Number of tokens the clipping search samples from M rows (0 on bad arguments). */
 int64_t awq_clip_token_count(int64_t M, int64_t max_tokens);
+/* With profiling on (awq_profile_enable), device times (ms) of the last clipping
+ * search's two kernels: [0] the Gram matrices, [1] the search. Returns 2. */
+int awq_clip_profile_last(float* ms, int n);
+
+/* Measured throughput (TFLOP/s, 2 flops per multiply-add) of the fp64 tensor-core
+ * MMA on the current device: a register-only loop of 8x8x4 fp64 MMAs, 4 CTAs of 8
+ * warps per SM, timed with CUDA events on `stream`. The roofline denominator of the
+ * clipping search's products. */
+int awq_fp64_mma_peak(double* tflops, awq_stream_t stream);
 
 int awq_version(void);
 

@@ -23,7 +23,7 @@ __all__ = [
     "tile_shape", "workspace_bytes", "release_cached", "profile_enable", "profile_last",
     "last_launch_count", "debug_set_fault", "status_string", "exported_functions",
     "activation_statistic", "candidate_scales", "qdq_candidates", "ClipOutput", "clip_search",
-    "clip_token_count",
+    "clip_token_count", "clip_profile_last", "fp64_mma_peak",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -86,6 +86,10 @@ def library() -> ctypes.CDLL:
     lib.awq_candidate_scales.argtypes = [vp, i64, i32, vp, vp]
     lib.awq_qdq_candidates.argtypes = [vp, i32, i64, i64, i32, i32, vp, vp, vp]
     lib.awq_clip_search.argtypes = [vp, vp, i32, vp, i64, i64, i64, i32, i32, i64, vp, vp, vp, vp, vp, vp, vp]
+    lib.awq_clip_profile_last.argtypes = [ctypes.POINTER(ctypes.c_float), i32]
+    lib.awq_clip_profile_last.restype = ctypes.c_int
+    lib.awq_fp64_mma_peak.argtypes = [ctypes.POINTER(ctypes.c_double), vp]
+    lib.awq_fp64_mma_peak.restype = ctypes.c_int
     lib.awq_clip_token_count.argtypes = [i64, i64]
     lib.awq_clip_token_count.restype = ctypes.c_int64
     for name in ("awq_activation_statistic", "awq_candidate_scales", "awq_qdq_candidates", "awq_clip_search"):
@@ -326,3 +330,18 @@ def clip_search(X: torch.Tensor, W: torch.Tensor, scales: torch.Tensor, group: i
                              _stream_handle(stream, dev))
     _check(st)
     return ClipOutput(max_val, best, codes, steps, zeros, errs)
+
+
+def clip_profile_last() -> dict:
+    """Device times (ms) of the last clipping search's kernels (profiling on)."""
+    ms = (ctypes.c_float * 2)()
+    library().awq_clip_profile_last(ms, 2)
+    return {"gram": ms[0], "clip_search": ms[1]}
+
+
+def fp64_mma_peak(device=None, stream=None) -> float:
+    """Measured fp64 tensor-core MMA throughput of the device, TFLOP/s."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    out = ctypes.c_double(0.0)
+    _check(library().awq_fp64_mma_peak(ctypes.byref(out), _stream_handle(stream, dev)))
+    return out.value

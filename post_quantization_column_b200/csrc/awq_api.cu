@@ -214,6 +214,21 @@ int* pinned_status_word(int dev) {
   return words[dev];
 }
 
+// Events around the two launches of the clipping search (profiling only).
+float g_clip_ms[2] = {0.0f, 0.0f};
+cudaEvent_t* clip_events(int dev) {
+  static cudaEvent_t ev[64][3];
+  static bool made[64] = {false};
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!made[dev]) {
+    for (auto& e : ev[dev])
+      if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    made[dev] = true;
+  }
+  return ev[dev];
+}
+
 // Per-device copy stream and events for awq_search_host, created on first use.
 struct CopyLane {
   static constexpr int kChunks = 8;
@@ -668,6 +683,7 @@ int awq_clip_search(const void* X, const void* W, int in_dtype, const float* sca
   a.codes = out_codes;
   a.steps = static_cast<__half*>(out_steps);
   a.zeros = static_cast<__half*>(out_zeros);
+  a.ev = g_profile ? clip_events(dev) : nullptr;
   int launches = 0, h_err = 0;
   int* pinned = pinned_status_word(dev);
   int* status_dst = pinned ? pinned : &h_err;
@@ -679,10 +695,55 @@ int awq_clip_search(const void* X, const void* W, int in_dtype, const float* sca
   if (se != cudaSuccess) return cuda_error(se, "stream synchronize");
   if (pinned) h_err = *pinned;
   g_last_launches = launches;
+  if (a.ev) {
+    cudaEventElapsedTime(&g_clip_ms[0], a.ev[0], a.ev[1]);
+    cudaEventElapsedTime(&g_clip_ms[1], a.ev[1], a.ev[2]);
+  }
   if (h_err & kErrBadScale) return set_error(AWQ_ERR_INVALID_ARG, "a scale is not a positive finite number");
   if (h_err & kErrNonfiniteX) return set_error(AWQ_ERR_NONFINITE, "non-finite value in X / s");
   if (h_err & kErrNonfiniteW) return set_error(AWQ_ERR_NONFINITE, "non-finite value in W");
   if (h_err) return set_error(AWQ_ERR_CUDA, "device status word " + std::to_string(h_err));
+  return AWQ_OK;
+}
+
+int awq_clip_profile_last(float* ms, int n) {
+  for (int i = 0; i < n && i < 2; ++i) ms[i] = g_clip_ms[i];
+  return 2;
+}
+
+int awq_fp64_mma_peak(double* tflops, awq_stream_t stream) {
+  t_last_error.clear();
+  if (!tflops) return set_error(AWQ_ERR_INVALID_ARG, "tflops is NULL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  bind_device(s, nullptr);
+  int dev = 0, num_sms = 0, st;
+  if ((st = check_device(&dev, &num_sms)) != AWQ_OK) return st;
+  cudaMemPool_t pool;
+  if ((st = get_pool(dev, &pool)) != AWQ_OK) return st;
+  const int blocks = 4 * num_sms, iters = 4096;
+  void* out = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(&out, static_cast<size_t>(blocks) * 256 * sizeof(double), pool, s);
+  if (e != cudaSuccess || !out) {
+    cudaGetLastError();
+    return set_error(AWQ_ERR_OOM, "probe buffer");
+  }
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  float ms = 0.0f;
+  if ((e = cudaEventCreate(&e0)) == cudaSuccess && (e = cudaEventCreate(&e1)) == cudaSuccess &&
+      (e = launch_fp64_mma_peak(static_cast<double*>(out), blocks, iters, s)) == cudaSuccess &&
+      (e = cudaEventRecord(e0, s)) == cudaSuccess &&
+      (e = launch_fp64_mma_peak(static_cast<double*>(out), blocks, iters, s)) == cudaSuccess &&
+      (e = cudaEventRecord(e1, s)) == cudaSuccess && (e = cudaEventSynchronize(e1)) == cudaSuccess)
+    e = cudaEventElapsedTime(&ms, e0, e1);
+  cudaFreeAsync(out, s);
+  cudaError_t se = cudaStreamSynchronize(s);
+  if (e0) cudaEventDestroy(e0);
+  if (e1) cudaEventDestroy(e1);
+  if (e != cudaSuccess) return cuda_error(e, "fp64 MMA probe");
+  if (se != cudaSuccess) return cuda_error(se, "stream synchronize");
+  // per launch: blocks x 8 warps x iters x 8 MMAs of 8 x 8 x 4 multiply-adds
+  const double flops = 2.0 * blocks * 8.0 * iters * 8.0 * 256.0;
+  *tflops = ms > 0.0f ? flops / (ms * 1e-3) / 1e12 : 0.0;
   return AWQ_OK;
 }
 

@@ -92,12 +92,16 @@ struct ClipArgs {
   __half* steps;       // [K / group][N]
   __half* zeros;       // [K / group][N]
   int* err;
+  cudaEvent_t* ev;     // nullptr, or 3 events recorded around the two launches
 };
 int64_t clip_token_stride(int64_t M, int64_t max_tokens);
 int64_t clip_token_count(int64_t M, int64_t max_tokens);
 // Gram matrices of the sampled scaled activations, then the per-(group, column) search
 // and the clipped artifact: two launches.
 cudaError_t launch_clip(const ClipArgs& a, cudaStream_t s, int* launches);
+// Register-only loop of fp64 tensor-core MMAs (8 accumulators per warp, `iters` x 8
+// MMAs of 8x8x4 per warp); `out` holds blocks * 256 doubles.
+cudaError_t launch_fp64_mma_peak(double* out, int blocks, int iters, cudaStream_t s);
 
 __host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 

@@ -493,6 +493,7 @@ template <typename T, int G>
 cudaError_t launch_clip_t(const ClipArgs& a, cudaStream_t st, int* launches) {
   const int64_t groups = a.K / G;
   const int64_t stride = clip_token_stride(a.M, a.max_tokens);
+  if (a.ev) cudaEventRecord(a.ev[0], st);
   {
     constexpr int TB = G < 64 ? G : 64;
     dim3 grid(static_cast<unsigned>(groups), (G / TB) * (G / TB));
@@ -502,6 +503,7 @@ cudaError_t launch_clip_t(const ClipArgs& a, cudaStream_t st, int* launches) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
+  if (a.ev) cudaEventRecord(a.ev[1], st);
   static unsigned long long done = 0;
   cudaError_t e = set_smem_limit_once(clip_kernel<T, G>, static_cast<int>(ClipTile<G>::kSmem), &done);
   if (e != cudaSuccess) return e;
@@ -510,6 +512,7 @@ cudaError_t launch_clip_t(const ClipArgs& a, cudaStream_t st, int* launches) {
       static_cast<const T*>(a.W), a.N, a.s, a.H, a.n_shrink, a.tokens, a.max_val, a.best, a.errors, a.codes, a.steps,
       a.zeros, a.err);
   *launches += 1;
+  if (a.ev) cudaEventRecord(a.ev[2], st);
   return cudaGetLastError();
 }
 
@@ -520,6 +523,27 @@ cudaError_t launch_clip_dtype(const ClipArgs& a, cudaStream_t st, int* launches)
     case 64: return launch_clip_t<T, 64>(a, st, launches);
     default: return launch_clip_t<T, 128>(a, st, launches);
   }
+}
+
+// Throughput probe of the fp64 tensor-core MMA: register operands, 8 independent
+// accumulators per warp, no memory traffic but one store per thread.
+__global__ void __launch_bounds__(256) fp64_mma_peak_kernel(double* out, int iters) {
+  const int lane = threadIdx.x & 31;
+  double a[4], b[2], d[8][2];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) a[i] = 1.0 + 1e-9 * (lane + i);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) b[i] = 1.0 - 1e-9 * (lane + i);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) d[i][0] = d[i][1] = 0.0;
+  for (int it = 0; it < iters; ++it) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mma_f64(d[i], a[i & 3], b[i >> 2]);
+  }
+  double s = 0.0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) s += d[i][0] + d[i][1];
+  out[static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x] = s;
 }
 
 }  // namespace
@@ -536,4 +560,12 @@ cudaError_t launch_clip(const ClipArgs& a, cudaStream_t s, int* launches) {
   return a.in_dtype == 0 ? launch_clip_dtype<__nv_bfloat16>(a, s, launches) : launch_clip_dtype<float>(a, s, launches);
 }
 
+}  // namespace awq
+
+namespace awq {
+// Blocks x 256 threads of the probe; `out` holds blocks * 256 doubles.
+cudaError_t launch_fp64_mma_peak(double* out, int blocks, int iters, cudaStream_t s) {
+  fp64_mma_peak_kernel<<<blocks, 256, 0, s>>>(out, iters);
+  return cudaGetLastError();
+}
 }  // namespace awq
