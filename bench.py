@@ -75,17 +75,19 @@ def recorded_traffic(kernel: str, workload: str):
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        rec = json.load(f)
-    if rec.get("kernel") != kernel or rec.get("workload") != workload:
-        return None
-    for rel, digest in rec.get("sources_sha256", {}).items():
-        full = os.path.join(ROOT, rel)
-        if not os.path.exists(full):
-            return None
-        with open(full, "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest() != digest:
+        recs = json.load(f).get("records", [])
+    for rec in recs:
+        if rec.get("kernel") != kernel or rec.get("workload") != workload:
+            continue
+        for rel, digest in rec.get("sources_sha256", {}).items():
+            full = os.path.join(ROOT, rel)
+            if not os.path.exists(full):
                 return None
-    return float(rec["dram_bytes_per_launch"])
+            with open(full, "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest() != digest:
+                    return None
+        return float(rec["dram_bytes_per_launch"])
+    return None
 
 
 def cpu_threads() -> int:
@@ -203,7 +205,8 @@ def measure_clip(awq, spec: LayerSpec, Xd, Wd, scales, stream, flush, steps: int
                      "peak_source": "fp64 tensor-core MMA throughput measured in this run (awq_fp64_mma_peak)",
                      "work": "2 * n_shrink * groups * N * g (g + 1) / 2 flops (distinct products of the "
                              "symmetric quadratic forms)",
-                     "traffic": None},
+                     "traffic": recorded_traffic("clip_kernel", spec.name),
+                     "traffic_unit": "DRAM bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"},
     }
 
 
