@@ -48,6 +48,7 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clip", action="store_true", help="skip the clipping-search measurement")
+    ap.add_argument("--no-w4a16", action="store_true", help="skip the W4A16 consumer measurement")
     return ap.parse_args(argv)
 
 
@@ -210,6 +211,46 @@ def measure_clip(awq, spec: LayerSpec, Xd, Wd, scales, stream, flush, steps: int
     }
 
 
+def measure_w4a16(awq, spec: LayerSpec, X, out, stream, flush, steps: int, peaks):
+    """The artifact's W4A16 consumer on the same layer: decode (1 token, fused GEMV; HBM
+    roofline over the 4.25-bit weight stream) and prefill (all M tokens, dequantize +
+    tensor-core GEMM; fp16 tensor roofline)."""
+    Xd = X.to(out.scales.device).float()
+    A = (Xd / out.scales[None, :]).half()  # activations divided by the chosen scales
+    res = {}
+    for label, M in (("decode", 1), ("prefill", spec.M)):
+        Am = A[:M].contiguous()
+        for _ in range(2):
+            awq.w4a16_matmul(Am, out.codes, out.steps, out.zeros, spec.group, stream=stream)
+        awq.profile_enable(True)
+        ms = []
+        for _ in range(steps):
+            flush.zero_()
+            awq.w4a16_matmul(Am, out.codes, out.steps, out.zeros, spec.group, stream=stream)
+            ms.append(awq.w4a16_profile_last())
+        launches = awq.last_launch_count()
+        t = statistics.median(ms)
+        groups = spec.K // spec.group
+        stream_bytes = spec.K * spec.N / 2 + 4 * groups * spec.N + 2 * M * spec.K + 4 * M * spec.N
+        flops = 2.0 * M * spec.K * spec.N
+        entry = {"M": M, "ms": t, "gpu_launches_per_call": launches, "TFLOP/s": flops / (t / 1e3) / 1e12,
+                 "GB/s": stream_bytes / (t / 1e3) / 1e9}
+        if label == "decode":
+            entry["roofline"] = {"bound": "hbm", "kernel": "gemv_kernel (fused dequantize + fp16 MMA)",
+                                 "achieved": entry["GB/s"], "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                                 "frac": entry["GB/s"] / float(peaks["hbm_gbs"]),
+                                 "work": "K N / 2 code bytes + 4 bytes per (group, column) + 2 M K + 4 M N"}
+        else:
+            entry["roofline"] = {"bound": "tensor", "kernel": "dequant_kernel + loss_gemm_kernel mode 2 (fp16)",
+                                 "achieved": entry["TFLOP/s"], "peak": float(peaks["bf16_tflops"]),
+                                 "unit": "TFLOP/s", "frac": entry["TFLOP/s"] / float(peaks["bf16_tflops"]),
+                                 "peak_source": "bf16 dense burst peak (fp16 runs at the same rate)",
+                                 "work": "2 M K N flops (both kernels' time)"}
+        res[label] = entry
+    awq.profile_enable(True)
+    return res
+
+
 def cpu_clip_sample(spec: LayerSpec, target_s: float, n_shrink: int = 10):
     """The clipping oracle as it stands on a column slice (full X, same scales reading)."""
     import oracle as O
@@ -368,9 +409,12 @@ def run_ours(args, rank, world, local):
         barrier()
         e2e_ms = float(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)))
 
-        # the next row of the pipeline: clipping search with the chosen scales
+        # the next rows of the pipeline: clipping search with the chosen scales, and the
+        # artifact's W4A16 consumer
         clip = None if args.no_clip else measure_clip(awq, spec, Xd, Wd, out.scales, stream, flush,
                                                       max(3, min(args.steps, 10)))
+        w4a16 = None if args.no_w4a16 else measure_w4a16(awq, spec, X, out, stream, flush,
+                                                         max(5, min(args.steps, 20)), measured_peaks()[0])
 
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
 
@@ -420,6 +464,8 @@ def run_ours(args, rank, world, local):
     }
     if clip is not None:
         line["clip_search"] = clip
+    if w4a16 is not None:
+        line["w4a16"] = w4a16
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(spec, args.cpu_seconds)
         if clip is not None:

@@ -194,6 +194,31 @@ int awq_clip_profile_last(float* ms, int n);
  * clipping search's products. */
 int awq_fp64_mma_peak(double* tflops, awq_stream_t stream);
 
+/* ---- W4A16 consumer of the artifact ---------------------------------------------
+ * [AWQ-P1] §7: the artifact feeds a W4A16 kernel, checked by decoding it and comparing
+ * the kernel's output with a reference; §8: 4-bit weights, 16-bit activations; §6: the
+ * scales are folded into the operation that produces the activations.
+ *   Y[m][n] = sum_k A[m][k] * w16[k][n],  w16[k][n] = fp16((q[k][n] - z[g][n]) * step[g][n])
+ * A [M][K] fp16 activations already divided by the scales (A = fp16(X / s)); codes
+ * [K][N/8] int32, steps and zeros [K/group][N] fp16 (the artifact of awq_search or
+ * awq_clip_search); Y [M][N] fp32. Every product is exact in fp32 and the sums are fp32.
+ * M <= 16 runs a fused dequantize + GEMV (bound by the 4.25-bit weight stream) and is
+ * asynchronous: the call returns once the work is enqueued on `stream` (launch errors
+ * are reported; Y is ready when the stream reaches that point). Larger M dequantizes
+ * to an N x K fp16 work space (N K 2 bytes from the library's pool), runs the
+ * tensor-core GEMM and synchronizes `stream` (its waits are bounded and reported as
+ * AWQ_ERR_TIMEOUT). Same preconditions as awq_search on K, N and group; all pointers
+ * device memory, 16-byte aligned. NaN or Inf in A propagates to Y. */
+int awq_w4a16_matmul(const void* A, const int32_t* codes, const void* steps,
+                     const void* zeros, int64_t M, int64_t K, int64_t N, int group,
+                     float* Y, awq_stream_t stream);
+/* With profiling on (awq_profile_enable): device time (ms) of the last call's kernels,
+ * waiting for them if needed; -1 when the last call was not profiled. */
+float awq_w4a16_profile_last(void);
+/* The dequantized operand alone: out_wt [N][K] fp16 (K contiguous) = w16 transposed. */
+int awq_w4a16_dequant(const int32_t* codes, const void* steps, const void* zeros,
+                      int64_t K, int64_t N, int group, void* out_wt, awq_stream_t stream);
+
 int awq_version(void);
 
 /* ---- Searching without allocating -------------------------------------------

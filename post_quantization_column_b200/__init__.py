@@ -23,7 +23,7 @@ __all__ = [
     "tile_shape", "workspace_bytes", "release_cached", "profile_enable", "profile_last",
     "last_launch_count", "debug_set_fault", "status_string", "exported_functions",
     "activation_statistic", "candidate_scales", "qdq_candidates", "ClipOutput", "clip_search",
-    "clip_token_count", "clip_profile_last", "fp64_mma_peak",
+    "clip_token_count", "clip_profile_last", "fp64_mma_peak", "w4a16_matmul", "w4a16_dequant", "w4a16_profile_last",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -90,9 +90,14 @@ def library() -> ctypes.CDLL:
     lib.awq_clip_profile_last.restype = ctypes.c_int
     lib.awq_fp64_mma_peak.argtypes = [ctypes.POINTER(ctypes.c_double), vp]
     lib.awq_fp64_mma_peak.restype = ctypes.c_int
+    lib.awq_w4a16_matmul.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, vp, vp]
+    lib.awq_w4a16_dequant.argtypes = [vp, vp, vp, i64, i64, i32, vp, vp]
+    lib.awq_w4a16_profile_last.argtypes = []
+    lib.awq_w4a16_profile_last.restype = ctypes.c_float
     lib.awq_clip_token_count.argtypes = [i64, i64]
     lib.awq_clip_token_count.restype = ctypes.c_int64
-    for name in ("awq_activation_statistic", "awq_candidate_scales", "awq_qdq_candidates", "awq_clip_search"):
+    for name in ("awq_activation_statistic", "awq_candidate_scales", "awq_qdq_candidates", "awq_clip_search",
+                 "awq_w4a16_matmul", "awq_w4a16_dequant"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -345,3 +350,45 @@ def fp64_mma_peak(device=None, stream=None) -> float:
     out = ctypes.c_double(0.0)
     _check(library().awq_fp64_mma_peak(ctypes.byref(out), _stream_handle(stream, dev)))
     return out.value
+
+
+def _artifact_args(codes, steps, zeros, group):
+    if not (codes.is_cuda and steps.is_cuda and zeros.is_cuda):
+        raise ValueError("the artifact must be on the device")
+    if codes.dtype != torch.int32 or steps.dtype != torch.float16 or zeros.dtype != torch.float16:
+        raise TypeError("codes int32, steps and zeros float16")
+    K = codes.shape[0]
+    N = steps.shape[1]
+    if codes.shape != (K, N // 8) or steps.shape != (K // group, N) or zeros.shape != steps.shape:
+        raise ValueError("codes (K, N/8), steps and zeros (K/group, N)")
+    return codes.contiguous(), steps.contiguous(), zeros.contiguous(), K, N
+
+
+def w4a16_matmul(A: torch.Tensor, codes: torch.Tensor, steps: torch.Tensor, zeros: torch.Tensor, group: int = 128,
+                 *, stream=None) -> torch.Tensor:
+    """Y = A w16 with w16 = fp16((q - z) step) from the packed artifact; A (M, K) fp16 on the
+    device, already divided by the scales. Returns (M, N) fp32 (for M <= 16 the call is
+    asynchronous on `stream`)."""
+    codes, steps, zeros, K, N = _artifact_args(codes, steps, zeros, group)
+    if A.dtype != torch.float16 or not A.is_cuda or A.dim() != 2 or A.shape[1] != K:
+        raise ValueError("A must be a (M, K) float16 CUDA tensor")
+    A = A.contiguous()
+    Y = torch.empty(A.shape[0], N, dtype=torch.float32, device=A.device)
+    _check(library().awq_w4a16_matmul(_ptr(A), _ptr(codes), _ptr(steps), _ptr(zeros), A.shape[0], K, N, group,
+                                      _ptr(Y), _stream_handle(stream, A.device)))
+    return Y
+
+
+def w4a16_dequant(codes: torch.Tensor, steps: torch.Tensor, zeros: torch.Tensor, group: int = 128, *,
+                  stream=None) -> torch.Tensor:
+    """The dequantized operand, transposed: (N, K) fp16, K contiguous."""
+    codes, steps, zeros, K, N = _artifact_args(codes, steps, zeros, group)
+    out = torch.empty(N, K, dtype=torch.float16, device=codes.device)
+    _check(library().awq_w4a16_dequant(_ptr(codes), _ptr(steps), _ptr(zeros), K, N, group, _ptr(out),
+                                       _stream_handle(stream, codes.device)))
+    return out
+
+
+def w4a16_profile_last() -> float:
+    """Device time (ms) of the last W4A16 call's kernels when profiling is on, else -1."""
+    return float(library().awq_w4a16_profile_last())

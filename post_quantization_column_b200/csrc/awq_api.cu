@@ -229,6 +229,23 @@ cudaEvent_t* clip_events(int dev) {
   return ev[dev];
 }
 
+// Events around the kernels of the W4A16 consumer (profiling only).
+bool g_w4a16_profiled = false;
+cudaEvent_t* g_w4a16_last_ev = nullptr;
+cudaEvent_t* w4a16_events(int dev) {
+  static cudaEvent_t ev[64][2];
+  static bool made[64] = {false};
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!made[dev]) {
+    for (auto& e : ev[dev])
+      if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    made[dev] = true;
+  }
+  g_w4a16_last_ev = ev[dev];
+  return ev[dev];
+}
+
 // Per-device copy stream and events for awq_search_host, created on first use.
 struct CopyLane {
   static constexpr int kChunks = 8;
@@ -703,6 +720,160 @@ int awq_clip_search(const void* X, const void* W, int in_dtype, const float* sca
   if (h_err & kErrNonfiniteX) return set_error(AWQ_ERR_NONFINITE, "non-finite value in X / s");
   if (h_err & kErrNonfiniteW) return set_error(AWQ_ERR_NONFINITE, "non-finite value in W");
   if (h_err) return set_error(AWQ_ERR_CUDA, "device status word " + std::to_string(h_err));
+  return AWQ_OK;
+}
+
+// ---- W4A16 consumer of the artifact --------------------------------------------------
+namespace {
+int validate_w4a16(const void* A, const void* codes, const void* steps, const void* zeros, int64_t M, int64_t K,
+                   int64_t N, int group, const void* Y) {
+  if (!codes || !steps || !zeros || (M > 0 && (!A || !Y)))
+    return set_error(AWQ_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (group != 32 && group != 64 && group != 128)
+    return set_error(AWQ_ERR_INVALID_ARG, "group must be 32, 64 or 128");
+  if (M <= 0 || K <= 0 || N <= 0) return set_error(AWQ_ERR_SHAPE, "M, K and N must be positive");
+  if (M >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) || N >= (int64_t(1) << 31))
+    return set_error(AWQ_ERR_SHAPE, "M, K and N must be below 2^31");
+  if (K % group) return set_error(AWQ_ERR_SHAPE, "group must divide K");
+  if (K / group > 65535) return set_error(AWQ_ERR_SHAPE, "K / group must not exceed 65535");
+  if (N % 8) return set_error(AWQ_ERR_SHAPE, "N must be a multiple of 8 (eight codes per int32)");
+  if (!aligned16(A) || !aligned16(codes) || !aligned16(steps) || !aligned16(zeros) || !aligned16(Y))
+    return set_error(AWQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  return AWQ_OK;
+}
+}  // namespace
+
+int awq_w4a16_matmul(const void* A, const int32_t* codes, const void* steps, const void* zeros, int64_t M, int64_t K,
+                     int64_t N, int group, float* Y, awq_stream_t stream) {
+  t_last_error.clear();
+  int st = validate_w4a16(A, codes, steps, zeros, M, K, N, group, Y);
+  if (st != AWQ_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  bind_device(s, codes);
+  int dev = 0, num_sms = 0;
+  if ((st = check_device(&dev, &num_sms)) != AWQ_OK) return st;
+  if (!is_device_memory(A) || !is_device_memory(codes) || !is_device_memory(steps) || !is_device_memory(zeros) ||
+      !is_device_memory(Y))
+    return set_error(AWQ_ERR_INVALID_ARG, "inputs and outputs must be device memory");
+  cudaMemPool_t pool;
+  if ((st = get_pool(dev, &pool)) != AWQ_OK) return st;
+  const bool gemv = M <= kW4A16GemvMaxM;
+  const size_t ws_bytes = gemv ? 256 + align_up(static_cast<size_t>(gemv_split_floats(M, K, N, group, num_sms)) * 4)
+                               : 256 + align_up(static_cast<size_t>(N) * K * 2);
+  void* ws = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, ws_bytes, pool, s);
+  if (e != cudaSuccess || !ws) {
+    cudaGetLastError();
+    return set_error(AWQ_ERR_OOM, "W4A16 work space of " + std::to_string(ws_bytes) + " bytes");
+  }
+  int* err = static_cast<int*>(ws);
+  void* body = static_cast<uint8_t*>(ws) + 256;
+  W4A16Args a;
+  a.A = static_cast<const __half*>(A);
+  a.codes = codes;
+  a.steps = static_cast<const __half*>(steps);
+  a.zeros = static_cast<const __half*>(zeros);
+  a.M = M;
+  a.K = K;
+  a.N = N;
+  a.group = group;
+  a.Y = Y;
+  int launches = 0, h_err = 0;
+  cudaEvent_t* ev = g_profile ? w4a16_events(dev) : nullptr;
+  if (gemv) {
+    // asynchronous: no device-side error conditions, nothing to read back
+    if (ev) cudaEventRecord(ev[0], s);
+    e = launch_w4a16_gemv(a, num_sms, static_cast<float*>(body), s, &launches);
+    if (ev) cudaEventRecord(ev[1], s);
+    g_w4a16_profiled = ev != nullptr;
+    cudaFreeAsync(ws, s);
+    if (e != cudaSuccess) return cuda_error(e, "W4A16 GEMV");
+    g_last_launches = launches;
+    return AWQ_OK;
+  }
+  int* pinned = pinned_status_word(dev);
+  int* status_dst = pinned ? pinned : &h_err;
+  int status = AWQ_OK;
+  const char* where = "";
+  do {
+    if ((e = cudaMemsetAsync(err, 0, 16, s)) != cudaSuccess) { where = "cudaMemsetAsync"; break; }
+    if (ev) cudaEventRecord(ev[0], s);
+    {
+      __half* Wt = static_cast<__half*>(body);
+      if ((e = launch_w4a16_dequant(codes, a.steps, a.zeros, K, N, group, Wt, s, &launches)) != cudaSuccess) {
+        where = "W4A16 dequantization";
+        break;
+      }
+      LossGemmArgs ga;
+      ga.Xb = reinterpret_cast<const __nv_bfloat16*>(A);  // 2-byte elements; the MMA reads them as fp16
+      ga.Wt = reinterpret_cast<const __nv_bfloat16*>(Wt);
+      ga.M = M;
+      ga.K = K;
+      ga.N = N;
+      ga.n_grid = 0;
+      ga.Y = Y;
+      ga.partial = nullptr;
+      ga.err = err;
+      ga.timeout_ns = g_timeout_ns;
+      ga.fault_mode = 0;
+      ga.num_sms = num_sms;
+      ga.f16 = 1;
+      CUtensorMap mapA, mapB;
+      const char* why = "";
+      if ((e = make_operand_maps(ga, &mapA, &mapB, &why, kTileN)) != cudaSuccess) {
+        status = set_error(AWQ_ERR_CUDA, std::string("TMA descriptor: ") + why);
+        break;
+      }
+      if ((e = launch_loss_gemm(ga, mapA, mapB, 2, s, &launches)) != cudaSuccess) { where = "W4A16 GEMM"; break; }
+      if (ev) cudaEventRecord(ev[1], s);
+      g_w4a16_profiled = ev != nullptr;
+    }
+    e = cudaMemcpyAsync(status_dst, err, sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) where = "status read-back";
+  } while (false);
+  if (status == AWQ_OK && e != cudaSuccess) status = cuda_error(e, where);
+  cudaFreeAsync(ws, s);
+  cudaError_t se = cudaStreamSynchronize(s);
+  if (status == AWQ_OK && se != cudaSuccess) status = cuda_error(se, "stream synchronize");
+  if (pinned) h_err = *pinned;
+  if (status == AWQ_OK) {
+    g_last_launches = launches;
+    if (h_err & kErrTimeout) status = set_error(AWQ_ERR_TIMEOUT, "a bounded wait in the W4A16 GEMM ran out");
+    else if (h_err) status = set_error(AWQ_ERR_CUDA, "device status word " + std::to_string(h_err));
+  }
+  return status;
+}
+
+float awq_w4a16_profile_last(void) {
+  if (!g_w4a16_profiled || !g_w4a16_last_ev) return -1.0f;
+  float ms = -1.0f;
+  if (cudaEventSynchronize(g_w4a16_last_ev[1]) != cudaSuccess ||
+      cudaEventElapsedTime(&ms, g_w4a16_last_ev[0], g_w4a16_last_ev[1]) != cudaSuccess) {
+    cudaGetLastError();
+    return -1.0f;
+  }
+  return ms;
+}
+
+int awq_w4a16_dequant(const int32_t* codes, const void* steps, const void* zeros, int64_t K, int64_t N, int group,
+                      void* out_wt, awq_stream_t stream) {
+  t_last_error.clear();
+  static __align__(16) int dummy[4];
+  int st = validate_w4a16(dummy, codes, steps, zeros, 1, K, N, group, out_wt);
+  if (st != AWQ_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  bind_device(s, codes);
+  int dev = 0, num_sms = 0;
+  if ((st = check_device(&dev, &num_sms)) != AWQ_OK) return st;
+  if (!is_device_memory(codes) || !is_device_memory(steps) || !is_device_memory(zeros) || !is_device_memory(out_wt))
+    return set_error(AWQ_ERR_INVALID_ARG, "inputs and outputs must be device memory");
+  int launches = 0;
+  cudaError_t e = launch_w4a16_dequant(codes, static_cast<const __half*>(steps), static_cast<const __half*>(zeros), K,
+                                       N, group, static_cast<__half*>(out_wt), s, &launches);
+  cudaError_t se = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_error(e, "W4A16 dequantization");
+  if (se != cudaSuccess) return cuda_error(se, "stream synchronize");
+  g_last_launches = launches;
   return AWQ_OK;
 }
 

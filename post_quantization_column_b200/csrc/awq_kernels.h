@@ -56,6 +56,7 @@ struct LossGemmArgs {
   uint64_t timeout_ns;
   int fault_mode;
   int num_sms;
+  int f16 = 0;               // mode 2 only: fp16 operands (the tensor maps move 2-byte elements either way)
 };
 // Which loss GEMM runs: 1 = the one-SM kernel (default), 2 = the two-SM
 // (cta_group::2) kernel, selected with AWQ_GEMM_VARIANT=2 in the environment.
@@ -66,7 +67,9 @@ inline int operand_b_box_rows() { return gemm_variant() == 2 ? kTileN / 2 : kTil
 // Builds the TMA descriptors (driver entry point) for the two operands.
 cudaError_t make_operand_maps(const LossGemmArgs& a, CUtensorMap* mapA, CUtensorMap* mapB,
                               const char** why, int b_box_rows);
-// mode 0: Y = X_b W_b into the tiled buffer; mode 1: per-tile sum of (X_b W_hat_i - Y)^2.
+// mode 0: Y = X_b W_b into the tiled buffer; mode 1: per-tile sum of (X_b W_hat_i - Y)^2;
+// mode 2: Y = X_b Wt[0]^T written row-major fp32 into a.Y (M x N, pitch N), always on
+// the one-SM kernel (make the maps with b_box_rows = kTileN).
 cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, const CUtensorMap& mapB,
                              int mode, cudaStream_t s, int* launches);
 
@@ -102,6 +105,25 @@ cudaError_t launch_clip(const ClipArgs& a, cudaStream_t s, int* launches);
 // Register-only loop of fp64 tensor-core MMAs (8 accumulators per warp, `iters` x 8
 // MMAs of 8x8x4 per warp); `out` holds blocks * 256 doubles.
 cudaError_t launch_fp64_mma_peak(double* out, int blocks, int iters, cudaStream_t s);
+
+// ---- W4A16 consumer of the artifact (AWQ-P1 §7-§8) ---------------------------------
+struct W4A16Args {
+  const __half* A;        // [M][K] fp16 activations (already divided by the scales)
+  const int32_t* codes;   // [K][N/8]
+  const __half* steps;    // [K/group][N]
+  const __half* zeros;    // [K/group][N]
+  int64_t M, K, N;
+  int group;
+  float* Y;               // [M][N] fp32
+};
+constexpr int kW4A16GemvMaxM = 16;
+// Fused dequantization + GEMV for M <= kW4A16GemvMaxM; `part` holds
+// gemv_split_floats(...) floats when that is non-zero (a second launch sums the splits).
+cudaError_t launch_w4a16_gemv(const W4A16Args& a, int num_sms, float* part, cudaStream_t s, int* launches);
+int64_t gemv_split_floats(int64_t M, int64_t K, int64_t N, int group, int num_sms);
+// w16 transposed: Wt[n][k] = fp16((q - z) step), N x K with K contiguous.
+cudaError_t launch_w4a16_dequant(const int32_t* codes, const __half* steps, const __half* zeros, int64_t K, int64_t N,
+                                 int group, __half* Wt, cudaStream_t s, int* launches);
 
 __host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 

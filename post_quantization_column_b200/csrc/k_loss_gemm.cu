@@ -2,11 +2,13 @@
 // Activation" §4: every candidate is scored by the mean squared difference between the
 // original output and the candidate output, the difference cast to FP32).
 //
-// One persistent kernel, two modes:
+// One persistent kernel, three modes:
 //   mode 0: Y = X_b W_b, written once to HBM in a tile-major layout;
 //   mode 1: for every (candidate i, output tile): acc = X_b W_hat_i,b on the tensor
 //           cores, and the epilogue adds (acc - Y)^2 over the tile and writes one fp64
-//           partial sum. The candidate output Y_hat is never written to HBM.
+//           partial sum. The candidate output Y_hat is never written to HBM;
+//   mode 2: a plain product A B^T (B stored K-major), written row-major in fp32 with
+//           the ragged rows and columns masked (the packed artifact's consumer).
 //
 // Blackwell structure (sm_100a): 128 x 256 output tiles, K in 64-element (128-byte)
 // slices; a 4-stage TMA -> shared-memory ring (128-byte swizzle, no multicast); one
@@ -49,7 +51,9 @@ struct GemmParams {
   int n_grid;
   int tiles_m, tiles_n;
   int nk;
-  float* Y;
+  int64_t M, N, ldo;  // mode 2: output rows, columns and row pitch
+  int f16;            // mode 2: operands are fp16 (else bf16)
+  float* Y;           // modes 0-1: the tiled reference output; mode 2: the row-major output
   double* partial;
   int* err;
   uint64_t timeout_ns;
@@ -128,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
-  const int64_t n_units = (p.mode == 0 ? 1 : p.n_grid) * tiles;
+  const int64_t n_units = (p.mode == 1 ? p.n_grid : 1) * tiles;
   const uint64_t budget = p.timeout_ns;
 
   auto fail = [&]() {
@@ -146,7 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int64_t u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         int c, mt, nt;
         unit_coords(u, p, c, mt, nt);
-        const int slot = p.mode == 0 ? 0 : c + 1;
+        const int slot = p.mode == 1 ? c + 1 : 0;
         for (int kb = 0; kb < p.nk; ++kb) {
           if (!mbar_wait_bounded(empty + stage, phase ^ 1u, abort_flag, budget)) {
             ok = false;
@@ -177,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+      const uint32_t idesc = p.f16 ? idesc_f16_f32(BM, BN) : idesc_bf16_f32(BM, BN);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -244,7 +248,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(j0), v);
         tmem_ld_wait();
         float4* yrow = ytile + (j0 / 4) * BM + row;  // tile layout [BN/4][BM][4]
-        if (p.mode == 0) {
+        if (p.mode == 2) {
+          const int64_t grow = static_cast<int64_t>(mt) * BM + row;
+          if (grow < p.M) {
+            const int64_t col0 = static_cast<int64_t>(nt) * BN + j0;
+            float4* orow = reinterpret_cast<float4*>(p.Y + grow * p.ldo + col0);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)  // N % 8 == 0: a float4 lies wholly inside or outside
+              if (col0 + 4 * q < p.N)
+                orow[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                      __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+          }
+        } else if (p.mode == 0) {
 #pragma unroll
           for (int q = 0; q < 8; ++q)
             yrow[q * BM] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
@@ -642,7 +657,7 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
                              cudaStream_t s, int* launches) {
   const int tiles_m = static_cast<int>(ceil_div(a.M, BM));
   const int tiles_n = static_cast<int>(ceil_div(a.N, BN));
-  if (gemm_variant() == 2) {
+  if (gemm_variant() == 2 && mode != 2) {
     static unsigned long long attr_done = 0;
     cudaError_t e = set_smem_limit_once(loss_gemm_pair_kernel, kPairSmemBytes, &attr_done);
     if (e != cudaSuccess) return e;
@@ -694,13 +709,17 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
   p.tiles_m = tiles_m;
   p.tiles_n = tiles_n;
   p.nk = static_cast<int>(ceil_div(a.K, BK));
+  p.M = a.M;
+  p.N = a.N;
+  p.ldo = a.N;
+  p.f16 = a.f16;
   p.Y = a.Y;
   p.partial = a.partial;
   p.err = a.err;
   p.timeout_ns = a.timeout_ns;
   p.fault_mode = a.fault_mode;
   const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
-  const int64_t units = (mode == 0 ? 1 : a.n_grid) * tiles;
+  const int64_t units = (mode == 1 ? a.n_grid : 1) * tiles;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(units, a.num_sms));
   loss_gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(mapA, mapB, p);
   *launches += 1;
