@@ -79,6 +79,14 @@ typedef enum awq_status {
 
 enum { AWQ_DTYPE_BF16 = 0, AWQ_DTYPE_F32 = 1 };
 
+/* The candidates' quantizer. AWQ_QUANT_ASYM is the search's asymmetric zero-point
+ * quantizer (AWQ-P1 §7, steps 3-4 below). AWQ_QUANT_SYM is the symmetric [-7, 7] absmax
+ * teaching quantizer of AWQ-P1 §2: per (group, column) step = max|W'| / 7 (1 for an
+ * all-zero group or when the quotient underflows), q = clamp(rint(W'/step), -7, 7),
+ * reconstruction q * step; the artifact stores it in the same layout as codes q + 7
+ * with zero point 7, so step * (code - zero) decodes both. */
+enum { AWQ_QUANT_ASYM = 0, AWQ_QUANT_SYM = 1 };
+
 /* The search on bf16 X [M][K] and bf16 W [K][N] (device pointers). */
 int awq_search(const void* X, const void* W, int64_t M, int64_t K, int64_t N,
                int group, int n_grid, float* out_scales, int32_t* out_codes,
@@ -102,6 +110,13 @@ int awq_search_ex(const void* X, const void* W, int in_dtype, int64_t M, int64_t
                   int32_t* out_codes, void* out_steps, void* out_zeros,
                   float* out_losses, double* out_tile_sq_err, int64_t tile_sq_err_len,
                   awq_stream_t stream);
+
+/* The search with the candidates quantized by `quantizer` (AWQ_QUANT_ASYM gives
+ * awq_search_ex without tile partials). */
+int awq_search_quant(const void* X, const void* W, int in_dtype, int64_t M, int64_t K,
+                     int64_t N, int group, int n_grid, int quantizer, float* out_scales,
+                     int32_t* out_codes, void* out_steps, void* out_zeros, float* out_losses,
+                     awq_stream_t stream);
 
 /* End-to-end form with HOST buffers: copies X and W to the device on `stream`,
  * runs awq_search_ex, copies the outputs back (out_losses may be NULL). Pinned
@@ -160,7 +175,7 @@ int awq_debug_set_fault(int mode, int64_t timeout_ns);
  * output column n of the scaled layer W' = fl32(s W) (the layer once the scales are
  * folded in, AWQ-P1 §6; `scales` [K] fp32, typically awq_search's out_scales):
  *   c_i = fl32(absmax_g,n * fl32(1 - i/20)),  i = 0 .. n_shrink-1  (10 in the page: 1 .. 0.55)
- *   delta_i = Q(clamp(W'_g[:, n], -c_i, c_i)) - W'_g[:, n]   (Q = the quantizer of step 3)
+ *   delta_i = Q(clamp(W'_g[:, n], -c_i, c_i)) - W'_g[:, n]   (Q = `quantizer`, AWQ_QUANT_*)
  *   e_i = mean over sampled tokens t of (sum_{k in g} X'[t,k] delta_i[k])^2,  X' = fl32(X / s)
  *   i* = first argmin of e_i (fp64); the output is the clipped group's artifact.
  * Sampled tokens: rows 0, d, 2d, ... of X with d = max(1, M / max_tokens), at most
@@ -179,7 +194,7 @@ int awq_debug_set_fault(int mode, int64_t timeout_ns);
  * projections unclipped) is the caller's decision. */
 int awq_clip_search(const void* X, const void* W, int in_dtype, const float* scales,
                     int64_t M, int64_t K, int64_t N, int group, int n_shrink,
-                    int64_t max_tokens, float* out_max_val, int32_t* out_best,
+                    int64_t max_tokens, int quantizer, float* out_max_val, int32_t* out_best,
                     double* out_errors, int32_t* out_codes, void* out_steps,
                     void* out_zeros, awq_stream_t stream);
 /* Number of tokens the clipping search samples from M rows (0 on bad arguments). */

@@ -29,7 +29,7 @@ from dataclasses import dataclass
 
 import numpy as np
 
-from .awq_oracle import asym_qdq, sym_teaching_qdq, scale_weights, pack_codes, fp16_rne, first_argmin
+from .awq_oracle import asym_qdq, sym_teaching_qdq, sym_artifact, scale_weights, pack_codes, fp16_rne, first_argmin
 
 __all__ = ["clip_factors", "sample_tokens", "ClipResult", "clip_search", "clipped_artifact", "N_SHRINK",
            "SHRINK_GRID", "MAX_TOKENS"]
@@ -98,11 +98,14 @@ def clip_search(X, W, s, group: int, n_shrink: int = N_SHRINK, *, quantizer: str
     return ClipResult(errors=errors, best=best, max_val=max_val, thresholds=thresholds)
 
 
-def clipped_artifact(W, s, group: int, max_val):
+def clipped_artifact(W, s, group: int, max_val, quantizer: str = "asym"):
     """Codes (packed), fp16 steps and fp16 zeros of Q(clamp(s * W, -max_val, max_val))."""
     W = np.asarray(W, dtype=np.float32)
     Wp = scale_weights(W, np.asarray(s, dtype=np.float32))
     c = np.repeat(np.asarray(max_val, dtype=np.float32), group, axis=0)
     wc = np.minimum(np.maximum(Wp, -c), c).astype(np.float32)
-    q, step, zero, _ = asym_qdq(wc, group)
+    if quantizer == "asym":
+        q, step, zero, _ = asym_qdq(wc, group)
+    else:
+        q, step, zero = sym_artifact(wc, group)
     return pack_codes(q), fp16_rne(step), zero.astype(np.float16)

@@ -57,7 +57,7 @@ __all__ = [
     "bf16_rne", "fp16_rne", "activation_statistic", "candidate_alphas",
     "candidate_scales", "scale_weights", "asym_qdq", "sym_teaching_qdq", "fold_back",
     "candidate_what", "squared_error_mean", "output_loss", "block_squared_error", "first_argmin",
-    "pack_codes", "unpack_codes", "decode_artifact", "bits_per_weight",
+    "pack_codes", "unpack_codes", "decode_artifact", "bits_per_weight", "sym_artifact",
     "SearchResult", "search", "CLAMP_MIN", "Q_MAX",
 ]
 
@@ -173,7 +173,9 @@ def sym_teaching_qdq(Wp, group: int):
         raise ValueError("a group must contain finite values")
     Wg = _groups(Wp, group)
     peak = np.abs(Wg).max(axis=1)
-    step = np.where(peak == 0, dt(1), (peak / dt(7)).astype(dt)).astype(dt)
+    step = (peak / dt(7)).astype(dt)
+    # an all-zero group gets step 1 (AWQ-P1 §2); so does a quotient that underflows to 0
+    step = np.where((peak == 0) | (step == 0), dt(1), step).astype(dt)
     q = np.clip(np.rint((Wg / step[:, None, :]).astype(dt)), -7, 7).astype(dt)
     rec = (q * step[:, None, :]).astype(dt)
     K, N = Wp.shape
@@ -324,9 +326,22 @@ def search(X, W, group: int = 128, n_grid: int = 20, *, quantizer: str = "asym",
     res.extra["Y"] = Y
     if quantizer == "asym":
         q, step, zero, _ = asym_qdq(scale_weights(W, S[best]), group)
-        res.q, res.step, res.zero = q, step, zero
-        if N % 8 == 0:
-            res.codes = pack_codes(q)
-        res.steps_f16 = fp16_rne(step)
-        res.zeros_f16 = zero.astype(np.float16)
+    elif quantizer == "sym_teaching":
+        q, step, zero = sym_artifact(scale_weights(W, S[best]), group)
+    else:
+        return res
+    res.q, res.step, res.zero = q, step, zero
+    if N % 8 == 0:
+        res.codes = pack_codes(q)
+    res.steps_f16 = fp16_rne(step)
+    res.zeros_f16 = zero.astype(np.float16)
     return res
+
+
+def sym_artifact(Wp, group: int):
+    """The teaching quantizer's codes in the unsigned 4-bit artifact: code = q + 7 in
+    0..14 with zero point 7, so step * (code - zero) = q * step (AWQ-P1 §2 quantizer,
+    §7 artifact)."""
+    q, step, _ = sym_teaching_qdq(Wp, group)
+    zero = np.full(step.shape, 7.0, dtype=np.asarray(Wp).dtype)
+    return (q + 7).astype(np.int32), step, zero

@@ -85,7 +85,8 @@ def library() -> ctypes.CDLL:
     lib.awq_activation_statistic.argtypes = [vp, i32, i64, i64, vp, vp]
     lib.awq_candidate_scales.argtypes = [vp, i64, i32, vp, vp]
     lib.awq_qdq_candidates.argtypes = [vp, i32, i64, i64, i32, i32, vp, vp, vp]
-    lib.awq_clip_search.argtypes = [vp, vp, i32, vp, i64, i64, i64, i32, i32, i64, vp, vp, vp, vp, vp, vp, vp]
+    lib.awq_clip_search.argtypes = [vp, vp, i32, vp, i64, i64, i64, i32, i32, i64, i32, vp, vp, vp, vp, vp, vp, vp]
+    lib.awq_search_quant.argtypes = [vp, vp, i32, i64, i64, i64, i32, i32, i32, vp, vp, vp, vp, vp, vp]
     lib.awq_clip_profile_last.argtypes = [ctypes.POINTER(ctypes.c_float), i32]
     lib.awq_clip_profile_last.restype = ctypes.c_int
     lib.awq_fp64_mma_peak.argtypes = [ctypes.POINTER(ctypes.c_double), vp]
@@ -97,6 +98,7 @@ def library() -> ctypes.CDLL:
     lib.awq_clip_token_count.argtypes = [i64, i64]
     lib.awq_clip_token_count.restype = ctypes.c_int64
     for name in ("awq_activation_statistic", "awq_candidate_scales", "awq_qdq_candidates", "awq_clip_search",
+                 "awq_search_quant",
                  "awq_w4a16_matmul", "awq_w4a16_dequant"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -202,9 +204,16 @@ def _alloc_outputs(K, N, group, n_grid, device, pin=False):
             torch.empty(n_grid, dtype=torch.float32, **kw))
 
 
+QUANTIZERS = {"asym": 0, "sym": 1}
+
+
 def search(X: torch.Tensor, W: torch.Tensor, group: int = 128, n_grid: int = 20, *,
-           stream: torch.cuda.Stream | None = None, tile_sq_err: bool = False) -> SearchOutput:
-    """Run the search on device tensors X (M, K) and W (K, N) of the same dtype."""
+           stream: torch.cuda.Stream | None = None, tile_sq_err: bool = False,
+           quantizer: str = "asym") -> SearchOutput:
+    """Run the search on device tensors X (M, K) and W (K, N) of the same dtype.
+
+    ``quantizer`` "asym" (the search's zero-point quantizer) or "sym" (the symmetric
+    [-7, 7] teaching quantizer, artifact codes q + 7 with zero point 7)."""
     if X.dim() != 2 or W.dim() != 2 or X.shape[1] != W.shape[0]:
         raise ValueError("X must be (M, K) and W must be (K, N)")
     if X.dtype != W.dtype:
@@ -223,6 +232,16 @@ def search(X: torch.Tensor, W: torch.Tensor, group: int = 128, n_grid: int = 20,
     if tile_sq_err:
         tm, tn = tile_shape()
         tiles = torch.empty(n_grid, -(-M // tm), -(-N // tn), dtype=torch.float64, device=X.device)
+    if quantizer not in QUANTIZERS:
+        raise ValueError(f"quantizer must be one of {sorted(QUANTIZERS)}")
+    if quantizer != "asym":
+        if tile_sq_err:
+            raise ValueError("tile partials are available for the asymmetric quantizer only")
+        st = lib.awq_search_quant(_ptr(X), _ptr(W), _dtype_code(X), M, K, N, group, n_grid, QUANTIZERS[quantizer],
+                                  _ptr(scales), _ptr(codes), _ptr(steps), _ptr(zeros), _ptr(losses),
+                                  _stream_handle(stream, X.device))
+        _check(st)
+        return SearchOutput(scales, codes, steps, zeros, losses, None)
     st = lib.awq_search_ex(_ptr(X), _ptr(W), _dtype_code(X), M, K, N, group, n_grid, _ptr(scales), _ptr(codes),
                            _ptr(steps), _ptr(zeros), _ptr(losses), _ptr(tiles),
                            tiles.numel() if tiles is not None else 0, _stream_handle(stream, X.device))
@@ -303,7 +322,7 @@ def clip_token_count(M: int, max_tokens: int = 512) -> int:
 
 
 def clip_search(X: torch.Tensor, W: torch.Tensor, scales: torch.Tensor, group: int = 128, n_shrink: int = 10,
-                max_tokens: int = 512, *, errors: bool = False,
+                max_tokens: int = 512, *, errors: bool = False, quantizer: str = "asym",
                 stream: torch.cuda.Stream | None = None) -> ClipOutput:
     """Clipping search after the scaling on device tensors X (M, K), W (K, N) and the
     chosen scales (K,) fp32: per (group, column) threshold, its index, and the artifact
@@ -330,8 +349,10 @@ def clip_search(X: torch.Tensor, W: torch.Tensor, scales: torch.Tensor, group: i
     steps = torch.empty(G, N, dtype=torch.float16, device=dev)
     zeros = torch.empty(G, N, dtype=torch.float16, device=dev)
     errs = torch.empty(n_shrink, G, N, dtype=torch.float64, device=dev) if errors else None
+    if quantizer not in QUANTIZERS:
+        raise ValueError(f"quantizer must be one of {sorted(QUANTIZERS)}")
     st = lib.awq_clip_search(_ptr(X), _ptr(W), _dtype_code(X), _ptr(scales), M, K, N, group, n_shrink, max_tokens,
-                             _ptr(max_val), _ptr(best), _ptr(errs), _ptr(codes), _ptr(steps), _ptr(zeros),
+                             QUANTIZERS[quantizer], _ptr(max_val), _ptr(best), _ptr(errs), _ptr(codes), _ptr(steps), _ptr(zeros),
                              _stream_handle(stream, dev))
     _check(st)
     return ClipOutput(max_val, best, codes, steps, zeros, errs)

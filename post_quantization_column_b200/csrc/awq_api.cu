@@ -283,7 +283,10 @@ struct HostFeed {
 
 int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid,
                   float* out_scales, int32_t* out_codes, void* out_steps, void* out_zeros, float* out_losses,
-                  double* out_tile_sq_err, int64_t tile_sq_err_len, cudaStream_t s, const HostFeed* feed = nullptr) {
+                  double* out_tile_sq_err, int64_t tile_sq_err_len, cudaStream_t s, const HostFeed* feed = nullptr,
+                  int quantizer = kQuantAsym) {
+  if (quantizer != kQuantAsym && quantizer != kQuantSym)
+    return set_error(AWQ_ERR_INVALID_ARG, "quantizer must be AWQ_QUANT_ASYM or AWQ_QUANT_SYM");
   int st = validate(X, W, in_dtype, M, K, N, group, n_grid, out_scales, out_codes, out_steps, out_zeros, true);
   if (st != AWQ_OK) return st;
   if (out_losses && !aligned16(out_losses)) {
@@ -356,10 +359,10 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
         const int64_t gn = std::min(feed->groups_per_chunk, groups - g0);
         if (gn <= 0) break;
         if ((e = cudaStreamWaitEvent(s, feed->w_ready[c], 0)) == cudaSuccess)
-          e = launch_qdq_groups(W, in_dtype, K, N, group, n_grid, S, Wt, err, g0, gn, s, &launches);
+          e = launch_qdq_groups(W, in_dtype, K, N, group, n_grid, S, Wt, err, g0, gn, s, &launches, quantizer);
       }
     } else {
-      e = launch_qdq(W, in_dtype, K, N, group, n_grid, S, Wt, err, s, &launches);
+      e = launch_qdq(W, in_dtype, K, N, group, n_grid, S, Wt, err, s, &launches, quantizer);
     }
     if (e != cudaSuccess) {
       where = "qdq kernel";
@@ -395,7 +398,7 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
     }
     ev.mark(kPhPack);
     if ((e = launch_pack(W, in_dtype, K, N, group, n_grid, S, losses, best, out_codes, static_cast<__half*>(out_steps),
-                         static_cast<__half*>(out_zeros), out_scales, s, &launches)) != cudaSuccess) {
+                         static_cast<__half*>(out_zeros), out_scales, s, &launches, quantizer)) != cudaSuccess) {
       where = "pack kernel";
       break;
     }
@@ -467,6 +470,14 @@ int awq_search_f32(const float* X, const float* W, int64_t M, int64_t K, int64_t
                    awq_stream_t stream) {
   return awq_search_ex(X, W, AWQ_DTYPE_F32, M, K, N, group, n_grid, out_scales, out_codes, out_steps, out_zeros,
                        out_losses, nullptr, 0, stream);
+}
+
+int awq_search_quant(const void* X, const void* W, int in_dtype, int64_t M, int64_t K, int64_t N, int group,
+                     int n_grid, int quantizer, float* out_scales, int32_t* out_codes, void* out_steps,
+                     void* out_zeros, float* out_losses, awq_stream_t stream) {
+  t_last_error.clear();
+  return search_device(X, W, in_dtype, M, K, N, group, n_grid, out_scales, out_codes, out_steps, out_zeros,
+                       out_losses, nullptr, 0, reinterpret_cast<cudaStream_t>(stream), nullptr, quantizer);
 }
 
 int awq_search_host(const void* X_host, const void* W_host, int in_dtype, int64_t M, int64_t K, int64_t N, int group,
@@ -650,7 +661,7 @@ int awq_qdq_candidates(const void* W, int in_dtype, int64_t K, int64_t N, int gr
 
 // ---- clipping search after the scaling ---------------------------------------------
 int awq_clip_search(const void* X, const void* W, int in_dtype, const float* scales, int64_t M, int64_t K, int64_t N,
-                    int group, int n_shrink, int64_t max_tokens, float* out_max_val, int32_t* out_best,
+                    int group, int n_shrink, int64_t max_tokens, int quantizer, float* out_max_val, int32_t* out_best,
                     double* out_errors, int32_t* out_codes, void* out_steps, void* out_zeros, awq_stream_t stream) {
   t_last_error.clear();
   int st = validate(X, W, in_dtype, M, K, N, group, 1, out_max_val, out_codes, out_steps, out_zeros, false);
@@ -658,6 +669,8 @@ int awq_clip_search(const void* X, const void* W, int in_dtype, const float* sca
   if (!scales) return set_error(AWQ_ERR_INVALID_ARG, "scales is NULL");
   if (n_shrink < 1 || n_shrink > kMaxShrink) return set_error(AWQ_ERR_INVALID_ARG, "n_shrink must be in 1..20");
   if (max_tokens < 1) return set_error(AWQ_ERR_INVALID_ARG, "max_tokens must be positive");
+  if (quantizer != kQuantAsym && quantizer != kQuantSym)
+    return set_error(AWQ_ERR_INVALID_ARG, "quantizer must be AWQ_QUANT_ASYM or AWQ_QUANT_SYM");
   if (!aligned16(X) || !aligned16(W) || (reinterpret_cast<uintptr_t>(scales) & 3u) ||
       (reinterpret_cast<uintptr_t>(out_max_val) & 3u) || (reinterpret_cast<uintptr_t>(out_best) & 3u) ||
       (reinterpret_cast<uintptr_t>(out_errors) & 7u) || (reinterpret_cast<uintptr_t>(out_codes) & 3u) ||
@@ -701,6 +714,7 @@ int awq_clip_search(const void* X, const void* W, int in_dtype, const float* sca
   a.steps = static_cast<__half*>(out_steps);
   a.zeros = static_cast<__half*>(out_zeros);
   a.ev = g_profile ? clip_events(dev) : nullptr;
+  a.quantizer = quantizer;
   int launches = 0, h_err = 0;
   int* pinned = pinned_status_word(dev);
   int* status_dst = pinned ? pinned : &h_err;

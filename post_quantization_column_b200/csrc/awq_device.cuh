@@ -32,7 +32,13 @@ constexpr double kClampMin = 1e-4;   // lower bound on a^alpha before normalisin
 struct QdqParams {
   float step;
   float zero;  // integral, 0..15
+  float qmax;  // largest code: 15 (asymmetric) or 14 (symmetric, codes q + 7)
 };
+
+// Which quantizer the candidates use: the asymmetric zero-point one of AWQ-P1 §7 (the
+// search's), or the symmetric [-7, 7] absmax teaching quantizer of AWQ-P1 §2, stored
+// in the same unsigned artifact as codes q + 7 with zero point 7.
+enum : int { kQuantAsym = 0, kQuantSym = 1 };
 
 __device__ __forceinline__ QdqParams qdq_params(float mn, float mx) {
   QdqParams p;
@@ -43,12 +49,30 @@ __device__ __forceinline__ QdqParams qdq_params(float mn, float mx) {
   z = __fadd_rn(z, 0.0f);  // the zero point is an integer: rint(-0.25) = -0 becomes +0
   p.step = step;
   p.zero = z;
+  p.qmax = 15.0f;
   return p;
+}
+
+// step = max |w| / 7 (1 for an all-zero group or on underflow); q = clamp(rint(w / step), -7, 7)
+// is stored as q + 7.
+__device__ __forceinline__ QdqParams qdq_params_sym(float mn, float mx) {
+  QdqParams p;
+  const float peak = fmaxf(fabsf(mn), fabsf(mx));
+  float step = __fdiv_rn(peak, 7.0f);
+  if (peak == 0.0f || step == 0.0f) step = 1.0f;
+  p.step = step;
+  p.zero = 7.0f;
+  p.qmax = 14.0f;
+  return p;
+}
+
+__device__ __forceinline__ QdqParams qdq_params_q(float mn, float mx, int quantizer) {
+  return quantizer == kQuantSym ? qdq_params_sym(mn, mx) : qdq_params(mn, mx);
 }
 
 __device__ __forceinline__ float qdq_code(float wp, QdqParams p) {
   float q = __fadd_rn(rintf(__fdiv_rn(wp, p.step)), p.zero);
-  return fminf(fmaxf(q, 0.0f), 15.0f);
+  return fminf(fmaxf(q, 0.0f), p.qmax);
 }
 
 // W_hat = ((q - z) * step) / s  — the fold-back of AWQ-P1 §4, in fp32.

@@ -29,20 +29,23 @@ cudaError_t launch_to_bf16(const float* x, int64_t n, __nv_bfloat16* out, cudaSt
                            int* launches);
 
 // ---- scale + QDQ + fold-back of every candidate (AWQ-P1 §4, §7) -------------------
+// `quantizer`: 0 the asymmetric zero-point quantizer (AWQ-P1 §7), 1 the symmetric [-7, 7]
+// teaching quantizer (AWQ-P1 §2), stored as codes q + 7 with zero point 7.
 // Writes Wt[0] = bf16(W)^T and Wt[1 + i] = bf16(W_hat_i)^T, each N x K (K contiguous).
 cudaError_t launch_qdq(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid,
-                       const float* S, __nv_bfloat16* Wt, int* err, cudaStream_t s, int* launches);
+                       const float* S, __nv_bfloat16* Wt, int* err, cudaStream_t s, int* launches,
+                       int quantizer = 0);
 // The same for the groups group0 .. group0 + groups - 1 only (rows group0*group ..).
 cudaError_t launch_qdq_groups(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid,
                               const float* S, __nv_bfloat16* Wt, int* err, int64_t group0, int64_t groups,
-                              cudaStream_t s, int* launches);
+                              cudaStream_t s, int* launches, int quantizer = 0);
 
 // ---- artifact of the chosen candidate (AWQ-P1 §7; QUANT-P4 §5.3) ------------------
 // The chosen candidate is the first minimum of `losses` (AWQ-P1 §3); its index is
 // also written to *best.
 cudaError_t launch_pack(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid, const float* S,
                         const float* losses, int* best, int32_t* codes, __half* steps, __half* zeros,
-                        float* out_scales, cudaStream_t s, int* launches);
+                        float* out_scales, cudaStream_t s, int* launches, int quantizer = 0);
 
 // ---- loss GEMM (AWQ-P1 §4) ---------------------------------------------------------
 struct LossGemmArgs {
@@ -96,6 +99,7 @@ struct ClipArgs {
   __half* zeros;       // [K / group][N]
   int* err;
   cudaEvent_t* ev;     // nullptr, or 3 events recorded around the two launches
+  int quantizer;       // 0 asymmetric, 1 symmetric teaching quantizer
 };
 int64_t clip_token_stride(int64_t M, int64_t max_tokens);
 int64_t clip_token_count(int64_t M, int64_t max_tokens);

@@ -4,7 +4,8 @@
 // For every input group g and output column n of the scaled layer (W' = fl32(s W),
 // X' = fl32(X / s), the layer once the scales are folded in, same page §6), the search
 // tries the thresholds c_i = fl32(absmax * fl32(1 - i/20)), i = 0 .. n_shrink-1, clamps
-// the group to [-c_i, c_i], quantizes it with the asymmetric 4-bit quantizer (§7), and
+// the group to [-c_i, c_i], quantizes it with the asymmetric 4-bit quantizer (§7; or the
+// symmetric teaching quantizer of §2), and
 // scores the candidate by the mean squared error of the group's partial dot product
 // over the sampled tokens:
 //     e_i = (1/T) sum_t ( sum_{k in g} X'[t,k] delta_i[k] )^2 = delta_i^T H_g delta_i / T,
@@ -207,7 +208,7 @@ __global__ void __launch_bounds__(kClipThreads, 1)
     clip_kernel(const T* __restrict__ W, int64_t N, const float* __restrict__ s, const double* __restrict__ H,
                 int n_shrink, int tokens, float* __restrict__ max_val, int32_t* __restrict__ best_out,
                 double* __restrict__ errors, int32_t* __restrict__ codes, __half* __restrict__ steps,
-                __half* __restrict__ zeros, int* err) {
+                __half* __restrict__ zeros, int* err, int quantizer) {
   using CT = ClipTile<G>;
   constexpr int MJ = CT::kSliceCols / 8;  // 8-column MMA tiles per warp
   extern __shared__ __align__(16) uint8_t smem[];
@@ -311,10 +312,10 @@ __global__ void __launch_bounds__(kClipThreads, 1)
       // the step; a quotient within 2^-15 of a half-integer takes the exact division.
       double* dbuf = sD + (it & 1) * G * kClipCols;
       const float c = __fmul_rn(amax, sF[it]);
-      const QdqParams p = qdq_params(clamp_to(mn, c), clamp_to(mx, c));
+      const QdqParams p = qdq_params_q(clamp_to(mn, c), clamp_to(mx, c), quantizer);
       const float recip = __frcp_rn(p.step);
       const bool col_exact = !(p.step >= kTinyStep && recip <= kHugeRecip);
-      const float lo = -p.zero, hi = 15.0f - p.zero;
+      const float lo = -p.zero, hi = p.qmax - p.zero;
 #pragma unroll
       for (int j = 0; j < CT::EPT; ++j) {
         const float wc = clamp_to(wp[j], c);
@@ -465,7 +466,7 @@ __global__ void __launch_bounds__(kClipThreads, 1)
   // int32 along N; steps and zeros as fp16
   const int bi = sBest[n];
   const float c = __fmul_rn(amax, sF[bi]);
-  const QdqParams p = qdq_params(clamp_to(mn, c), clamp_to(mx, c));
+  const QdqParams p = qdq_params_q(clamp_to(mn, c), clamp_to(mx, c), quantizer);
   uint8_t* sQ = reinterpret_cast<uint8_t*>(sD);  // [G][64] codes
 #pragma unroll
   for (int j = 0; j < CT::EPT; ++j)
@@ -510,7 +511,7 @@ cudaError_t launch_clip_t(const ClipArgs& a, cudaStream_t st, int* launches) {
   dim3 grid(static_cast<unsigned>(ceil_div(a.N, kClipCols)), static_cast<unsigned>(groups));
   clip_kernel<T, G><<<grid, kClipThreads, ClipTile<G>::kSmem, st>>>(
       static_cast<const T*>(a.W), a.N, a.s, a.H, a.n_shrink, a.tokens, a.max_val, a.best, a.errors, a.codes, a.steps,
-      a.zeros, a.err);
+      a.zeros, a.err, a.quantizer);
   *launches += 1;
   if (a.ev) cudaEventRecord(a.ev[2], st);
   return cudaGetLastError();

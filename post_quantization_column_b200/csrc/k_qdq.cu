@@ -120,7 +120,7 @@ struct ColumnQdq {
 // butterfly over the low lane bits), then compute each column's parameters once per
 // column-group — even row-lanes column 0, odd ones column 1 — and broadcast them.
 template <int RL>
-__device__ __forceinline__ void column_qdq(float (&mn)[2], float (&mx)[2], ColumnQdq (&cq)[2]) {
+__device__ __forceinline__ void column_qdq(float (&mn)[2], float (&mx)[2], ColumnQdq (&cq)[2], int quantizer) {
 #pragma unroll
   for (int o = 1; o < RL; o <<= 1) {
 #pragma unroll
@@ -131,7 +131,7 @@ __device__ __forceinline__ void column_qdq(float (&mn)[2], float (&mx)[2], Colum
   }
   const int lane = threadIdx.x & 31;
   const int odd = lane & 1;
-  const QdqParams p = qdq_params(odd ? mn[1] : mn[0], odd ? mx[1] : mx[0]);
+  const QdqParams p = qdq_params_q(odd ? mn[1] : mn[0], odd ? mx[1] : mx[0], quantizer);
   const float r = __frcp_rn(p.step);
   const int exact = !(p.step >= kTinyStep && r <= kHugeRecip);
   const int base = lane & ~(RL - 1);
@@ -139,16 +139,17 @@ __device__ __forceinline__ void column_qdq(float (&mn)[2], float (&mx)[2], Colum
   for (int j = 0; j < 2; ++j) {
     cq[j].p.step = __shfl_sync(0xffffffffu, p.step, base + j);
     cq[j].p.zero = __shfl_sync(0xffffffffu, p.zero, base + j);
+    cq[j].p.qmax = p.qmax;  // the same for every column of the launch
     cq[j].recip = __shfl_sync(0xffffffffu, r, base + j);
     cq[j].exact = __shfl_sync(0xffffffffu, exact, base + j) != 0;
   }
 }
 
-// Whether every scaled weight of a column rounds inside [-z, 15 - z] without
+// Whether every scaled weight of a column rounds inside [-z, qmax - z] without
 // clamping: t = w' * (1/step) is monotone in w', so its extremes are the range times
 // the reciprocal, and a margin of 2^-15 covers the difference to the exact quotient.
 __device__ __forceinline__ bool clamp_free(float mn, float mx, const ColumnQdq& c) {
-  const float lo = -c.p.zero, hi = 15.0f - c.p.zero;
+  const float lo = -c.p.zero, hi = c.p.qmax - c.p.zero;
   return !c.exact && __fmul_rn(mn, c.recip) >= lo - kNearHalf && __fmul_rn(mx, c.recip) <= hi + kNearHalf;
 }
 
@@ -157,13 +158,13 @@ __device__ __forceinline__ bool clamp_free(float mn, float mx, const ColumnQdq& 
 template <bool kClamp>
 __device__ __forceinline__ bool fold_back_8(const float (&s)[8], const float (&w)[8], const float* rs,
                                             const ColumnQdq& c, float (&out)[8]) {
-  const float lo = -c.p.zero, hi = 15.0f - c.p.zero;
+  const float lo = -c.p.zero, hi = c.p.qmax - c.p.zero;
   bool need = false;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     float t = __fmul_rn(__fmul_rn(s[i], w[i]), c.recip);
     if (kClamp) t = fminf(fmaxf(t, lo), hi);
-    const float qz = round_small(t);  // q - z, an integer in [-z, 15 - z]
+    const float qz = round_small(t);  // q - z, an integer in [-z, qmax - z]
     need |= fabsf(__fsub_rn(t, qz)) >= kNearHalf;
     const float v = __fmul_rn(__fmul_rn(qz, c.p.step), rs[i]);
     need |= near_bf16_midpoint(v);
@@ -175,7 +176,7 @@ __device__ __forceinline__ bool fold_back_8(const float (&s)[8], const float (&w
 template <typename T, int G>
 __global__ void __launch_bounds__(Tile<G>::kThreads, Tile<G>::kBlocksPerSm)
     qdq_kernel(const T* __restrict__ W, int64_t K, int64_t N, int n_grid, const float* __restrict__ S,
-               __nv_bfloat16* __restrict__ Wt, int* err, int64_t group0) {
+               __nv_bfloat16* __restrict__ Wt, int* err, int64_t group0, int quantizer) {
   using L = Tile<G>;
   extern __shared__ float smem[];
   float* sWT = smem;                                 // [64][kPitch]
@@ -237,7 +238,7 @@ __global__ void __launch_bounds__(Tile<G>::kThreads, Tile<G>::kBlocksPerSm)
       }
     }
     ColumnQdq cq[2];
-    column_qdq<L::RL>(mn, mx, cq);
+    column_qdq<L::RL>(mn, mx, cq, quantizer);
     const bool no_clamp =
         __all_sync(0xffffffffu, clamp_free(mn[0], mx[0], cq[0]) && clamp_free(mn[1], mx[1], cq[1]));
 
@@ -298,7 +299,8 @@ template <typename T, int G>
 __global__ void __launch_bounds__(Tile<G>::kThreads, Tile<G>::kBlocksPerSm)
     pack_kernel(const T* __restrict__ W, int64_t K, int64_t N, int n_grid, const float* __restrict__ S,
                 const float* __restrict__ losses, int* __restrict__ best_out, int32_t* __restrict__ codes,
-                __half* __restrict__ steps, __half* __restrict__ zeros, float* __restrict__ out_scales) {
+                __half* __restrict__ steps, __half* __restrict__ zeros, float* __restrict__ out_scales,
+                int quantizer) {
   using L = Tile<G>;
   __shared__ float sWT[kQdqCols * L::kPitch];
   __shared__ __align__(16) uint8_t sQ[G][kQdqCols];
@@ -355,13 +357,13 @@ __global__ void __launch_bounds__(Tile<G>::kThreads, Tile<G>::kBlocksPerSm)
       }
     }
     ColumnQdq cq[2];
-    column_qdq<L::RL>(mn, mx, cq);
+    column_qdq<L::RL>(mn, mx, cq, quantizer);
 
     float q[2][8];
     bool need = cq[0].exact || cq[1].exact;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-      const float lo = -cq[j].p.zero, hi = 15.0f - cq[j].p.zero;
+      const float lo = -cq[j].p.zero, hi = cq[j].p.qmax - cq[j].p.zero;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const float tc = fminf(fmaxf(__fmul_rn(wp[j][i], cq[j].recip), lo), hi);
@@ -410,7 +412,7 @@ __global__ void __launch_bounds__(Tile<G>::kThreads, Tile<G>::kBlocksPerSm)
 
 template <typename T, int G>
 cudaError_t launch_qdq_t(const T* W, int64_t K, int64_t N, int n_grid, const float* S, __nv_bfloat16* Wt,
-                         int* err, int64_t group0, int64_t groups, cudaStream_t s) {
+                         int* err, int64_t group0, int64_t groups, cudaStream_t s, int quantizer) {
   using L = Tile<G>;
   const size_t smem = (static_cast<size_t>(kQdqCols) * L::kPitch + 2 * static_cast<size_t>(n_grid) * L::kSkewPitch) *
                       sizeof(float);
@@ -420,14 +422,14 @@ cudaError_t launch_qdq_t(const T* W, int64_t K, int64_t N, int n_grid, const flo
   cudaError_t e = set_smem_limit_once(qdq_kernel<T, G>, smem_max, &attr_done);
   if (e != cudaSuccess) return e;
   dim3 grid(static_cast<unsigned>(ceil_div(N, kQdqCols)), static_cast<unsigned>(groups));
-  qdq_kernel<T, G><<<grid, L::kThreads, smem, s>>>(W, K, N, n_grid, S, Wt, err, group0);
+  qdq_kernel<T, G><<<grid, L::kThreads, smem, s>>>(W, K, N, n_grid, S, Wt, err, group0, quantizer);
   return cudaGetLastError();
 }
 
 template <typename T, int G>
 cudaError_t launch_pack_t(const T* W, int64_t K, int64_t N, int n_grid, const float* S, const float* losses,
                           int* best, int32_t* codes, __half* steps, __half* zeros, float* out_scales,
-                          cudaStream_t s) {
+                          cudaStream_t s, int quantizer) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -435,7 +437,7 @@ cudaError_t launch_pack_t(const T* W, int64_t K, int64_t N, int n_grid, const fl
   const int64_t per_sm = Tile<G>::kBlocksPerSm;  // resident CTAs per SM at <= 64 registers
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, per_sm * sms));
   pack_kernel<T, G><<<grid, Tile<G>::kThreads, 0, s>>>(W, K, N, n_grid, S, losses, best, codes, steps, zeros,
-                                                       out_scales);
+                                                       out_scales, quantizer);
   return cudaGetLastError();
 }
 
@@ -443,46 +445,46 @@ cudaError_t launch_pack_t(const T* W, int64_t K, int64_t N, int n_grid, const fl
 
 cudaError_t launch_qdq_groups(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid,
                               const float* S, __nv_bfloat16* Wt, int* err, int64_t group0, int64_t groups,
-                              cudaStream_t s, int* launches) {
+                              cudaStream_t s, int* launches, int quantizer) {
   *launches += 1;
   if (in_dtype == 0) {
     const auto* w = static_cast<const __nv_bfloat16*>(W);
     switch (group) {
-      case 32: return launch_qdq_t<__nv_bfloat16, 32>(w, K, N, n_grid, S, Wt, err, group0, groups, s);
-      case 64: return launch_qdq_t<__nv_bfloat16, 64>(w, K, N, n_grid, S, Wt, err, group0, groups, s);
-      default: return launch_qdq_t<__nv_bfloat16, 128>(w, K, N, n_grid, S, Wt, err, group0, groups, s);
+      case 32: return launch_qdq_t<__nv_bfloat16, 32>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer);
+      case 64: return launch_qdq_t<__nv_bfloat16, 64>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer);
+      default: return launch_qdq_t<__nv_bfloat16, 128>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer);
     }
   }
   const auto* w = static_cast<const float*>(W);
   switch (group) {
-    case 32: return launch_qdq_t<float, 32>(w, K, N, n_grid, S, Wt, err, group0, groups, s);
-    case 64: return launch_qdq_t<float, 64>(w, K, N, n_grid, S, Wt, err, group0, groups, s);
-    default: return launch_qdq_t<float, 128>(w, K, N, n_grid, S, Wt, err, group0, groups, s);
+    case 32: return launch_qdq_t<float, 32>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer);
+    case 64: return launch_qdq_t<float, 64>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer);
+    default: return launch_qdq_t<float, 128>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer);
   }
 }
 
 cudaError_t launch_qdq(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid, const float* S,
-                       __nv_bfloat16* Wt, int* err, cudaStream_t s, int* launches) {
-  return launch_qdq_groups(W, in_dtype, K, N, group, n_grid, S, Wt, err, 0, K / group, s, launches);
+                       __nv_bfloat16* Wt, int* err, cudaStream_t s, int* launches, int quantizer) {
+  return launch_qdq_groups(W, in_dtype, K, N, group, n_grid, S, Wt, err, 0, K / group, s, launches, quantizer);
 }
 
 cudaError_t launch_pack(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid, const float* S,
                         const float* losses, int* best, int32_t* codes, __half* steps, __half* zeros,
-                        float* out_scales, cudaStream_t s, int* launches) {
+                        float* out_scales, cudaStream_t s, int* launches, int quantizer) {
   *launches += 1;
   if (in_dtype == 0) {
     const auto* w = static_cast<const __nv_bfloat16*>(W);
     switch (group) {
-      case 32: return launch_pack_t<__nv_bfloat16, 32>(w, K, N, n_grid, S, losses, best, codes, steps, zeros, out_scales, s);
-      case 64: return launch_pack_t<__nv_bfloat16, 64>(w, K, N, n_grid, S, losses, best, codes, steps, zeros, out_scales, s);
-      default: return launch_pack_t<__nv_bfloat16, 128>(w, K, N, n_grid, S, losses, best, codes, steps, zeros, out_scales, s);
+      case 32: return launch_pack_t<__nv_bfloat16, 32>(w, K, N, n_grid, S, losses, best, codes, steps, zeros, out_scales, s, quantizer);
+      case 64: return launch_pack_t<__nv_bfloat16, 64>(w, K, N, n_grid, S, losses, best, codes, steps, zeros, out_scales, s, quantizer);
+      default: return launch_pack_t<__nv_bfloat16, 128>(w, K, N, n_grid, S, losses, best, codes, steps, zeros, out_scales, s, quantizer);
     }
   }
   const auto* w = static_cast<const float*>(W);
   switch (group) {
-    case 32: return launch_pack_t<float, 32>(w, K, N, n_grid, S, losses, best, codes, steps, zeros, out_scales, s);
-    case 64: return launch_pack_t<float, 64>(w, K, N, n_grid, S, losses, best, codes, steps, zeros, out_scales, s);
-    default: return launch_pack_t<float, 128>(w, K, N, n_grid, S, losses, best, codes, steps, zeros, out_scales, s);
+    case 32: return launch_pack_t<float, 32>(w, K, N, n_grid, S, losses, best, codes, steps, zeros, out_scales, s, quantizer);
+    case 64: return launch_pack_t<float, 64>(w, K, N, n_grid, S, losses, best, codes, steps, zeros, out_scales, s, quantizer);
+    default: return launch_pack_t<float, 128>(w, K, N, n_grid, S, losses, best, codes, steps, zeros, out_scales, s, quantizer);
   }
 }
 

@@ -93,12 +93,14 @@ def test_clip_search_validation_happens_on_the_host(lib):
     buf = ctypes.create_string_buffer(64)
     p = ctypes.cast(buf, ctypes.c_void_p)
     args = lambda **kw: [kw.get("X", p), p, 0, kw.get("s", p), 16, 128, 64, kw.get("group", 128),
-                         kw.get("n_shrink", 10), kw.get("tokens", 512), p, null, null, p, p, p, null]
+                         kw.get("n_shrink", 10), kw.get("tokens", 512), kw.get("quantizer", 0), p, null, null,
+                         p, p, p, null]
     assert lib.awq_clip_search(*args(X=null)) == 1
     assert lib.awq_clip_search(*args(s=null)) == 1
     assert lib.awq_clip_search(*args(n_shrink=0)) == 1
     assert lib.awq_clip_search(*args(n_shrink=21)) == 1
     assert lib.awq_clip_search(*args(tokens=0)) == 1
     assert lib.awq_clip_search(*args(group=48)) == 1
-    assert b"n_shrink" in lib.awq_last_error_message() or b"max_tokens" in lib.awq_last_error_message() \
-        or b"group" in lib.awq_last_error_message()
+    assert b"group" in lib.awq_last_error_message()
+    assert lib.awq_clip_search(*args(quantizer=2)) == 1
+    assert b"quantizer" in lib.awq_last_error_message()

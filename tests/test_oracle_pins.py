@@ -310,3 +310,21 @@ def test_bits_per_weight_budget():
     # AWQ-P1 §8: group 128 with fp16 step + fp16 zero -> 4.25 bits/weight, ~3.76x vs 16-bit
     assert O.bits_per_weight(4096, 4096, 128) == 4.25
     assert 16 / O.bits_per_weight(4096, 4096, 128) == pytest.approx(3.76, abs=0.005)
+
+
+def test_symmetric_artifact_decodes_to_the_teaching_quantizer():
+    """The teaching quantizer (AWQ-P1 §2) in the unsigned artifact: code = q + 7, zero 7;
+    the page's worked example at S = diag(10, 1) has q = [7, 7], so the codes are 14."""
+    Wp = np.array([[1.0], [1.0]], np.float32)  # 10 * 0.1 and 1 * 1 in one group
+    q, step, zero = O.sym_artifact(Wp, 2)
+    assert q[:, 0].tolist() == [14, 14] and zero.tolist() == [[7.0]]
+    assert step[0, 0] == np.float32(1.0) / np.float32(7.0)
+    rng = np.random.default_rng(31)
+    W = (rng.standard_normal((256, 16)) * 0.02).astype(np.float32)
+    W[:128, 3] = 0.0                                   # an all-zero group: step 1, codes 7
+    q, step, zero = O.sym_artifact(W, 128)
+    assert q.min() >= 0 and q.max() <= 14 and np.all(q[:128, 3] == 7) and step[0, 3] == 1.0
+    rec = O.sym_teaching_qdq(W, 128)[2]
+    dec = O.decode_artifact(O.pack_codes(q), O.fp16_rne(step), zero.astype(np.float16), 128, 16)
+    st = np.repeat(step, 128, axis=0)
+    assert np.all(np.abs(dec - rec) <= 7 * st * 2.0 ** -11 + 1e-30)
