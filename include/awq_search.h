@@ -209,6 +209,25 @@ int awq_clip_profile_last(float* ms, int n);
  * clipping search's products. */
 int awq_fp64_mma_peak(double* tflops, awq_stream_t stream);
 
+/* ---- Module-level objective: an MLP block ------------------------------------------
+ * [AWQ-P1] §4: a candidate may be scored on the output of the whole module. For a
+ * Llama-shaped MLP block with input X (M x K), gate and up projections searched jointly
+ * as W_gu = [W_gate | W_up] (K x 2F, one scale vector) and the down projection W_down
+ * (F x K_out, kept as it is):
+ *   Y_i = h_i W_down,b,  h_i = bf16(fl32(silu(G_i) * U_i)),  [G_i | U_i] = X_b W_hat_i,b
+ *   L_i = ||Y_i - Y_ref||_F^2 / (M K_out),  Y_ref the block with bf16(W_gu)
+ * silu(x) = x / (1 + exp(-x)) in fp32; the GEMMs take bf16 operands and accumulate in
+ * fp32. Steps 1-4 and 6 as awq_search (statistic and scales from X; QDQ, argmin and the
+ * artifact of W_gu: out_codes [K][2F/8], out_steps/out_zeros [K/group][2F]).
+ * Preconditions as awq_search with N = 2F, plus F and K_out multiples of 8; W_down has
+ * the dtype of X and W_gu. Work space from the library's pool: the candidates
+ * ((n_grid + 1) 2F K bf16), the first GEMM's output (M 2F fp32), h (M F bf16), the
+ * transposed down projection and the reference output. Synchronizes `stream`. */
+int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_dtype,
+                   int64_t M, int64_t K, int64_t F, int64_t K_out, int group, int n_grid,
+                   float* out_scales, int32_t* out_codes, void* out_steps, void* out_zeros,
+                   float* out_losses, awq_stream_t stream);
+
 /* ---- W4A16 consumer of the artifact ---------------------------------------------
  * [AWQ-P1] §7: the artifact feeds a W4A16 kernel, checked by decoding it and comparing
  * the kernel's output with a reference; §8: 4-bit weights, 16-bit activations; §6: the

@@ -23,7 +23,7 @@ __all__ = [
     "tile_shape", "workspace_bytes", "release_cached", "profile_enable", "profile_last",
     "last_launch_count", "debug_set_fault", "status_string", "exported_functions",
     "activation_statistic", "candidate_scales", "qdq_candidates", "ClipOutput", "clip_search",
-    "clip_token_count", "clip_profile_last", "fp64_mma_peak", "w4a16_matmul", "w4a16_dequant", "w4a16_profile_last",
+    "clip_token_count", "clip_profile_last", "fp64_mma_peak", "w4a16_matmul", "w4a16_dequant", "w4a16_profile_last", "search_mlp", "QUANTIZERS",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -87,6 +87,7 @@ def library() -> ctypes.CDLL:
     lib.awq_qdq_candidates.argtypes = [vp, i32, i64, i64, i32, i32, vp, vp, vp]
     lib.awq_clip_search.argtypes = [vp, vp, i32, vp, i64, i64, i64, i32, i32, i64, i32, vp, vp, vp, vp, vp, vp, vp]
     lib.awq_search_quant.argtypes = [vp, vp, i32, i64, i64, i64, i32, i32, i32, vp, vp, vp, vp, vp, vp]
+    lib.awq_search_mlp.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp]
     lib.awq_clip_profile_last.argtypes = [ctypes.POINTER(ctypes.c_float), i32]
     lib.awq_clip_profile_last.restype = ctypes.c_int
     lib.awq_fp64_mma_peak.argtypes = [ctypes.POINTER(ctypes.c_double), vp]
@@ -98,7 +99,7 @@ def library() -> ctypes.CDLL:
     lib.awq_clip_token_count.argtypes = [i64, i64]
     lib.awq_clip_token_count.restype = ctypes.c_int64
     for name in ("awq_activation_statistic", "awq_candidate_scales", "awq_qdq_candidates", "awq_clip_search",
-                 "awq_search_quant",
+                 "awq_search_quant", "awq_search_mlp",
                  "awq_w4a16_matmul", "awq_w4a16_dequant"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -413,3 +414,24 @@ def w4a16_dequant(codes: torch.Tensor, steps: torch.Tensor, zeros: torch.Tensor,
 def w4a16_profile_last() -> float:
     """Device time (ms) of the last W4A16 call's kernels when profiling is on, else -1."""
     return float(library().awq_w4a16_profile_last())
+
+
+def search_mlp(X: torch.Tensor, W_gu: torch.Tensor, W_down: torch.Tensor, group: int = 128, n_grid: int = 20, *,
+               stream: torch.cuda.Stream | None = None) -> SearchOutput:
+    """Scale search of the gate and up projections W_gu = [W_gate | W_up] (K, 2F) scored on
+    the MLP block output down(silu(X W_gate) * (X W_up)) with W_down (F, K_out)."""
+    if not (X.is_cuda and W_gu.is_cuda and W_down.is_cuda):
+        raise ValueError("search_mlp() takes CUDA tensors")
+    if not (X.dtype == W_gu.dtype == W_down.dtype):
+        raise TypeError("X, W_gu and W_down must share a dtype")
+    X, W_gu, W_down = X.contiguous(), W_gu.contiguous(), W_down.contiguous()
+    M, K = X.shape
+    N = W_gu.shape[1]
+    F, K_out = W_down.shape
+    if W_gu.shape[0] != K or N != 2 * F:
+        raise ValueError("W_gu must be (K, 2F) and W_down (F, K_out)")
+    scales, codes, steps, zeros, losses = _alloc_outputs(K, N, group, n_grid, X.device)
+    _check(library().awq_search_mlp(_ptr(X), _ptr(W_gu), _ptr(W_down), _dtype_code(X), M, K, F, K_out, group, n_grid,
+                                    _ptr(scales), _ptr(codes), _ptr(steps), _ptr(zeros), _ptr(losses),
+                                    _stream_handle(stream, X.device)))
+    return SearchOutput(scales, codes, steps, zeros, losses)

@@ -832,6 +832,7 @@ int awq_w4a16_matmul(const void* A, const int32_t* codes, const void* steps, con
       ga.fault_mode = 0;
       ga.num_sms = num_sms;
       ga.f16 = 1;
+      ga.slot_base = 0;
       CUtensorMap mapA, mapB;
       const char* why = "";
       if ((e = make_operand_maps(ga, &mapA, &mapB, &why, kTileN)) != cudaSuccess) {
@@ -889,6 +890,169 @@ int awq_w4a16_dequant(const int32_t* codes, const void* steps, const void* zeros
   if (se != cudaSuccess) return cuda_error(se, "stream synchronize");
   g_last_launches = launches;
   return AWQ_OK;
+}
+
+// ---- MLP-block objective --------------------------------------------------------------
+int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_dtype, int64_t M, int64_t K,
+                   int64_t F, int64_t K_out, int group, int n_grid, float* out_scales, int32_t* out_codes,
+                   void* out_steps, void* out_zeros, float* out_losses, awq_stream_t stream) {
+  t_last_error.clear();
+  int st = validate(X, W_gu, in_dtype, M, K, 2 * F, group, n_grid, out_scales, out_codes, out_steps, out_zeros, true);
+  if (st != AWQ_OK) return st;
+  if (!W_down || !aligned16(W_down)) return set_error(AWQ_ERR_INVALID_ARG, "W_down must be a 16-byte aligned pointer");
+  if (F <= 0 || K_out <= 0 || F % 8 || K_out % 8 || K_out >= (int64_t(1) << 31))
+    return set_error(AWQ_ERR_SHAPE, "F and K_out must be positive multiples of 8");
+  if (out_losses && (reinterpret_cast<uintptr_t>(out_losses) & 3u))
+    return set_error(AWQ_ERR_INVALID_ARG, "out_losses misaligned");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  bind_device(s, X);
+  int dev = 0, num_sms = 0;
+  if ((st = check_device(&dev, &num_sms)) != AWQ_OK) return st;
+  if (!is_device_memory(X) || !is_device_memory(W_gu) || !is_device_memory(W_down) || !is_device_memory(out_scales) ||
+      !is_device_memory(out_codes) || !is_device_memory(out_steps) || !is_device_memory(out_zeros) ||
+      (out_losses && !is_device_memory(out_losses)))
+    return set_error(AWQ_ERR_INVALID_ARG, "inputs and outputs must be device memory");
+  const int64_t N = 2 * F;
+  const int64_t tiles2 = ceil_div(M, kTileM) * ceil_div(K_out, kTileN);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += align_up(bytes);
+    return at;
+  };
+  const size_t o_err = take(16), o_a = take(static_cast<size_t>(K) * 4), o_S = take(static_cast<size_t>(n_grid) * K * 4),
+               o_best = take(16), o_losses = take(static_cast<size_t>(n_grid) * 4),
+               o_Xb = in_dtype == AWQ_DTYPE_F32 ? take(static_cast<size_t>(M) * K * 2) : 0,
+               o_Wt = take(static_cast<size_t>(n_grid + 1) * N * K * 2), o_H = take(static_cast<size_t>(M) * N * 4),
+               o_h = take(static_cast<size_t>(M) * F * 2), o_WdT = take(static_cast<size_t>(K_out) * F * 2),
+               o_Y = take(static_cast<size_t>(tiles2) * kTileM * kTileN * 4),
+               o_part = take(static_cast<size_t>(n_grid) * tiles2 * 8);
+  cudaMemPool_t pool;
+  if ((st = get_pool(dev, &pool)) != AWQ_OK) return st;
+  void* ws = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, off, pool, s);
+  if (e != cudaSuccess || !ws) {
+    cudaGetLastError();
+    return set_error(AWQ_ERR_OOM, "work space of " + std::to_string(off) + " bytes");
+  }
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  int* err = reinterpret_cast<int*>(b + o_err);
+  float* a = reinterpret_cast<float*>(b + o_a);
+  float* S = reinterpret_cast<float*>(b + o_S);
+  int* best = reinterpret_cast<int*>(b + o_best);
+  float* losses = reinterpret_cast<float*>(b + o_losses);
+  __nv_bfloat16* Wt = reinterpret_cast<__nv_bfloat16*>(b + o_Wt);
+  float* H = reinterpret_cast<float*>(b + o_H);
+  __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(b + o_h);
+  __nv_bfloat16* WdT = reinterpret_cast<__nv_bfloat16*>(b + o_WdT);
+  float* Y = reinterpret_cast<float*>(b + o_Y);
+  double* part = reinterpret_cast<double*>(b + o_part);
+  const __nv_bfloat16* Xb = in_dtype == AWQ_DTYPE_F32 ? reinterpret_cast<__nv_bfloat16*>(b + o_Xb)
+                                                      : static_cast<const __nv_bfloat16*>(X);
+  int launches = 0, h_err = 0, status = AWQ_OK;
+  const char* where = "";
+  do {
+    if ((e = cudaMemsetAsync(err, 0, 16, s)) != cudaSuccess) { where = "cudaMemsetAsync"; break; }
+    if ((e = launch_statistic(X, in_dtype, M, K, 1, nullptr, a, err, s, &launches)) != cudaSuccess) {
+      where = "statistic kernel";
+      break;
+    }
+    if ((e = launch_scales(a, K, n_grid, S, s, &launches)) != cudaSuccess) { where = "scales kernel"; break; }
+    if (in_dtype == AWQ_DTYPE_F32 &&
+        (e = launch_to_bf16(static_cast<const float*>(X), M * K, const_cast<__nv_bfloat16*>(Xb), s, &launches)) !=
+            cudaSuccess) {
+      where = "bf16 operand kernel";
+      break;
+    }
+    if ((e = launch_qdq(W_gu, in_dtype, K, N, group, n_grid, S, Wt, err, s, &launches)) != cudaSuccess) {
+      where = "qdq kernel";
+      break;
+    }
+    if ((e = launch_transpose_bf16(W_down, in_dtype, F, K_out, WdT, s, &launches)) != cudaSuccess) {
+      where = "down-projection transpose";
+      break;
+    }
+    // GEMM 1: H = X_b [W_gate | W_up]_slot, row-major fp32 (mode 2)
+    LossGemmArgs g1;
+    g1.Xb = Xb;
+    g1.Wt = Wt;
+    g1.M = M;
+    g1.K = K;
+    g1.N = N;
+    g1.n_grid = n_grid;
+    g1.Y = H;
+    g1.partial = nullptr;
+    g1.err = err;
+    g1.timeout_ns = g_timeout_ns;
+    g1.fault_mode = 0;
+    g1.num_sms = num_sms;
+    // GEMM 2: h W_down^T; mode 0 writes the reference block output (tiled), mode 1 the
+    // per-tile squared error of one candidate against it
+    LossGemmArgs g2 = g1;
+    g2.Xb = h;
+    g2.Wt = WdT;
+    g2.K = F;
+    g2.N = K_out;
+    g2.n_grid = 0;  // one operand slot for the tensor map
+    g2.Y = Y;
+    g2.slot_base = 0;
+    CUtensorMap a1, b1, a2, b2;
+    const char* why = "";
+    if ((e = make_operand_maps(g1, &a1, &b1, &why, kTileN)) != cudaSuccess ||
+        (e = make_operand_maps(g2, &a2, &b2, &why, kTileN)) != cudaSuccess) {
+      status = set_error(AWQ_ERR_CUDA, std::string("TMA descriptor: ") + why);
+      break;
+    }
+    g2.n_grid = 1;  // one candidate per launch
+    for (int c = -1; c < n_grid && e == cudaSuccess; ++c) {
+      g1.slot_base = c + 1;  // slot 0: bf16(W), the reference block
+      if ((e = launch_loss_gemm(g1, a1, b1, 2, s, &launches)) != cudaSuccess) { where = "block GEMM 1"; break; }
+      if ((e = launch_silu_mul(H, M, F, h, s, &launches)) != cudaSuccess) { where = "silu-mul kernel"; break; }
+      g2.partial = part + static_cast<int64_t>(c < 0 ? 0 : c) * tiles2;
+      if ((e = launch_loss_gemm(g2, a2, b2, c < 0 ? 0 : 1, s, &launches)) != cudaSuccess) {
+        where = "block GEMM 2";
+        break;
+      }
+    }
+    if (e != cudaSuccess) break;
+    if ((e = launch_loss_reduce(part, tiles2, n_grid, M, K_out, losses, s, &launches)) != cudaSuccess) {
+      where = "loss reduction kernel";
+      break;
+    }
+    if ((e = launch_pack(W_gu, in_dtype, K, N, group, n_grid, S, losses, best, out_codes,
+                         static_cast<__half*>(out_steps), static_cast<__half*>(out_zeros), out_scales, s,
+                         &launches)) != cudaSuccess) {
+      where = "pack kernel";
+      break;
+    }
+    if (out_losses &&
+        (e = cudaMemcpyAsync(out_losses, losses, static_cast<size_t>(n_grid) * 4, cudaMemcpyDeviceToDevice, s)) !=
+            cudaSuccess) {
+      where = "copy of the losses";
+      break;
+    }
+  } while (false);
+  int* pinned = pinned_status_word(dev);
+  int* status_dst = pinned ? pinned : &h_err;
+  if (status == AWQ_OK && e == cudaSuccess) {
+    e = cudaMemcpyAsync(status_dst, err, sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) where = "status read-back";
+  }
+  if (status == AWQ_OK && e != cudaSuccess) status = cuda_error(e, where);
+  cudaFreeAsync(ws, s);
+  cudaError_t se = cudaStreamSynchronize(s);
+  if (status == AWQ_OK && se != cudaSuccess) status = cuda_error(se, "stream synchronize");
+  if (pinned) h_err = *pinned;
+  if (status == AWQ_OK) {
+    g_last_launches = launches;
+    if (h_err & kErrTimeout)
+      status = set_error(AWQ_ERR_TIMEOUT, "a bounded wait in a block GEMM ran out");
+    else if (h_err & (kErrNonfiniteX | kErrNonfiniteW))
+      status = set_error(AWQ_ERR_NONFINITE, (h_err & kErrNonfiniteX) ? "non-finite value in X" : "non-finite value in W");
+    else if (h_err)
+      status = set_error(AWQ_ERR_CUDA, "device status word " + std::to_string(h_err));
+  }
+  return status;
 }
 
 int awq_clip_profile_last(float* ms, int n) {

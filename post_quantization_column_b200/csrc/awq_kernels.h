@@ -60,6 +60,8 @@ struct LossGemmArgs {
   int fault_mode;
   int num_sms;
   int f16 = 0;               // mode 2 only: fp16 operands (the tensor maps move 2-byte elements either way)
+  int slot_base = 1;         // B slot of candidate 0 (mode 1; the search's slot 0 is bf16(W)) or the
+                             // slot multiplied (mode 2); values other than 1 run on the one-SM kernel
 };
 // Which loss GEMM runs: 1 = the one-SM kernel (default), 2 = the two-SM
 // (cta_group::2) kernel, selected with AWQ_GEMM_VARIANT=2 in the environment.
@@ -128,6 +130,13 @@ int64_t gemv_split_floats(int64_t M, int64_t K, int64_t N, int group, int num_sm
 // w16 transposed: Wt[n][k] = fp16((q - z) step), N x K with K contiguous.
 cudaError_t launch_w4a16_dequant(const int32_t* codes, const __half* steps, const __half* zeros, int64_t K, int64_t N,
                                  int group, __half* Wt, cudaStream_t s, int* launches);
+
+// ---- MLP-block objective (AWQ-P1 §4: the candidate scored on the module output) -----
+// h[m][f] = bf16(fl32(silu(H[m][f]) * H[m][F + f])), H = [X W_gate | X W_up] in fp32 (M x 2F).
+cudaError_t launch_silu_mul(const float* H, int64_t M, int64_t F, __nv_bfloat16* h, cudaStream_t s, int* launches);
+// Wt[o][f] = bf16(W[f][o]): the down projection as a K-major operand (in_dtype 0 bf16, 1 fp32).
+cudaError_t launch_transpose_bf16(const void* W, int in_dtype, int64_t rows, int64_t cols, __nv_bfloat16* Wt,
+                                  cudaStream_t s, int* launches);
 
 __host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 

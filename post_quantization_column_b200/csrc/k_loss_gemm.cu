@@ -53,6 +53,7 @@ struct GemmParams {
   int nk;
   int64_t M, N, ldo;  // mode 2: output rows, columns and row pitch
   int f16;            // mode 2: operands are fp16 (else bf16)
+  int slot_base;      // B slot of candidate 0 (mode 1) or the slot multiplied (mode 2)
   float* Y;           // modes 0-1: the tiled reference output; mode 2: the row-major output
   double* partial;
   int* err;
@@ -150,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int64_t u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         int c, mt, nt;
         unit_coords(u, p, c, mt, nt);
-        const int slot = p.mode == 1 ? c + 1 : 0;
+        const int slot = p.mode == 1 ? c + p.slot_base : (p.mode == 2 ? p.slot_base : 0);
         for (int kb = 0; kb < p.nk; ++kb) {
           if (!mbar_wait_bounded(empty + stage, phase ^ 1u, abort_flag, budget)) {
             ok = false;
@@ -657,7 +658,7 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
                              cudaStream_t s, int* launches) {
   const int tiles_m = static_cast<int>(ceil_div(a.M, BM));
   const int tiles_n = static_cast<int>(ceil_div(a.N, BN));
-  if (gemm_variant() == 2 && mode != 2) {
+  if (gemm_variant() == 2 && mode != 2 && a.slot_base == 1) {
     static unsigned long long attr_done = 0;
     cudaError_t e = set_smem_limit_once(loss_gemm_pair_kernel, kPairSmemBytes, &attr_done);
     if (e != cudaSuccess) return e;
@@ -713,6 +714,7 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
   p.N = a.N;
   p.ldo = a.N;
   p.f16 = a.f16;
+  p.slot_base = a.slot_base;
   p.Y = a.Y;
   p.partial = a.partial;
   p.err = a.err;

@@ -116,3 +116,16 @@ def outlier_channels(spec: LayerSpec) -> np.ndarray:
 def as_f32_numpy(t: torch.Tensor) -> np.ndarray:
     """Exact float32 view of a bf16/fp32 host tensor, for the CPU side."""
     return t.detach().to("cpu").float().contiguous().numpy()
+
+
+def generate_down(spec: LayerSpec, K_out: int, w_std: float = 0.015) -> torch.Tensor:
+    """The down projection (F x K_out, F = N / 2) of an MLP block whose [gate | up] weights
+    are `generate(spec)`'s W; its own Philox substream (the fifth of the layer's seed), so X
+    and W are unchanged. Same storage dtype as the layer."""
+    if spec.N % 2:
+        raise ValueError("the [gate | up] layer has an even number of columns")
+    g = _streams(spec.seed, 5)[4]
+    w = g.standard_normal((spec.N // 2, K_out), dtype=np.float32)
+    w *= np.float32(w_std)
+    t = torch.from_numpy(w)
+    return t.to(torch.bfloat16) if spec.dtype == "bf16" else t
