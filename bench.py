@@ -49,6 +49,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clip", action="store_true", help="skip the clipping-search measurement")
     ap.add_argument("--no-w4a16", action="store_true", help="skip the W4A16 consumer measurement")
+    ap.add_argument("--no-mlp-block", action="store_true", help="skip the MLP-block objective measurement")
     return ap.parse_args(argv)
 
 
@@ -251,6 +252,44 @@ def measure_w4a16(awq, spec: LayerSpec, X, out, stream, flush, steps: int, peaks
     return res
 
 
+MLP_BLOCK = "llama7b_mlp_gate_up_4096x4096x22016"  # [gate | up] of the block; the down projection 11008 x 4096
+
+
+def measure_mlp_block(awq, stream, flush, steps: int, peaks, k_out: int = 4096):
+    """The module-level objective on a Llama-7B MLP block: the gate and up projections
+    searched on down(silu(gate) * up). Device time of the whole call (CUDA events);
+    the work is every candidate's two GEMMs plus the reference block's."""
+    from workloads import generate_down
+    spec = WORKLOADS[MLP_BLOCK]
+    X, W_gu = generate(spec)
+    W_down = generate_down(spec, k_out)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    Xd, Wg, Wd = X.to(dev), W_gu.to(dev), W_down.to(dev)
+    for _ in range(2):
+        out = awq.search_mlp(Xd, Wg, Wd, spec.group, spec.n_grid, stream=stream)
+    s_ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        s_ev[i].record(stream)
+        out = awq.search_mlp(Xd, Wg, Wd, spec.group, spec.n_grid, stream=stream)
+        e_ev[i].record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.mean(s.elapsed_time(e) for s, e in zip(s_ev, e_ev))
+    F = spec.N // 2
+    flops = (spec.n_grid + 1) * (2.0 * spec.M * spec.K * spec.N + 2.0 * spec.M * F * k_out)
+    achieved = flops / (ms / 1e3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    del Xd, Wg, Wd
+    return {"workload": f"{MLP_BLOCK} + down {F}x{k_out}", "ms_per_search": ms, "steps": steps,
+            "gpu_launches_per_search": awq.last_launch_count(), "chosen_alpha_index": out.best,
+            "TFLOP/s": achieved,
+            "roofline": {"bound": "tensor", "kernel": "loss_gemm_kernel modes 2 and 1 (+ silu-mul, QDQ, pack)",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_source": "measured bf16_tflops (burst)",
+                         "work": "(n_grid + 1) x (2 M K 2F + 2 M F K_out) flops over the whole call"}}
+
+
 def cpu_clip_sample(spec: LayerSpec, target_s: float, n_shrink: int = 10):
     """The clipping oracle as it stands on a column slice (full X, same scales reading)."""
     import oracle as O
@@ -415,6 +454,7 @@ def run_ours(args, rank, world, local):
                                                       max(3, min(args.steps, 10)))
         w4a16 = None if args.no_w4a16 else measure_w4a16(awq, spec, X, out, stream, flush,
                                                          max(5, min(args.steps, 20)), measured_peaks()[0])
+        mlp = None if args.no_mlp_block else measure_mlp_block(awq, stream, flush, 3, measured_peaks()[0])
 
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
 
@@ -466,6 +506,8 @@ def run_ours(args, rank, world, local):
         line["clip_search"] = clip
     if w4a16 is not None:
         line["w4a16"] = w4a16
+    if mlp is not None:
+        line["mlp_block"] = mlp
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(spec, args.cpu_seconds)
         if clip is not None:
