@@ -249,6 +249,18 @@ int awq_w4a16_matmul(const void* A, const int32_t* codes, const void* steps,
 /* With profiling on (awq_profile_enable): device time (ms) of the last call's kernels,
  * waiting for them if needed; -1 when the last call was not profiled. */
 float awq_w4a16_profile_last(void);
+/* Decode on repacked codes. awq_w4a16_repack rewrites the artifact's codes (K x N/8
+ * int32; K % 32 == 0, N % 64 == 0) once, e.g. at load time, into the order the decode
+ * kernel reads them: for every 16 rows, 64 columns and MMA lane, 16 contiguous bytes,
+ * nibbles arranged so that one shift and one mask give an fp16 pair. Same size as the
+ * codes; synchronizes `stream`. awq_w4a16_matmul_packed is awq_w4a16_matmul for M <= 16
+ * on that layout (same result definition, steps and zeros unchanged), asynchronous on
+ * `stream`. */
+int awq_w4a16_repack(const int32_t* codes, int64_t K, int64_t N, int32_t* out_packed,
+                     awq_stream_t stream);
+int awq_w4a16_matmul_packed(const void* A, const int32_t* packed, const void* steps,
+                            const void* zeros, int64_t M, int64_t K, int64_t N, int group,
+                            float* Y, awq_stream_t stream);
 /* The dequantized operand alone: out_wt [N][K] fp16 (K contiguous) = w16 transposed. */
 int awq_w4a16_dequant(const int32_t* codes, const void* steps, const void* zeros,
                       int64_t K, int64_t N, int group, void* out_wt, awq_stream_t stream);

@@ -23,7 +23,7 @@ __all__ = [
     "tile_shape", "workspace_bytes", "release_cached", "profile_enable", "profile_last",
     "last_launch_count", "debug_set_fault", "status_string", "exported_functions",
     "activation_statistic", "candidate_scales", "qdq_candidates", "ClipOutput", "clip_search",
-    "clip_token_count", "clip_profile_last", "fp64_mma_peak", "w4a16_matmul", "w4a16_dequant", "w4a16_profile_last", "search_mlp", "QUANTIZERS",
+    "clip_token_count", "clip_profile_last", "fp64_mma_peak", "w4a16_matmul", "w4a16_dequant", "w4a16_profile_last", "search_mlp", "QUANTIZERS", "w4a16_repack", "w4a16_matmul_packed",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -94,13 +94,15 @@ def library() -> ctypes.CDLL:
     lib.awq_fp64_mma_peak.restype = ctypes.c_int
     lib.awq_w4a16_matmul.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, vp, vp]
     lib.awq_w4a16_dequant.argtypes = [vp, vp, vp, i64, i64, i32, vp, vp]
+    lib.awq_w4a16_repack.argtypes = [vp, i64, i64, vp, vp]
+    lib.awq_w4a16_matmul_packed.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, vp, vp]
     lib.awq_w4a16_profile_last.argtypes = []
     lib.awq_w4a16_profile_last.restype = ctypes.c_float
     lib.awq_clip_token_count.argtypes = [i64, i64]
     lib.awq_clip_token_count.restype = ctypes.c_int64
     for name in ("awq_activation_statistic", "awq_candidate_scales", "awq_qdq_candidates", "awq_clip_search",
                  "awq_search_quant", "awq_search_mlp",
-                 "awq_w4a16_matmul", "awq_w4a16_dequant"):
+                 "awq_w4a16_matmul", "awq_w4a16_dequant", "awq_w4a16_repack", "awq_w4a16_matmul_packed"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -435,3 +437,27 @@ def search_mlp(X: torch.Tensor, W_gu: torch.Tensor, W_down: torch.Tensor, group:
                                     _ptr(scales), _ptr(codes), _ptr(steps), _ptr(zeros), _ptr(losses),
                                     _stream_handle(stream, X.device)))
     return SearchOutput(scales, codes, steps, zeros, losses)
+
+
+def w4a16_repack(codes: torch.Tensor, *, stream=None) -> torch.Tensor:
+    """The artifact's codes (K, N/8) int32 rewritten in the decode kernel's order (same size)."""
+    if not codes.is_cuda or codes.dtype != torch.int32 or codes.dim() != 2:
+        raise ValueError("codes must be a (K, N/8) int32 CUDA tensor")
+    codes = codes.contiguous()
+    K, N = codes.shape[0], codes.shape[1] * 8
+    out = torch.empty_like(codes)
+    _check(library().awq_w4a16_repack(_ptr(codes), K, N, _ptr(out), _stream_handle(stream, codes.device)))
+    return out
+
+
+def w4a16_matmul_packed(A: torch.Tensor, packed: torch.Tensor, steps: torch.Tensor, zeros: torch.Tensor,
+                        group: int = 128, *, stream=None) -> torch.Tensor:
+    """w4a16_matmul for at most 16 tokens on repacked codes (asynchronous on `stream`)."""
+    packed, steps, zeros, K, N = _artifact_args(packed, steps, zeros, group)
+    if A.dtype != torch.float16 or not A.is_cuda or A.dim() != 2 or A.shape[1] != K:
+        raise ValueError("A must be a (M, K) float16 CUDA tensor")
+    A = A.contiguous()
+    Y = torch.empty(A.shape[0], N, dtype=torch.float32, device=A.device)
+    _check(library().awq_w4a16_matmul_packed(_ptr(A), _ptr(packed), _ptr(steps), _ptr(zeros), A.shape[0], K, N,
+                                             group, _ptr(Y), _stream_handle(stream, A.device)))
+    return Y

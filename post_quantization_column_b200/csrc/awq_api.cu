@@ -859,6 +859,74 @@ int awq_w4a16_matmul(const void* A, const int32_t* codes, const void* steps, con
   return status;
 }
 
+int awq_w4a16_repack(const int32_t* codes, int64_t K, int64_t N, int32_t* out_packed, awq_stream_t stream) {
+  t_last_error.clear();
+  if (!codes || !out_packed) return set_error(AWQ_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (K <= 0 || N <= 0 || K % 32 || N % 64 || K >= (int64_t(1) << 31) || N >= (int64_t(1) << 31))
+    return set_error(AWQ_ERR_SHAPE, "K must be a positive multiple of 32 and N of 64");
+  if (!aligned16(codes) || !aligned16(out_packed))
+    return set_error(AWQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  bind_device(s, codes);
+  int dev = 0, num_sms = 0, st;
+  if ((st = check_device(&dev, &num_sms)) != AWQ_OK) return st;
+  if (!is_device_memory(codes) || !is_device_memory(out_packed))
+    return set_error(AWQ_ERR_INVALID_ARG, "codes and out_packed must be device memory");
+  int launches = 0;
+  cudaError_t e = launch_w4a16_repack(codes, K, N, reinterpret_cast<uint32_t*>(out_packed), s, &launches);
+  cudaError_t se = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_error(e, "repack");
+  if (se != cudaSuccess) return cuda_error(se, "stream synchronize");
+  g_last_launches = launches;
+  return AWQ_OK;
+}
+
+int awq_w4a16_matmul_packed(const void* A, const int32_t* packed, const void* steps, const void* zeros, int64_t M,
+                            int64_t K, int64_t N, int group, float* Y, awq_stream_t stream) {
+  t_last_error.clear();
+  int st = validate_w4a16(A, packed, steps, zeros, M, K, N, group, Y);
+  if (st != AWQ_OK) return st;
+  if (M > kW4A16GemvMaxM) return set_error(AWQ_ERR_SHAPE, "the repacked layout serves at most 16 tokens");
+  if (N % 64) return set_error(AWQ_ERR_SHAPE, "the repacked layout needs N % 64 == 0");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  bind_device(s, packed);
+  int dev = 0, num_sms = 0;
+  if ((st = check_device(&dev, &num_sms)) != AWQ_OK) return st;
+  if (!is_device_memory(A) || !is_device_memory(packed) || !is_device_memory(steps) || !is_device_memory(zeros) ||
+      !is_device_memory(Y))
+    return set_error(AWQ_ERR_INVALID_ARG, "inputs and outputs must be device memory");
+  cudaMemPool_t pool;
+  if ((st = get_pool(dev, &pool)) != AWQ_OK) return st;
+  const size_t ws_bytes = 256 + align_up(static_cast<size_t>(gemv_split_floats(M, K, N, group, num_sms, true)) * 4);
+  void* ws = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, ws_bytes, pool, s);
+  if (e != cudaSuccess || !ws) {
+    cudaGetLastError();
+    return set_error(AWQ_ERR_OOM, "W4A16 work space");
+  }
+  W4A16Args a;
+  a.A = static_cast<const __half*>(A);
+  a.codes = packed;
+  a.steps = static_cast<const __half*>(steps);
+  a.zeros = static_cast<const __half*>(zeros);
+  a.M = M;
+  a.K = K;
+  a.N = N;
+  a.group = group;
+  a.Y = Y;
+  int launches = 0;
+  cudaEvent_t* ev = g_profile ? w4a16_events(dev) : nullptr;
+  if (ev) cudaEventRecord(ev[0], s);
+  e = launch_w4a16_gemv_packed(a, reinterpret_cast<const uint32_t*>(packed), num_sms,
+                               reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + 256), s, &launches);
+  if (ev) cudaEventRecord(ev[1], s);
+  g_w4a16_profiled = ev != nullptr;
+  cudaFreeAsync(ws, s);
+  if (e != cudaSuccess) return cuda_error(e, "W4A16 GEMV (repacked)");
+  g_last_launches = launches;
+  return AWQ_OK;
+}
+
 float awq_w4a16_profile_last(void) {
   if (!g_w4a16_profiled || !g_w4a16_last_ev) return -1.0f;
   float ms = -1.0f;

@@ -126,7 +126,13 @@ constexpr int kW4A16GemvMaxM = 16;
 // Fused dequantization + GEMV for M <= kW4A16GemvMaxM; `part` holds
 // gemv_split_floats(...) floats when that is non-zero (a second launch sums the splits).
 cudaError_t launch_w4a16_gemv(const W4A16Args& a, int num_sms, float* part, cudaStream_t s, int* launches);
-int64_t gemv_split_floats(int64_t M, int64_t K, int64_t N, int group, int num_sms);
+int64_t gemv_split_floats(int64_t M, int64_t K, int64_t N, int group, int num_sms, bool packed = false);
+// The codes in the decode kernel's order (N % 64 == 0): same size as the codes.
+cudaError_t launch_w4a16_repack(const int32_t* codes, int64_t K, int64_t N, uint32_t* packed, cudaStream_t s,
+                                int* launches);
+// The decode GEMV on repacked codes (M <= kW4A16GemvMaxM, N % 64 == 0); `part` as above.
+cudaError_t launch_w4a16_gemv_packed(const W4A16Args& a, const uint32_t* packed, int num_sms, float* part,
+                                     cudaStream_t s, int* launches);
 // w16 transposed: Wt[n][k] = fp16((q - z) step), N x K with K contiguous.
 cudaError_t launch_w4a16_dequant(const int32_t* codes, const __half* steps, const __half* zeros, int64_t K, int64_t N,
                                  int group, __half* Wt, cudaStream_t s, int* launches);

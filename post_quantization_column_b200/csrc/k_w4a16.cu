@@ -287,6 +287,201 @@ __global__ void __launch_bounds__(kDqThreads)
   }
 }
 
+// ---- the consumer's repacked layout ---------------------------------------------------
+// For decode the codes are read in the order the MMA fragments use them: for every
+// 16-row step s, 64-column block cb and lane (g, t), 16 bytes (4 words) hold the lane's
+// 32 nibbles. Word u serves column tiles j = 2u and 2u + 1; its nibble p (0..3) and
+// p + 4 are the pair (rows r, r + 1) of fragment p: tile 2u + (p >> 1), rows 2t (p even)
+// or 2t + 8 (p odd), column 8 j + g. So (word >> 4p) & 0x000F000F puts the pair in the two
+// halves, one shift and one logic op per two weights, and a warp reads 512 contiguous
+// bytes per step.
+__global__ void repack_kernel(const int32_t* __restrict__ codes, int64_t K, int64_t N, uint32_t* __restrict__ P) {
+  const int64_t words = N / 8, cbs = N / 64;
+  const int64_t total = (K / 16) * cbs * 32 * 4;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int u = static_cast<int>(i % 4);
+    const int lane = static_cast<int>((i / 4) % 32);
+    const int64_t cb = (i / 128) % cbs, s = i / (128 * cbs);
+    const int g = lane >> 2, t = lane & 3;
+    uint32_t out = 0;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const int j = 2 * u + (p >> 1);
+      const int64_t row = 16 * s + ((p & 1) ? 2 * t + 8 : 2 * t);
+      const int64_t w = cb * 8 + j;
+      const uint32_t lo = (static_cast<uint32_t>(__ldg(codes + row * words + w)) >> (4 * g)) & 0xFu;
+      const uint32_t hi = (static_cast<uint32_t>(__ldg(codes + (row + 1) * words + w)) >> (4 * g)) & 0xFu;
+      out |= (lo << (4 * p)) | (hi << (4 * (p + 4)));
+    }
+    P[i] = out;
+  }
+}
+
+// The decode GEMV on the repacked codes: as gemv_kernel, but a step is one 16-byte copy per
+// lane into a per-warp ring of kPRing stages in shared memory (cp.async, kPRing - 1 steps
+// ahead, so about 8 KB per warp are in flight), the group's steps and zeros travel in the
+// same ring (16 lanes copy the 64 columns' 128 + 128 bytes with the group's first step),
+// and each fp16 pair costs one shift and one logic op before the packed (1024 + q) -
+// (1024 + z) and the multiply by the step.
+constexpr int kPRing = 16;                          // steps in flight per warp (a power of two)
+constexpr int kPActBytes = 16 * 1024;               // activations staged per CTA when they fit (2 CTAs per SM)
+constexpr int kPRingBytes = kPRing * 32 * 16;       // 8 KB of codes per warp
+// Parameter buffers per warp: a group's steps and zeros are copied with its first step,
+// up to kPRing - 1 steps before that step is computed, and must outlive the whole group,
+// so PB * S > kPRing + S - 2 for S = G / 16 steps per group: 16, 8 and 4 for G = 32, 64, 128.
+template <int G>
+struct PackedSmem {
+  static constexpr int S = G / 16;
+  static constexpr int PB = G == 32 ? 16 : (G == 64 ? 8 : 4);
+  static_assert(PB * S > kPRing + S - 2, "parameter buffers must outlive their group");
+  static constexpr int kParamBytes = PB * 2 * 64 * 2;  // PB groups of 64 steps + 64 zeros (fp16)
+  static constexpr int kWarpBytes = kPRingBytes + kParamBytes;
+  static constexpr int kSmem = (kGemvThreads / 32) * kWarpBytes;
+};
+
+template <int G>
+__global__ void __launch_bounds__(kGemvThreads)
+    gemv_packed_kernel(const __half* __restrict__ A, int M, const uint4* __restrict__ P,
+                       const __half* __restrict__ steps, const __half* __restrict__ zeros, int64_t K, int64_t N,
+                       int64_t k_per_split, float* __restrict__ out) {
+  __shared__ float red[kGemvThreads / 32][16][kGemvCols];
+  extern __shared__ __align__(16) uint8_t pdyn[];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int64_t cbs = N / 64, cb = blockIdx.x;
+  const int64_t k0 = static_cast<int64_t>(blockIdx.y) * k_per_split;
+  const int64_t k1 = min(K, k0 + k_per_split);
+  // warps take whole groups of the split (contiguous runs), so parameters change only
+  // between the unrolled steps of one group
+  constexpr int kStepsPerGroup = G / 16;
+  const int n_groups = static_cast<int>((k1 - k0) / G);
+  const int gpw = (n_groups + kGemvThreads / 32 - 1) / (kGemvThreads / 32);
+  const int g_begin = min(n_groups, warp * gpw), g_end = min(n_groups, g_begin + gpw);
+  const int s0 = g_begin * kStepsPerGroup, s1 = g_end * kStepsPerGroup;
+  using PS = PackedSmem<G>;
+  uint8_t* ring = pdyn + warp * PS::kWarpBytes;
+  // the CTA's slice of the activations, staged once when it fits (M k_per_split halves)
+  __half* sAct = reinterpret_cast<__half*>(pdyn + PS::kSmem);
+  const bool staged = static_cast<int64_t>(M) * k_per_split * 2 <= kPActBytes;
+  if (staged) {
+    const int kn = static_cast<int>(k1 - k0);
+    for (int i = threadIdx.x; i < M * (kn / 8); i += kGemvThreads) {
+      const int m = i / (kn / 8), v = i % (kn / 8);
+      *reinterpret_cast<uint4*>(sAct + m * k_per_split + 8 * v) =
+          __ldg(reinterpret_cast<const uint4*>(A + static_cast<int64_t>(m) * K + k0 + 8 * v));
+    }
+    __syncthreads();
+  }
+  __half* params = reinterpret_cast<__half*>(ring + kPRingBytes);  // [PB][2][64]
+
+  float acc[8][4];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
+
+  auto issue = [&](int s) {
+    if (s < s1) {
+      const int64_t gs = k0 / 16 + s;  // global step
+      const uint32_t dst = smem_u32(ring + (s & (kPRing - 1)) * 512 + lane * 16);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(P + (gs * cbs + cb) * 32 + lane)
+                   : "memory");
+      if (gs % kStepsPerGroup == 0 && lane < 16) {  // runs start on group boundaries
+        const int64_t grp = (gs * 16) / G;
+        const __half* src = (lane < 8 ? steps : zeros) + grp * N + cb * 64 + 8 * (lane & 7);
+        const uint32_t pd = smem_u32(params + (grp & (PS::PB - 1)) * 128 + (lane < 8 ? 0 : 64) + 8 * (lane & 7));
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(pd), "l"(src) : "memory");
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+#pragma unroll 1
+  for (int q = 0; q < kPRing - 1; ++q) issue(s0 + q);
+
+  __half2 z2[8], st2[8];
+  const __half k1024 = __float2half_rn(1024.0f);
+  const __half* sArow0 = sAct + gq * k_per_split + 2 * tq;      // staged activations of token g
+  const __half* sArow1 = sArow0 + 8 * k_per_split;              // and of token g + 8
+#pragma unroll 1
+  for (int gi = g_begin; gi < g_end; ++gi) {
+    const int64_t grp = k0 / G + gi;
+#pragma unroll
+    for (int ss = 0; ss < kStepsPerGroup; ++ss) {
+      const int s = gi * kStepsPerGroup + ss;
+      issue(s + kPRing - 1);
+      asm volatile("cp.async.wait_group %0;" ::"n"(kPRing - 1) : "memory");
+      __syncwarp();  // the group's steps and zeros were copied by other lanes
+      if (ss == 0) {
+        const __half* pr = params + (grp & (PS::PB - 1)) * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const __half st = pr[8 * j + gq];
+          const __half zb = __hadd(pr[64 + 8 * j + gq], k1024);  // exact: z is an integer <= 15
+          st2[j] = __halves2half2(st, st);
+          z2[j] = __halves2half2(zb, zb);
+        }
+      }
+      const uint4 v = *reinterpret_cast<const uint4*>(ring + (s & (kPRing - 1)) * 512 + lane * 16);
+      const int kk = 16 * s;  // row offset inside the split
+      uint32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0;
+      if (staged) {
+        if (gq < M) {
+          a0 = *reinterpret_cast<const uint32_t*>(sArow0 + kk);
+          a2 = *reinterpret_cast<const uint32_t*>(sArow0 + kk + 8);
+        }
+        if (gq + 8 < M) {
+          a1 = *reinterpret_cast<const uint32_t*>(sArow1 + kk);
+          a3 = *reinterpret_cast<const uint32_t*>(sArow1 + kk + 8);
+        }
+      } else {
+        const int64_t kb = k0 + kk;
+        if (gq < M) {
+          const __half* ar = A + static_cast<int64_t>(gq) * K + kb + 2 * tq;
+          a0 = __ldg(reinterpret_cast<const uint32_t*>(ar));
+          a2 = __ldg(reinterpret_cast<const uint32_t*>(ar + 8));
+        }
+        if (gq + 8 < M) {
+          const __half* ar = A + static_cast<int64_t>(gq + 8) * K + kb + 2 * tq;
+          a1 = __ldg(reinterpret_cast<const uint32_t*>(ar));
+          a3 = __ldg(reinterpret_cast<const uint32_t*>(ar + 8));
+        }
+      }
+      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int j = 2 * u + h;
+          uint32_t b[2];
+#pragma unroll
+          for (int which = 0; which < 2; ++which) {
+            const int p = 2 * h + which;
+            const uint32_t biased = ((wv[u] >> (4 * p)) & 0x000F000Fu) | 0x64006400u;  // halves 1024 + q
+            b[which] = half2_as_u32(__hmul2(__hsub2(u32_as_half2(biased), z2[j]), st2[j]));
+          }
+          mma_f16_16816(acc[j], a0, a1, a2, a3, b[0], b[1]);
+        }
+      }
+    }
+    __syncwarp();  // all lanes are past this group's parameters before a later group overwrites them
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    red[warp][gq][8 * j + 2 * tq] = acc[j][0];
+    red[warp][gq][8 * j + 2 * tq + 1] = acc[j][1];
+    red[warp][gq + 8][8 * j + 2 * tq] = acc[j][2];
+    red[warp][gq + 8][8 * j + 2 * tq + 1] = acc[j][3];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < M * kGemvCols; i += kGemvThreads) {
+    const int m = i / kGemvCols, c = i % kGemvCols;
+    float sum = red[0][m][c];
+#pragma unroll
+    for (int q = 1; q < kGemvThreads / 32; ++q) sum = __fadd_rn(sum, red[q][m][c]);
+    out[(static_cast<int64_t>(blockIdx.y) * M + m) * N + cb * 64 + c] = sum;
+  }
+}
+
 // Splits of whole groups so that the grid fills the SMs a few times over.
 int64_t gemv_splits(int64_t K, int64_t N, int group, int num_sms) {
   const int64_t col_blocks = ceil_div(N, kGemvCols);
@@ -318,10 +513,45 @@ cudaError_t launch_gemv_g(const W4A16Args& a, int num_sms, float* part, cudaStre
   return cudaGetLastError();
 }
 
+// The repacked kernel gives its warps whole groups: a split holds at least 8 groups when
+// the layer has that many.
+int64_t gemv_packed_splits(int64_t K, int64_t N, int group, int num_sms) {
+  const int64_t col_blocks = N / 64;
+  const int64_t groups = K / group;
+  int64_t splits = std::max<int64_t>(1, std::min<int64_t>(groups / 8, ceil_div(8 * num_sms, col_blocks)));
+  const int64_t gps = ceil_div(groups, splits);
+  return ceil_div(groups, gps);
+}
+
+template <int G>
+cudaError_t launch_gemv_packed_g(const W4A16Args& a, const uint32_t* packed, int num_sms, float* part,
+                                 cudaStream_t s, int* launches) {
+  const int64_t col_blocks = a.N / 64;
+  const int64_t splits = gemv_packed_splits(a.K, a.N, G, num_sms);
+  const int64_t k_per_split = ceil_div(a.K / G, splits) * G;
+  float* dst = splits == 1 ? a.Y : part;
+  static unsigned long long done = 0;
+  const int smem = PackedSmem<G>::kSmem +
+                   (a.M * k_per_split * 2 <= kPActBytes ? static_cast<int>(a.M * k_per_split * 2) : 0);
+  cudaError_t e0 = set_smem_limit_once(gemv_packed_kernel<G>, PackedSmem<G>::kSmem + kPActBytes, &done);
+  if (e0 != cudaSuccess) return e0;
+  gemv_packed_kernel<G><<<dim3(static_cast<unsigned>(col_blocks), static_cast<unsigned>(splits)), kGemvThreads,
+                          smem, s>>>(a.A, static_cast<int>(a.M), reinterpret_cast<const uint4*>(packed), a.steps, a.zeros,
+                               a.K, a.N, k_per_split, dst);
+  *launches += 1;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || splits == 1) return e;
+  const int64_t mn = a.M * a.N;
+  const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(ceil_div(mn, 256), 4 * num_sms));
+  split_sum_kernel<<<blocks, 256, 0, s>>>(part, static_cast<int>(splits), mn, a.Y);
+  *launches += 1;
+  return cudaGetLastError();
+}
+
 }  // namespace
 
-int64_t gemv_split_floats(int64_t M, int64_t K, int64_t N, int group, int num_sms) {
-  const int64_t splits = gemv_splits(K, N, group, num_sms);
+int64_t gemv_split_floats(int64_t M, int64_t K, int64_t N, int group, int num_sms, bool packed) {
+  const int64_t splits = packed ? gemv_packed_splits(K, N, group, num_sms) : gemv_splits(K, N, group, num_sms);
   return splits > 1 ? splits * M * N : 0;
 }
 
@@ -342,4 +572,25 @@ cudaError_t launch_w4a16_dequant(const int32_t* codes, const __half* steps, cons
   return cudaGetLastError();
 }
 
+}  // namespace awq
+
+namespace awq {
+cudaError_t launch_w4a16_repack(const int32_t* codes, int64_t K, int64_t N, uint32_t* packed, cudaStream_t s,
+                                int* launches) {
+  const int64_t total = K * N / 8;
+  const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(ceil_div(total, 256), 148 * 16));
+  repack_kernel<<<blocks, 256, 0, s>>>(codes, K, N, packed);
+  *launches += 1;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_w4a16_gemv_packed(const W4A16Args& a, const uint32_t* packed, int num_sms, float* part,
+                                     cudaStream_t s, int* launches) {
+  if (a.M < 1 || a.M > kW4A16GemvMaxM || a.N % 64) return cudaErrorInvalidValue;
+  switch (a.group) {
+    case 32: return launch_gemv_packed_g<32>(a, packed, num_sms, part, s, launches);
+    case 64: return launch_gemv_packed_g<64>(a, packed, num_sms, part, s, launches);
+    default: return launch_gemv_packed_g<128>(a, packed, num_sms, part, s, launches);
+  }
+}
 }  // namespace awq

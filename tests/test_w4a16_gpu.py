@@ -121,3 +121,28 @@ def test_full_size_sampled_columns(name, M):
     st, zr = steps.cpu().numpy(), zeros.cpu().numpy()
     for c0, c1 in [(0, 64), (N // 2 - 32, N // 2 + 32), (N - 72, N)]:
         _check_output(Y[:, c0:c1], A16, codes[:, c0 // 8:c1 // 8], st[:, c0:c1], zr[:, c0:c1], g)
+
+
+@pytest.mark.parametrize("M", [1, 5, 16])
+@pytest.mark.parametrize("K,N,group", [(256, 256, 128), (160, 128, 32), (384, 576, 64)])
+def test_repacked_decode_matches_oracle(M, K, N, group):
+    codes, steps, zeros = _random_artifact(K, N, group, 7 * M + N)
+    c, st, zr = _dev(codes, steps, zeros)
+    packed = awq.w4a16_repack(c)
+    A = (np.random.default_rng(M + 1).standard_normal((M, K)) * 2).astype(np.float16)
+    Y = awq.w4a16_matmul_packed(torch.from_numpy(A).cuda(), packed, st, zr, group).cpu().numpy()
+    _check_output(Y, A, codes, steps, zeros, group)
+
+
+def test_repacked_decode_full_size_70b_columns():
+    spec = WORKLOADS["llama70b_mlp_gate_up_16384x8192x57344"]
+    K, N, g = spec.K, spec.N, spec.group
+    rng = np.random.default_rng(9)
+    q_dev = torch.randint(-2 ** 31, 2 ** 31 - 1, (K, N // 8), dtype=torch.int32, device="cuda")
+    steps = torch.from_numpy((rng.random((K // g, N)) * 0.01 + 1e-4).astype(np.float16)).cuda()
+    zeros = torch.from_numpy(rng.integers(0, 16, size=(K // g, N)).astype(np.float16)).cuda()
+    A16 = rng.standard_normal((3, K)).astype(np.float16)
+    Y = awq.w4a16_matmul_packed(torch.from_numpy(A16).cuda(), awq.w4a16_repack(q_dev), steps, zeros, g).cpu().numpy()
+    codes, st, zr = q_dev.cpu().numpy(), steps.cpu().numpy(), zeros.cpu().numpy()
+    for c0, c1 in [(0, 64), (N // 2 - 64, N // 2 + 64), (N - 128, N)]:
+        _check_output(Y[:, c0:c1], A16, codes[:, c0 // 8:c1 // 8], st[:, c0:c1], zr[:, c0:c1], g)
