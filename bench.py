@@ -212,42 +212,67 @@ def measure_clip(awq, spec: LayerSpec, Xd, Wd, scales, stream, flush, steps: int
     }
 
 
+def _time_w4a16(awq, fn, flush, steps):
+    for _ in range(2):
+        fn()
+    awq.profile_enable(True)
+    ms = []
+    for _ in range(steps):
+        flush.zero_()
+        fn()
+        ms.append(awq.w4a16_profile_last())
+    return statistics.median(ms), awq.last_launch_count()
+
+
 def measure_w4a16(awq, spec: LayerSpec, X, out, stream, flush, steps: int, peaks):
-    """The artifact's W4A16 consumer on the same layer: decode (1 token, fused GEMV; HBM
-    roofline over the 4.25-bit weight stream) and prefill (all M tokens, dequantize +
-    tensor-core GEMM; fp16 tensor roofline)."""
+    """The artifact's W4A16 consumer on the same layer: decode (1 token on the repacked
+    codes, fused GEMV; HBM roofline over the 4.25-bit weight stream), the same on a
+    Llama-70B gate+up-shaped artifact (where the stream, 250 MB, dwarfs launch latency),
+    and prefill (all M tokens, dequantize + tensor-core GEMM; fp16 tensor roofline)."""
     Xd = X.to(out.scales.device).float()
     A = (Xd / out.scales[None, :]).half()  # activations divided by the chosen scales
+    hbm = float(peaks["hbm_gbs"])
+
+    def decode_entry(K, N, group, t, launches, kernel):
+        stream_bytes = K * N / 2 + 4 * (K // group) * N + 2 * K + 4 * N
+        gbs = stream_bytes / (t / 1e3) / 1e9
+        return {"M": 1, "K": K, "N": N, "ms": t, "gpu_launches_per_call": launches, "GB/s": gbs,
+                "roofline": {"bound": "hbm", "kernel": kernel, "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                             "frac": gbs / hbm, "work": "K N / 2 code bytes + 4 bytes per (group, column) + 2 K + 4 N"}}
+
     res = {}
-    for label, M in (("decode", 1), ("prefill", spec.M)):
-        Am = A[:M].contiguous()
-        for _ in range(2):
-            awq.w4a16_matmul(Am, out.codes, out.steps, out.zeros, spec.group, stream=stream)
-        awq.profile_enable(True)
-        ms = []
-        for _ in range(steps):
-            flush.zero_()
-            awq.w4a16_matmul(Am, out.codes, out.steps, out.zeros, spec.group, stream=stream)
-            ms.append(awq.w4a16_profile_last())
-        launches = awq.last_launch_count()
-        t = statistics.median(ms)
-        groups = spec.K // spec.group
-        stream_bytes = spec.K * spec.N / 2 + 4 * groups * spec.N + 2 * M * spec.K + 4 * M * spec.N
-        flops = 2.0 * M * spec.K * spec.N
-        entry = {"M": M, "ms": t, "gpu_launches_per_call": launches, "TFLOP/s": flops / (t / 1e3) / 1e12,
-                 "GB/s": stream_bytes / (t / 1e3) / 1e9}
-        if label == "decode":
-            entry["roofline"] = {"bound": "hbm", "kernel": "gemv_kernel (fused dequantize + fp16 MMA)",
-                                 "achieved": entry["GB/s"], "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
-                                 "frac": entry["GB/s"] / float(peaks["hbm_gbs"]),
-                                 "work": "K N / 2 code bytes + 4 bytes per (group, column) + 2 M K + 4 M N"}
-        else:
-            entry["roofline"] = {"bound": "tensor", "kernel": "dequant_kernel + loss_gemm_kernel mode 2 (fp16)",
-                                 "achieved": entry["TFLOP/s"], "peak": float(peaks["bf16_tflops"]),
-                                 "unit": "TFLOP/s", "frac": entry["TFLOP/s"] / float(peaks["bf16_tflops"]),
-                                 "peak_source": "bf16 dense burst peak (fp16 runs at the same rate)",
-                                 "work": "2 M K N flops (both kernels' time)"}
-        res[label] = entry
+    packed = awq.w4a16_repack(out.codes, stream=stream)  # once, as at load time
+    A1 = A[:1].contiguous()
+    t, n = _time_w4a16(awq, lambda: awq.w4a16_matmul_packed(A1, packed, out.steps, out.zeros, spec.group,
+                                                             stream=stream), flush, steps)
+    res["decode"] = decode_entry(spec.K, spec.N, spec.group, t, n, "gemv_packed_kernel (repacked codes)")
+    t, n = _time_w4a16(awq, lambda: awq.w4a16_matmul(A1, out.codes, out.steps, out.zeros, spec.group,
+                                                      stream=stream), flush, steps)
+    res["decode_plain_layout"] = decode_entry(spec.K, spec.N, spec.group, t, n, "gemv_kernel (artifact layout)")
+    big = WORKLOADS["llama70b_mlp_gate_up_16384x8192x57344"]
+    gen = torch.Generator(device=out.codes.device).manual_seed(0)
+    codes70 = torch.randint(-2 ** 31, 2 ** 31 - 1, (big.K, big.N // 8), dtype=torch.int32, device=out.codes.device,
+                            generator=gen)
+    steps70 = (torch.rand(big.K // big.group, big.N, device=out.codes.device, generator=gen) * 0.01 + 1e-4).half()
+    zeros70 = torch.randint(0, 16, (big.K // big.group, big.N), device=out.codes.device, generator=gen).half()
+    packed70 = awq.w4a16_repack(codes70, stream=stream)
+    A70 = torch.randn(1, big.K, device=out.codes.device, generator=gen).half()
+    t, n = _time_w4a16(awq, lambda: awq.w4a16_matmul_packed(A70, packed70, steps70, zeros70, big.group,
+                                                             stream=stream), flush, steps)
+    res["decode_70b_gate_up_shape"] = decode_entry(big.K, big.N, big.group, t, n,
+                                                   "gemv_packed_kernel (random artifact of the 70B gate+up shape)")
+    del codes70, steps70, zeros70, packed70
+    M = spec.M
+    Am = A[:M].contiguous()
+    t, launches = _time_w4a16(awq, lambda: awq.w4a16_matmul(Am, out.codes, out.steps, out.zeros, spec.group,
+                                                             stream=stream), flush, steps)
+    tflops = 2.0 * M * spec.K * spec.N / (t / 1e3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    res["prefill"] = {"M": M, "ms": t, "gpu_launches_per_call": launches, "TFLOP/s": tflops,
+                      "roofline": {"bound": "tensor", "kernel": "dequant_kernel + loss_gemm_kernel mode 2 (fp16)",
+                                   "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
+                                   "peak_source": "bf16 dense burst peak (fp16 runs at the same rate)",
+                                   "work": "2 M K N flops (both kernels' time)"}}
     awq.profile_enable(True)
     return res
 
