@@ -484,6 +484,8 @@ def run_ours(args, rank, world, local):
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
 
     flops = spec.candidate_flops
+    gemm_kernel = ("loss_gemm_pair_kernel" if awq.loss_gemm_variant(spec.M, spec.K, spec.N, spec.n_grid) == 2
+                   else "loss_gemm_kernel")
     value = weak_scaling_tflops(world, args.steps, flops, total_ms)
     layers_per_s = world * args.steps / (total_ms / 1e3)
     e2e_value = weak_scaling_tflops(world, e2e_steps, flops, e2e_ms)
@@ -504,11 +506,10 @@ def run_ours(args, rank, world, local):
                    "l2": "flushed between steps (256 MiB device write outside the timed events)"},
         "layers_per_s": layers_per_s,
         "roofline": {"bound": "tensor",
-                     "kernel": ("loss_gemm_pair_kernel" if os.environ.get("AWQ_GEMM_VARIANT", "1").startswith("2")
-                                else "loss_gemm_kernel") + " (candidate GEMMs + fused squared error)",
+                     "kernel": gemm_kernel + " (candidate GEMMs + fused squared error)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} bf16_tflops (burst)",
-                     "traffic": recorded_traffic("loss_gemm_kernel", spec.name),
+                     "traffic": recorded_traffic(gemm_kernel, spec.name),
                      "traffic_unit": "DRAM bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
                      "ms_per_launch": gemm_avg},
         "other_kernels": {

@@ -267,6 +267,11 @@ int awq_w4a16_dequant(const int32_t* codes, const void* steps, const void* zeros
 
 int awq_version(void);
 
+/* The loss-GEMM kernel a search of this size runs: 1 = the one-SM kernel (the default
+ * for every size), 2 = the two-SM (cta_group::2) kernel when AWQ_GEMM_VARIANT=2 is set in
+ * the environment. */
+int awq_loss_gemm_variant(int64_t M, int64_t K, int64_t N, int n_grid);
+
 /* ---- Searching without allocating -------------------------------------------
  * No counterpart in the paper or the pages: this is a deployment variant of
  * awq_search_ex for callers that cannot call cudaMalloc — e.g. a plugin whose host

@@ -381,9 +381,10 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
     ga.timeout_ns = g_timeout_ns;
     ga.fault_mode = g_fault_mode;
     ga.num_sms = num_sms;
+    ga.variant = gemm_variant(M, K, N, n_grid);
     CUtensorMap mapA, mapB;
     const char* why = "";
-    if ((e = make_operand_maps(ga, &mapA, &mapB, &why, operand_b_box_rows())) != cudaSuccess) {
+    if ((e = make_operand_maps(ga, &mapA, &mapB, &why, operand_b_box_rows(ga.variant))) != cudaSuccess) {
       status = set_error(AWQ_ERR_CUDA, std::string("TMA descriptor: ") + why);
       break;
     }
@@ -1231,5 +1232,7 @@ int awq_debug_set_fault(int mode, int64_t timeout_ns) {
 }
 
 int awq_version(void) { return kVersion; }
+
+int awq_loss_gemm_variant(int64_t M, int64_t K, int64_t N, int n_grid) { return gemm_variant(M, K, N, n_grid); }
 
 }  // extern "C"

@@ -60,15 +60,17 @@ struct LossGemmArgs {
   int fault_mode;
   int num_sms;
   int f16 = 0;               // mode 2 only: fp16 operands (the tensor maps move 2-byte elements either way)
+  int variant = 1;           // 1 the one-SM kernel, 2 the two-SM kernel (modes 0 and 1, slot_base 1)
   int slot_base = 1;         // B slot of candidate 0 (mode 1; the search's slot 0 is bf16(W)) or the
                              // slot multiplied (mode 2); values other than 1 run on the one-SM kernel
 };
-// Which loss GEMM runs: 1 = the one-SM kernel (default), 2 = the two-SM
+// Which loss GEMM runs for a search of this size: 1 = the one-SM kernel (every size; it
+// measured as fast or faster than the pair kernel on every workload), 2 = the two-SM
 // (cta_group::2) kernel, selected with AWQ_GEMM_VARIANT=2 in the environment.
-int gemm_variant();
+int gemm_variant(int64_t M, int64_t K, int64_t N, int n_grid);
 // Rows of the W_hat box one CTA loads: the full 256-column tile, or half of it when a
 // CTA pair shares the tile.
-inline int operand_b_box_rows() { return gemm_variant() == 2 ? kTileN / 2 : kTileN; }
+inline int operand_b_box_rows(int variant) { return variant == 2 ? kTileN / 2 : kTileN; }
 // Builds the TMA descriptors (driver entry point) for the two operands.
 cudaError_t make_operand_maps(const LossGemmArgs& a, CUtensorMap* mapA, CUtensorMap* mapB,
                               const char** why, int b_box_rows);

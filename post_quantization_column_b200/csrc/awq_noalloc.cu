@@ -182,9 +182,10 @@ extern "C" int awq_search_noalloc(const void* X, const void* W, int in_dtype, in
     ga.timeout_ns = 2000ull * 1000 * 1000;
     ga.fault_mode = 0;
     ga.num_sms = num_sms;
+    ga.variant = gemm_variant(M, K, N, n_grid);
     CUtensorMap mapA, mapB;
     const char* why = "";
-    if ((e = make_operand_maps(ga, &mapA, &mapB, &why, operand_b_box_rows())) != cudaSuccess) { where = why; break; }
+    if ((e = make_operand_maps(ga, &mapA, &mapB, &why, operand_b_box_rows(ga.variant))) != cudaSuccess) { where = why; break; }
     if ((e = launch_loss_gemm(ga, mapA, mapB, 0, s, &launches)) != cudaSuccess) { where = "reference GEMM"; break; }
     if ((e = launch_loss_gemm(ga, mapA, mapB, 1, s, &launches)) != cudaSuccess) { where = "loss GEMM"; break; }
     if ((e = launch_loss_reduce(loss_partial, tiles, n_grid, M, N, losses, s, &launches)) != cudaSuccess) {
