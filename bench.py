@@ -309,7 +309,7 @@ def measure_mlp_block(awq, stream, flush, steps: int, peaks, k_out: int = 4096):
     return {"workload": f"{MLP_BLOCK} + down {F}x{k_out}", "ms_per_search": ms, "steps": steps,
             "gpu_launches_per_search": awq.last_launch_count(), "chosen_alpha_index": out.best,
             "TFLOP/s": achieved,
-            "roofline": {"bound": "tensor", "kernel": "loss_gemm_kernel modes 2 and 1 (+ silu-mul, QDQ, pack)",
+            "roofline": {"bound": "tensor", "kernel": "loss_gemm_kernel modes 3 and 1 (silu-mul fused in the first GEMM epilogue; + QDQ, pack)",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                          "peak_source": "measured bf16_tflops (burst)",
                          "work": "(n_grid + 1) x (2 M K 2F + 2 M F K_out) flops over the whole call"}}

@@ -10,6 +10,7 @@
 #include "awq_kernels.h"
 
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -983,6 +984,11 @@ int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_d
     return set_error(AWQ_ERR_INVALID_ARG, "inputs and outputs must be device memory");
   const int64_t N = 2 * F;
   const int64_t tiles2 = ceil_div(M, kTileM) * ceil_div(K_out, kTileN);
+  // The silu-mul runs in the first GEMM's epilogue when its tiles can hold both halves of
+  // 128 intermediate columns (F % 128 == 0); AWQ_MLP_UNFUSED=1 keeps the separate
+  // elementwise kernel (the two give identical bits).
+  const char* unfused_env = getenv("AWQ_MLP_UNFUSED");
+  const bool fused = F % (kTileN / 2) == 0 && !(unfused_env && unfused_env[0] == '1');
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t at = off;
@@ -992,7 +998,8 @@ int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_d
   const size_t o_err = take(16), o_a = take(static_cast<size_t>(K) * 4), o_S = take(static_cast<size_t>(n_grid) * K * 4),
                o_best = take(16), o_losses = take(static_cast<size_t>(n_grid) * 4),
                o_Xb = in_dtype == AWQ_DTYPE_F32 ? take(static_cast<size_t>(M) * K * 2) : 0,
-               o_Wt = take(static_cast<size_t>(n_grid + 1) * N * K * 2), o_H = take(static_cast<size_t>(M) * N * 4),
+               o_Wt = take(static_cast<size_t>(n_grid + 1) * N * K * 2),
+               o_H = fused ? 0 : take(static_cast<size_t>(M) * N * 4),
                o_h = take(static_cast<size_t>(M) * F * 2), o_WdT = take(static_cast<size_t>(K_out) * F * 2),
                o_Y = take(static_cast<size_t>(tiles2) * kTileM * kTileN * 4),
                o_part = take(static_cast<size_t>(n_grid) * tiles2 * 8);
@@ -1011,7 +1018,7 @@ int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_d
   int* best = reinterpret_cast<int*>(b + o_best);
   float* losses = reinterpret_cast<float*>(b + o_losses);
   __nv_bfloat16* Wt = reinterpret_cast<__nv_bfloat16*>(b + o_Wt);
-  float* H = reinterpret_cast<float*>(b + o_H);
+  float* H = fused ? nullptr : reinterpret_cast<float*>(b + o_H);
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(b + o_h);
   __nv_bfloat16* WdT = reinterpret_cast<__nv_bfloat16*>(b + o_WdT);
   float* Y = reinterpret_cast<float*>(b + o_Y);
@@ -1033,7 +1040,8 @@ int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_d
       where = "bf16 operand kernel";
       break;
     }
-    if ((e = launch_qdq(W_gu, in_dtype, K, N, group, n_grid, S, Wt, err, s, &launches)) != cudaSuccess) {
+    if ((e = launch_qdq(W_gu, in_dtype, K, N, group, n_grid, S, Wt, err, s, &launches, 0, fused ? F : 0)) !=
+        cudaSuccess) {
       where = "qdq kernel";
       break;
     }
@@ -1041,7 +1049,9 @@ int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_d
       where = "down-projection transpose";
       break;
     }
-    // GEMM 1: H = X_b [W_gate | W_up]_slot, row-major fp32 (mode 2)
+    // GEMM 1: h = bf16(silu(X_b W_gate) (X_b W_up)) with the silu-mul in the epilogue
+    // (mode 3), or H = X_b [W_gate | W_up]_slot row-major fp32 (mode 2) and the
+    // elementwise kernel
     LossGemmArgs g1;
     g1.Xb = Xb;
     g1.Wt = Wt;
@@ -1049,7 +1059,8 @@ int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_d
     g1.K = K;
     g1.N = N;
     g1.n_grid = n_grid;
-    g1.Y = H;
+    g1.Y = fused ? nullptr : H;
+    g1.H = fused ? h : nullptr;
     g1.partial = nullptr;
     g1.err = err;
     g1.timeout_ns = g_timeout_ns;
@@ -1064,6 +1075,7 @@ int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_d
     g2.N = K_out;
     g2.n_grid = 0;  // one operand slot for the tensor map
     g2.Y = Y;
+    g2.H = nullptr;
     g2.slot_base = 0;
     CUtensorMap a1, b1, a2, b2;
     const char* why = "";
@@ -1075,8 +1087,14 @@ int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_d
     g2.n_grid = 1;  // one candidate per launch
     for (int c = -1; c < n_grid && e == cudaSuccess; ++c) {
       g1.slot_base = c + 1;  // slot 0: bf16(W), the reference block
-      if ((e = launch_loss_gemm(g1, a1, b1, 2, s, &launches)) != cudaSuccess) { where = "block GEMM 1"; break; }
-      if ((e = launch_silu_mul(H, M, F, h, s, &launches)) != cudaSuccess) { where = "silu-mul kernel"; break; }
+      if ((e = launch_loss_gemm(g1, a1, b1, fused ? 3 : 2, s, &launches)) != cudaSuccess) {
+        where = "block GEMM 1";
+        break;
+      }
+      if (!fused && (e = launch_silu_mul(H, M, F, h, s, &launches)) != cudaSuccess) {
+        where = "silu-mul kernel";
+        break;
+      }
       g2.partial = part + static_cast<int64_t>(c < 0 ? 0 : c) * tiles2;
       if ((e = launch_loss_gemm(g2, a2, b2, c < 0 ? 0 : 1, s, &launches)) != cudaSuccess) {
         where = "block GEMM 2";

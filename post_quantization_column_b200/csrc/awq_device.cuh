@@ -80,6 +80,14 @@ __device__ __forceinline__ float qdq_fold_back(float q, QdqParams p, float s) {
   return __fdiv_rn(__fmul_rn(__fsub_rn(q, p.zero), p.step), s);
 }
 
+// The MLP block's intermediate value silu(g) u = (g / (1 + exp(-g))) u in fp32, each
+// operation rounded once ("AWQ：为什么 4-bit 权重量化要先观察 Activation" §4, a candidate
+// scored on its module's output). The standalone elementwise kernel and the fused GEMM
+// epilogue both call this, so the two paths give identical bits.
+__device__ __forceinline__ float silu_mul_f32(float g, float u) {
+  return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+}
+
 template <typename T>
 __device__ __forceinline__ float to_f32(T v);
 template <>

@@ -32,13 +32,16 @@ cudaError_t launch_to_bf16(const float* x, int64_t n, __nv_bfloat16* out, cudaSt
 // `quantizer`: 0 the asymmetric zero-point quantizer (AWQ-P1 §7), 1 the symmetric [-7, 7]
 // teaching quantizer (AWQ-P1 §2), stored as codes q + 7 with zero point 7.
 // Writes Wt[0] = bf16(W)^T and Wt[1 + i] = bf16(W_hat_i)^T, each N x K (K contiguous).
+// `interleave` = F > 0 (N = 2F, F % 128 == 0) writes the columns of [W_gate | W_up] in the
+// order the fused MLP GEMM reads them: every 256 rows are 128 gate columns followed by the
+// 128 up columns of the same outputs.
 cudaError_t launch_qdq(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid,
                        const float* S, __nv_bfloat16* Wt, int* err, cudaStream_t s, int* launches,
-                       int quantizer = 0);
+                       int quantizer = 0, int64_t interleave = 0);
 // The same for the groups group0 .. group0 + groups - 1 only (rows group0*group ..).
 cudaError_t launch_qdq_groups(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid,
                               const float* S, __nv_bfloat16* Wt, int* err, int64_t group0, int64_t groups,
-                              cudaStream_t s, int* launches, int quantizer = 0);
+                              cudaStream_t s, int* launches, int quantizer = 0, int64_t interleave = 0);
 
 // ---- artifact of the chosen candidate (AWQ-P1 §7; QUANT-P4 §5.3) ------------------
 // The chosen candidate is the first minimum of `losses` (AWQ-P1 §3); its index is
@@ -62,7 +65,8 @@ struct LossGemmArgs {
   int f16 = 0;               // mode 2 only: fp16 operands (the tensor maps move 2-byte elements either way)
   int variant = 1;           // 1 the one-SM kernel, 2 the two-SM kernel (modes 0 and 1, slot_base 1)
   int slot_base = 1;         // B slot of candidate 0 (mode 1; the search's slot 0 is bf16(W)) or the
-                             // slot multiplied (mode 2); values other than 1 run on the one-SM kernel
+                             // slot multiplied (modes 2, 3); values other than 1 run on the one-SM kernel
+  __nv_bfloat16* H = nullptr;  // mode 3: the MLP block's intermediate h, M x N/2 row-major bf16
 };
 // Which loss GEMM runs for a search of this size: 1 = the one-SM kernel (every size; it
 // measured as fast or faster than the pair kernel on every workload), 2 = the two-SM
@@ -76,7 +80,10 @@ cudaError_t make_operand_maps(const LossGemmArgs& a, CUtensorMap* mapA, CUtensor
                               const char** why, int b_box_rows);
 // mode 0: Y = X_b W_b into the tiled buffer; mode 1: per-tile sum of (X_b W_hat_i - Y)^2;
 // mode 2: Y = X_b Wt[0]^T written row-major fp32 into a.Y (M x N, pitch N), always on
-// the one-SM kernel (make the maps with b_box_rows = kTileN).
+// the one-SM kernel (make the maps with b_box_rows = kTileN);
+// mode 3: the MLP block's first GEMM with the silu-mul fused in its epilogue: the B slot
+// holds [W_gate | W_up] interleaved by 128 columns (launch_qdq's `interleave`), and
+// h = bf16(fl32(silu(g) u)) is written row-major into a.H (M x N/2), one-SM kernel only.
 cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, const CUtensorMap& mapB,
                              int mode, cudaStream_t s, int* launches);
 

@@ -8,7 +8,11 @@
 //           cores, and the epilogue adds (acc - Y)^2 over the tile and writes one fp64
 //           partial sum. The candidate output Y_hat is never written to HBM;
 //   mode 2: a plain product A B^T (B stored K-major), written row-major in fp32 with
-//           the ragged rows and columns masked (the packed artifact's consumer).
+//           the ragged rows and columns masked (the packed artifact's consumer);
+//   mode 3: the MLP block's first GEMM, B = [W_gate | W_up] interleaved by 128 columns so
+//           that a 256-column tile holds the gate and up halves of 128 intermediate
+//           columns; the epilogue writes h = bf16(silu(g) u) row-major and never stores
+//           the fp32 halves.
 //
 // Blackwell structure (sm_100a): 128 x 256 output tiles, K in 64-element (128-byte)
 // slices; a 4-stage TMA -> shared-memory ring (128-byte swizzle, no multicast); one
@@ -53,8 +57,9 @@ struct GemmParams {
   int nk;
   int64_t M, N, ldo;  // mode 2: output rows, columns and row pitch
   int f16;            // mode 2: operands are fp16 (else bf16)
-  int slot_base;      // B slot of candidate 0 (mode 1) or the slot multiplied (mode 2)
+  int slot_base;      // B slot of candidate 0 (mode 1) or the slot multiplied (modes 2, 3)
   float* Y;           // modes 0-1: the tiled reference output; mode 2: the row-major output
+  __nv_bfloat16* H;   // mode 3: the row-major bf16 intermediate (pitch ldo)
   double* partial;
   int* err;
   uint64_t timeout_ns;
@@ -151,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int64_t u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         int c, mt, nt;
         unit_coords(u, p, c, mt, nt);
-        const int slot = p.mode == 1 ? c + p.slot_base : (p.mode == 2 ? p.slot_base : 0);
+        const int slot = p.mode == 1 ? c + p.slot_base : (p.mode >= 2 ? p.slot_base : 0);
         for (int kb = 0; kb < p.nk; ++kb) {
           if (!mbar_wait_bounded(empty + stage, phase ^ 1u, abort_flag, budget)) {
             ok = false;
@@ -240,6 +245,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      if (p.mode == 3) {
+        // columns j (gate) and BN/2 + j (up) of the accumulator are the two halves of
+        // intermediate column nt * BN/2 + j
+        const int64_t grow = static_cast<int64_t>(mt) * BM + row;
+#pragma unroll 1
+        for (int j0 = 0; j0 < BN / 2; j0 += 32) {
+          uint32_t g[32], up[32];
+          tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(j0), g);
+          tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(BN / 2 + j0), up);
+          tmem_ld_wait();
+          if (grow < p.M) {
+            uint4* orow = reinterpret_cast<uint4*>(p.H + grow * p.ldo + static_cast<int64_t>(nt) * (BN / 2) + j0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint32_t w[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int k = 8 * q + 2 * e;
+                const __nv_bfloat162 hv =
+                    __floats2bfloat162_rn(silu_mul_f32(__uint_as_float(g[k]), __uint_as_float(up[k])),
+                                          silu_mul_f32(__uint_as_float(g[k + 1]), __uint_as_float(up[k + 1])));
+                w[e] = *reinterpret_cast<const uint32_t*>(&hv);
+              }
+              orow[q] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(tempty + acc);
+        continue;
+      }
       const int64_t tile = static_cast<int64_t>(mt) * p.tiles_n + nt;
       float4* ytile = reinterpret_cast<float4*>(p.Y + tile * (BM * BN));
       float sq = 0.0f;
@@ -665,7 +701,7 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
                              cudaStream_t s, int* launches) {
   const int tiles_m = static_cast<int>(ceil_div(a.M, BM));
   const int tiles_n = static_cast<int>(ceil_div(a.N, BN));
-  if (a.variant == 2 && mode != 2 && a.slot_base == 1) {
+  if (a.variant == 2 && mode < 2 && a.slot_base == 1) {
     static unsigned long long attr_done = 0;
     cudaError_t e = set_smem_limit_once(loss_gemm_pair_kernel, kPairSmemBytes, &attr_done);
     if (e != cudaSuccess) return e;
@@ -719,7 +755,8 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
   p.nk = static_cast<int>(ceil_div(a.K, BK));
   p.M = a.M;
   p.N = a.N;
-  p.ldo = a.N;
+  p.ldo = mode == 3 ? a.N / 2 : a.N;
+  p.H = a.H;
   p.f16 = a.f16;
   p.slot_base = a.slot_base;
   p.Y = a.Y;

@@ -30,10 +30,7 @@ __global__ void __launch_bounds__(kActThreads)
     float v[4] = {g.x, g.y, g.z, g.w};
     const float w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float sg = __fdiv_rn(v[j], __fadd_rn(1.0f, expf(-v[j])));
-      v[j] = __fmul_rn(sg, w[j]);
-    }
+    for (int j = 0; j < 4; ++j) v[j] = silu_mul_f32(v[j], w[j]);
     const __nv_bfloat162 lo = __floats2bfloat162_rn(v[0], v[1]);
     const __nv_bfloat162 hi = __floats2bfloat162_rn(v[2], v[3]);
     uint2 o;

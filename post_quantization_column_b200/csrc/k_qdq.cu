@@ -71,6 +71,16 @@ struct Tile {
 // the qdq kernel's row order; the pack kernel reads its own unskewed copy).
 __device__ __forceinline__ int skew(int r) { return r + 2 * (r >> 5); }
 
+// Output row of column n in the candidate operand. With interleave = F > 0 (W = [W_gate |
+// W_up], 2F columns, F % 128 == 0) every 256 rows hold 128 gate columns followed by the
+// 128 up columns of the same outputs, so one 128 x 256 GEMM tile holds both halves of the
+// MLP block's 128 intermediate columns; otherwise the identity.
+__device__ __forceinline__ int64_t interleaved_column(int64_t n, int64_t interleave) {
+  if (interleave <= 0) return n;
+  const int64_t half = n >= interleave ? 1 : 0, f = n - half * interleave;
+  return (f >> 7) * 256 + half * 128 + (f & 127);
+}
+
 __device__ __forceinline__ float round_small(float x) {
   return __fsub_rn(__fadd_rn(x, kRoundMagic), kRoundMagic);
 }
@@ -256,7 +266,7 @@ __device__ __noinline__ void exact_run(float2 w0, float2 w1, float2 w2, float2 w
 template <typename T, int G>
 __global__ void __launch_bounds__(Tile<G>::kThreads, Tile<G>::kBlocksPerSm)
     qdq_kernel(const T* __restrict__ W, int64_t K, int64_t N, int n_grid, const float* __restrict__ S,
-               __nv_bfloat16* __restrict__ Wt, int* err, int64_t group0, int quantizer) {
+               __nv_bfloat16* __restrict__ Wt, int* err, int64_t group0, int quantizer, int64_t interleave) {
   using L = Tile<G>;
   extern __shared__ float smem[];
   float* sWT = smem;                                    // [64][kPitch]
@@ -294,8 +304,8 @@ __global__ void __launch_bounds__(Tile<G>::kThreads, Tile<G>::kBlocksPerSm)
   const int col0 = warp * L::kColsPerWarp + cg * 2;
   const int row0 = (rl >> 1) * kRowsPerLane + own * (G / 2);
   const bool active = n0 + col0 < N;  // N is even: both columns are in or both out
-  __nv_bfloat16* const dst0 = Wt + (n0 + col0 + own) * K + k0 + row0;
-  const int64_t dst1_off = own ? -K : K;  // the lane's other column
+  __nv_bfloat16* const dst0 = Wt + interleaved_column(n0 + col0 + own, interleave) * K + k0 + row0;
+  const int64_t dst1_off = own ? -K : K;  // the lane's other column (a pair never straddles 128 columns)
 
   float2 w2[2][4];
 #pragma unroll
@@ -591,7 +601,8 @@ __global__ void __launch_bounds__(Tile<G>::kThreads, Tile<G>::kBlocksPerSm)
 
 template <typename T, int G>
 cudaError_t launch_qdq_t(const T* W, int64_t K, int64_t N, int n_grid, const float* S, __nv_bfloat16* Wt,
-                         int* err, int64_t group0, int64_t groups, cudaStream_t s, int quantizer) {
+                         int* err, int64_t group0, int64_t groups, cudaStream_t s, int quantizer,
+                         int64_t interleave) {
   using L = Tile<G>;
   auto bytes = [](int grid_points) {
     return (static_cast<size_t>(L::kCols) * L::kPitch + 2 * static_cast<size_t>(grid_points) * L::kSkewPitch +
@@ -602,7 +613,8 @@ cudaError_t launch_qdq_t(const T* W, int64_t K, int64_t N, int n_grid, const flo
   cudaError_t e = set_smem_limit_once(qdq_kernel<T, G>, static_cast<int>(bytes(64)), &attr_done);
   if (e != cudaSuccess) return e;
   dim3 grid(static_cast<unsigned>(ceil_div(N, static_cast<int64_t>(L::kCols))), static_cast<unsigned>(groups));
-  qdq_kernel<T, G><<<grid, L::kThreads, bytes(n_grid), s>>>(W, K, N, n_grid, S, Wt, err, group0, quantizer);
+  qdq_kernel<T, G><<<grid, L::kThreads, bytes(n_grid), s>>>(W, K, N, n_grid, S, Wt, err, group0, quantizer,
+                                                            interleave);
   return cudaGetLastError();
 }
 
@@ -625,27 +637,28 @@ cudaError_t launch_pack_t(const T* W, int64_t K, int64_t N, int n_grid, const fl
 
 cudaError_t launch_qdq_groups(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid,
                               const float* S, __nv_bfloat16* Wt, int* err, int64_t group0, int64_t groups,
-                              cudaStream_t s, int* launches, int quantizer) {
+                              cudaStream_t s, int* launches, int quantizer, int64_t interleave) {
   *launches += 1;
   if (in_dtype == 0) {
     const auto* w = static_cast<const __nv_bfloat16*>(W);
     switch (group) {
-      case 32: return launch_qdq_t<__nv_bfloat16, 32>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer);
-      case 64: return launch_qdq_t<__nv_bfloat16, 64>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer);
-      default: return launch_qdq_t<__nv_bfloat16, 128>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer);
+      case 32: return launch_qdq_t<__nv_bfloat16, 32>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer, interleave);
+      case 64: return launch_qdq_t<__nv_bfloat16, 64>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer, interleave);
+      default: return launch_qdq_t<__nv_bfloat16, 128>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer, interleave);
     }
   }
   const auto* w = static_cast<const float*>(W);
   switch (group) {
-    case 32: return launch_qdq_t<float, 32>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer);
-    case 64: return launch_qdq_t<float, 64>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer);
-    default: return launch_qdq_t<float, 128>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer);
+    case 32: return launch_qdq_t<float, 32>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer, interleave);
+    case 64: return launch_qdq_t<float, 64>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer, interleave);
+    default: return launch_qdq_t<float, 128>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer, interleave);
   }
 }
 
 cudaError_t launch_qdq(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid, const float* S,
-                       __nv_bfloat16* Wt, int* err, cudaStream_t s, int* launches, int quantizer) {
-  return launch_qdq_groups(W, in_dtype, K, N, group, n_grid, S, Wt, err, 0, K / group, s, launches, quantizer);
+                       __nv_bfloat16* Wt, int* err, cudaStream_t s, int* launches, int quantizer, int64_t interleave) {
+  return launch_qdq_groups(W, in_dtype, K, N, group, n_grid, S, Wt, err, 0, K / group, s, launches, quantizer,
+                           interleave);
 }
 
 cudaError_t launch_pack(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid, const float* S,

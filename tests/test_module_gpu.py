@@ -81,3 +81,17 @@ def test_mlp_block_is_deterministic():
     a, b = awq.search_mlp(X, W_gu, W_down, 128, 20), awq.search_mlp(X, W_gu, W_down, 128, 20)
     for name in ("scales", "codes", "steps", "zeros", "losses"):
         assert torch.equal(getattr(a, name), getattr(b, name)), name
+
+
+def test_fused_epilogue_matches_separate_elementwise_kernel(monkeypatch):
+    """F % 128 == 0 runs the silu-mul in the first GEMM's epilogue (gate and up columns
+    interleaved by 128 in the candidate operand); the separate elementwise kernel must give
+    the same bits, losses included."""
+    spec = custom_spec(200, 256, 2 * 256, dtype="bf16", seed=5)
+    X, W_gu = (t.cuda() for t in generate(spec))
+    W_down = generate_down(spec, 264).cuda()
+    fused = awq.search_mlp(X, W_gu, W_down, 128, 20)
+    monkeypatch.setenv("AWQ_MLP_UNFUSED", "1")
+    plain = awq.search_mlp(X, W_gu, W_down, 128, 20)
+    for name in ("scales", "codes", "steps", "zeros", "losses"):
+        assert torch.equal(getattr(fused, name), getattr(plain, name)), name
