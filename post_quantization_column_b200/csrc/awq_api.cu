@@ -989,6 +989,13 @@ int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_d
   // elementwise kernel (the two give identical bits).
   const char* unfused_env = getenv("AWQ_MLP_UNFUSED");
   const bool fused = F % (kTileN / 2) == 0 && !(unfused_env && unfused_env[0] == '1');
+  // The fused path runs each GEMM once for a batch of candidates (their intermediates h
+  // side by side, up to 4 GiB), so the second GEMM's few hundred tiles of one candidate
+  // do not each end in a partial wave.
+  const int64_t h_bytes = M * F * 2;
+  const int h_batch = fused ? static_cast<int>(std::max<int64_t>(
+                                  1, std::min<int64_t>(n_grid, (int64_t(4) << 30) / std::max<int64_t>(h_bytes, 1))))
+                            : 0;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t at = off;
@@ -1000,7 +1007,8 @@ int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_d
                o_Xb = in_dtype == AWQ_DTYPE_F32 ? take(static_cast<size_t>(M) * K * 2) : 0,
                o_Wt = take(static_cast<size_t>(n_grid + 1) * N * K * 2),
                o_H = fused ? 0 : take(static_cast<size_t>(M) * N * 4),
-               o_h = take(static_cast<size_t>(M) * F * 2), o_WdT = take(static_cast<size_t>(K_out) * F * 2),
+               o_h = take(static_cast<size_t>(1 + h_batch) * M * F * 2),
+               o_WdT = take(static_cast<size_t>(K_out) * F * 2),
                o_Y = take(static_cast<size_t>(tiles2) * kTileM * kTileN * 4),
                o_part = take(static_cast<size_t>(n_grid) * tiles2 * 8);
   cudaMemPool_t pool;
@@ -1077,28 +1085,51 @@ int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_d
     g2.Y = Y;
     g2.H = nullptr;
     g2.slot_base = 0;
-    CUtensorMap a1, b1, a2, b2;
+    CUtensorMap a1, b1, a2, b2, a2b, b2b;
     const char* why = "";
+    // the batched second GEMM: A = the stack of intermediates [1 + h_batch][M][F]
+    LossGemmArgs g2b = g2;
+    g2b.a_slotted = 1;
+    g2b.a_slots = 1 + h_batch;
     if ((e = make_operand_maps(g1, &a1, &b1, &why, kTileN)) != cudaSuccess ||
-        (e = make_operand_maps(g2, &a2, &b2, &why, kTileN)) != cudaSuccess) {
+        (e = make_operand_maps(g2, &a2, &b2, &why, kTileN)) != cudaSuccess ||
+        (fused && (e = make_operand_maps(g2b, &a2b, &b2b, &why, kTileN)) != cudaSuccess)) {
       status = set_error(AWQ_ERR_CUDA, std::string("TMA descriptor: ") + why);
       break;
     }
     g2.n_grid = 1;  // one candidate per launch
-    for (int c = -1; c < n_grid && e == cudaSuccess; ++c) {
-      g1.slot_base = c + 1;  // slot 0: bf16(W), the reference block
-      if ((e = launch_loss_gemm(g1, a1, b1, fused ? 3 : 2, s, &launches)) != cudaSuccess) {
-        where = "block GEMM 1";
-        break;
+    if (fused) {
+      // reference block: h_0 = block intermediate with bf16(W), then Y = h_0 W_down^T
+      g1.slot_base = 0;
+      g1.cands = 1;
+      if ((e = launch_loss_gemm(g1, a1, b1, 3, s, &launches)) != cudaSuccess) { where = "block GEMM 1"; break; }
+      g2.partial = part;
+      if ((e = launch_loss_gemm(g2, a2, b2, 0, s, &launches)) != cudaSuccess) { where = "block GEMM 2"; break; }
+      for (int c0 = 0; c0 < n_grid && e == cudaSuccess; c0 += h_batch) {
+        const int nb = std::min(h_batch, n_grid - c0);
+        g1.slot_base = 1 + c0;  // candidate c0 + i in B slot 1 + c0 + i ...
+        g1.cands = nb;
+        g1.H = h + h_bytes / 2;  // ... writes h slot 1 + i
+        g1.h_stride = h_bytes / 2;
+        if ((e = launch_loss_gemm(g1, a1, b1, 3, s, &launches)) != cudaSuccess) { where = "block GEMM 1"; break; }
+        g2b.a_slot_base = 1;
+        g2b.cands = nb;
+        g2b.b_per_cand = 0;  // every candidate against the same W_down
+        g2b.slot_base = 0;
+        g2b.n_grid = nb;
+        g2b.partial = part + static_cast<int64_t>(c0) * tiles2;
+        if ((e = launch_loss_gemm(g2b, a2b, b2b, 1, s, &launches)) != cudaSuccess) { where = "block GEMM 2"; break; }
       }
-      if (!fused && (e = launch_silu_mul(H, M, F, h, s, &launches)) != cudaSuccess) {
-        where = "silu-mul kernel";
-        break;
-      }
-      g2.partial = part + static_cast<int64_t>(c < 0 ? 0 : c) * tiles2;
-      if ((e = launch_loss_gemm(g2, a2, b2, c < 0 ? 0 : 1, s, &launches)) != cudaSuccess) {
-        where = "block GEMM 2";
-        break;
+    } else {
+      for (int c = -1; c < n_grid && e == cudaSuccess; ++c) {
+        g1.slot_base = c + 1;  // slot 0: bf16(W), the reference block
+        if ((e = launch_loss_gemm(g1, a1, b1, 2, s, &launches)) != cudaSuccess) { where = "block GEMM 1"; break; }
+        if ((e = launch_silu_mul(H, M, F, h, s, &launches)) != cudaSuccess) { where = "silu-mul kernel"; break; }
+        g2.partial = part + static_cast<int64_t>(c < 0 ? 0 : c) * tiles2;
+        if ((e = launch_loss_gemm(g2, a2, b2, c < 0 ? 0 : 1, s, &launches)) != cudaSuccess) {
+          where = "block GEMM 2";
+          break;
+        }
       }
     }
     if (e != cudaSuccess) break;

@@ -67,6 +67,12 @@ struct LossGemmArgs {
   int slot_base = 1;         // B slot of candidate 0 (mode 1; the search's slot 0 is bf16(W)) or the
                              // slot multiplied (modes 2, 3); values other than 1 run on the one-SM kernel
   __nv_bfloat16* H = nullptr;  // mode 3: the MLP block's intermediate h, M x N/2 row-major bf16
+  int64_t h_stride = 0;        // mode 3: elements between successive candidates' h
+  int cands = 0;               // modes 1, 3: candidates this launch walks (0: n_grid for mode 1, 1 for mode 3)
+  int b_per_cand = 1;          // modes 1, 3: candidate c reads B slot slot_base + c (1) or slot_base (0)
+  int a_slotted = 0;           // A is a stack of a_slots operands [a_slots][M][K]; c reads a_slot_base + c
+  int a_slot_base = 0;
+  int a_slots = 1;
 };
 // Which loss GEMM runs for a search of this size: 1 = the one-SM kernel (every size; it
 // measured as fast or faster than the pair kernel on every workload), 2 = the two-SM

@@ -57,9 +57,14 @@ struct GemmParams {
   int nk;
   int64_t M, N, ldo;  // mode 2: output rows, columns and row pitch
   int f16;            // mode 2: operands are fp16 (else bf16)
-  int slot_base;      // B slot of candidate 0 (mode 1) or the slot multiplied (modes 2, 3)
+  int slot_base;      // B slot of candidate 0 (modes 1, 3) or the slot multiplied (mode 2)
+  int cands;          // candidates this launch walks (modes 1 and 3)
+  int b_per_cand;     // modes 1, 3: B slot = slot_base + c (1) or slot_base for every c (0)
+  int a_slotted;      // A is a stack of slots (3-D map); candidate c reads slot a_slot_base + c
+  int a_slot_base;
   float* Y;           // modes 0-1: the tiled reference output; mode 2: the row-major output
-  __nv_bfloat16* H;   // mode 3: the row-major bf16 intermediate (pitch ldo)
+  __nv_bfloat16* H;   // mode 3: the row-major bf16 intermediate of candidate 0 (pitch ldo)
+  int64_t h_stride;   // mode 3: elements between successive candidates' intermediates
   double* partial;
   int* err;
   uint64_t timeout_ns;
@@ -138,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
-  const int64_t n_units = (p.mode == 1 ? p.n_grid : 1) * tiles;
+  const int64_t n_units = (p.mode == 1 || p.mode == 3 ? p.cands : 1) * tiles;
   const uint64_t budget = p.timeout_ns;
 
   auto fail = [&]() {
@@ -156,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int64_t u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         int c, mt, nt;
         unit_coords(u, p, c, mt, nt);
-        const int slot = p.mode == 1 ? c + p.slot_base : (p.mode >= 2 ? p.slot_base : 0);
+        const int slot = p.mode == 0 ? 0 : p.slot_base + ((p.mode == 1 || p.mode == 3) && p.b_per_cand ? c : 0);
         for (int kb = 0; kb < p.nk; ++kb) {
           if (!mbar_wait_bounded(empty + stage, phase ^ 1u, abort_flag, budget)) {
             ok = false;
@@ -165,7 +170,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool skip = p.fault_mode == 1 && p.mode == 1 && u == blockIdx.x && kb == 0;
           if (!skip) {
             mbar_arrive_expect_tx(full + stage, kStageBytes);
-            tma_load_2d(&mapA, full + stage, sA + stage * kABytes, kb * BK, mt * BM);
+            if (p.a_slotted)
+              tma_load_3d(&mapA, full + stage, sA + stage * kABytes, kb * BK, mt * BM, p.a_slot_base + c);
+            else
+              tma_load_2d(&mapA, full + stage, sA + stage * kABytes, kb * BK, mt * BM);
             tma_load_3d(&mapB, full + stage, sB + stage * kBBytes, kb * BK, nt * BN, slot);
             issued |= 1u << stage;
             last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -256,7 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(BN / 2 + j0), up);
           tmem_ld_wait();
           if (grow < p.M) {
-            uint4* orow = reinterpret_cast<uint4*>(p.H + grow * p.ldo + static_cast<int64_t>(nt) * (BN / 2) + j0);
+            uint4* orow = reinterpret_cast<uint4*>(p.H + static_cast<int64_t>(c) * p.h_stride + grow * p.ldo +
+                                                   static_cast<int64_t>(nt) * (BN / 2) + j0);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               uint32_t w[4];
@@ -655,13 +664,15 @@ cudaError_t make_operand_maps(const LossGemmArgs& a, CUtensorMap* mapA, CUtensor
     *why = "cuTensorMapEncodeTiled unavailable";
     return cudaErrorNotSupported;
   }
-  // A = X_b [M][K]: dims (K, M), box (64, 128), 128-byte swizzle
-  const cuuint64_t dimsA[2] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(a.M)};
-  const cuuint64_t strideA[1] = {static_cast<cuuint64_t>(a.K) * 2};
-  const cuuint32_t boxA[2] = {BK, BM};
+  // A = X_b [M][K]: dims (K, M), box (64, 128), 128-byte swizzle; or a stack of a_slots
+  // such operands [a_slots][M][K]: dims (K, M, slots), box (64, 128, 1)
+  const cuuint64_t dimsA[3] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(a.M),
+                               static_cast<cuuint64_t>(a.a_slots)};
+  const cuuint64_t strideA[2] = {static_cast<cuuint64_t>(a.K) * 2, static_cast<cuuint64_t>(a.K) * a.M * 2};
+  const cuuint32_t boxA[3] = {BK, BM, 1};
   const cuuint32_t ones[3] = {1, 1, 1};
-  CUresult r = fn(mapA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16*>(a.Xb), dimsA, strideA, boxA,
-                  ones, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  CUresult r = fn(mapA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.a_slotted ? 3 : 2, const_cast<__nv_bfloat16*>(a.Xb),
+                  dimsA, strideA, boxA, ones, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     *why = "tensor map of X";
@@ -701,7 +712,7 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
                              cudaStream_t s, int* launches) {
   const int tiles_m = static_cast<int>(ceil_div(a.M, BM));
   const int tiles_n = static_cast<int>(ceil_div(a.N, BN));
-  if (a.variant == 2 && mode < 2 && a.slot_base == 1) {
+  if (a.variant == 2 && mode < 2 && a.slot_base == 1 && !a.a_slotted && a.b_per_cand && a.cands == 0) {
     static unsigned long long attr_done = 0;
     cudaError_t e = set_smem_limit_once(loss_gemm_pair_kernel, kPairSmemBytes, &attr_done);
     if (e != cudaSuccess) return e;
@@ -757,6 +768,11 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
   p.N = a.N;
   p.ldo = mode == 3 ? a.N / 2 : a.N;
   p.H = a.H;
+  p.h_stride = a.h_stride;
+  p.cands = a.cands > 0 ? a.cands : (mode == 1 ? a.n_grid : 1);
+  p.b_per_cand = a.b_per_cand;
+  p.a_slotted = a.a_slotted;
+  p.a_slot_base = a.a_slot_base;
   p.f16 = a.f16;
   p.slot_base = a.slot_base;
   p.Y = a.Y;
@@ -765,7 +781,7 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
   p.timeout_ns = a.timeout_ns;
   p.fault_mode = a.fault_mode;
   const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
-  const int64_t units = (mode == 1 ? a.n_grid : 1) * tiles;
+  const int64_t units = (mode == 1 || mode == 3 ? p.cands : 1) * tiles;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(units, a.num_sms));
   loss_gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(mapA, mapB, p);
   *launches += 1;
