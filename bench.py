@@ -245,7 +245,7 @@ def measure_w4a16(awq, spec: LayerSpec, X, out, stream, flush, steps: int, peaks
     A1 = A[:1].contiguous()
     t, n = _time_w4a16(awq, lambda: awq.w4a16_matmul_packed(A1, packed, out.steps, out.zeros, spec.group,
                                                              stream=stream), flush, steps)
-    res["decode"] = decode_entry(spec.K, spec.N, spec.group, t, n, "gemv_packed_kernel (repacked codes)")
+    res["decode"] = decode_entry(spec.K, spec.N, spec.group, t, n, "gemv_stream_kernel (repacked codes)")
     t, n = _time_w4a16(awq, lambda: awq.w4a16_matmul(A1, out.codes, out.steps, out.zeros, spec.group,
                                                       stream=stream), flush, steps)
     res["decode_plain_layout"] = decode_entry(spec.K, spec.N, spec.group, t, n, "gemv_kernel (artifact layout)")
@@ -260,7 +260,7 @@ def measure_w4a16(awq, spec: LayerSpec, X, out, stream, flush, steps: int, peaks
     t, n = _time_w4a16(awq, lambda: awq.w4a16_matmul_packed(A70, packed70, steps70, zeros70, big.group,
                                                              stream=stream), flush, steps)
     res["decode_70b_gate_up_shape"] = decode_entry(big.K, big.N, big.group, t, n,
-                                                   "gemv_packed_kernel (random artifact of the 70B gate+up shape)")
+                                                   "gemv_stream_kernel (random artifact of the 70B gate+up shape)")
     del codes70, steps70, zeros70, packed70
     M = spec.M
     Am = A[:M].contiguous()

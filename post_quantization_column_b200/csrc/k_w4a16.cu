@@ -288,13 +288,13 @@ __global__ void __launch_bounds__(kDqThreads)
 }
 
 // ---- the consumer's repacked layout ---------------------------------------------------
-// For decode the codes are read in the order the MMA fragments use them: for every
-// 16-row step s, 64-column block cb and lane (g, t), 16 bytes (4 words) hold the lane's
-// 32 nibbles. Word u serves column tiles j = 2u and 2u + 1; its nibble p (0..3) and
-// p + 4 are the pair (rows r, r + 1) of fragment p: tile 2u + (p >> 1), rows 2t (p even)
-// or 2t + 8 (p odd), column 8 j + g. So (word >> 4p) & 0x000F000F puts the pair in the two
-// halves, one shift and one logic op per two weights, and a warp reads 512 contiguous
-// bytes per step.
+// For decode the weights are the A operand of 16 x 8 x 16 MMAs (16 output columns by 16
+// rows of K per MMA) and the codes are read in fragment order: for every 16-row step s,
+// 64-column block cb and lane (g, t), 16 bytes (4 words) hold the lane's 32 nibbles.
+// Word u serves the 16 columns 16u .. 16u + 15; its nibbles p and p + 4 (p = 0..3) are
+// rows (r, r + 1) of column 16u + g + 8 (p & 1), r = 2t + 8 (p >> 1) — fragment register
+// a_p. Pairs 0 and 1 sit in bits 0-7 of each half of the word, pairs 2 and 3 in bits
+// 8-15, and a warp reads 512 contiguous bytes per step.
 __global__ void repack_kernel(const int32_t* __restrict__ codes, int64_t K, int64_t N, uint32_t* __restrict__ P) {
   const int64_t words = N / 8, cbs = N / 64;
   const int64_t total = (K / 16) * cbs * 32 * 4;
@@ -307,9 +307,8 @@ __global__ void repack_kernel(const int32_t* __restrict__ codes, int64_t K, int6
     uint32_t out = 0;
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-      const int j = 2 * u + (p >> 1);
-      const int64_t row = 16 * s + ((p & 1) ? 2 * t + 8 : 2 * t);
-      const int64_t w = cb * 8 + j;
+      const int64_t w = cb * 8 + 2 * u + (p & 1);  // column 16u + g + 8 (p & 1) is nibble g of this word
+      const int64_t row = 16 * s + 2 * t + 8 * (p >> 1);
       const uint32_t lo = (static_cast<uint32_t>(__ldg(codes + row * words + w)) >> (4 * g)) & 0xFu;
       const uint32_t hi = (static_cast<uint32_t>(__ldg(codes + (row + 1) * words + w)) >> (4 * g)) & 0xFu;
       out |= (lo << (4 * p)) | (hi << (4 * (p + 4)));
@@ -318,167 +317,221 @@ __global__ void repack_kernel(const int32_t* __restrict__ codes, int64_t K, int6
   }
 }
 
-// The decode GEMV on the repacked codes: as gemv_kernel, but a step is one 16-byte copy per
-// lane into a per-warp ring of kPRing stages in shared memory (cp.async, kPRing - 1 steps
-// ahead, so about 8 KB per warp are in flight), the group's steps and zeros travel in the
-// same ring (16 lanes copy the 64 columns' 128 + 128 bytes with the group's first step),
-// and each fp16 pair costs one shift and one logic op before the packed (1024 + q) -
-// (1024 + z) and the multiply by the step.
-constexpr int kPRing = 16;                          // steps in flight per warp (a power of two)
-constexpr int kPActBytes = 16 * 1024;               // activations staged per CTA when they fit (2 CTAs per SM)
-constexpr int kPRingBytes = kPRing * 32 * 16;       // 8 KB of codes per warp
-// Parameter buffers per warp: a group's steps and zeros are copied with its first step,
-// up to kPRing - 1 steps before that step is computed, and must outlive the whole group,
-// so PB * S > kPRing + S - 2 for S = G / 16 steps per group: 16, 8 and 4 for G = 32, 64, 128.
+// The decode GEMV on the repacked codes, as a persistent stream. The work is the list of
+// chunks (64-column block cb, group g), cb-major, split into equal contiguous runs, one
+// per warp of a grid sized to the SMs: every warp streams the same number of weights (to
+// one chunk), whatever the layer's shape, so no wave is left partly empty. A warp's run
+// crosses column blocks: it keeps one accumulator set, and when its run leaves a block
+// (or ends) it writes its partial sums to that block's slot for this warp, the block's
+// "piece". A second launch adds each block's pieces in warp order (fixed order,
+// deterministic).
+//
+// Per 16-row step a lane copies its 16 bytes (the repacked layout) into a per-warp ring
+// of kPRing stages in shared memory (cp.async, kPRing - 1 steps ahead, continuing across
+// chunks and blocks); a chunk's 64 steps and 64 zeros travel in the same ring with its
+// first step. Each fp16 pair of the B fragments costs one logic op (plus one shift per
+// two pairs, on the multiply pipe) before an exact packed q - z and the multiply by the
+// step.
+constexpr int kPRing = 8;                           // steps in flight per warp (a power of two)
+constexpr int kSActBytes = 32 * 1024;               // the activations are staged when M K halves fit
+constexpr int kPRingBytes = kPRing * 32 * 16;       // 4 KB of codes per warp
+// Parameter buffers per warp: a chunk's steps and zeros are copied with its first step,
+// up to kPRing - 1 steps before that step is computed, and must outlive the whole chunk,
+// so PB * S > kPRing + S - 2 for S = G / 16 steps per chunk: 8, 4 and 2 for G = 32, 64, 128.
 template <int G>
 struct PackedSmem {
   static constexpr int S = G / 16;
-  static constexpr int PB = G == 32 ? 16 : (G == 64 ? 8 : 4);
-  static_assert(PB * S > kPRing + S - 2, "parameter buffers must outlive their group");
-  static constexpr int kParamBytes = PB * 2 * 64 * 2;  // PB groups of 64 steps + 64 zeros (fp16)
+  static constexpr int PB = G == 32 ? 8 : (G == 64 ? 4 : 2);
+  static_assert(PB * S > kPRing + S - 2, "parameter buffers must outlive their chunk");
+  static constexpr int kParamBytes = PB * 2 * 64 * 2;  // PB chunks of 64 steps + 64 zeros (fp16)
   static constexpr int kWarpBytes = kPRingBytes + kParamBytes;
   static constexpr int kSmem = (kGemvThreads / 32) * kWarpBytes;
 };
 
-template <int G>
-__global__ void __launch_bounds__(kGemvThreads)
-    gemv_packed_kernel(const __half* __restrict__ A, int M, const uint4* __restrict__ P,
+// The warp whose run holds chunk l when T chunks are split over W warps (warp w starts at
+// floor(w T / W)): the last warp whose start is <= l.
+__host__ __device__ __forceinline__ int64_t chunk_owner(int64_t l, int64_t T, int64_t W) {
+  return ((l + 1) * W - 1) / T;
+}
+
+template <int G, int NT>
+__global__ void __launch_bounds__(kGemvThreads, NT == 1 ? 3 : 2)
+    gemv_stream_kernel(const __half* __restrict__ A, int M, const uint4* __restrict__ P,
                        const __half* __restrict__ steps, const __half* __restrict__ zeros, int64_t K, int64_t N,
-                       int64_t k_per_split, float* __restrict__ out) {
-  __shared__ float red[kGemvThreads / 32][16][kGemvCols];
+                       int64_t W, int pieces, float* __restrict__ part) {
+  constexpr int S = G / 16;
+  using PS = PackedSmem<G>;
   extern __shared__ __align__(16) uint8_t pdyn[];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int gq = lane >> 2, tq = lane & 3;
-  const int64_t cbs = N / 64, cb = blockIdx.x;
-  const int64_t k0 = static_cast<int64_t>(blockIdx.y) * k_per_split;
-  const int64_t k1 = min(K, k0 + k_per_split);
-  // warps take whole groups of the split (contiguous runs), so parameters change only
-  // between the unrolled steps of one group
-  constexpr int kStepsPerGroup = G / 16;
-  const int n_groups = static_cast<int>((k1 - k0) / G);
-  const int gpw = (n_groups + kGemvThreads / 32 - 1) / (kGemvThreads / 32);
-  const int g_begin = min(n_groups, warp * gpw), g_end = min(n_groups, g_begin + gpw);
-  const int s0 = g_begin * kStepsPerGroup, s1 = g_end * kStepsPerGroup;
-  using PS = PackedSmem<G>;
-  uint8_t* ring = pdyn + warp * PS::kWarpBytes;
-  // the CTA's slice of the activations, staged once when it fits (M k_per_split halves)
+  const int64_t cbs = N / 64, Gk = K / G, T = cbs * Gk;
+  const int64_t wg = static_cast<int64_t>(blockIdx.x) * (kGemvThreads / 32) + warp;
+
+  // the activations, staged once per CTA when they fit (M K halves)
   __half* sAct = reinterpret_cast<__half*>(pdyn + PS::kSmem);
-  const bool staged = static_cast<int64_t>(M) * k_per_split * 2 <= kPActBytes;
+  const bool staged = static_cast<int64_t>(M) * K * 2 <= kSActBytes;
   if (staged) {
-    const int kn = static_cast<int>(k1 - k0);
-    for (int i = threadIdx.x; i < M * (kn / 8); i += kGemvThreads) {
-      const int m = i / (kn / 8), v = i % (kn / 8);
-      *reinterpret_cast<uint4*>(sAct + m * k_per_split + 8 * v) =
-          __ldg(reinterpret_cast<const uint4*>(A + static_cast<int64_t>(m) * K + k0 + 8 * v));
-    }
+    const int64_t vecs = static_cast<int64_t>(M) * K / 8;
+    for (int64_t i = threadIdx.x; i < vecs; i += kGemvThreads)
+      reinterpret_cast<uint4*>(sAct)[i] = __ldg(reinterpret_cast<const uint4*>(A) + i);
     __syncthreads();
   }
+  if (wg >= W) return;  // W <= T: every warp below W has at least one chunk
+  const int64_t l0 = wg * T / W, l1 = (wg + 1) * T / W;
+  uint8_t* ring = pdyn + warp * PS::kWarpBytes;
   __half* params = reinterpret_cast<__half*>(ring + kPRingBytes);  // [PB][2][64]
 
-  float acc[8][4];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
-
-  auto issue = [&](int s) {
-    if (s < s1) {
-      const int64_t gs = k0 / 16 + s;  // global step
-      const uint32_t dst = smem_u32(ring + (s & (kPRing - 1)) * 512 + lane * 16);
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(P + (gs * cbs + cb) * 32 + lane)
-                   : "memory");
-      if (gs % kStepsPerGroup == 0 && lane < 16) {  // runs start on group boundaries
-        const int64_t grp = (gs * 16) / G;
-        const __half* src = (lane < 8 ? steps : zeros) + grp * N + cb * 64 + 8 * (lane & 7);
-        const uint32_t pd = smem_u32(params + (grp & (PS::PB - 1)) * 128 + (lane < 8 ? 0 : 64) + 8 * (lane & 7));
+  // ---- issue side: kPRing - 1 steps ahead of the compute side
+  int64_t i_cb = l0 / Gk, i_g = l0 % Gk, i_l = l0;
+  const uint4* i_ptr = P + (i_g * S * cbs + i_cb) * 32 + lane;
+  // issue(ssi): the step at position ssi of its chunk (ssi is a constant once unrolled)
+  auto issue = [&](int ssi) {
+    if (i_l < l1) {
+      const uint32_t dst = smem_u32(ring + ((i_l * S + ssi) & (kPRing - 1)) * 512 + lane * 16);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(i_ptr) : "memory");
+      if (ssi == 0 && lane < 16) {
+        const __half* src = (lane < 8 ? steps : zeros) + i_g * N + i_cb * 64 + 8 * (lane & 7);
+        const uint32_t pd = smem_u32(params + (i_l & (PS::PB - 1)) * 128 + (lane < 8 ? 0 : 64) + 8 * (lane & 7));
         asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(pd), "l"(src) : "memory");
+      }
+      i_ptr += cbs * 32;
+      if (ssi == S - 1) {  // next chunk
+        ++i_l;
+        if (++i_g == Gk) {
+          i_g = 0;
+          ++i_cb;
+          i_ptr = P + i_cb * 32 + lane;
+        }
       }
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
-#pragma unroll 1
-  for (int q = 0; q < kPRing - 1; ++q) issue(s0 + q);
+#pragma unroll
+  for (int q = 0; q < kPRing - 1; ++q) issue(q % S);
 
-  __half2 z2[8], st2[8];
-  const __half k1024 = __float2half_rn(1024.0f);
-  const __half* sArow0 = sAct + gq * k_per_split + 2 * tq;      // staged activations of token g
-  const __half* sArow1 = sArow0 + 8 * k_per_split;              // and of token g + 8
+  // ---- compute side: acc[i][u] is the 16 x 8 tile of columns 16u .. and tokens 8i ..
+  float acc[NT][4][4];
+#pragma unroll
+  for (int i = 0; i < NT; ++i)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc[i][u][0] = acc[i][u][1] = acc[i][u][2] = acc[i][u][3] = 0.0f;
+  const __half k1024 = __float2half_rn(1024.0f), k64 = __float2half_rn(64.0f);
+  const __half2 sixteenth = __float2half2_rn(0.0625f);
+  const __half* sArow0 = sAct + static_cast<int64_t>(gq) * K + 2 * tq;      // staged row of token g
+  const __half* sArow1 = sArow0 + 8 * K;                                     // and of token g + 8
+  const __half* gArow0 = A + static_cast<int64_t>(gq) * K + 2 * tq;
+  const __half* gArow1 = gArow0 + 8 * K;
+  int64_t c_cb = l0 / Gk, c_g = l0 % Gk;
 #pragma unroll 1
-  for (int gi = g_begin; gi < g_end; ++gi) {
-    const int64_t grp = k0 / G + gi;
+  for (int64_t l = l0; l < l1; ++l) {
+    // per word u: column 16u + g (even pairs: 1024 + z, step) and 16u + g + 8 (odd pairs:
+    // -(64 + z), step)
+    __half2 z2[4], zn2[4], st2[8];
 #pragma unroll
-    for (int ss = 0; ss < kStepsPerGroup; ++ss) {
-      const int s = gi * kStepsPerGroup + ss;
-      issue(s + kPRing - 1);
+    for (int ss = 0; ss < S; ++ss) {
+      issue((ss + kPRing - 1) % S);
       asm volatile("cp.async.wait_group %0;" ::"n"(kPRing - 1) : "memory");
-      __syncwarp();  // the group's steps and zeros were copied by other lanes
+      __syncwarp();  // the chunk's steps and zeros were copied by other lanes
       if (ss == 0) {
-        const __half* pr = params + (grp & (PS::PB - 1)) * 128;
+        const __half* pr = params + (l & (PS::PB - 1)) * 128;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 8; ++j) {  // column 8j + g of the block
           const __half st = pr[8 * j + gq];
-          const __half zb = __hadd(pr[64 + 8 * j + gq], k1024);  // exact: z is an integer <= 15
+          const __half z = pr[64 + 8 * j + gq];
           st2[j] = __halves2half2(st, st);
-          z2[j] = __halves2half2(zb, zb);
+          if (j % 2 == 0) {
+            const __half zb = __hadd(z, k1024);  // 1024 + z, exact: z is an integer <= 15
+            z2[j / 2] = __halves2half2(zb, zb);
+          } else {
+            const __half zn = __hneg(__hadd(z, k64));  // -(64 + z), exact
+            zn2[j / 2] = __halves2half2(zn, zn);
+          }
         }
       }
-      const uint4 v = *reinterpret_cast<const uint4*>(ring + (s & (kPRing - 1)) * 512 + lane * 16);
-      const int kk = 16 * s;  // row offset inside the split
-      uint32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0;
+      const uint4 v = *reinterpret_cast<const uint4*>(ring + ((l * S + ss) & (kPRing - 1)) * 512 + lane * 16);
+      const int64_t kk = (c_g * S + ss) * 16;  // row of the step
+      // B fragments: tokens g (and g + 8), rows 2t, 2t + 1 and 2t + 8, 2t + 9 of the step
+      uint32_t b0 = 0, b1 = 0, b2 = 0, b3 = 0;
       if (staged) {
         if (gq < M) {
-          a0 = *reinterpret_cast<const uint32_t*>(sArow0 + kk);
-          a2 = *reinterpret_cast<const uint32_t*>(sArow0 + kk + 8);
+          b0 = *reinterpret_cast<const uint32_t*>(sArow0 + kk);
+          b1 = *reinterpret_cast<const uint32_t*>(sArow0 + kk + 8);
         }
-        if (gq + 8 < M) {
-          a1 = *reinterpret_cast<const uint32_t*>(sArow1 + kk);
-          a3 = *reinterpret_cast<const uint32_t*>(sArow1 + kk + 8);
+        if (NT == 2 && gq + 8 < M) {
+          b2 = *reinterpret_cast<const uint32_t*>(sArow1 + kk);
+          b3 = *reinterpret_cast<const uint32_t*>(sArow1 + kk + 8);
         }
       } else {
-        const int64_t kb = k0 + kk;
         if (gq < M) {
-          const __half* ar = A + static_cast<int64_t>(gq) * K + kb + 2 * tq;
-          a0 = __ldg(reinterpret_cast<const uint32_t*>(ar));
-          a2 = __ldg(reinterpret_cast<const uint32_t*>(ar + 8));
+          b0 = __ldg(reinterpret_cast<const uint32_t*>(gArow0 + kk));
+          b1 = __ldg(reinterpret_cast<const uint32_t*>(gArow0 + kk + 8));
         }
-        if (gq + 8 < M) {
-          const __half* ar = A + static_cast<int64_t>(gq + 8) * K + kb + 2 * tq;
-          a1 = __ldg(reinterpret_cast<const uint32_t*>(ar));
-          a3 = __ldg(reinterpret_cast<const uint32_t*>(ar + 8));
+        if (NT == 2 && gq + 8 < M) {
+          b2 = __ldg(reinterpret_cast<const uint32_t*>(gArow1 + kk));
+          b3 = __ldg(reinterpret_cast<const uint32_t*>(gArow1 + kk + 8));
         }
       }
       const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
+        // pairs 0, 1 in bits 0-7 of each half, pairs 2, 3 after a shift by 8 (taken on the
+        // multiply pipe as the high word of w * 2^24). Even pair: halves 1024 + q minus
+        // (1024 + z); odd pair: halves 1024 + 16 q times 1/16 minus (64 + z) in one fused
+        // step (every value exact); then times the step.
+        const uint32_t w8 = __umulhi(wv[u], 1u << 24);
+        uint32_t a[4];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const int j = 2 * u + h;
-          uint32_t b[2];
-#pragma unroll
-          for (int which = 0; which < 2; ++which) {
-            const int p = 2 * h + which;
-            const uint32_t biased = ((wv[u] >> (4 * p)) & 0x000F000Fu) | 0x64006400u;  // halves 1024 + q
-            b[which] = half2_as_u32(__hmul2(__hsub2(u32_as_half2(biased), z2[j]), st2[j]));
-          }
-          mma_f16_16816(acc[j], a0, a1, a2, a3, b[0], b[1]);
+          const uint32_t src = h ? w8 : wv[u];
+          const uint32_t lo = (src & 0x000F000Fu) | 0x64006400u;
+          const uint32_t hi = (src & 0x00F000F0u) | 0x64006400u;
+          a[2 * h] = half2_as_u32(__hmul2(__hsub2(u32_as_half2(lo), z2[u]), st2[2 * u]));
+          a[2 * h + 1] = half2_as_u32(__hmul2(__hfma2(u32_as_half2(hi), sixteenth, zn2[u]), st2[2 * u + 1]));
         }
+        mma_f16_16816(acc[0][u], a[0], a[1], a[2], a[3], b0, b1);
+        if (NT == 2) mma_f16_16816(acc[NT - 1][u], a[0], a[1], a[2], a[3], b2, b3);
       }
     }
-    __syncwarp();  // all lanes are past this group's parameters before a later group overwrites them
+    // the chunk is done: leave the column block at its end or at the end of the run
+    if (++c_g == Gk || l + 1 == l1) {
+      const int64_t piece = wg - chunk_owner(c_cb * Gk, T, W);
+      float* dst = part + (c_cb * pieces + piece) * static_cast<int64_t>(M) * 64;
+#pragma unroll
+      for (int i = 0; i < NT; ++i)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          // D rows are columns 16u + g (+ 8), D columns are tokens 8i + 2t (+ 1)
+          const int m0 = 8 * i + 2 * tq, n0 = 16 * u + gq;
+          if (m0 < M) {
+            dst[m0 * 64 + n0] = acc[i][u][0];
+            dst[m0 * 64 + n0 + 8] = acc[i][u][2];
+          }
+          if (m0 + 1 < M) {
+            dst[(m0 + 1) * 64 + n0] = acc[i][u][1];
+            dst[(m0 + 1) * 64 + n0 + 8] = acc[i][u][3];
+          }
+          acc[i][u][0] = acc[i][u][1] = acc[i][u][2] = acc[i][u][3] = 0.0f;
+        }
+      c_g = 0;
+      ++c_cb;
+    }
+    __syncwarp();  // all lanes are past this chunk's parameters before a later chunk overwrites them
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    red[warp][gq][8 * j + 2 * tq] = acc[j][0];
-    red[warp][gq][8 * j + 2 * tq + 1] = acc[j][1];
-    red[warp][gq + 8][8 * j + 2 * tq] = acc[j][2];
-    red[warp][gq + 8][8 * j + 2 * tq + 1] = acc[j][3];
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < M * kGemvCols; i += kGemvThreads) {
-    const int m = i / kGemvCols, c = i % kGemvCols;
-    float sum = red[0][m][c];
-#pragma unroll
-    for (int q = 1; q < kGemvThreads / 32; ++q) sum = __fadd_rn(sum, red[q][m][c]);
-    out[(static_cast<int64_t>(blockIdx.y) * M + m) * N + cb * 64 + c] = sum;
+}
+
+// Y[m][n] = the sum of column block n / 64's pieces, in warp order.
+__global__ void piece_sum_kernel(const float* __restrict__ part, int pieces, int M, int64_t N, int64_t Gk, int64_t W,
+                                 float* __restrict__ Y) {
+  const int64_t MN = static_cast<int64_t>(M) * N, T = (N / 64) * Gk;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < MN;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t m = i / N, n = i % N, cb = n / 64;
+    const int64_t count = chunk_owner(cb * Gk + Gk - 1, T, W) - chunk_owner(cb * Gk, T, W) + 1;
+    const float* src = part + (cb * pieces * M + m) * 64 + n % 64;
+    float s = src[0];
+    for (int64_t q = 1; q < count; ++q) s = __fadd_rn(s, src[q * M * 64]);
+    Y[i] = s;
   }
 }
 
@@ -513,37 +566,69 @@ cudaError_t launch_gemv_g(const W4A16Args& a, int num_sms, float* part, cudaStre
   return cudaGetLastError();
 }
 
-// The repacked kernel gives its warps whole groups: a split holds at least 8 groups when
-// the layer has that many.
-int64_t gemv_packed_splits(int64_t K, int64_t N, int group, int num_sms) {
-  const int64_t col_blocks = N / 64;
-  const int64_t groups = K / group;
-  int64_t splits = std::max<int64_t>(1, std::min<int64_t>(groups / 8, ceil_div(8 * num_sms, col_blocks)));
-  const int64_t gps = ceil_div(groups, splits);
-  return ceil_div(groups, gps);
+template <int G>
+int stream_smem(int64_t M, int64_t K) {
+  return PackedSmem<G>::kSmem + (M * K * 2 <= kSActBytes ? static_cast<int>(M * K * 2) : 0);
+}
+
+// Resident CTAs per SM of a decode variant (queried once, at the largest shared-memory
+// size the launcher uses).
+template <int G, int NT>
+int stream_ctas_per_sm() {
+  static const int per_sm = [] {
+    static unsigned long long done = 0;
+    int n = 0;
+    if (set_smem_limit_once(gemv_stream_kernel<G, NT>, PackedSmem<G>::kSmem + kSActBytes, &done) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_stream_kernel<G, NT>, kGemvThreads,
+                                                      PackedSmem<G>::kSmem + kSActBytes) != cudaSuccess) {
+      cudaGetLastError();
+      n = 1;
+    }
+    return std::max(n, 1);
+  }();
+  return per_sm;
+}
+
+// Warps of the streaming decode: as many CTAs of 8 warps as the SMs hold at once, and
+// never more warps than chunks.
+template <int G>
+int64_t gemv_stream_warps(int64_t M, int64_t K, int64_t N, int num_sms) {
+  const int per_sm = M <= 8 ? stream_ctas_per_sm<G, 1>() : stream_ctas_per_sm<G, 2>();
+  const int64_t T = (N / 64) * (K / G);
+  return std::max<int64_t>(1, std::min<int64_t>(T, static_cast<int64_t>(per_sm) * num_sms * (kGemvThreads / 32)));
+}
+
+// Slots per column block for its pieces: a block's Gk chunks meet at most
+// ceil((Gk - 1) W / T) + 1 warps' runs (the sum kernel uses each block's exact count).
+int gemv_stream_pieces(int64_t K, int64_t N, int group, int64_t W) {
+  const int64_t Gk = K / group, T = (N / 64) * Gk;
+  return static_cast<int>(ceil_div((Gk - 1) * W, T) + 1);
+}
+
+template <int G>
+int64_t gemv_stream_part_floats(int64_t M, int64_t K, int64_t N, int num_sms) {
+  return (N / 64) * gemv_stream_pieces(K, N, G, gemv_stream_warps<G>(M, K, N, num_sms)) * M * 64;
 }
 
 template <int G>
 cudaError_t launch_gemv_packed_g(const W4A16Args& a, const uint32_t* packed, int num_sms, float* part,
                                  cudaStream_t s, int* launches) {
-  const int64_t col_blocks = a.N / 64;
-  const int64_t splits = gemv_packed_splits(a.K, a.N, G, num_sms);
-  const int64_t k_per_split = ceil_div(a.K / G, splits) * G;
-  float* dst = splits == 1 ? a.Y : part;
-  static unsigned long long done = 0;
-  const int smem = PackedSmem<G>::kSmem +
-                   (a.M * k_per_split * 2 <= kPActBytes ? static_cast<int>(a.M * k_per_split * 2) : 0);
-  cudaError_t e0 = set_smem_limit_once(gemv_packed_kernel<G>, PackedSmem<G>::kSmem + kPActBytes, &done);
+  const int64_t W = gemv_stream_warps<G>(a.M, a.K, a.N, num_sms);
+  const int pieces = gemv_stream_pieces(a.K, a.N, G, W);
+  const unsigned ctas = static_cast<unsigned>(ceil_div(W, static_cast<int64_t>(kGemvThreads / 32)));
+  auto kernel = a.M <= 8 ? gemv_stream_kernel<G, 1> : gemv_stream_kernel<G, 2>;
+  static unsigned long long done1 = 0, done2 = 0;  // the limit is per device
+  cudaError_t e0 = set_smem_limit_once(kernel, PackedSmem<G>::kSmem + kSActBytes, a.M <= 8 ? &done1 : &done2);
   if (e0 != cudaSuccess) return e0;
-  gemv_packed_kernel<G><<<dim3(static_cast<unsigned>(col_blocks), static_cast<unsigned>(splits)), kGemvThreads,
-                          smem, s>>>(a.A, static_cast<int>(a.M), reinterpret_cast<const uint4*>(packed), a.steps, a.zeros,
-                               a.K, a.N, k_per_split, dst);
+  kernel<<<ctas, kGemvThreads, stream_smem<G>(a.M, a.K), s>>>(a.A, static_cast<int>(a.M),
+                                                              reinterpret_cast<const uint4*>(packed), a.steps,
+                                                              a.zeros, a.K, a.N, W, pieces, part);
   *launches += 1;
   cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess || splits == 1) return e;
+  if (e != cudaSuccess) return e;
   const int64_t mn = a.M * a.N;
   const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(ceil_div(mn, 256), 4 * num_sms));
-  split_sum_kernel<<<blocks, 256, 0, s>>>(part, static_cast<int>(splits), mn, a.Y);
+  piece_sum_kernel<<<blocks, 256, 0, s>>>(part, pieces, static_cast<int>(a.M), a.N, a.K / G, W, a.Y);
   *launches += 1;
   return cudaGetLastError();
 }
@@ -551,7 +636,14 @@ cudaError_t launch_gemv_packed_g(const W4A16Args& a, const uint32_t* packed, int
 }  // namespace
 
 int64_t gemv_split_floats(int64_t M, int64_t K, int64_t N, int group, int num_sms, bool packed) {
-  const int64_t splits = packed ? gemv_packed_splits(K, N, group, num_sms) : gemv_splits(K, N, group, num_sms);
+  if (packed) {
+    switch (group) {
+      case 32: return gemv_stream_part_floats<32>(M, K, N, num_sms);
+      case 64: return gemv_stream_part_floats<64>(M, K, N, num_sms);
+      default: return gemv_stream_part_floats<128>(M, K, N, num_sms);
+    }
+  }
+  const int64_t splits = gemv_splits(K, N, group, num_sms);
   return splits > 1 ? splits * M * N : 0;
 }
 
