@@ -251,11 +251,13 @@ int awq_w4a16_matmul(const void* A, const int32_t* codes, const void* steps,
 float awq_w4a16_profile_last(void);
 /* Decode on repacked codes. awq_w4a16_repack rewrites the artifact's codes (K x N/8
  * int32; K % 32 == 0, N % 64 == 0) once, e.g. at load time, into the order the decode
- * kernel reads them: for every 16 rows, 64 columns and MMA lane, 16 contiguous bytes,
- * nibbles arranged so that one shift and one mask give an fp16 pair. Same size as the
- * codes; synchronizes `stream`. awq_w4a16_matmul_packed is awq_w4a16_matmul for M <= 16
- * on that layout (same result definition, steps and zeros unchanged), asynchronous on
- * `stream`. */
+ * kernel reads them: for every 16 rows, 64 columns and MMA lane, 16 contiguous bytes in
+ * the A-fragment order of 16 x 8 x 16 MMAs whose A operand is the weights (16 columns by
+ * 16 rows), nibbles arranged so that one mask (plus one shift per two pairs) gives an
+ * fp16 pair. Same size as the codes; synchronizes `stream`. A layout written by an older
+ * build is not compatible: repack again. awq_w4a16_matmul_packed is awq_w4a16_matmul for
+ * M <= 16 on that layout (same result definition, steps and zeros unchanged; fixed-order,
+ * deterministic sums), asynchronous on `stream`. */
 int awq_w4a16_repack(const int32_t* codes, int64_t K, int64_t N, int32_t* out_packed,
                      awq_stream_t stream);
 int awq_w4a16_matmul_packed(const void* A, const int32_t* packed, const void* steps,
