@@ -125,6 +125,18 @@ int awq_search_host(const void* X_host, const void* W_host, int in_dtype, int64_
                     int64_t K, int64_t N, int group, int n_grid, float* out_scales_host,
                     int32_t* out_codes_host, void* out_steps_host, void* out_zeros_host,
                     float* out_losses_host, awq_stream_t stream);
+/* The same for n_layers layers of one shape (X_hosts[i] M x K, W_hosts[i] K x N; the
+ * output arrays hold one host pointer per layer, out_losses_host or its entries may be
+ * NULL). Layer i + 1's inputs are copied to the device while layer i is searched (two
+ * device slots) and layer i's artifact is copied back while layer i + 1 runs, so with
+ * pinned host memory the transfers hide behind the searches. Returns when every output
+ * has landed; stops at the first failing layer and returns its status (the outputs of
+ * the layers before it are complete). */
+int awq_search_host_batch(int n_layers, const void* const* X_hosts, const void* const* W_hosts,
+                          int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid,
+                          float* const* out_scales_host, int32_t* const* out_codes_host,
+                          void* const* out_steps_host, void* const* out_zeros_host,
+                          float* const* out_losses_host, awq_stream_t stream);
 
 /* ---- The steps one at a time (same kernels as awq_search; device pointers) ----
  * Step 1 (AWQ-P1 §1): out_a[K] = mean_m |X[m,j]| (fp64 sum, one rounding to fp32).

@@ -19,7 +19,7 @@ from dataclasses import dataclass
 import torch
 
 __all__ = [
-    "AwqError", "SearchOutput", "search", "search_host", "library", "library_path", "header_path",
+    "AwqError", "SearchOutput", "search", "search_host", "search_host_batch", "library", "library_path", "header_path",
     "tile_shape", "workspace_bytes", "release_cached", "profile_enable", "profile_last",
     "last_launch_count", "debug_set_fault", "status_string", "exported_functions",
     "activation_statistic", "candidate_scales", "qdq_candidates", "ClipOutput", "clip_search",
@@ -65,7 +65,9 @@ def library() -> ctypes.CDLL:
     lib.awq_search_f32.argtypes = [vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp]
     lib.awq_search_ex.argtypes = [vp, vp, i32, i64, i64, i64, i32, i32, vp, vp, vp, vp, f32p, f64p, i64, vp]
     lib.awq_search_host.argtypes = [vp, vp, i32, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp]
-    for name in ("awq_search", "awq_search_f32", "awq_search_ex", "awq_search_host", "awq_release_cached",
+    lib.awq_search_host_batch.argtypes = [i32, vp, vp, i32, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp]
+    for name in ("awq_search", "awq_search_f32", "awq_search_ex", "awq_search_host", "awq_search_host_batch",
+                 "awq_release_cached",
                  "awq_profile_enable", "awq_profile_last", "awq_last_launch_count", "awq_debug_set_fault",
                  "awq_version"):
         getattr(lib, name).restype = ctypes.c_int
@@ -309,6 +311,41 @@ def search_host(X: torch.Tensor, W: torch.Tensor, group: int = 128, n_grid: int 
                              _ptr(steps), _ptr(zeros), _ptr(losses), _stream_handle(stream, dev))
     _check(st)
     return SearchOutput(scales, codes, steps, zeros, losses)
+
+
+def search_host_batch(Xs: list, Ws: list, group: int = 128, n_grid: int = 20, *,
+                      stream: torch.cuda.Stream | None = None, outs: list | None = None,
+                      device: int | torch.device | None = None) -> list:
+    """search_host() for several layers of one shape: layer i + 1's inputs are copied while
+    layer i is searched and layer i's artifact is copied back while layer i + 1 runs."""
+    if len(Xs) != len(Ws) or not Xs:
+        raise ValueError("Xs and Ws must be equally long, non-empty lists")
+    X0, W0 = Xs[0], Ws[0]
+    for X, W in zip(Xs, Ws):
+        if X.is_cuda or W.is_cuda:
+            raise ValueError("search_host_batch() takes host tensors")
+        if X.dtype != X0.dtype or W.dtype != X0.dtype or X.shape != X0.shape or W.shape != W0.shape:
+            raise TypeError("every layer needs the same shapes and dtype")
+    Xs = [X.contiguous() for X in Xs]
+    Ws = [W.contiguous() for W in Ws]
+    M, K = X0.shape
+    N = W0.shape[1]
+    if outs is None:
+        outs = [_alloc_outputs(K, N, group, n_grid, None, pin=True) for _ in Xs]
+    if len(outs) != len(Xs):
+        raise ValueError("outs needs one output tuple per layer")
+    n = len(Xs)
+
+    def arr(ptrs):
+        return (ctypes.c_void_p * n)(*ptrs)
+
+    keep = [arr([_ptr(x) for x in Xs]), arr([_ptr(w) for w in Ws])] + [arr([_ptr(o[k]) for o in outs])
+                                                                        for k in range(5)]
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    st = library().awq_search_host_batch(n, keep[0], keep[1], _dtype_code(X0), M, K, N, group, n_grid, keep[2],
+                                         keep[3], keep[4], keep[5], keep[6], _stream_handle(stream, dev))
+    _check(st)
+    return [SearchOutput(*o) for o in outs]
 
 
 @dataclass

@@ -565,6 +565,154 @@ int awq_search_host(const void* X_host, const void* W_host, int in_dtype, int64_
   return status;
 }
 
+// ---- many layers from host memory, transfers overlapped with the searches -------------
+// Inputs go through two device slots: while layer i is searched on `stream`, a copy stream
+// uploads layer i + 1 into the other slot (X, then W in chunks the search consumes as they
+// land), and a third stream copies layer i's artifact back while layer i + 1 runs.
+int awq_search_host_batch(int n_layers, const void* const* X_hosts, const void* const* W_hosts, int in_dtype,
+                          int64_t M, int64_t K, int64_t N, int group, int n_grid, float* const* out_scales_host,
+                          int32_t* const* out_codes_host, void* const* out_steps_host, void* const* out_zeros_host,
+                          float* const* out_losses_host, awq_stream_t stream) {
+  t_last_error.clear();
+  if (n_layers < 1 || !X_hosts || !W_hosts || !out_scales_host || !out_codes_host || !out_steps_host ||
+      !out_zeros_host)
+    return set_error(AWQ_ERR_INVALID_ARG, "n_layers must be >= 1 and the pointer arrays non-null");
+  for (int i = 0; i < n_layers; ++i) {
+    const int st = validate(X_hosts[i], W_hosts[i], in_dtype, M, K, N, group, n_grid, out_scales_host[i],
+                            out_codes_host[i], out_steps_host[i], out_zeros_host[i], false);
+    if (st != AWQ_OK) return st;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  bind_device(s, nullptr);
+  int dev = 0, num_sms = 0;
+  int st = check_device(&dev, &num_sms);
+  if (st != AWQ_OK) return st;
+  cudaMemPool_t pool;
+  if ((st = get_pool(dev, &pool)) != AWQ_OK) return st;
+  const size_t eb = in_dtype == AWQ_DTYPE_BF16 ? 2 : 4;
+  const size_t G = static_cast<size_t>(K / group);
+  const size_t bx = static_cast<size_t>(M) * K * eb, bw = static_cast<size_t>(K) * N * eb;
+  const size_t bs = static_cast<size_t>(K) * 4, bc = static_cast<size_t>(K) * (N / 8) * 4;
+  const size_t bst = G * N * 2, bl = static_cast<size_t>(n_grid) * 4;
+  // per slot: X, W, scales, codes, steps, zeros, losses
+  const size_t sizes[7] = {bx, bw, bs, bc, bst, bst, bl};
+  size_t off[7], slot_bytes = 0;
+  for (int k = 0; k < 7; ++k) {
+    off[k] = slot_bytes;
+    slot_bytes += align_up(sizes[k]);
+  }
+  constexpr int kChunks = CopyLane::kChunks;
+  struct Slot {
+    cudaEvent_t x_ready = nullptr, in_free = nullptr, out_done = nullptr, w_ready[kChunks] = {};
+  } slots[2];
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t alloc_done = nullptr, search_done = nullptr, h2d_done = nullptr, d2h_done = nullptr;
+  bool ok = cudaStreamCreateWithFlags(&h2d, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&d2h, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&alloc_done, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&search_done, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&h2d_done, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&d2h_done, cudaEventDisableTiming) == cudaSuccess;
+  for (auto& sl : slots) {
+    ok = ok && cudaEventCreateWithFlags(&sl.x_ready, cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&sl.in_free, cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&sl.out_done, cudaEventDisableTiming) == cudaSuccess;
+    for (auto& ev : sl.w_ready) ok = ok && cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) == cudaSuccess;
+  }
+  void* buf = nullptr;
+  int status = AWQ_OK;
+  cudaError_t e = cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    status = set_error(AWQ_ERR_CUDA, "could not create the batch's streams and events");
+  } else if ((e = cudaMallocFromPoolAsync(&buf, 2 * slot_bytes, pool, s)) != cudaSuccess || !buf) {
+    cudaGetLastError();
+    buf = nullptr;
+    status = set_error(AWQ_ERR_OOM, "device slots for the batch");
+  }
+  const int chunks = static_cast<int>(std::min<size_t>(kChunks, G));
+  const int64_t groups_per_chunk = static_cast<int64_t>((G + chunks - 1) / chunks);
+  const size_t chunk_bytes = static_cast<size_t>(groups_per_chunk) * group * N * eb;
+  auto slot_ptr = [&](int i, int k) { return static_cast<uint8_t*>(buf) + (i & 1) * slot_bytes + off[k]; };
+  // uploads of layer i into slot i % 2, once the search of layer i - 2 is done with it
+  auto upload = [&](int i) -> cudaError_t {
+    Slot& sl = slots[i & 1];
+    cudaError_t r = i >= 2 ? cudaStreamWaitEvent(h2d, sl.in_free, 0) : cudaSuccess;
+    if (r == cudaSuccess) r = cudaMemcpyAsync(slot_ptr(i, 0), X_hosts[i], bx, cudaMemcpyHostToDevice, h2d);
+    if (r == cudaSuccess) r = cudaEventRecord(sl.x_ready, h2d);
+    for (int c = 0; c < chunks && r == cudaSuccess; ++c) {
+      const size_t at = static_cast<size_t>(c) * chunk_bytes;
+      const size_t n = std::min(chunk_bytes, bw - std::min(bw, at));
+      if (n > 0)
+        r = cudaMemcpyAsync(slot_ptr(i, 1) + at, static_cast<const uint8_t*>(W_hosts[i]) + at, n,
+                            cudaMemcpyHostToDevice, h2d);
+      if (r == cudaSuccess) r = cudaEventRecord(sl.w_ready[c], h2d);
+    }
+    return r;
+  };
+  if (status == AWQ_OK) {
+    if ((e = cudaEventRecord(alloc_done, s)) != cudaSuccess || (e = cudaStreamWaitEvent(h2d, alloc_done, 0)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(d2h, alloc_done, 0)) != cudaSuccess || (e = upload(0)) != cudaSuccess)
+      status = cuda_error(e, "host-to-device copy");
+  }
+  for (int i = 0; i < n_layers && status == AWQ_OK; ++i) {
+    Slot& sl = slots[i & 1];
+    if (i + 1 < n_layers && (e = upload(i + 1)) != cudaSuccess) {
+      status = cuda_error(e, "host-to-device copy");
+      break;
+    }
+    if (i >= 2 && (e = cudaStreamWaitEvent(s, sl.out_done, 0)) != cudaSuccess) {
+      status = cuda_error(e, "stream wait");
+      break;
+    }
+    HostFeed feed;
+    feed.chunks = chunks;
+    feed.groups_per_chunk = groups_per_chunk;
+    feed.x_ready = sl.x_ready;
+    feed.w_ready = sl.w_ready;
+    status = search_device(slot_ptr(i, 0), slot_ptr(i, 1), in_dtype, M, K, N, group, n_grid,
+                           reinterpret_cast<float*>(slot_ptr(i, 2)), reinterpret_cast<int32_t*>(slot_ptr(i, 3)),
+                           slot_ptr(i, 4), slot_ptr(i, 5), reinterpret_cast<float*>(slot_ptr(i, 6)), nullptr, 0, s,
+                           &feed);
+    if (status != AWQ_OK) break;
+    if ((e = cudaEventRecord(sl.in_free, s)) != cudaSuccess || (e = cudaEventRecord(search_done, s)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(d2h, search_done, 0)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(out_scales_host[i], slot_ptr(i, 2), bs, cudaMemcpyDeviceToHost, d2h)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(out_codes_host[i], slot_ptr(i, 3), bc, cudaMemcpyDeviceToHost, d2h)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(out_steps_host[i], slot_ptr(i, 4), bst, cudaMemcpyDeviceToHost, d2h)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(out_zeros_host[i], slot_ptr(i, 5), bst, cudaMemcpyDeviceToHost, d2h)) != cudaSuccess ||
+        (out_losses_host && out_losses_host[i] &&
+         (e = cudaMemcpyAsync(out_losses_host[i], slot_ptr(i, 6), bl, cudaMemcpyDeviceToHost, d2h)) != cudaSuccess) ||
+        (e = cudaEventRecord(sl.out_done, d2h)) != cudaSuccess) {
+      status = cuda_error(e, "device-to-host copy");
+      break;
+    }
+  }
+  // both copy streams are done with the slots before they return to the pool
+  if (h2d && d2h && alloc_done) {
+    cudaEventRecord(h2d_done, h2d);
+    cudaEventRecord(d2h_done, d2h);
+    cudaStreamWaitEvent(s, h2d_done, 0);
+    cudaStreamWaitEvent(s, d2h_done, 0);
+  }
+  if (buf) cudaFreeAsync(buf, s);
+  cudaError_t se = cudaStreamSynchronize(s);
+  if (h2d) cudaStreamSynchronize(h2d);
+  if (d2h) cudaStreamSynchronize(d2h);
+  if (status == AWQ_OK && se != cudaSuccess) status = cuda_error(se, "stream synchronize");
+  for (auto& sl : slots) {
+    for (cudaEvent_t ev : {sl.x_ready, sl.in_free, sl.out_done})
+      if (ev) cudaEventDestroy(ev);
+    for (cudaEvent_t ev : sl.w_ready)
+      if (ev) cudaEventDestroy(ev);
+  }
+  for (cudaEvent_t ev : {alloc_done, search_done, h2d_done, d2h_done})
+    if (ev) cudaEventDestroy(ev);
+  if (h2d) cudaStreamDestroy(h2d);
+  if (d2h) cudaStreamDestroy(d2h);
+  return status;
+}
+
 // ---- the steps one at a time (same kernels as the search) --------------------------
 int awq_activation_statistic(const void* X, int in_dtype, int64_t M, int64_t K, float* out_a, awq_stream_t stream) {
   t_last_error.clear();

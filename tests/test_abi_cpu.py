@@ -22,7 +22,8 @@ def lib():
 
 def test_header_declares_the_search_entry_points():
     names = awq.exported_functions()
-    for required in ("awq_search", "awq_search_f32", "awq_search_ex", "awq_search_host", "awq_status_string"):
+    for required in ("awq_search", "awq_search_f32", "awq_search_ex", "awq_search_host", "awq_search_host_batch",
+                     "awq_status_string"):
         assert required in names
 
 

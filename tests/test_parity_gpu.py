@@ -104,6 +104,17 @@ def test_host_entry_point_matches_device_entry_point():
         assert torch.equal(getattr(d, name).cpu(), getattr(h, name)), name
 
 
+def test_host_batch_matches_one_layer_at_a_time():
+    """Five layers through the batched host entry point (inputs of layer i + 1 uploaded
+    while layer i runs, two device slots reused) give each layer's own artifact."""
+    layers = [generate(custom_spec(256, 384, 520, seed=20 + i)) for i in range(5)]
+    outs = awq.search_host_batch([X.pin_memory() for X, _ in layers], [W.pin_memory() for _, W in layers])
+    for (X, W), o in zip(layers, outs):
+        d = awq.search(X.cuda(), W.cuda())
+        for name in ("scales", "codes", "steps", "zeros", "losses"):
+            assert torch.equal(getattr(d, name).cpu(), getattr(o, name)), name
+
+
 def test_nonfinite_inputs_are_rejected():
     spec = custom_spec(64, 128, 64, seed=3)
     X, W = generate(spec)
