@@ -129,9 +129,11 @@ int awq_search_host(const void* X_host, const void* W_host, int in_dtype, int64_
  * output arrays hold one host pointer per layer, out_losses_host or its entries may be
  * NULL). Layer i + 1's inputs are copied to the device while layer i is searched (two
  * device slots) and layer i's artifact is copied back while layer i + 1 runs, so with
- * pinned host memory the transfers hide behind the searches. Returns when every output
- * has landed; stops at the first failing layer and returns its status (the outputs of
- * the layers before it are complete). */
+ * pinned host memory the transfers hide behind the searches. The whole batch is enqueued
+ * at once and the call returns when every output has landed. A layer whose kernels
+ * report a problem (non-finite input, a bounded wait that ran out) does not stop the
+ * others: the call returns the status of the first such layer, and that layer's outputs
+ * are undefined; an error while enqueueing stops the batch there. */
 int awq_search_host_batch(int n_layers, const void* const* X_hosts, const void* const* W_hosts,
                           int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid,
                           float* const* out_scales_host, int32_t* const* out_codes_host,

@@ -282,10 +282,19 @@ struct HostFeed {
   int64_t groups_per_chunk = 0;
 };
 
+// The call's status from the device status word the kernels set.
+int status_from_word(int h_err) {
+  if (h_err & kErrTimeout) return set_error(AWQ_ERR_TIMEOUT, "a bounded wait in the loss GEMM ran out");
+  if (h_err & (kErrNonfiniteX | kErrNonfiniteW))
+    return set_error(AWQ_ERR_NONFINITE, (h_err & kErrNonfiniteX) ? "non-finite value in X" : "non-finite value in W");
+  if (h_err) return set_error(AWQ_ERR_CUDA, "device status word " + std::to_string(h_err));
+  return AWQ_OK;
+}
+
 int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid,
                   float* out_scales, int32_t* out_codes, void* out_steps, void* out_zeros, float* out_losses,
                   double* out_tile_sq_err, int64_t tile_sq_err_len, cudaStream_t s, const HostFeed* feed = nullptr,
-                  int quantizer = kQuantAsym) {
+                  int quantizer = kQuantAsym, int* async_status = nullptr) {
   if (quantizer != kQuantAsym && quantizer != kQuantSym)
     return set_error(AWQ_ERR_INVALID_ARG, "quantizer must be AWQ_QUANT_ASYM or AWQ_QUANT_SYM");
   int st = validate(X, W, in_dtype, M, K, N, group, n_grid, out_scales, out_codes, out_steps, out_zeros, true);
@@ -419,6 +428,17 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
     }
   } while (false);
 
+  if (async_status) {
+    // the caller reads the device status word later (pinned host memory), after a sync
+    if (status == AWQ_OK && e == cudaSuccess) {
+      e = cudaMemcpyAsync(async_status, err, sizeof(int), cudaMemcpyDeviceToHost, s);
+      if (e != cudaSuccess) where = "status read-back";
+    }
+    if (status == AWQ_OK && e != cudaSuccess) status = cuda_error(e, where);
+    cudaFreeAsync(ws, s);
+    g_last_launches = launches;
+    return status;
+  }
   int h_err = 0;
   int* pinned = pinned_status_word(dev);
   int* status_dst = pinned ? pinned : &h_err;
@@ -434,12 +454,7 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
   if (status == AWQ_OK) {
     ev.collect();
     g_last_launches = launches;
-    if (h_err & kErrTimeout)
-      status = set_error(AWQ_ERR_TIMEOUT, "a bounded wait in the loss GEMM ran out");
-    else if (h_err & (kErrNonfiniteX | kErrNonfiniteW))
-      status = set_error(AWQ_ERR_NONFINITE, (h_err & kErrNonfiniteX) ? "non-finite value in X" : "non-finite value in W");
-    else if (h_err)
-      status = set_error(AWQ_ERR_CUDA, "device status word " + std::to_string(h_err));
+    status = status_from_word(h_err);
   }
   return status;
 }
@@ -567,8 +582,10 @@ int awq_search_host(const void* X_host, const void* W_host, int in_dtype, int64_
 
 // ---- many layers from host memory, transfers overlapped with the searches -------------
 // Inputs go through two device slots: while layer i is searched on `stream`, a copy stream
-// uploads layer i + 1 into the other slot (X, then W in chunks the search consumes as they
-// land), and a third stream copies layer i's artifact back while layer i + 1 runs.
+// uploads layer i + 1 into the other slot (X, then W in chunks the first search consumes
+// as they land), and a third stream copies layer i's artifact back while layer i + 1 runs.
+// The whole batch is enqueued without host waits (events order the slots' reuse); each
+// layer's device status word lands in pinned memory and is read after the final sync.
 int awq_search_host_batch(int n_layers, const void* const* X_hosts, const void* const* W_hosts, int in_dtype,
                           int64_t M, int64_t K, int64_t N, int group, int n_grid, float* const* out_scales_host,
                           int32_t* const* out_codes_host, void* const* out_steps_host, void* const* out_zeros_host,
@@ -620,11 +637,17 @@ int awq_search_host_batch(int n_layers, const void* const* X_hosts, const void* 
     for (auto& ev : sl.w_ready) ok = ok && cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) == cudaSuccess;
   }
   void* buf = nullptr;
+  int* words = nullptr;  // pinned: each layer's device status word, read after the final sync
   int status = AWQ_OK;
   cudaError_t e = cudaSuccess;
   if (!ok) {
     cudaGetLastError();
     status = set_error(AWQ_ERR_CUDA, "could not create the batch's streams and events");
+  } else if (cudaMallocHost(reinterpret_cast<void**>(&words), static_cast<size_t>(n_layers) * sizeof(int)) !=
+             cudaSuccess) {
+    cudaGetLastError();
+    words = nullptr;
+    status = set_error(AWQ_ERR_OOM, "pinned status words for the batch");
   } else if ((e = cudaMallocFromPoolAsync(&buf, 2 * slot_bytes, pool, s)) != cudaSuccess || !buf) {
     cudaGetLastError();
     buf = nullptr;
@@ -665,15 +688,23 @@ int awq_search_host_batch(int n_layers, const void* const* X_hosts, const void* 
       status = cuda_error(e, "stream wait");
       break;
     }
+    // the first layer is searched as its inputs land (X, then W chunk by chunk); later
+    // layers were uploaded during the previous search, so they wait for their whole
+    // upload and quantize W in one launch
     HostFeed feed;
     feed.chunks = chunks;
     feed.groups_per_chunk = groups_per_chunk;
     feed.x_ready = sl.x_ready;
     feed.w_ready = sl.w_ready;
+    if (i > 0 && ((e = cudaStreamWaitEvent(s, sl.x_ready, 0)) != cudaSuccess ||
+                  (e = cudaStreamWaitEvent(s, sl.w_ready[chunks - 1], 0)) != cudaSuccess)) {
+      status = cuda_error(e, "stream wait");
+      break;
+    }
     status = search_device(slot_ptr(i, 0), slot_ptr(i, 1), in_dtype, M, K, N, group, n_grid,
                            reinterpret_cast<float*>(slot_ptr(i, 2)), reinterpret_cast<int32_t*>(slot_ptr(i, 3)),
                            slot_ptr(i, 4), slot_ptr(i, 5), reinterpret_cast<float*>(slot_ptr(i, 6)), nullptr, 0, s,
-                           &feed);
+                           i == 0 ? &feed : nullptr, kQuantAsym, words + i);
     if (status != AWQ_OK) break;
     if ((e = cudaEventRecord(sl.in_free, s)) != cudaSuccess || (e = cudaEventRecord(search_done, s)) != cudaSuccess ||
         (e = cudaStreamWaitEvent(d2h, search_done, 0)) != cudaSuccess ||
@@ -700,6 +731,9 @@ int awq_search_host_batch(int n_layers, const void* const* X_hosts, const void* 
   if (h2d) cudaStreamSynchronize(h2d);
   if (d2h) cudaStreamSynchronize(d2h);
   if (status == AWQ_OK && se != cudaSuccess) status = cuda_error(se, "stream synchronize");
+  // the first layer whose kernels reported a problem decides the status
+  for (int i = 0; i < n_layers && status == AWQ_OK && words; ++i) status = status_from_word(words[i]);
+  if (words) cudaFreeHost(words);
   for (auto& sl : slots) {
     for (cudaEvent_t ev : {sl.x_ready, sl.in_free, sl.out_done})
       if (ev) cudaEventDestroy(ev);
