@@ -92,7 +92,7 @@ Layout plan(int in_dtype, int64_t M, int64_t K, int64_t N, int n_grid, int num_s
   L.row_chunks = statistic_row_chunks(M, K, in_dtype, num_sms);
   const int64_t tiles_m = ceil_div(M, kTileM), tiles_n = ceil_div(N, kTileN);
   L.tiles = tiles_m * tiles_n;
-  L.err = take(16);
+  L.err = take(16 + static_cast<size_t>(L.tiles) * 4);  // status word, then the loss GEMM's per-tile flags
   L.a = take(static_cast<size_t>(K) * 4);
   L.stat_partial = take(static_cast<size_t>(L.row_chunks) * K * 8);
   L.S = take(static_cast<size_t>(n_grid) * K * 4);
@@ -343,7 +343,11 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
   const char* where = "";
   int status = AWQ_OK;
   do {
-    if ((e = cudaMemsetAsync(err, 0, 16, s)) != cudaSuccess) { where = "cudaMemsetAsync"; break; }
+    // the status word and the loss GEMM's per-tile flags
+    if ((e = cudaMemsetAsync(err, 0, 16 + static_cast<size_t>(L.tiles) * 4, s)) != cudaSuccess) {
+      where = "cudaMemsetAsync";
+      break;
+    }
     if (feed && (e = cudaStreamWaitEvent(s, feed->x_ready, 0)) != cudaSuccess) { where = "waiting for X"; break; }
     ev.mark(kPhStatistic);
     if ((e = launch_statistic(X, in_dtype, M, K, L.row_chunks, stat_partial, a, err, s, &launches)) != cudaSuccess) {
@@ -399,9 +403,16 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
       break;
     }
     ev.mark(kPhGemmY);
-    if ((e = launch_loss_gemm(ga, mapA, mapB, 0, s, &launches)) != cudaSuccess) { where = "reference GEMM"; break; }
-    ev.mark(kPhGemmLoss);
-    if ((e = launch_loss_gemm(ga, mapA, mapB, 1, s, &launches)) != cudaSuccess) { where = "loss GEMM"; break; }
+    if (ga.variant == 1) {
+      // one launch: the reference tiles first, each candidate tile waits for its tile of Y
+      ga.ready = err + 4;
+      ev.mark(kPhGemmLoss);
+      if ((e = launch_loss_gemm(ga, mapA, mapB, 4, s, &launches)) != cudaSuccess) { where = "loss GEMM"; break; }
+    } else {
+      if ((e = launch_loss_gemm(ga, mapA, mapB, 0, s, &launches)) != cudaSuccess) { where = "reference GEMM"; break; }
+      ev.mark(kPhGemmLoss);
+      if ((e = launch_loss_gemm(ga, mapA, mapB, 1, s, &launches)) != cudaSuccess) { where = "loss GEMM"; break; }
+    }
     ev.mark(kPhReduce);
     if ((e = launch_loss_reduce(loss_partial, L.tiles, n_grid, M, N, losses, s, &launches)) != cudaSuccess) {
       where = "loss reduction kernel";

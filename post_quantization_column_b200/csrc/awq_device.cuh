@@ -156,6 +156,32 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// A flag another CTA of the same grid publishes: st.release.gpu after the data it
+// guards, ld.acquire.gpu before the data is read (through L2, not the L1 cache).
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Waits until *flag is non-zero; gives up when `*abort` becomes non-zero or after
+// `budget_ns` nanoseconds.
+__device__ __forceinline__ bool flag_wait_bounded(const int* flag, volatile int* abort, uint64_t budget_ns) {
+  if (ld_acquire_gpu(flag)) return true;
+  const uint64_t t0 = global_timer_ns();
+  uint32_t spins = 0;
+  while (true) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(flag)) return true;
+    if (++spins % 16u == 0u) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > budget_ns) return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------------
 // TMA (no multicast anywhere in this library)
 // ---------------------------------------------------------------------------------

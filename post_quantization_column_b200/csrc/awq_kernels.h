@@ -73,6 +73,7 @@ struct LossGemmArgs {
   int a_slotted = 0;           // A is a stack of a_slots operands [a_slots][M][K]; c reads a_slot_base + c
   int a_slot_base = 0;
   int a_slots = 1;
+  int* ready = nullptr;        // mode 4: per-tile flags (tiles_m * tiles_n ints), zero at launch
 };
 // Which loss GEMM runs for a search of this size: 1 = the one-SM kernel (every size; it
 // measured as fast or faster than the pair kernel on every workload), 2 = the two-SM
@@ -87,6 +88,8 @@ cudaError_t make_operand_maps(const LossGemmArgs& a, CUtensorMap* mapA, CUtensor
 // mode 0: Y = X_b W_b into the tiled buffer; mode 1: per-tile sum of (X_b W_hat_i - Y)^2;
 // mode 2: Y = X_b Wt[0]^T written row-major fp32 into a.Y (M x N, pitch N), always on
 // the one-SM kernel (make the maps with b_box_rows = kTileN);
+// mode 4: modes 0 and 1 in one launch (reference tiles first, flags in a.ready; one-SM
+// kernel only; the grid never exceeds the SMs, so every awaited flag belongs to a running CTA);
 // mode 3: the MLP block's first GEMM with the silu-mul fused in its epilogue: the B slot
 // holds [W_gate | W_up] interleaved by 128 columns (launch_qdq's `interleave`), and
 // h = bf16(fl32(silu(g) u)) is written row-major into a.H (M x N/2), one-SM kernel only.

@@ -9,6 +9,12 @@
 //           partial sum. The candidate output Y_hat is never written to HBM;
 //   mode 2: a plain product A B^T (B stored K-major), written row-major in fp32 with
 //           the ragged rows and columns masked (the packed artifact's consumer);
+//   mode 4: modes 0 and 1 in one launch: units 0 .. tiles - 1 are the reference tiles
+//           (B slot 0), the rest the candidates' (slot 1 + c). A reference tile's epilogue
+//           publishes a per-tile flag after its Y stores; a candidate tile's epilogue waits
+//           for the flag (bounded) before it reads Y. Every CTA finishes its reference tiles
+//           before it starts a candidate tile, and the grid never exceeds the SMs (one CTA
+//           each), so every flag a CTA waits for is set by a CTA that is running;
 //   mode 3: the MLP block's first GEMM, B = [W_gate | W_up] interleaved by 128 columns so
 //           that a 256-column tile holds the gate and up halves of 128 intermediate
 //           columns; the epilogue writes h = bf16(silu(g) u) row-major and never stores
@@ -62,7 +68,8 @@ struct GemmParams {
   int b_per_cand;     // modes 1, 3: B slot = slot_base + c (1) or slot_base for every c (0)
   int a_slotted;      // A is a stack of slots (3-D map); candidate c reads slot a_slot_base + c
   int a_slot_base;
-  float* Y;           // modes 0-1: the tiled reference output; mode 2: the row-major output
+  float* Y;           // modes 0, 1, 4: the tiled reference output; mode 2: the row-major output
+  int* ready;         // mode 4: per-tile flags, zero at launch, set once a reference tile is in Y
   __nv_bfloat16* H;   // mode 3: the row-major bf16 intermediate of candidate 0 (pitch ldo)
   int64_t h_stride;   // mode 3: elements between successive candidates' intermediates
   double* partial;
@@ -143,7 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
-  const int64_t n_units = (p.mode == 1 || p.mode == 3 ? p.cands : 1) * tiles;
+  const int64_t n_units = (p.mode == 1 || p.mode == 3 ? p.cands : (p.mode == 4 ? p.n_grid + 1 : 1)) * tiles;
   const uint64_t budget = p.timeout_ns;
 
   auto fail = [&]() {
@@ -158,16 +165,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       uint32_t issued = 0, last_parity = 0;  // per-stage bits
       bool ok = true;
+      bool fault_pending = p.fault_mode == 1;
       for (int64_t u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         int c, mt, nt;
         unit_coords(u, p, c, mt, nt);
-        const int slot = p.mode == 0 ? 0 : p.slot_base + ((p.mode == 1 || p.mode == 3) && p.b_per_cand ? c : 0);
+        const int slot = p.mode == 0 ? 0
+                         : p.mode == 4 ? c  // 0: bf16(W), then candidate c - 1 in slot c
+                                       : p.slot_base + ((p.mode == 1 || p.mode == 3) && p.b_per_cand ? c : 0);
         for (int kb = 0; kb < p.nk; ++kb) {
           if (!mbar_wait_bounded(empty + stage, phase ^ 1u, abort_flag, budget)) {
             ok = false;
             break;
           }
-          const bool skip = p.fault_mode == 1 && p.mode == 1 && u == blockIdx.x && kb == 0;
+          // fault injection: the first candidate unit of the CTA loses its first copy
+          const bool skip = fault_pending && (p.mode == 1 || (p.mode == 4 && c > 0)) && kb == 0;
+          if (skip) fault_pending = false;
           if (!skip) {
             mbar_arrive_expect_tx(full + stage, kStageBytes);
             if (p.a_slotted)
@@ -286,6 +298,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       const int64_t tile = static_cast<int64_t>(mt) * p.tiles_n + nt;
+      // mode 4: unit c = 0 is a reference tile, c > 0 candidate c - 1's
+      const bool ref_tile = p.mode == 0 || (p.mode == 4 && c == 0);
+      const bool loss_tile = p.mode == 1 || (p.mode == 4 && c > 0);
+      const int lc = p.mode == 4 ? c - 1 : c;
+      if (p.mode == 4 && c > 0) {
+        // the reference tile this candidate tile is compared with must be in Y
+        int ready = 1;
+        if (ew == 0 && lane == 0) ready = flag_wait_bounded(p.ready + tile, abort_flag, budget);
+        if (named_barrier_or(3, kEpiThreads, !ready)) {
+          if (!ready) fail();
+          break;
+        }
+      }
       float4* ytile = reinterpret_cast<float4*>(p.Y + tile * (BM * BN));
       float sq = 0.0f;
 #pragma unroll 1
@@ -305,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 orow[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
                                       __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
           }
-        } else if (p.mode == 0) {
+        } else if (ref_tile) {
 #pragma unroll
           for (int q = 0; q < 8; ++q)
             yrow[q * BM] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
@@ -313,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            const float4 y = __ldg(yrow + q * BM);
+            const float4 y = __ldcg(yrow + q * BM);  // through L2: mode 4 wrote it in this launch
             const float d0 = __uint_as_float(v[4 * q]) - y.x;
             const float d1 = __uint_as_float(v[4 * q + 1]) - y.y;
             const float d2 = __uint_as_float(v[4 * q + 2]) - y.z;
@@ -327,14 +352,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(tempty + acc);
-      if (p.mode == 1) {
+      if (p.mode == 4 && ref_tile) {
+        // publish: every thread's Y stores, then the tile's flag
+        __threadfence();
+        named_barrier_sync(4, kEpiThreads);
+        if (ew == 0 && lane == 0) st_release_gpu(p.ready + tile, 1);
+      }
+      if (loss_tile) {
         double ds = static_cast<double>(sq);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
         if (lane == 0) red[acc * 4 + ew] = ds;
         named_barrier_sync(2, kEpiThreads);
         if (ew == 0 && lane == 0)
-          p.partial[static_cast<int64_t>(c) * tiles + tile] =
+          p.partial[static_cast<int64_t>(lc) * tiles + tile] =
               ((red[acc * 4 + 0] + red[acc * 4 + 1]) + red[acc * 4 + 2]) + red[acc * 4 + 3];
       }
     }
@@ -712,6 +743,7 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
                              cudaStream_t s, int* launches) {
   const int tiles_m = static_cast<int>(ceil_div(a.M, BM));
   const int tiles_n = static_cast<int>(ceil_div(a.N, BN));
+  if (mode == 4 && (a.slot_base != 1 || !a.ready || a.a_slotted || !a.b_per_cand)) return cudaErrorInvalidValue;
   if (a.variant == 2 && mode < 2 && a.slot_base == 1 && !a.a_slotted && a.b_per_cand && a.cands == 0) {
     static unsigned long long attr_done = 0;
     cudaError_t e = set_smem_limit_once(loss_gemm_pair_kernel, kPairSmemBytes, &attr_done);
@@ -776,12 +808,13 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
   p.f16 = a.f16;
   p.slot_base = a.slot_base;
   p.Y = a.Y;
+  p.ready = a.ready;
   p.partial = a.partial;
   p.err = a.err;
   p.timeout_ns = a.timeout_ns;
   p.fault_mode = a.fault_mode;
   const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
-  const int64_t units = (mode == 1 || mode == 3 ? p.cands : 1) * tiles;
+  const int64_t units = (mode == 1 || mode == 3 ? p.cands : (mode == 4 ? a.n_grid + 1 : 1)) * tiles;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(units, a.num_sms));
   loss_gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(mapA, mapB, p);
   *launches += 1;

@@ -115,6 +115,19 @@ def test_host_batch_matches_one_layer_at_a_time():
             assert torch.equal(getattr(d, name).cpu(), getattr(o, name)), name
 
 
+def test_host_batch_reports_a_bad_layer_and_finishes_the_others():
+    layers = [generate(custom_spec(128, 256, 264, seed=40 + i)) for i in range(3)]
+    Xs = [X.pin_memory() for X, _ in layers]
+    Xs[1][3, 5] = float("nan")
+    outs = [awq._alloc_outputs(256, 264, 128, 20, None, pin=True) for _ in range(3)]
+    with pytest.raises(awq.AwqError) as e:
+        awq.search_host_batch(Xs, [W.pin_memory() for _, W in layers], outs=outs)
+    assert e.value.status == 3
+    for i in (0, 2):
+        d = awq.search(layers[i][0].cuda(), layers[i][1].cuda())
+        assert torch.equal(d.codes.cpu(), outs[i][1]) and torch.equal(d.scales.cpu(), outs[i][0])
+
+
 def test_nonfinite_inputs_are_rejected():
     spec = custom_spec(64, 128, 64, seed=3)
     X, W = generate(spec)
@@ -153,7 +166,8 @@ def test_launch_count_and_profile():
         prof = awq.profile_last()
     finally:
         awq.profile_enable(False)
-    # statistic + scales + qdq + reference GEMM + loss GEMM + reduce + pack
-    assert awq.last_launch_count() == 7
+    # statistic + scales + qdq + one GEMM launch for the reference output and the candidates
+    # (two with the two-SM variant) + reduce + pack
+    assert awq.last_launch_count() == (6 if awq.loss_gemm_variant(256, 256, 512, 20) == 1 else 7)
     assert set(prof) >= {"statistic", "scales", "qdq", "gemm_reference", "gemm_loss", "loss_reduce", "pack"}
     assert all(v >= 0 for v in prof.values()) and prof["gemm_loss"] > 0
