@@ -273,6 +273,45 @@ CopyLane* copy_lane(int dev) {
   return &L;
 }
 
+// Streams, events and pinned status words of the batched host search, created once per
+// device and reused; a batch holds the lane's mutex for its whole call.
+struct BatchLane {
+  struct Slot {
+    cudaEvent_t x_ready = nullptr, in_free = nullptr, out_done = nullptr;
+    cudaEvent_t w_ready[CopyLane::kChunks] = {};
+  };
+  std::mutex mu;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t alloc_done = nullptr, search_done = nullptr, h2d_done = nullptr, d2h_done = nullptr;
+  Slot slots[2];
+  int* words = nullptr;
+  int words_cap = 0;
+};
+
+BatchLane* batch_lane(int dev) {
+  static BatchLane lanes[64];
+  static bool made[64] = {false};
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mu);
+  BatchLane& L = lanes[dev];
+  if (!made[dev]) {
+    auto ev = [](cudaEvent_t* e) { return cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess; };
+    bool ok = cudaStreamCreateWithFlags(&L.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&L.d2h, cudaStreamNonBlocking) == cudaSuccess && ev(&L.alloc_done) &&
+              ev(&L.search_done) && ev(&L.h2d_done) && ev(&L.d2h_done);
+    for (auto& sl : L.slots) {
+      ok = ok && ev(&sl.x_ready) && ev(&sl.in_free) && ev(&sl.out_done);
+      for (auto& w : sl.w_ready) ok = ok && ev(&w);
+    }
+    if (!ok) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    made[dev] = true;
+  }
+  return &L;
+}
+
 // Inputs that are still arriving from the host: the search waits for X before the
 // statistic and for each chunk of W's row groups before quantizing those groups.
 struct HostFeed {
@@ -630,34 +669,28 @@ int awq_search_host_batch(int n_layers, const void* const* X_hosts, const void* 
     slot_bytes += align_up(sizes[k]);
   }
   constexpr int kChunks = CopyLane::kChunks;
-  struct Slot {
-    cudaEvent_t x_ready = nullptr, in_free = nullptr, out_done = nullptr, w_ready[kChunks] = {};
-  } slots[2];
-  cudaStream_t h2d = nullptr, d2h = nullptr;
-  cudaEvent_t alloc_done = nullptr, search_done = nullptr, h2d_done = nullptr, d2h_done = nullptr;
-  bool ok = cudaStreamCreateWithFlags(&h2d, cudaStreamNonBlocking) == cudaSuccess &&
-            cudaStreamCreateWithFlags(&d2h, cudaStreamNonBlocking) == cudaSuccess &&
-            cudaEventCreateWithFlags(&alloc_done, cudaEventDisableTiming) == cudaSuccess &&
-            cudaEventCreateWithFlags(&search_done, cudaEventDisableTiming) == cudaSuccess &&
-            cudaEventCreateWithFlags(&h2d_done, cudaEventDisableTiming) == cudaSuccess &&
-            cudaEventCreateWithFlags(&d2h_done, cudaEventDisableTiming) == cudaSuccess;
-  for (auto& sl : slots) {
-    ok = ok && cudaEventCreateWithFlags(&sl.x_ready, cudaEventDisableTiming) == cudaSuccess &&
-         cudaEventCreateWithFlags(&sl.in_free, cudaEventDisableTiming) == cudaSuccess &&
-         cudaEventCreateWithFlags(&sl.out_done, cudaEventDisableTiming) == cudaSuccess;
-    for (auto& ev : sl.w_ready) ok = ok && cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) == cudaSuccess;
-  }
+  BatchLane* lane = batch_lane(dev);
+  if (!lane) return set_error(AWQ_ERR_CUDA, "could not create the batch's streams and events");
+  std::lock_guard<std::mutex> hold(lane->mu);  // one batch at a time per device
+  BatchLane::Slot* slots = lane->slots;
+  cudaStream_t h2d = lane->h2d, d2h = lane->d2h;
+  cudaEvent_t alloc_done = lane->alloc_done, search_done = lane->search_done, h2d_done = lane->h2d_done,
+              d2h_done = lane->d2h_done;
   void* buf = nullptr;
-  int* words = nullptr;  // pinned: each layer's device status word, read after the final sync
   int status = AWQ_OK;
   cudaError_t e = cudaSuccess;
-  if (!ok) {
-    cudaGetLastError();
-    status = set_error(AWQ_ERR_CUDA, "could not create the batch's streams and events");
-  } else if (cudaMallocHost(reinterpret_cast<void**>(&words), static_cast<size_t>(n_layers) * sizeof(int)) !=
-             cudaSuccess) {
-    cudaGetLastError();
-    words = nullptr;
+  if (lane->words_cap < n_layers) {  // pinned: each layer's device status word, read after the final sync
+    if (lane->words) cudaFreeHost(lane->words);
+    lane->words = nullptr;
+    lane->words_cap = 0;
+    if (cudaMallocHost(reinterpret_cast<void**>(&lane->words), static_cast<size_t>(n_layers) * sizeof(int)) ==
+        cudaSuccess)
+      lane->words_cap = n_layers;
+    else
+      cudaGetLastError();
+  }
+  int* words = lane->words_cap >= n_layers ? lane->words : nullptr;
+  if (!words) {
     status = set_error(AWQ_ERR_OOM, "pinned status words for the batch");
   } else if ((e = cudaMallocFromPoolAsync(&buf, 2 * slot_bytes, pool, s)) != cudaSuccess || !buf) {
     cudaGetLastError();
@@ -670,7 +703,7 @@ int awq_search_host_batch(int n_layers, const void* const* X_hosts, const void* 
   auto slot_ptr = [&](int i, int k) { return static_cast<uint8_t*>(buf) + (i & 1) * slot_bytes + off[k]; };
   // uploads of layer i into slot i % 2, once the search of layer i - 2 is done with it
   auto upload = [&](int i) -> cudaError_t {
-    Slot& sl = slots[i & 1];
+    BatchLane::Slot& sl = slots[i & 1];
     cudaError_t r = i >= 2 ? cudaStreamWaitEvent(h2d, sl.in_free, 0) : cudaSuccess;
     if (r == cudaSuccess) r = cudaMemcpyAsync(slot_ptr(i, 0), X_hosts[i], bx, cudaMemcpyHostToDevice, h2d);
     if (r == cudaSuccess) r = cudaEventRecord(sl.x_ready, h2d);
@@ -690,7 +723,7 @@ int awq_search_host_batch(int n_layers, const void* const* X_hosts, const void* 
       status = cuda_error(e, "host-to-device copy");
   }
   for (int i = 0; i < n_layers && status == AWQ_OK; ++i) {
-    Slot& sl = slots[i & 1];
+    BatchLane::Slot& sl = slots[i & 1];
     if (i + 1 < n_layers && (e = upload(i + 1)) != cudaSuccess) {
       status = cuda_error(e, "host-to-device copy");
       break;
@@ -731,7 +764,7 @@ int awq_search_host_batch(int n_layers, const void* const* X_hosts, const void* 
     }
   }
   // both copy streams are done with the slots before they return to the pool
-  if (h2d && d2h && alloc_done) {
+  {
     cudaEventRecord(h2d_done, h2d);
     cudaEventRecord(d2h_done, d2h);
     cudaStreamWaitEvent(s, h2d_done, 0);
@@ -744,17 +777,6 @@ int awq_search_host_batch(int n_layers, const void* const* X_hosts, const void* 
   if (status == AWQ_OK && se != cudaSuccess) status = cuda_error(se, "stream synchronize");
   // the first layer whose kernels reported a problem decides the status
   for (int i = 0; i < n_layers && status == AWQ_OK && words; ++i) status = status_from_word(words[i]);
-  if (words) cudaFreeHost(words);
-  for (auto& sl : slots) {
-    for (cudaEvent_t ev : {sl.x_ready, sl.in_free, sl.out_done})
-      if (ev) cudaEventDestroy(ev);
-    for (cudaEvent_t ev : sl.w_ready)
-      if (ev) cudaEventDestroy(ev);
-  }
-  for (cudaEvent_t ev : {alloc_done, search_done, h2d_done, d2h_done})
-    if (ev) cudaEventDestroy(ev);
-  if (h2d) cudaStreamDestroy(h2d);
-  if (d2h) cudaStreamDestroy(d2h);
   return status;
 }
 
