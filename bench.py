@@ -213,12 +213,16 @@ def measure_clip(awq, spec: LayerSpec, Xd, Wd, scales, stream, flush, steps: int
 
 
 def _time_w4a16(awq, fn, flush, steps):
+    """Device time of one call (the library's own events around its launches). A short
+    device-side spin after the L2 flush keeps the GPU busy while the host enqueues the
+    call, so the events see the kernels, not the host's launch latency."""
     for _ in range(2):
         fn()
     awq.profile_enable(True)
     ms = []
     for _ in range(steps):
         flush.zero_()
+        torch.cuda._sleep(200_000)  # about 0.1 ms at the B200's clocks
         fn()
         ms.append(awq.w4a16_profile_last())
     return statistics.median(ms), awq.last_launch_count()

@@ -529,8 +529,17 @@ __global__ void piece_sum_kernel(const float* __restrict__ part, int pieces, int
     const int64_t m = i / N, n = i % N, cb = n / 64;
     const int64_t count = chunk_owner(cb * Gk + Gk - 1, T, W) - chunk_owner(cb * Gk, T, W) + 1;
     const float* src = part + (cb * pieces * M + m) * 64 + n % 64;
+    const int64_t stride = static_cast<int64_t>(M) * 64;  // one piece
     float s = src[0];
-    for (int64_t q = 1; q < count; ++q) s = __fadd_rn(s, src[q * M * 64]);
+    // eight loads in flight at a time, the additions still in piece order
+    for (int64_t q0 = 1; q0 < count; q0 += 8) {
+      float v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[k] = q0 + k < count ? src[(q0 + k) * stride] : 0.0f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (q0 + k < count) s = __fadd_rn(s, v[k]);
+    }
     Y[i] = s;
   }
 }
