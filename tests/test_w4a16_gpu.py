@@ -123,8 +123,8 @@ def test_full_size_sampled_columns(name, M):
         _check_output(Y[:, c0:c1], A16, codes[:, c0 // 8:c1 // 8], st[:, c0:c1], zr[:, c0:c1], g)
 
 
-@pytest.mark.parametrize("M", [1, 5, 16])
-@pytest.mark.parametrize("K,N,group", [(256, 256, 128), (160, 128, 32), (384, 576, 64)])
+@pytest.mark.parametrize("M", [1, 5, 9, 16])
+@pytest.mark.parametrize("K,N,group", [(256, 256, 128), (160, 128, 32), (384, 576, 64), (128, 1024, 128)])
 def test_repacked_decode_matches_oracle(M, K, N, group):
     codes, steps, zeros = _random_artifact(K, N, group, 7 * M + N)
     c, st, zr = _dev(codes, steps, zeros)
