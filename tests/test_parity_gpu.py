@@ -36,6 +36,8 @@ def test_single_linear_layer_fp32():
     (64, 256, 256, 128, 1, "normal", "bf16"),        # a single candidate
     (260, 512, 1032, 128, 20, "abs_normal", "f32"),  # fp32 inputs, ragged tails
     (1, 128, 8, 128, 20, "normal", "bf16"),          # one token, one packed word
+    (96, 256, 264, 128, 64, "normal", "bf16"),       # the largest grid (64 candidates)
+    (64, 160, 136, 32, 64, "abs_normal", "bf16"),    # largest grid with group 32
 ])
 def test_small_layers(M, K, N, group, n_grid, law, dtype):
     spec = custom_spec(M, K, N, dtype=dtype, law=law, group=group, n_grid=n_grid, seed=M + K + N,
