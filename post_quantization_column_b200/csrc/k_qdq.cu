@@ -236,6 +236,19 @@ __device__ __forceinline__ bool fold_back_pairs(const float2 (&wp)[4], const flo
   float dmax = 0.0f;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
+    if (!kClamp && !kExactT) {
+      // The usual case, one operation shorter: a fused multiply-add rounds the exact
+      // product w' (1/step) onto -1.5 2^23, which gives -(q - z) once 1.5 2^23 is added back
+      // (the product is not rounded first, which only brings it closer to the quotient), and
+      // a second one gives w' (1/step) - (q - z) for the half-integer check.
+      const float2 nrc = make_float2(-c.recip, -c.recip);
+      const float2 nqz = __fadd2_rn(__ffma2_rn(wp[i], nrc, nmagic), magic);  // -(q - z)
+      const float2 d = __ffma2_rn(wp[i], rc, nqz);
+      dmax = fmax3(dmax, fabsf(d.x), fabsf(d.y));
+      const float2 v = div2_rn(__fmul2_rn(nqz, nst), ns[i], rs[i]);  // ((q - z) step) / s
+      out[i] = bf16x2_bits(v.x, v.y);
+      continue;
+    }
     float2 t = kExactT ? div2_rn(wp[i], nst, rc) : __fmul2_rn(wp[i], rc);
     if (kClamp) {
       t.x = fminf(fmaxf(t.x, lo), hi);
