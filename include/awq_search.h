@@ -234,8 +234,13 @@ int awq_fp64_mma_peak(double* tflops, awq_stream_t stream);
  * fp32. Steps 1-4 and 6 as awq_search (statistic and scales from X; QDQ, argmin and the
  * artifact of W_gu: out_codes [K][2F/8], out_steps/out_zeros [K/group][2F]).
  * Preconditions as awq_search with N = 2F, plus F and K_out multiples of 8; W_down has
- * the dtype of X and W_gu. Work space from the library's pool: the candidates
- * ((n_grid + 1) 2F K bf16), the first GEMM's output (M 2F fp32), h (M F bf16), the
+ * the dtype of X and W_gu. When F % 128 == 0 the silu-mul runs in the first GEMM's
+ * epilogue (gate and up columns interleaved by 128 in the candidate operand) and each
+ * GEMM runs once for a batch of candidates; otherwise the first GEMM writes [G | U] in
+ * fp32 and a separate kernel forms h, one candidate at a time. Both give the same bits;
+ * AWQ_MLP_UNFUSED=1 in the environment selects the second form. Work space from the
+ * library's pool: the candidates ((n_grid + 1) 2F K bf16), h for the reference and a
+ * batch of candidates (up to 4 GiB; the unfused form: M 2F fp32 plus M F bf16), the
  * transposed down projection and the reference output. Synchronizes `stream`. */
 int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_dtype,
                    int64_t M, int64_t K, int64_t F, int64_t K_out, int group, int n_grid,
