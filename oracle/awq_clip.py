@@ -8,7 +8,7 @@ channel and every input group separately, the search tries thresholds of 1, 0.95
 to [-threshold, threshold], quantizes it, and scores the candidate by the mean squared
 error of the group's partial dot product over sampled tokens; the lowest error wins.
 
-Readings (also in DESIGN.md):
+Readings:
 * the weights searched are the scaled ones, W' = fl32(s * W), with the scales the
   scale search chose, and the partial outputs use the scaled activations
   X' = fl32(X / s) — the layer as it stands once the scales are folded in (AWQ-P1 §6);

@@ -7,7 +7,7 @@ MLP block. Here the searched projections are the gate and up projections of a
 Llama-shaped MLP, which read the same input and share one scale vector; the block
 output is down(act(X W_gate) * (X W_up)).
 
-Readings (also in DESIGN.md):
+Readings:
 * W_gu = [W_gate | W_up] (K x 2F) is searched jointly, as the gate+up layers are;
 * act = SiLU, x / (1 + exp(-x)) (the activation of the Llama-shaped blocks);
 * the down projection keeps its original weights during the search;

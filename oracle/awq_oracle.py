@@ -20,7 +20,7 @@ Notation (AWQ-P1 §1, §7): X is M x K (M calibration tokens, K input channels),
 K x N (N output channels), groups run along K, a group is `group` consecutive rows
 of one column of W.
 
-Readings where the pages are silent or garbled (each also listed in the design doc):
+Readings where the pages are silent or garbled:
 
 * statistic: |X| summed in fp64, divided by M in fp64, rounded once to fp32;
 * scales: alpha_i = i / n_grid; raw = max(a^alpha, 1e-4) (clamp BEFORE the

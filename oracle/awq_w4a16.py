@@ -8,7 +8,7 @@ a separate choice; §6: the scales are folded into the operation that produces t
 activations, so the linear layer receives X / s. "model-quantization / 05 core modules"
 (QUANT-P4) §5.3: int4 codes packed eight per int32 with separate fp16 scale tensors.
 
-Readings (also in DESIGN.md):
+Readings:
 * activations: A = fp16(fl32(X / s)) — 16-bit activations already divided by the scales;
 * dequantized weight: w16[k][n] = fp16((q[k][n] - z[g][n]) * step[g][n]) with the
   artifact's fp16 step and zero (q - z is an integer of magnitude at most 15, so the
