@@ -106,13 +106,15 @@ def test_host_entry_point_matches_device_entry_point():
         assert torch.equal(getattr(d, name).cpu(), getattr(h, name)), name
 
 
-def test_host_batch_matches_one_layer_at_a_time():
+@pytest.mark.parametrize("dtype,group", [("bf16", 128), ("f32", 64)])
+def test_host_batch_matches_one_layer_at_a_time(dtype, group):
     """Five layers through the batched host entry point (inputs of layer i + 1 uploaded
     while layer i runs, two device slots reused) give each layer's own artifact."""
-    layers = [generate(custom_spec(256, 384, 520, seed=20 + i)) for i in range(5)]
-    outs = awq.search_host_batch([X.pin_memory() for X, _ in layers], [W.pin_memory() for _, W in layers])
+    layers = [generate(custom_spec(256, 384, 520, dtype=dtype, group=group, seed=20 + i)) for i in range(5)]
+    outs = awq.search_host_batch([X.pin_memory() for X, _ in layers], [W.pin_memory() for _, W in layers],
+                                 group)
     for (X, W), o in zip(layers, outs):
-        d = awq.search(X.cuda(), W.cuda())
+        d = awq.search(X.cuda(), W.cuda(), group)
         for name in ("scales", "codes", "steps", "zeros", "losses"):
             assert torch.equal(getattr(d, name).cpu(), getattr(o, name)), name
 
