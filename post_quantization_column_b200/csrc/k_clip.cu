@@ -301,148 +301,157 @@ __global__ void __launch_bounds__(kClipThreads, 1)
   const double tokens_d = static_cast<double>(tokens);
 
   // One barrier per threshold: in step it, the deltas of threshold it are built into
-  // buffer it % 2 while the products of threshold it - 1 run on the other buffer and
-  // the column sums of threshold it - 2 are reduced. Odd warps multiply first and
-  // build second, even warps the other way round, so the ALU work of one half of the
-  // warps overlaps the tensor-core work of the other half.
-  auto build = [&](int it) {
-    if (it < n_shrink) {
-      // clamp -> QDQ -> delta. Clamping is monotone, so the clamped group's min and
-      // max are the clamped min and max. Codes use a correctly rounded reciprocal of
-      // the step; a quotient within 2^-15 of a half-integer takes the exact division.
-      double* dbuf = sD + (it & 1) * G * kClipCols;
-      const float c = __fmul_rn(amax, sF[it]);
-      const QdqParams p = qdq_params_q(clamp_to(mn, c), clamp_to(mx, c), quantizer);
-      const float recip = __frcp_rn(p.step);
-      const bool col_exact = !(p.step >= kTinyStep && recip <= kHugeRecip);
-      const float lo = -p.zero, hi = p.qmax - p.zero;
-#pragma unroll
-      for (int j = 0; j < CT::EPT; ++j) {
-        const float wc = clamp_to(wp[j], c);
-        const float tv = fminf(fmaxf(__fmul_rn(wc, recip), lo), hi);
-        float qz = __fsub_rn(__fadd_rn(tv, kRoundMagic), kRoundMagic);  // q - z
-        if (col_exact || fabsf(__fsub_rn(tv, qz)) >= kNearHalf) qz = __fsub_rn(qdq_code(wc, p), p.zero);
-        const float rec = __fmul_rn(qz, p.step);
-        dbuf[d_index(r + CT::kRowStep * j, n)] = __dsub_rn(static_cast<double>(rec), static_cast<double>(wp[j]));
-      }
-    }
+  // buffer it % 2 while the products of threshold it - 1 run on the other buffer and the
+  // column sums of threshold it - 2 are reduced. Each warp interleaves the two: its share
+  // of the build is spread over the units of its product run, so the ALU work of the
+  // build issues while the warp's own tensor-core MMAs are in flight.
+  struct BuildParams {
+    double* dbuf;
+    float c, recip, lo, hi;
+    QdqParams p;
+    bool col_exact;
   };
-  auto product = [&](int it) {
-    if (it >= 1 && it <= n_shrink) {
-      const double* dbuf = sD + ((it - 1) & 1) * G * kClipCols;
-      double ep[MJ][2];  // column sums of this lane: columns colw + 8 jt + 2 tq + {0, 1}
-      double acc[4][MJ][2];
+  auto build_params = [&](int it) {
+    // clamp -> QDQ -> delta. Clamping is monotone, so the clamped group's min and max are
+    // the clamped min and max. Codes use a correctly rounded reciprocal of the step; a
+    // quotient within 2^-15 of a half-integer takes the exact division.
+    BuildParams bp;
+    bp.dbuf = sD + (it & 1) * G * kClipCols;
+    bp.c = __fmul_rn(amax, sF[it]);
+    bp.p = qdq_params_q(clamp_to(mn, bp.c), clamp_to(mx, bp.c), quantizer);
+    bp.recip = __frcp_rn(bp.p.step);
+    bp.col_exact = !(bp.p.step >= kTinyStep && bp.recip <= kHugeRecip);
+    bp.lo = -bp.p.zero;
+    bp.hi = bp.p.qmax - bp.p.zero;
+    return bp;
+  };
+  auto build_one = [&](const BuildParams& bp, int j) {  // element j of this thread's share
+    const float wc = clamp_to(wp[j], bp.c);
+    const float tv = fminf(fmaxf(__fmul_rn(wc, bp.recip), bp.lo), bp.hi);
+    float qz = __fsub_rn(__fadd_rn(tv, kRoundMagic), kRoundMagic);  // q - z
+    if (bp.col_exact || fabsf(__fsub_rn(tv, qz)) >= kNearHalf) qz = __fsub_rn(qdq_code(wc, bp.p), bp.p.zero);
+    const float rec = __fmul_rn(qz, bp.p.step);
+    bp.dbuf[d_index(r + CT::kRowStep * j, n)] = __dsub_rn(static_cast<double>(rec), static_cast<double>(wp[j]));
+  };
+  auto build = [&](int it) {  // the whole share at once (the first threshold: no products to hide it behind)
+    const BuildParams bp = build_params(it);
 #pragma unroll
-      for (int jt = 0; jt < MJ; ++jt) {
-        ep[jt][0] = ep[jt][1] = 0.0;
+    for (int j = 0; j < CT::EPT; ++j) build_one(bp, j);
+  };
+  // products of threshold it - 1; with_build: threshold it's deltas built alongside
+  auto product = [&](int it, bool with_build) {
+    constexpr int kUnits = CT::kStepsPerWarp / 2;  // two k-steps per unit
+    const double* dbuf = sD + ((it - 1) & 1) * G * kClipCols;
+    BuildParams bp;
+    if (with_build) bp = build_params(it);
+    double ep[MJ][2];  // column sums of this lane: columns colw + 8 jt + 2 tq + {0, 1}
+    double acc[4][MJ][2];
 #pragma unroll
-        for (int i4 = 0; i4 < 4; ++i4) acc[i4][jt][0] = acc[i4][jt][1] = 0.0;
-      }
-      auto fold = [&](int blk) {  // ep += Delta_blk .* Q_blk, then clear Q
+    for (int jt = 0; jt < MJ; ++jt) {
+      ep[jt][0] = ep[jt][1] = 0.0;
 #pragma unroll
-        for (int i4 = 0; i4 < 4; ++i4) {
-          const int row = 32 * blk + 8 * i4 + gq;
+      for (int i4 = 0; i4 < 4; ++i4) acc[i4][jt][0] = acc[i4][jt][1] = 0.0;
+    }
+    auto fold = [&](int blk) {  // ep += Delta_blk .* Q_blk, then clear Q
 #pragma unroll
-          for (int jt = 0; jt < MJ; ++jt) {
-            const double2 dv = *reinterpret_cast<const double2*>(dbuf + d_index(row, colw + 8 * jt + 2 * tq));
-            ep[jt][0] = __fma_rn(dv.x, acc[i4][jt][0], ep[jt][0]);
-            ep[jt][1] = __fma_rn(dv.y, acc[i4][jt][1], ep[jt][1]);
-            acc[i4][jt][0] = acc[i4][jt][1] = 0.0;
-          }
-        }
-      };
-      auto double_q = [&]() {  // exact: the weight-2 sums
-#pragma unroll
-        for (int i4 = 0; i4 < 4; ++i4)
-#pragma unroll
-          for (int jt = 0; jt < MJ; ++jt) {
-            acc[i4][jt][0] = __dadd_rn(acc[i4][jt][0], acc[i4][jt][0]);
-            acc[i4][jt][1] = __dadd_rn(acc[i4][jt][1], acc[i4][jt][1]);
-          }
-      };
-      // The run, as segments of one item each: row block b, column block cb, steps
-      // ks0 .. ks0 + cnt - 1. Inside a segment every load is a fixed offset from one of
-      // four per-lane pointers: with x = tq & 1 the swizzle maps the fragment columns
-      // 8 m + gq of row 4 s + tq to 8 (m ^ x) + (gq ^ 4 (tq >> 1)), so pointers pa0 / pa1
-      // (pd0 / pd1) serve the even / odd MMA rows (columns) and each step moves them by
-      // 4 rows. Runs start and end on even steps, so the inner loop takes two steps.
-      const int x = tq & 1;
-      const int lane_off = gq ^ (4 * (tq >> 1));
-      int b = b_start, j = j_start, ks = ks_start, remaining = CT::kStepsPerWarp;
-      bool on_diag = false;
-      while (remaining > 0) {
-        const int n_off = CT::NB - 1 - b;  // weight-2 blocks right of the diagonal
-        const int cb = j < n_off ? b + 1 + j : b;
-        const int cnt = min(8 - ks, remaining);
-        on_diag = cb == b;
-        if (on_diag && ks == 0) double_q();  // entering the diagonal block
-        const double* hrow = sH + ((cb * (cb + 1) / 2 + b) * 32 + 4 * ks + tq) * 32 + lane_off;
-        const double* pa0 = hrow + 8 * x;
-        const double* pa1 = hrow + 8 * (1 - x);
-        const double* drow = dbuf + (32 * cb + 4 * ks + tq) * kClipCols + colw + lane_off;
-        const double* pd0 = drow + 8 * x;
-        const double* pd1 = drow + 8 * (1 - x);
-#pragma unroll 1
-        for (int u = 0; u < cnt; u += 2) {
-#pragma unroll
-          for (int v = 0; v < 2; ++v) {
-            const int oa = (u + v) * 128, od = (u + v) * 4 * kClipCols;
-            const double a0 = pa0[oa], a1 = pa1[oa], a2 = pa0[oa + 16], a3 = pa1[oa + 16];
-            const double b0 = pd0[od], b1 = pd1[od];
-            mma_f64(acc[0][0], a0, b0);
-            mma_f64(acc[0][1], a0, b1);
-            mma_f64(acc[1][0], a1, b0);
-            mma_f64(acc[1][1], a1, b1);
-            mma_f64(acc[2][0], a2, b0);
-            mma_f64(acc[2][1], a2, b1);
-            mma_f64(acc[3][0], a3, b0);
-            mma_f64(acc[3][1], a3, b1);
-          }
-        }
-        remaining -= cnt;
-        ks += cnt;
-        if (ks == 8) {
-          ks = 0;
-          if (++j == CT::NB - b) {
-            fold(b);
-            ++b;
-            j = 0;
-          }
-        }
-      }
-      if (b < CT::NB) {  // the run ended inside row block b (a no-op after a clean block end)
-        if (!on_diag) double_q();  // it never reached the diagonal block
-        fold(b);
-      }
-      // combine the 8 lanes (gq) that hold partial sums of the same columns
-#pragma unroll
-      for (int jt = 0; jt < MJ; ++jt)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          double v = ep[jt][h];
-          v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, 4));
-          v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, 8));
-          v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, 16));
-          ep[jt][h] = v;
-        }
-      if (gq == 0) {
-        double* red = sRed + ((it - 1) & 1) * CT::kWarps * CT::kSliceCols + warp * CT::kSliceCols;
+      for (int i4 = 0; i4 < 4; ++i4) {
+        const int row = 32 * blk + 8 * i4 + gq;
 #pragma unroll
         for (int jt = 0; jt < MJ; ++jt) {
-          red[8 * jt + 2 * tq] = ep[jt][0];
-          red[8 * jt + 2 * tq + 1] = ep[jt][1];
+          const double2 dv = *reinterpret_cast<const double2*>(dbuf + d_index(row, colw + 8 * jt + 2 * tq));
+          ep[jt][0] = __fma_rn(dv.x, acc[i4][jt][0], ep[jt][0]);
+          ep[jt][1] = __fma_rn(dv.y, acc[i4][jt][1], ep[jt][1]);
+          acc[i4][jt][0] = acc[i4][jt][1] = 0.0;
         }
+      }
+    };
+    auto double_q = [&]() {  // exact: the weight-2 sums
+#pragma unroll
+      for (int i4 = 0; i4 < 4; ++i4)
+#pragma unroll
+        for (int jt = 0; jt < MJ; ++jt) {
+          acc[i4][jt][0] = __dadd_rn(acc[i4][jt][0], acc[i4][jt][0]);
+          acc[i4][jt][1] = __dadd_rn(acc[i4][jt][1], acc[i4][jt][1]);
+        }
+    };
+    // The run, as units of two k-steps (runs start and end on even steps, so a unit never
+    // crosses a 32-row block): row block b, column block cb, steps ks, ks + 1. Every load
+    // is a fixed offset from one of four per-lane pointers: with x = tq & 1 the swizzle
+    // maps the fragment columns 8 m + gq of row 4 s + tq to 8 (m ^ x) + (gq ^ 4 (tq >> 1)),
+    // so pointers pa0 / pa1 (pd0 / pd1) serve the even / odd MMA rows (columns).
+    const int x = tq & 1;
+    const int lane_off = gq ^ (4 * (tq >> 1));
+    int b = b_start, j = j_start, ks = ks_start;
+    bool on_diag = false;
+#pragma unroll
+    for (int unit = 0; unit < kUnits; ++unit) {
+      const int n_off = CT::NB - 1 - b;  // weight-2 blocks right of the diagonal
+      const int cb = j < n_off ? b + 1 + j : b;
+      on_diag = cb == b;
+      if (on_diag && ks == 0) double_q();  // entering the diagonal block
+      const double* hrow = sH + ((cb * (cb + 1) / 2 + b) * 32 + 4 * ks + tq) * 32 + lane_off;
+      const double* pa0 = hrow + 8 * x;
+      const double* pa1 = hrow + 8 * (1 - x);
+      const double* drow = dbuf + (32 * cb + 4 * ks + tq) * kClipCols + colw + lane_off;
+      const double* pd0 = drow + 8 * x;
+      const double* pd1 = drow + 8 * (1 - x);
+#pragma unroll
+      for (int v = 0; v < 2; ++v) {
+        const int oa = v * 128, od = v * 4 * kClipCols;
+        const double a0 = pa0[oa], a1 = pa1[oa], a2 = pa0[oa + 16], a3 = pa1[oa + 16];
+        const double b0 = pd0[od], b1 = pd1[od];
+        mma_f64(acc[0][0], a0, b0);
+        mma_f64(acc[0][1], a0, b1);
+        mma_f64(acc[1][0], a1, b0);
+        mma_f64(acc[1][1], a1, b1);
+        mma_f64(acc[2][0], a2, b0);
+        mma_f64(acc[2][1], a2, b1);
+        mma_f64(acc[3][0], a3, b0);
+        mma_f64(acc[3][1], a3, b1);
+      }
+      if (with_build) {  // this unit's slice of the next threshold's deltas
+#pragma unroll
+        for (int e = unit * CT::EPT / kUnits; e < (unit + 1) * CT::EPT / kUnits; ++e) build_one(bp, e);
+      }
+      ks += 2;
+      if (ks == 8) {
+        ks = 0;
+        if (++j == CT::NB - b) {
+          fold(b);
+          ++b;
+          j = 0;
+        }
+      }
+    }
+    if (b < CT::NB) {  // the run ended inside row block b (a no-op after a clean block end)
+      if (!on_diag) double_q();  // it never reached the diagonal block
+      fold(b);
+    }
+    // combine the 8 lanes (gq) that hold partial sums of the same columns
+#pragma unroll
+    for (int jt = 0; jt < MJ; ++jt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        double v = ep[jt][h];
+        v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, 4));
+        v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, 8));
+        v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, 16));
+        ep[jt][h] = v;
+      }
+    if (gq == 0) {
+      double* red = sRed + ((it - 1) & 1) * CT::kWarps * CT::kSliceCols + warp * CT::kSliceCols;
+#pragma unroll
+      for (int jt = 0; jt < MJ; ++jt) {
+        red[8 * jt + 2 * tq] = ep[jt][0];
+        red[8 * jt + 2 * tq + 1] = ep[jt][1];
       }
     }
   };
   for (int it = 0; it < n_shrink + 2; ++it) {
-    if (warp & 1) {
-      product(it);
+    if (it >= 1 && it <= n_shrink)
+      product(it, it < n_shrink);
+    else if (it < n_shrink)
       build(it);
-    } else {
-      build(it);
-      product(it);
-    }
     if (it >= 2 && lane < 4) {
       const int i = it - 2;
       const double* red = sRed + (i & 1) * CT::kWarps * CT::kSliceCols;
