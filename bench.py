@@ -541,7 +541,8 @@ def run_ours(args, rank, world, local):
                     "GB/s": qdq_bytes / (statistics.mean(qdq_ms) / 1e3) / 1e9,
                     "hbm_frac": qdq_bytes / (statistics.mean(qdq_ms) / 1e3) / 1e9 / float(peaks["hbm_gbs"])},
             "statistic": {"ms": statistics.mean(stat_ms),
-                          "GB/s": stat_bytes / (statistics.mean(stat_ms) / 1e3) / 1e9},
+                          "GB/s": stat_bytes / (statistics.mean(stat_ms) / 1e3) / 1e9,
+                          "hbm_frac": stat_bytes / (statistics.mean(stat_ms) / 1e3) / 1e9 / float(peaks["hbm_gbs"])},
             "pack": {"ms": statistics.mean(pack_ms)},
         },
         "phases_ms": {k: v / args.steps for k, v in phase_tot.items()},

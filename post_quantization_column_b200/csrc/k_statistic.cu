@@ -6,11 +6,12 @@
 // Both reductions run as one launch of 8-CTA thread-block clusters and combine their
 // partial results through distributed shared memory in a fixed order, so they need no
 // global scratch and no second pass:
-//  * statistic: a cluster owns 64 columns (bf16; 32 for fp32); its 8 CTAs split the
-//    rows, each thread walks rows with 16-byte column vectors (a warp reads 128-byte
-//    row segments; fp64 accumulation), the CTA sums its 32 row-threads, and CTA rank 0
-//    sums the 8 CTAs' partials, divides by M once in fp64 and rounds once to fp32.
-//    HBM-bound: one read of X, with enough CTAs (8 per 64 columns) to keep HBM busy.
+//  * statistic: a cluster owns 8 or 16 16-byte column vectors (64 or 128 bf16 columns,
+//    32 or 64 fp32 ones; the wider form once the narrow grid would exceed a wave of
+//    resident CTAs); its 8 CTAs split the rows, each thread walks rows with one column
+//    vector, 8 loads in flight (fp64 accumulation), the CTA sums its row-threads, and
+//    CTA rank 0 sums the 8 CTAs' partials, divides by M once in fp64 and rounds once to
+//    fp32. HBM-bound: one read of X in 128- or 256-byte row segments.
 //  * scales: a cluster owns one candidate alpha_i; its 8 CTAs split K, exchange their
 //    max/min of raw = max(a^alpha, 1e-4) and each normalises its share by
 //    sqrt(max * min) — fp64 throughout, one rounding to fp32.
@@ -25,14 +26,17 @@ namespace awq {
 namespace {
 
 constexpr int kCluster = 8;       // CTAs per cluster (portable size)
-constexpr int kStatVecs = 8;      // 16-byte column vectors per CTA (a warp reads 128-byte row segments)
-constexpr int kStatRows = 32;     // row-threads per column vector
-constexpr int kStatThreads = kStatVecs * kStatRows;
+constexpr int kStatThreads = 256;
+constexpr int kStatBatch = 8;     // row loads in flight per thread
+constexpr int kStatCtasPerSm = 4;  // resident statistic CTAs per SM (registers)
 
-template <typename T>
+// VECS 16-byte column vectors per CTA: a warp reads 32 / VECS rows of 16 VECS bytes.
+template <typename T, int VECS>
 __global__ void __cluster_dims__(1, kCluster, 1) __launch_bounds__(kStatThreads)
     statistic_kernel(const T* __restrict__ X, int64_t M, int64_t K, float* __restrict__ a, int* err) {
   constexpr int VEC = 16 / sizeof(T);
+  constexpr int kStatVecs = VECS;
+  constexpr int kStatRows = kStatThreads / VECS;  // row-threads per column vector
   constexpr int kCols = kStatVecs * VEC;  // columns per cluster
   __shared__ double red[kStatRows][kStatVecs][VEC];
   __shared__ double part[kCols];          // this CTA's column sums, read by rank 0
@@ -46,15 +50,24 @@ __global__ void __cluster_dims__(1, kCluster, 1) __launch_bounds__(kStatThreads)
 #pragma unroll
   for (int i = 0; i < VEC; ++i) acc[i] = 0.0;
   if (c0 < K) {  // K % 32 == 0, so a vector lies wholly inside or outside
+    // Rows r0, r0 + stride, ... in that order; kStatBatch loads are issued before any is
+    // used, so a thread waits for one DRAM round trip per batch, not per row.
     const T* base = X + c0;
     const int64_t stride = static_cast<int64_t>(kStatRows) * kCluster;
-#pragma unroll 4
-    for (int64_t r = static_cast<int64_t>(rank) * kStatRows + ty; r < M; r += stride) {
-      const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(base + r * K));
+    auto add = [&](const uint4& raw) {
       const T* e = reinterpret_cast<const T*>(&raw);
 #pragma unroll
       for (int i = 0; i < VEC; ++i) acc[i] += fabs(static_cast<double>(to_f32<T>(e[i])));
+    };
+    int64_t r = static_cast<int64_t>(rank) * kStatRows + ty;
+    for (; r + (kStatBatch - 1) * stride < M; r += stride * kStatBatch) {
+      uint4 raw[kStatBatch];
+#pragma unroll
+      for (int b = 0; b < kStatBatch; ++b) raw[b] = __ldcs(reinterpret_cast<const uint4*>(base + (r + b * stride) * K));
+#pragma unroll
+      for (int b = 0; b < kStatBatch; ++b) add(raw[b]);
     }
+    for (; r < M; r += stride) add(__ldcs(reinterpret_cast<const uint4*>(base + r * K)));
   }
 #pragma unroll
   for (int i = 0; i < VEC; ++i) red[ty][tx][i] = acc[i];
@@ -155,13 +168,30 @@ int statistic_row_chunks(int64_t, int64_t, int, int) { return 1; }
 
 cudaError_t launch_statistic(const void* X, int in_dtype, int64_t M, int64_t K, int /*row_chunks*/,
                              double* /*partial*/, float* a, int* err, cudaStream_t s, int* launches) {
+  // Clusters of 8 column vectors (64 bf16 / 32 fp32 columns, 128-byte row segments) while
+  // they fit in one wave of resident CTAs; wider clusters of 16 vectors (256-byte
+  // segments) for larger K, which halves the CTAs and keeps the grid to about one wave.
+  int dev = 0, num_sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
   const int vec = in_dtype == 0 ? 8 : 4;
-  dim3 grid(static_cast<unsigned>(ceil_div(K, static_cast<int64_t>(kStatVecs) * vec)), kCluster);
-  if (in_dtype == 0)
-    statistic_kernel<__nv_bfloat16><<<grid, kStatThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(X), M, K, a,
-                                                                   err);
-  else
-    statistic_kernel<float><<<grid, kStatThreads, 0, s>>>(static_cast<const float*>(X), M, K, a, err);
+  const bool wide = ceil_div(K, static_cast<int64_t>(8 * vec)) * kCluster > static_cast<int64_t>(kStatCtasPerSm) * num_sms;
+  const int vecs = wide ? 16 : 8;
+  dim3 grid(static_cast<unsigned>(ceil_div(K, static_cast<int64_t>(vecs) * vec)), kCluster);
+  if (in_dtype == 0) {
+    const auto* x = static_cast<const __nv_bfloat16*>(X);
+    if (wide)
+      statistic_kernel<__nv_bfloat16, 16><<<grid, kStatThreads, 0, s>>>(x, M, K, a, err);
+    else
+      statistic_kernel<__nv_bfloat16, 8><<<grid, kStatThreads, 0, s>>>(x, M, K, a, err);
+  } else {
+    const auto* x = static_cast<const float*>(X);
+    if (wide)
+      statistic_kernel<float, 16><<<grid, kStatThreads, 0, s>>>(x, M, K, a, err);
+    else
+      statistic_kernel<float, 8><<<grid, kStatThreads, 0, s>>>(x, M, K, a, err);
+  }
   *launches += 1;
   return cudaGetLastError();
 }

@@ -49,6 +49,18 @@ def test_statistic_bit_exact(name):
     assert np.array_equal(_bits(a), _bits(ref))
 
 
+@pytest.mark.parametrize("M,K,dtype", [(1000, 4832, "bf16"), (777, 2400, "f32"), (37, 4096, "bf16"),
+                                       (3001, 256, "f32"), (130, 11008, "bf16")])
+def test_statistic_ragged_shapes(M, K, dtype):
+    # row counts that leave a partial batch of row loads, and K that leaves the last
+    # cluster's column block partly outside X, in both cluster widths (64/128 bf16 columns
+    # per cluster for K up to / above about 4.7k; 32/64 fp32 ones up to / above 2.4k)
+    X, _ = generate(custom_spec(M, K, 8, dtype=dtype, seed=5))
+    a = awq.activation_statistic(X.cuda()).cpu().numpy()
+    ref = O.activation_statistic(as_f32_numpy(X))
+    assert np.array_equal(_bits(a), _bits(ref))
+
+
 @pytest.mark.parametrize("name", list(WORKLOADS))
 def test_scales_bit_exact_for_every_candidate(name):
     spec = WORKLOADS[name]
