@@ -26,10 +26,11 @@
 // the IEEE divisions. Rounding to an integer uses (x + 1.5*2^23) - 1.5*2^23, exact
 // round-half-to-even for |x| < 2^22.
 //
-// pack_kernel: the same tile walk for the chosen candidate only (the first argmin of
-// the fp32 losses, computed by every CTA): codes go through shared memory and are
-// packed eight per int32 along N (QUANT-P4 §5.3), steps and zeros are written as fp16,
-// and the chosen scales are copied out.
+// pack_kernel: the same quantizer for the chosen candidate only (the first argmin of
+// the fp32 losses, computed by every warp), one warp per group x 32-column strip with no
+// shared memory: codes are packed eight per int32 along N in registers (QUANT-P4 §5.3)
+// and stored directly, steps and zeros are written as fp16, and the chosen scales are
+// copied out.
 #include "awq_device.cuh"
 #include "awq_kernels.h"
 
@@ -460,155 +461,201 @@ __global__ void __launch_bounds__(Tile<G>::kThreads, Tile<G>::kBlocksPerSm)
   }
 }
 
-// Register-staged tile loads for the persistent pack kernel: each thread holds its
-// share of the next G x 64 tile (16-byte vectors) while the current tile is computed.
+// Lane layout of the pack kernel: each warp quantizes one group x kCols strip on its
+// own, with no shared memory and no block barrier. Lane (lr, lc) = (lane / 4, lane % 4)
+// holds the 16-byte vector of VEC adjacent columns (lc VEC .. lc VEC + VEC - 1 of the
+// strip) in rows lr, lr + 8, ..., so every load instruction reads eight 64-byte row runs.
 template <typename T, int G>
-struct TileLoad {
-  static constexpr int VEC = 16 / sizeof(T);
-  static constexpr int VPR = kQdqCols / VEC;
-  static constexpr int kPerThread = G * VPR / Tile<G>::kThreads;  // 2 (bf16) or 4 (fp32)
-  uint4 v[kPerThread];
-
-  __device__ __forceinline__ void load(const T* __restrict__ W, int64_t N, int64_t k0, int64_t n0) {
-#pragma unroll
-    for (int it = 0; it < kPerThread; ++it) {
-      const int idx = threadIdx.x + it * Tile<G>::kThreads;
-      const int r = idx / VPR, vv = idx % VPR;
-      const int64_t col = n0 + static_cast<int64_t>(vv) * VEC;
-      v[it] = col < N ? __ldcs(reinterpret_cast<const uint4*>(W + (k0 + r) * N + col)) : make_uint4(0, 0, 0, 0);
-    }
-  }
-  __device__ __forceinline__ void store(float* sWT) const {
-#pragma unroll
-    for (int it = 0; it < kPerThread; ++it) {
-      const int idx = threadIdx.x + it * Tile<G>::kThreads;
-      const int r = idx / VPR, vv = idx % VPR;
-      const T* e = reinterpret_cast<const T*>(&v[it]);
-#pragma unroll
-      for (int i = 0; i < VEC; ++i) sWT[(vv * VEC + i) * Tile<G>::kPitch + r] = to_f32<T>(e[i]);
-    }
-  }
+struct PackShape {
+  static constexpr int VEC = 16 / sizeof(T);  // columns per lane: 8 (bf16) or 4 (fp32)
+  static constexpr int LC = 4;                // lanes across the strip
+  static constexpr int LR = 8;                // lanes down the group
+  static constexpr int RPL = G / LR;          // rows per lane: 16, 8, 4
+  static constexpr int kCols = LC * VEC;      // columns per warp: 32 or 16
+  static constexpr int kWarps = 4;
+  static constexpr int kThreads = 32 * kWarps;
 };
 
-// Persistent: each CTA walks tiles blockIdx.x, + gridDim.x, ... (column tiles of one
-// group are adjacent), loading the next tile into registers while it quantizes the
-// current one, so HBM reads overlap the arithmetic.
+// A read-only load the compiler cannot merge with an earlier one of the same address, so
+// the first pass's value need not stay live in a register (an L1 hit).
+__device__ __forceinline__ float reload_f32(const float* p) {
+  float v;
+  asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
+  return v;
+}
+
+template <typename T>
+__device__ __forceinline__ void unpack16(const uint4& raw, float (&w)[16 / sizeof(T)]) {
+  const T* e = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+  for (int j = 0; j < static_cast<int>(16 / sizeof(T)); ++j) w[j] = to_f32<T>(e[j]);
+}
+
+// Codes of the chosen candidate with its group steps and zeros, packed eight per int32
+// along N. Per lane: the group range of each of its columns over its rows, finished by a
+// butterfly over the eight row-lanes; each row-lane then computes one column's parameters
+// (the definition's divisions) and shares them; codes come from the correctly rounded
+// reciprocal of the step with the same half-integer check as the candidate kernel, and a
+// row holding a code that only the exact quotient decides is redone with the IEEE
+// division after the pass. A lane's VEC codes of a row form one int32 (bf16) or its low
+// or high 16 bits (fp32), stored directly.
 template <typename T, int G>
-__global__ void __launch_bounds__(Tile<G>::kThreads, Tile<G>::kBlocksPerSm)
+__global__ void __launch_bounds__(PackShape<T, G>::kThreads, 4)
     pack_kernel(const T* __restrict__ W, int64_t K, int64_t N, int n_grid, const float* __restrict__ S,
                 const float* __restrict__ losses, int* __restrict__ best_out, int32_t* __restrict__ codes,
                 __half* __restrict__ steps, __half* __restrict__ zeros, float* __restrict__ out_scales,
                 int quantizer) {
-  using L = Tile<G>;
-  __shared__ float sWT[kQdqCols * L::kPitch];
-  // codes of the tile, row-major; rows 68 bytes apart so that the row-lanes' stores
-  // (rows 8 apart) spread over the banks
-  constexpr int kQPitch = kQdqCols + 4;
-  __shared__ __align__(16) uint8_t sQ[G * kQPitch];
-  __shared__ float sScale[G];
-  __shared__ int sBest;
-
-  const int64_t tiles_n = ceil_div(N, kQdqCols);
-  const int64_t tiles = tiles_n * (K / G);
+  using P = PackShape<T, G>;
+  constexpr int VEC = P::VEC;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lc = lane % P::LC, lr = lane / P::LC;
+  const int64_t k0 = static_cast<int64_t>(blockIdx.y) * G;
+  const int64_t n0 = (static_cast<int64_t>(blockIdx.x) * P::kWarps + warp) * P::kCols;
+  const int64_t nl = n0 + lc * VEC;  // the lane's first column
+  const bool active = nl < N;        // N % 8 == 0: a lane's columns are all in or all out
   const int64_t words = N / 8;
 
-  // the chosen candidate: first minimum of the fp32 losses
-  if (threadIdx.x == 0) {
-    int b = 0;
-    for (int c = 1; c < n_grid; ++c)
-      if (losses[c] < losses[b]) b = c;
-    sBest = b;
-    if (blockIdx.x == 0) *best_out = b;
+  uint4 raw[P::RPL];
+  if (active) {
+#pragma unroll
+    for (int i = 0; i < P::RPL; ++i) raw[i] = __ldcs(reinterpret_cast<const uint4*>(W + (k0 + lr + 8 * i) * N + nl));
+  } else {
+#pragma unroll
+    for (int i = 0; i < P::RPL; ++i) raw[i] = make_uint4(0u, 0u, 0u, 0u);
   }
 
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int rl = lane % L::RL, cg = lane / L::RL;
-  const int col0 = warp * L::kColsPerWarp + cg * 2;
-  const int row0 = rl * kRowsPerLane;
-
-  TileLoad<T, G> next;
-  int64_t t = blockIdx.x;
-  if (t < tiles) next.load(W, N, (t / tiles_n) * G, (t % tiles_n) * kQdqCols);
-  __syncthreads();
-  const float* Sbest = S + static_cast<int64_t>(sBest) * K;
-
-  for (; t < tiles; t += gridDim.x) {
-    const int64_t k0 = (t / tiles_n) * G, n0 = (t % tiles_n) * kQdqCols;
-    next.store(sWT);
-    for (int r = threadIdx.x; r < G; r += L::kThreads) {
-      const float sv = Sbest[k0 + r];
-      sScale[r] = sv;
-      if (n0 == 0) out_scales[k0 + r] = sv;
-    }
-    __syncthreads();
-    const int64_t tn = t + gridDim.x;
-    if (tn < tiles) next.load(W, N, (tn / tiles_n) * G, (tn % tiles_n) * kQdqCols);
-
-    float wp[2][8];
-    float mn[2], mx[2];
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      mn[j] = INFINITY;
-      mx[j] = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        wp[j][i] = __fmul_rn(sScale[row0 + i], sWT[(col0 + j) * L::kPitch + row0 + i]);
-        mn[j] = fminf(mn[j], wp[j][i]);
-        mx[j] = fmaxf(mx[j], wp[j][i]);
+  // the chosen candidate: first minimum of the fp32 losses
+  int best = 0;
+  if (lane == 0) {
+    float bv = losses[0];
+    for (int c = 1; c < n_grid; ++c) {
+      const float v = losses[c];
+      if (v < bv) {
+        bv = v;
+        best = c;
       }
     }
-    ColumnQdq cq[2];
-    column_qdq<L::RL>(mn, mx, cq, quantizer);
+    if (blockIdx.x == 0 && blockIdx.y == 0 && warp == 0) *best_out = best;
+  }
+  best = __shfl_sync(0xffffffffu, best, 0);
+  const float* Sb = S + static_cast<int64_t>(best) * K + k0;
+  float s[P::RPL];
+#pragma unroll
+  for (int i = 0; i < P::RPL; ++i) s[i] = Sb[lr + 8 * i];
+  if (n0 == 0 && lc == 0) {
+#pragma unroll
+    for (int i = 0; i < P::RPL; ++i) out_scales[k0 + lr + 8 * i] = s[i];
+  }
 
-    float q[2][8];
-    bool need = cq[0].exact || cq[1].exact;
+  // group range of the lane's columns, then across the row-lanes
+  float mn[VEC], mx[VEC];
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const float lo = -cq[j].p.zero, hi = cq[j].p.qmax - cq[j].p.zero;
+  for (int j = 0; j < VEC; ++j) {
+    mn[j] = INFINITY;
+    mx[j] = -INFINITY;
+  }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float tc = fminf(fmaxf(__fmul_rn(wp[j][i], cq[j].recip), lo), hi);
-        const float qz = round_small(tc);
-        need |= fabsf(__fsub_rn(tc, qz)) >= kNearHalf;
-        q[j][i] = __fadd_rn(qz, cq[j].p.zero);
-      }
+  for (int i = 0; i < P::RPL; ++i) {
+    float w[VEC];
+    unpack16<T>(raw[i], w);
+#pragma unroll
+    for (int j = 0; j < VEC; ++j) {
+      const float wp = __fmul_rn(s[i], w[j]);
+      mn[j] = fminf(mn[j], wp);
+      mx[j] = fmaxf(mx[j], wp);
     }
-    if (__any_sync(0xffffffffu, need) && need) {
+  }
 #pragma unroll
-      for (int j = 0; j < 2; ++j)
+  for (int o = P::LC; o < 32; o <<= 1)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) q[j][i] = qdq_code(wp[j][i], cq[j].p);
+    for (int j = 0; j < VEC; ++j) {
+      mn[j] = fminf(mn[j], __shfl_xor_sync(0xffffffffu, mn[j], o));
+      mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], o));
     }
-#pragma unroll
-    for (int i = 0; i < 8; ++i)  // the lane's two adjacent columns of a row as one 16-bit store
-      *reinterpret_cast<uint16_t*>(&sQ[(row0 + i) * kQPitch + col0]) =
-          static_cast<uint16_t>(static_cast<uint32_t>(q[0][i]) | (static_cast<uint32_t>(q[1][i]) << 8));
 
-    const int64_t n = n0 + col0;
-    if (rl == 0 && n < N) {
-      const int64_t g = k0 / G;
-      *reinterpret_cast<__half2*>(steps + g * N + n) = __halves2half2(__float2half_rn(cq[0].p.step),
-                                                                      __float2half_rn(cq[1].p.step));
-      *reinterpret_cast<__half2*>(zeros + g * N + n) = __halves2half2(__float2half_rn(cq[0].p.zero),
-                                                                      __float2half_rn(cq[1].p.zero));
-    }
-    __syncthreads();
-    // eight codes (one 8-byte run of a tile row) -> one int32, nibble i = column 8w + i
-    for (int idx = threadIdx.x; idx < G * (kQdqCols / 8); idx += L::kThreads) {
-      const int r = idx / (kQdqCols / 8), wd = idx % (kQdqCols / 8);
-      const int64_t word = n0 / 8 + wd;
-      if (word >= words) continue;
-      const uint2 b = make_uint2(*reinterpret_cast<const uint32_t*>(&sQ[r * kQPitch + wd * 8]),
-                                 *reinterpret_cast<const uint32_t*>(&sQ[r * kQPitch + wd * 8 + 4]));
-      uint32_t packed = 0;
+  // row-lane lr computes the parameters of column lr % VEC of its strip, and shares them
+  const int jc = lr % VEC;
+  float cmn = mn[0], cmx = mx[0];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        packed |= ((b.x >> (8 * i)) & 0xFu) << (4 * i);
-        packed |= ((b.y >> (8 * i)) & 0xFu) << (4 * (i + 4));
-      }
-      codes[(k0 + r) * words + word] = static_cast<int32_t>(packed);
+  for (int j = 1; j < VEC; ++j)
+    if (jc == j) {
+      cmn = mn[j];
+      cmx = mx[j];
     }
-    __syncthreads();  // sWT, sQ and sScale are rewritten by the next tile
+  const QdqParams pc = qdq_params_q(cmn, cmx, quantizer);
+  const float rc = __frcp_rn(pc.step);
+  const int exact_c = !(pc.step >= kTinyStep && rc <= kHugeRecip);
+  if (active && lr < VEC) {
+    const int64_t o = (k0 / G) * N + nl + jc;
+    steps[o] = __float2half_rn(pc.step);
+    zeros[o] = __float2half_rn(pc.zero);
+  }
+  QdqParams p[VEC];
+  float rcp[VEC];
+  int zi[VEC];
+  bool col_exact = false;
+#pragma unroll
+  for (int j = 0; j < VEC; ++j) {
+    const int src = j * P::LC + lc;
+    p[j].step = __shfl_sync(0xffffffffu, pc.step, src);
+    p[j].zero = __shfl_sync(0xffffffffu, pc.zero, src);
+    p[j].qmax = pc.qmax;
+    rcp[j] = __shfl_sync(0xffffffffu, rc, src);
+    col_exact |= __shfl_sync(0xffffffffu, exact_c, src) != 0;
+    zi[j] = static_cast<int>(p[j].zero);
+  }
+
+  // codes: q - z = rint(clamp(w' (1/step), -z, qmax - z)); 1.5 2^23 + (q - z) carries q - z
+  // in its low bits, so (bits + z) & 15 is the code. W' is formed again from the raw
+  // vectors (the empty asm hides them from the compiler, which would otherwise keep the
+  // first pass's VEC x RPL products live in registers).
+#pragma unroll
+  for (int i = 0; i < P::RPL; ++i)
+    asm volatile("" : "+r"(raw[i].x), "+r"(raw[i].y), "+r"(raw[i].z), "+r"(raw[i].w));
+  uint32_t redo = 0;
+  int32_t* const crow = codes + k0 * words + nl / 8;
+#pragma unroll
+  for (int i = 0; i < P::RPL; ++i) {
+    float w[VEC];
+    unpack16<T>(raw[i], w);
+    const float si = reload_f32(Sb + lr + 8 * i);
+    uint32_t word = 0;
+    bool need = false;
+#pragma unroll
+    for (int j = 0; j < VEC; ++j) {
+      const float wp = __fmul_rn(si, w[j]);
+      const float tc = fminf(fmaxf(__fmul_rn(wp, rcp[j]), -p[j].zero), p[j].qmax - p[j].zero);
+      const float m = __fadd_rn(tc, kRoundMagic);
+      need |= fabsf(__fsub_rn(tc, __fsub_rn(m, kRoundMagic))) >= kNearHalf;
+      word |= ((__float_as_uint(m) + static_cast<uint32_t>(zi[j])) & 0xFu) << (4 * j);
+    }
+    redo |= static_cast<uint32_t>(need) << i;
+    if (active) {
+      if (VEC == 8)
+        crow[(lr + 8 * i) * words] = static_cast<int32_t>(word);
+      else
+        reinterpret_cast<uint16_t*>(crow + (lr + 8 * i) * words)[lc & 1] = static_cast<uint16_t>(word);
+    }
+  }
+  if (col_exact) redo = (1u << P::RPL) - 1u;
+  // rows with a code decided only by the exact quotient (or columns outside the range
+  // guards): the definition's division, rewriting the lane's own stores
+  while (redo && active) {
+    const int i = __ffs(redo) - 1;
+    redo &= redo - 1;
+    const int64_t r = lr + 8 * i;
+    const uint4 v = *reinterpret_cast<const uint4*>(W + (k0 + r) * N + nl);
+    const float sv = Sb[r];
+    float w[VEC];
+    unpack16<T>(v, w);
+    uint32_t word = 0;
+#pragma unroll
+    for (int j = 0; j < VEC; ++j)
+      word |= static_cast<uint32_t>(qdq_code(__fmul_rn(sv, w[j]), p[j])) << (4 * j);
+    if (VEC == 8)
+      crow[r * words] = static_cast<int32_t>(word);
+    else
+      reinterpret_cast<uint16_t*>(crow + r * words)[lc & 1] = static_cast<uint16_t>(word);
   }
 }
 
@@ -635,14 +682,11 @@ template <typename T, int G>
 cudaError_t launch_pack_t(const T* W, int64_t K, int64_t N, int n_grid, const float* S, const float* losses,
                           int* best, int32_t* codes, __half* steps, __half* zeros, float* out_scales,
                           cudaStream_t s, int quantizer) {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t tiles = ceil_div(N, kQdqCols) * (K / G);
-  const int64_t per_sm = Tile<G>::kBlocksPerSm;  // resident CTAs per SM at <= 64 registers
-  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, per_sm * sms));
-  pack_kernel<T, G><<<grid, Tile<G>::kThreads, 0, s>>>(W, K, N, n_grid, S, losses, best, codes, steps, zeros,
-                                                       out_scales, quantizer);
+  using P = PackShape<T, G>;
+  dim3 grid(static_cast<unsigned>(ceil_div(N, static_cast<int64_t>(P::kWarps) * P::kCols)),
+            static_cast<unsigned>(K / G));
+  pack_kernel<T, G><<<grid, P::kThreads, 0, s>>>(W, K, N, n_grid, S, losses, best, codes, steps, zeros, out_scales,
+                                                 quantizer);
   return cudaGetLastError();
 }
 
