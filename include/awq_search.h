@@ -118,6 +118,22 @@ int awq_search_quant(const void* X, const void* W, int in_dtype, int64_t M, int6
                      int32_t* out_codes, void* out_steps, void* out_zeros, float* out_losses,
                      awq_stream_t stream);
 
+/* Asynchronous form of awq_search_ex (no tile partials): enqueues the whole search on
+ * `stream` and returns without waiting. Argument checks happen before anything is
+ * enqueued and their errors are returned at once; errors the kernels detect (non-finite
+ * input, a bounded wait that ran out) are reported through `status_word`, a 4-byte word
+ * of PINNED host memory (cudaHostAlloc / cudaMallocHost) that the call's last copy
+ * writes. After synchronizing `stream` the caller passes the word to awq_search_status,
+ * which returns the call's status (AWQ_OK or the error awq_search_ex would have
+ * returned) and sets awq_last_error_message. The outputs, the status word, X and W must stay
+ * allocated until the stream has passed the call. Consecutive calls on one stream run
+ * back to back, with no host round trip between them. */
+int awq_search_async(const void* X, const void* W, int in_dtype, int64_t M, int64_t K,
+                     int64_t N, int group, int n_grid, float* out_scales, int32_t* out_codes,
+                     void* out_steps, void* out_zeros, float* out_losses, int32_t* status_word,
+                     awq_stream_t stream);
+int awq_search_status(int32_t status_word);
+
 /* End-to-end form with HOST buffers: copies X and W to the device on `stream`,
  * runs awq_search_ex, copies the outputs back (out_losses may be NULL). Pinned
  * host memory makes the copies asynchronous; pageable memory also works. */
@@ -173,6 +189,13 @@ const char* awq_last_error_message(void);
  * times (ms) of the last call and returns the number of phases. */
 int awq_profile_enable(int on);
 int awq_profile_last(float* ms, int n);
+/* Profiled calls also get a ticket: awq_profile_last_ticket returns the calling thread's
+ * last one (-1 if none); awq_profile_collect writes up to `n` phase times (ms) of that
+ * call once its work has completed (e.g. an awq_search_async call after the stream has
+ * been synchronized) and returns the number of phases, or -1 if the call is still
+ * running or 256 later profiled calls on its device have reused its events. */
+int64_t awq_profile_last_ticket(void);
+int awq_profile_collect(int64_t ticket, float* ms, int n);
 const char* awq_profile_phase_name(int phase);
 /* Kernel launches the last call made (all of them this library's own kernels). */
 int awq_last_launch_count(void);

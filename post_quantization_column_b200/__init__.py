@@ -19,7 +19,7 @@ from dataclasses import dataclass
 import torch
 
 __all__ = [
-    "AwqError", "SearchOutput", "search", "search_host", "search_host_batch", "library", "library_path", "header_path",
+    "AwqError", "SearchOutput", "search", "search_async", "PendingSearch", "search_host", "search_host_batch", "library", "library_path", "header_path",
     "tile_shape", "workspace_bytes", "release_cached", "profile_enable", "profile_last",
     "last_launch_count", "debug_set_fault", "status_string", "exported_functions",
     "activation_statistic", "candidate_scales", "qdq_candidates", "ClipOutput", "clip_search",
@@ -66,6 +66,14 @@ def library() -> ctypes.CDLL:
     lib.awq_search_ex.argtypes = [vp, vp, i32, i64, i64, i64, i32, i32, vp, vp, vp, vp, f32p, f64p, i64, vp]
     lib.awq_search_host.argtypes = [vp, vp, i32, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp]
     lib.awq_search_host_batch.argtypes = [i32, vp, vp, i32, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp]
+    lib.awq_search_async.argtypes = [vp, vp, i32, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+    lib.awq_search_async.restype = ctypes.c_int
+    lib.awq_search_status.argtypes = [ctypes.c_int32]
+    lib.awq_search_status.restype = ctypes.c_int
+    lib.awq_profile_last_ticket.argtypes = []
+    lib.awq_profile_last_ticket.restype = ctypes.c_int64
+    lib.awq_profile_collect.argtypes = [ctypes.c_int64, ctypes.POINTER(ctypes.c_float), i32]
+    lib.awq_profile_collect.restype = ctypes.c_int
     for name in ("awq_search", "awq_search_f32", "awq_search_ex", "awq_search_host", "awq_search_host_batch",
                  "awq_release_cached",
                  "awq_profile_enable", "awq_profile_last", "awq_last_launch_count", "awq_debug_set_fault",
@@ -254,6 +262,62 @@ def search(X: torch.Tensor, W: torch.Tensor, group: int = 128, n_grid: int = 20,
                            tiles.numel() if tiles is not None else 0, _stream_handle(stream, X.device))
     _check(st)
     return SearchOutput(scales, codes, steps, zeros, losses, tiles)
+
+
+class PendingSearch:
+    """A search enqueued by search_async(): ``wait()`` synchronizes its stream, raises
+    AwqError if the kernels reported an error, and returns the SearchOutput;
+    ``profile()`` (after wait, with profiling on) gives the call's phase times in ms."""
+
+    def __init__(self, out: SearchOutput, status: torch.Tensor, stream, device, ticket: int):
+        self.out, self._status, self._stream, self._device, self._ticket = out, status, stream, device, ticket
+        self._done = False
+
+    def wait(self) -> SearchOutput:
+        if not self._done:
+            (self._stream or torch.cuda.current_stream(self._device)).synchronize()
+            self._done = True
+        _check(library().awq_search_status(int(self._status[0])))
+        return self.out
+
+    def profile(self) -> dict:
+        lib = library()
+        buf = (ctypes.c_float * 16)()
+        n = lib.awq_profile_collect(self._ticket, buf, 16) if self._ticket >= 0 else -1
+        if n < 0:
+            raise RuntimeError("no phase times for this call (profiling off, still running, or reused)")
+        return {lib.awq_profile_phase_name(i).decode(): float(buf[i]) for i in range(n)}
+
+
+def search_async(X: torch.Tensor, W: torch.Tensor, group: int = 128, n_grid: int = 20, *,
+                 stream: torch.cuda.Stream | None = None) -> PendingSearch:
+    """search() without waiting: the whole search is enqueued on ``stream`` and the call
+    returns at once, so consecutive layers run back to back on the device. Argument
+    errors raise here; errors the kernels detect raise from ``wait()``."""
+    if X.dim() != 2 or W.dim() != 2 or X.shape[1] != W.shape[0]:
+        raise ValueError("X must be (M, K) and W must be (K, N)")
+    if X.dtype != W.dtype:
+        raise TypeError("X and W must share a dtype")
+    if not (X.is_cuda and W.is_cuda):
+        raise ValueError("search_async() takes CUDA tensors")
+    lib = library()
+    X = X.contiguous()
+    W = W.contiguous()
+    M, K = X.shape
+    N = W.shape[1]
+    if group <= 0 or K % group or N % 8:
+        raise ValueError("group must divide K and N must be a multiple of 8")
+    scales, codes, steps, zeros, losses = _alloc_outputs(K, N, group, n_grid, X.device)
+    status = torch.full((1,), -1, dtype=torch.int32, pin_memory=True)
+    _check(lib.awq_search_async(_ptr(X), _ptr(W), _dtype_code(X), M, K, N, group, n_grid, _ptr(scales), _ptr(codes),
+                                _ptr(steps), _ptr(zeros), _ptr(losses), status.data_ptr(),
+                                _stream_handle(stream, X.device)))
+    ticket = int(lib.awq_profile_last_ticket())
+    out = SearchOutput(scales, codes, steps, zeros, losses, None)
+    # keep the inputs alive until the stream has passed the call
+    pending = PendingSearch(out, status, stream, X.device, ticket)
+    pending._inputs = (X, W)
+    return pending
 
 
 def activation_statistic(X: torch.Tensor, *, stream=None) -> torch.Tensor:

@@ -169,10 +169,16 @@ int check_device(int* dev, int* num_sms) {
   return AWQ_OK;
 }
 
-// Phase events, created once per device and reused by every profiled call.
+// Phase events of profiled calls: a ring of event sets per device, created once, so
+// that the times of an asynchronous call can still be read after later calls have been
+// enqueued (until the ring wraps). Each profiled call takes the next set and a ticket.
+constexpr int kEvRing = 256;
+thread_local int64_t t_last_ticket = -1;
+
 struct Events {
-  static cudaEvent_t cache[64][kNumPhases + 1];
+  static cudaEvent_t cache[64][kEvRing][kNumPhases + 1];
   static bool made[64];
+  static int64_t next[64];
   cudaEvent_t* ev = nullptr;
   cudaStream_t s = nullptr;
   void create(bool enable, cudaStream_t stream) {
@@ -180,12 +186,16 @@ struct Events {
     if (!enable) return;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return;
+    std::lock_guard<std::mutex> lock(g_mu);
     if (!made[dev]) {
-      for (auto& e : cache[dev])
-        if (cudaEventCreate(&e) != cudaSuccess) return;
+      for (auto& set : cache[dev])
+        for (auto& e : set)
+          if (cudaEventCreate(&e) != cudaSuccess) return;
       made[dev] = true;
     }
-    ev = cache[dev];
+    const int64_t ticket = next[dev]++;
+    ev = cache[dev][ticket % kEvRing];
+    t_last_ticket = ticket * 64 + dev;
   }
   void mark(int i) {
     if (ev) cudaEventRecord(ev[i], s);
@@ -194,9 +204,29 @@ struct Events {
     if (!ev) return;
     for (int i = 0; i < kNumPhases; ++i) cudaEventElapsedTime(&g_phase_ms[i], ev[i], ev[i + 1]);
   }
+  // phase times of the call with this ticket, once its events have completed; false if
+  // the ticket's set has been reused or its events are not complete
+  static bool collect_ticket(int64_t ticket, float* ms) {
+    if (ticket < 0) return false;
+    const int dev = static_cast<int>(ticket % 64);
+    const int64_t seq = ticket / 64;
+    cudaEvent_t* set = nullptr;
+    {
+      std::lock_guard<std::mutex> lock(g_mu);
+      if (!made[dev] || seq >= next[dev] || next[dev] - seq > kEvRing) return false;
+      set = cache[dev][seq % kEvRing];
+    }
+    for (int i = 0; i < kNumPhases; ++i)
+      if (cudaEventElapsedTime(&ms[i], set[i], set[i + 1]) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+      }
+    return true;
+  }
 };
-cudaEvent_t Events::cache[64][kNumPhases + 1];
+cudaEvent_t Events::cache[64][kEvRing][kNumPhases + 1];
 bool Events::made[64] = {false};
+int64_t Events::next[64] = {0};
 
 // A pinned host word per device for the kernels' status, so reading it back is one
 // asynchronous copy followed by the stream synchronisation the call does anyway.
@@ -523,6 +553,26 @@ int awq_search_ex(const void* X, const void* W, int in_dtype, int64_t M, int64_t
   t_last_error.clear();
   return search_device(X, W, in_dtype, M, K, N, group, n_grid, out_scales, out_codes, out_steps, out_zeros,
                        out_losses, out_tile_sq_err, tile_sq_err_len, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int awq_search_async(const void* X, const void* W, int in_dtype, int64_t M, int64_t K, int64_t N, int group,
+                     int n_grid, float* out_scales, int32_t* out_codes, void* out_steps, void* out_zeros,
+                     float* out_losses, int32_t* status_word, awq_stream_t stream) {
+  t_last_error.clear();
+  if (!status_word) return set_error(AWQ_ERR_INVALID_ARG, "status_word is NULL");
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, status_word) != cudaSuccess || attr.type != cudaMemoryTypeHost) {
+    cudaGetLastError();
+    return set_error(AWQ_ERR_INVALID_ARG, "status_word must be pinned host memory");
+  }
+  return search_device(X, W, in_dtype, M, K, N, group, n_grid, out_scales, out_codes, out_steps, out_zeros,
+                       out_losses, nullptr, 0, reinterpret_cast<cudaStream_t>(stream), nullptr, kQuantAsym,
+                       status_word);
+}
+
+int awq_search_status(int32_t status_word) {
+  t_last_error.clear();
+  return status_from_word(status_word);
 }
 
 int awq_search(const void* X, const void* W, int64_t M, int64_t K, int64_t N, int group, int n_grid,
@@ -1479,6 +1529,16 @@ int awq_profile_enable(int on) {
 
 int awq_profile_last(float* ms, int n) {
   for (int i = 0; i < n && i < kNumPhases; ++i) ms[i] = g_phase_ms[i];
+  return kNumPhases;
+}
+
+int64_t awq_profile_last_ticket(void) { return t_last_ticket; }
+
+int awq_profile_collect(int64_t ticket, float* ms, int n) {
+  if (!ms || n < 0) return -1;
+  float all[kNumPhases];
+  if (!Events::collect_ticket(ticket, all)) return -1;
+  for (int i = 0; i < n && i < kNumPhases; ++i) ms[i] = all[i];
   return kNumPhases;
 }
 

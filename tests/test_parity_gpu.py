@@ -149,6 +149,56 @@ def test_nonfinite_inputs_are_rejected():
     awq.search(X.cuda(), W.cuda())
 
 
+def test_async_searches_back_to_back_match_the_synchronous_call():
+    """Four layers enqueued through search_async without waiting (different shapes and
+    dtypes on one stream), then waited for: each gives the synchronous call's artifact and
+    losses bit for bit, and profiled calls keep their own phase times."""
+    specs = [custom_spec(256, 384, 520, seed=50), custom_spec(300, 256, 264, dtype="f32", group=64, seed=51),
+             custom_spec(128, 512, 128, seed=52), custom_spec(256, 384, 520, seed=53)]
+    layers = [tuple(t.cuda() for t in generate(s)) for s in specs]
+    awq.profile_enable(True)
+    try:
+        pend = [awq.search_async(X, W, s.group, s.n_grid) for s, (X, W) in zip(specs, layers)]
+        outs = [p.wait() for p in pend]
+        profs = [p.profile() for p in pend]
+    finally:
+        awq.profile_enable(False)
+    for s, (X, W), o, prof in zip(specs, layers, outs, profs):
+        d = awq.search(X, W, s.group, s.n_grid)
+        for name in ("scales", "codes", "steps", "zeros", "losses"):
+            assert torch.equal(getattr(d, name), getattr(o, name)), (s.name, name)
+        assert set(prof) >= {"statistic", "qdq", "gemm_loss", "pack"}
+        assert all(v >= 0.0 for v in prof.values()) and prof["gemm_loss"] > 0.0
+
+
+def test_async_search_reports_kernel_errors_on_wait():
+    spec = custom_spec(64, 128, 64, seed=3)
+    X, W = generate(spec)
+    Xn = X.clone()
+    Xn[5, 7] = float("nan")
+    bad = awq.search_async(Xn.cuda(), W.cuda())
+    good = awq.search_async(X.cuda(), W.cuda())
+    with pytest.raises(awq.AwqError) as e:
+        bad.wait()
+    assert e.value.status == 3
+    ref = awq.search(X.cuda(), W.cuda())
+    assert torch.equal(good.wait().codes, ref.codes)
+
+
+def test_async_search_needs_a_pinned_status_word():
+    import ctypes
+    lib = awq.library()
+    X = torch.zeros(16, 128, dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros(128, 64, dtype=torch.bfloat16, device="cuda")
+    outs = awq._alloc_outputs(128, 64, 128, 20, X.device)
+    word = (ctypes.c_int32 * 1)()  # pageable host memory
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    st = lib.awq_search_async(p(X), p(W), 0, 16, 128, 64, 128, 20, p(outs[0]), p(outs[1]), p(outs[2]), p(outs[3]),
+                              p(outs[4]), ctypes.cast(word, ctypes.c_void_p),
+                              ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 1  # AWQ_ERR_INVALID_ARG
+
+
 def test_host_pointer_is_rejected_by_the_device_entry_point():
     import ctypes
     lib = awq.library()
