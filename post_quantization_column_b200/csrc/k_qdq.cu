@@ -462,14 +462,15 @@ __global__ void __launch_bounds__(Tile<G>::kThreads, Tile<G>::kBlocksPerSm)
 }
 
 // Lane layout of the pack kernel: each warp quantizes one group x kCols strip on its
-// own, with no shared memory and no block barrier. Lane (lr, lc) = (lane / 4, lane % 4)
+// own, with no shared memory and no block barrier. Lane (lr, lc) = (lane / LC, lane % LC)
 // holds the 16-byte vector of VEC adjacent columns (lc VEC .. lc VEC + VEC - 1 of the
-// strip) in rows lr, lr + 8, ..., so every load instruction reads eight 64-byte row runs.
+// strip) in rows lr, lr + LR, ..., so every load instruction reads eight 64-byte row runs.
+// (Two lanes across and 16 down, at 80 registers and 24 warps per SM, ran no faster.)
 template <typename T, int G>
 struct PackShape {
   static constexpr int VEC = 16 / sizeof(T);  // columns per lane: 8 (bf16) or 4 (fp32)
   static constexpr int LC = 4;                // lanes across the strip
-  static constexpr int LR = 8;                // lanes down the group
+  static constexpr int LR = 32 / LC;          // lanes down the group
   static constexpr int RPL = G / LR;          // rows per lane: 16, 8, 4
   static constexpr int kCols = LC * VEC;      // columns per warp: 32 or 16
   static constexpr int kWarps = 4;
@@ -518,7 +519,7 @@ __global__ void __launch_bounds__(PackShape<T, G>::kThreads, 4)
   uint4 raw[P::RPL];
   if (active) {
 #pragma unroll
-    for (int i = 0; i < P::RPL; ++i) raw[i] = __ldcs(reinterpret_cast<const uint4*>(W + (k0 + lr + 8 * i) * N + nl));
+    for (int i = 0; i < P::RPL; ++i) raw[i] = __ldcs(reinterpret_cast<const uint4*>(W + (k0 + lr + P::LR * i) * N + nl));
   } else {
 #pragma unroll
     for (int i = 0; i < P::RPL; ++i) raw[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -541,10 +542,10 @@ __global__ void __launch_bounds__(PackShape<T, G>::kThreads, 4)
   const float* Sb = S + static_cast<int64_t>(best) * K + k0;
   float s[P::RPL];
 #pragma unroll
-  for (int i = 0; i < P::RPL; ++i) s[i] = Sb[lr + 8 * i];
+  for (int i = 0; i < P::RPL; ++i) s[i] = Sb[lr + P::LR * i];
   if (n0 == 0 && lc == 0) {
 #pragma unroll
-    for (int i = 0; i < P::RPL; ++i) out_scales[k0 + lr + 8 * i] = s[i];
+    for (int i = 0; i < P::RPL; ++i) out_scales[k0 + lr + P::LR * i] = s[i];
   }
 
   // group range of the lane's columns, then across the row-lanes
@@ -618,7 +619,7 @@ __global__ void __launch_bounds__(PackShape<T, G>::kThreads, 4)
   for (int i = 0; i < P::RPL; ++i) {
     float w[VEC];
     unpack16<T>(raw[i], w);
-    const float si = reload_f32(Sb + lr + 8 * i);
+    const float si = reload_f32(Sb + lr + P::LR * i);
     uint32_t word = 0;
     bool need = false;
 #pragma unroll
@@ -632,9 +633,9 @@ __global__ void __launch_bounds__(PackShape<T, G>::kThreads, 4)
     redo |= static_cast<uint32_t>(need) << i;
     if (active) {
       if (VEC == 8)
-        crow[(lr + 8 * i) * words] = static_cast<int32_t>(word);
+        crow[(lr + P::LR * i) * words] = static_cast<int32_t>(word);
       else
-        reinterpret_cast<uint16_t*>(crow + (lr + 8 * i) * words)[lc & 1] = static_cast<uint16_t>(word);
+        reinterpret_cast<uint16_t*>(crow + (lr + P::LR * i) * words)[lc & 1] = static_cast<uint16_t>(word);
     }
   }
   if (col_exact) redo = (1u << P::RPL) - 1u;
@@ -643,7 +644,7 @@ __global__ void __launch_bounds__(PackShape<T, G>::kThreads, 4)
   while (redo && active) {
     const int i = __ffs(redo) - 1;
     redo &= redo - 1;
-    const int64_t r = lr + 8 * i;
+    const int64_t r = lr + P::LR * i;
     const uint4 v = *reinterpret_cast<const uint4*>(W + (k0 + r) * N + nl);
     const float sv = Sb[r];
     float w[VEC];
