@@ -485,6 +485,22 @@ __device__ __forceinline__ float reload_f32(const float* p) {
   return v;
 }
 
+// The VEC values of a 16-byte vector times s, as pairs (bf16 widened by a shift or a mask).
+template <typename T>
+__device__ __forceinline__ void scaled_pairs(const uint4& raw, float s, float2 (&out)[8 / sizeof(T)]) {
+  const float2 s2 = make_float2(s, s);
+  const uint32_t u[4] = {raw.x, raw.y, raw.z, raw.w};
+  if constexpr (sizeof(T) == 2) {
+#pragma unroll
+    for (int h = 0; h < 4; ++h)
+      out[h] = __fmul2_rn(s2, make_float2(__uint_as_float(u[h] << 16), __uint_as_float(u[h] & 0xFFFF0000u)));
+  } else {
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      out[h] = __fmul2_rn(s2, make_float2(__uint_as_float(u[2 * h]), __uint_as_float(u[2 * h + 1])));
+  }
+}
+
 template <typename T>
 __device__ __forceinline__ void unpack16(const uint4& raw, float (&w)[16 / sizeof(T)]) {
   const T* e = reinterpret_cast<const T*>(&raw);
@@ -548,7 +564,8 @@ __global__ void __launch_bounds__(PackShape<T, G>::kThreads, 4)
     for (int i = 0; i < P::RPL; ++i) out_scales[k0 + lr + P::LR * i] = s[i];
   }
 
-  // group range of the lane's columns, then across the row-lanes
+  // group range of the lane's columns over its rows (two rows per three-input min / max),
+  // then across the row-lanes
   float mn[VEC], mx[VEC];
 #pragma unroll
   for (int j = 0; j < VEC; ++j) {
@@ -556,14 +573,16 @@ __global__ void __launch_bounds__(PackShape<T, G>::kThreads, 4)
     mx[j] = -INFINITY;
   }
 #pragma unroll
-  for (int i = 0; i < P::RPL; ++i) {
-    float w[VEC];
-    unpack16<T>(raw[i], w);
+  for (int i = 0; i < P::RPL; i += 2) {
+    float2 a[VEC / 2], b[VEC / 2];
+    scaled_pairs<T>(raw[i], s[i], a);
+    scaled_pairs<T>(raw[i + 1], s[i + 1], b);
 #pragma unroll
-    for (int j = 0; j < VEC; ++j) {
-      const float wp = __fmul_rn(s[i], w[j]);
-      mn[j] = fminf(mn[j], wp);
-      mx[j] = fmaxf(mx[j], wp);
+    for (int h = 0; h < VEC / 2; ++h) {
+      mn[2 * h] = fmin3(mn[2 * h], a[h].x, b[h].x);
+      mx[2 * h] = fmax3(mx[2 * h], a[h].x, b[h].x);
+      mn[2 * h + 1] = fmin3(mn[2 * h + 1], a[h].y, b[h].y);
+      mx[2 * h + 1] = fmax3(mx[2 * h + 1], a[h].y, b[h].y);
     }
   }
 #pragma unroll
@@ -591,51 +610,63 @@ __global__ void __launch_bounds__(PackShape<T, G>::kThreads, 4)
     steps[o] = __float2half_rn(pc.step);
     zeros[o] = __float2half_rn(pc.zero);
   }
-  QdqParams p[VEC];
-  float rcp[VEC];
-  int zi[VEC];
+  // per column: 1/step, the clamp bounds lo = -z and hi = qmax - z (integers, so z = -lo
+  // and qmax = hi - lo exactly), -(1.5 2^23 + z), and the step for the exact path
+  float rcp[VEC], lo[VEC], hi[VEC], nmz[VEC], stp[VEC];
   bool col_exact = false;
 #pragma unroll
   for (int j = 0; j < VEC; ++j) {
     const int src = j * P::LC + lc;
-    p[j].step = __shfl_sync(0xffffffffu, pc.step, src);
-    p[j].zero = __shfl_sync(0xffffffffu, pc.zero, src);
-    p[j].qmax = pc.qmax;
+    stp[j] = __shfl_sync(0xffffffffu, pc.step, src);
+    const float z = __shfl_sync(0xffffffffu, pc.zero, src);
     rcp[j] = __shfl_sync(0xffffffffu, rc, src);
     col_exact |= __shfl_sync(0xffffffffu, exact_c, src) != 0;
-    zi[j] = static_cast<int>(p[j].zero);
+    lo[j] = -z;
+    hi[j] = __fsub_rn(pc.qmax, z);
+    nmz[j] = -__fadd_rn(kRoundMagic, z);
   }
 
-  // codes: q - z = rint(clamp(w' (1/step), -z, qmax - z)); 1.5 2^23 + (q - z) carries q - z
-  // in its low bits, so (bits + z) & 15 is the code. W' is formed again from the raw
-  // vectors (the empty asm hides them from the compiler, which would otherwise keep the
-  // first pass's VEC x RPL products live in registers).
+  // codes: t = clamp(w' (1/step), -z, qmax - z); m = RN(t + 1.5 2^23 + z) holds rint(t) + z
+  // = q in its low bits (the two agree unless t is a half-integer, which the check below
+  // sends to the exact path). The low bytes of a row's m values are gathered with byte
+  // permutes and their low nibbles merged into the packed word. W' is formed again from
+  // the raw vectors (the empty asm hides them from the compiler, which would otherwise keep
+  // the first pass's VEC x RPL products live in registers).
 #pragma unroll
   for (int i = 0; i < P::RPL; ++i)
     asm volatile("" : "+r"(raw[i].x), "+r"(raw[i].y), "+r"(raw[i].z), "+r"(raw[i].w));
+  const float2 minus1 = make_float2(-1.0f, -1.0f);
   uint32_t redo = 0;
   int32_t* const crow = codes + k0 * words + nl / 8;
 #pragma unroll
   for (int i = 0; i < P::RPL; ++i) {
-    float w[VEC];
-    unpack16<T>(raw[i], w);
-    const float si = reload_f32(Sb + lr + P::LR * i);
-    uint32_t word = 0;
-    bool need = false;
+    float2 wp[VEC / 2];
+    scaled_pairs<T>(raw[i], reload_f32(Sb + lr + P::LR * i), wp);
+    uint32_t mb[VEC];
+    float dmax = 0.0f;
 #pragma unroll
-    for (int j = 0; j < VEC; ++j) {
-      const float wp = __fmul_rn(si, w[j]);
-      const float tc = fminf(fmaxf(__fmul_rn(wp, rcp[j]), -p[j].zero), p[j].qmax - p[j].zero);
-      const float m = __fadd_rn(tc, kRoundMagic);
-      need |= fabsf(__fsub_rn(tc, __fsub_rn(m, kRoundMagic))) >= kNearHalf;
-      word |= ((__float_as_uint(m) + static_cast<uint32_t>(zi[j])) & 0xFu) << (4 * j);
+    for (int h = 0; h < VEC / 2; ++h) {
+      float2 tc = __fmul2_rn(wp[h], make_float2(rcp[2 * h], rcp[2 * h + 1]));
+      tc.x = fminf(fmaxf(tc.x, lo[2 * h]), hi[2 * h]);
+      tc.y = fminf(fmaxf(tc.y, lo[2 * h + 1]), hi[2 * h + 1]);
+      const float2 nm = make_float2(nmz[2 * h], nmz[2 * h + 1]);
+      const float2 m = __ffma2_rn(nm, minus1, tc);         // t + 1.5 2^23 + z, rounded once
+      const float2 d = __ffma2_rn(__fadd2_rn(m, nm), minus1, tc);  // t - rint(t), exact
+      dmax = fmax3(dmax, fabsf(d.x), fabsf(d.y));
+      mb[2 * h] = __float_as_uint(m.x);
+      mb[2 * h + 1] = __float_as_uint(m.y);
     }
-    redo |= static_cast<uint32_t>(need) << i;
+    redo |= static_cast<uint32_t>(dmax >= kNearHalf) << i;
     if (active) {
-      if (VEC == 8)
-        crow[(lr + P::LR * i) * words] = static_cast<int32_t>(word);
-      else
-        reinterpret_cast<uint16_t*>(crow + (lr + P::LR * i) * words)[lc & 1] = static_cast<uint16_t>(word);
+      if constexpr (VEC == 8) {
+        const uint32_t ev = __byte_perm(__byte_perm(mb[0], mb[2], 0x0040), __byte_perm(mb[4], mb[6], 0x0040), 0x5410);
+        const uint32_t od = __byte_perm(__byte_perm(mb[1], mb[3], 0x0040), __byte_perm(mb[5], mb[7], 0x0040), 0x5410);
+        crow[(lr + P::LR * i) * words] = static_cast<int32_t>((ev & 0x0F0F0F0Fu) | ((od << 4) & 0xF0F0F0F0u));
+      } else {
+        const uint32_t ev = __byte_perm(mb[0], mb[2], 0x0040), od = __byte_perm(mb[1], mb[3], 0x0040);
+        reinterpret_cast<uint16_t*>(crow + (lr + P::LR * i) * words)[lc & 1] =
+            static_cast<uint16_t>((ev & 0x0F0Fu) | ((od << 4) & 0xF0F0u));
+      }
     }
   }
   if (col_exact) redo = (1u << P::RPL) - 1u;
@@ -651,8 +682,10 @@ __global__ void __launch_bounds__(PackShape<T, G>::kThreads, 4)
     unpack16<T>(v, w);
     uint32_t word = 0;
 #pragma unroll
-    for (int j = 0; j < VEC; ++j)
-      word |= static_cast<uint32_t>(qdq_code(__fmul_rn(sv, w[j]), p[j])) << (4 * j);
+    for (int j = 0; j < VEC; ++j) {
+      const QdqParams pj{stp[j], -lo[j], __fsub_rn(hi[j], lo[j])};
+      word |= static_cast<uint32_t>(qdq_code(__fmul_rn(sv, w[j]), pj)) << (4 * j);
+    }
     if (VEC == 8)
       crow[r * words] = static_cast<int32_t>(word);
     else
