@@ -76,12 +76,11 @@ int get_pool(int dev, cudaMemPool_t* out) {
 }
 
 struct Layout {
-  size_t err, a, stat_partial, S, best, losses, Xb, Wt, Y, loss_partial, total;
-  int row_chunks;
+  size_t err, a, S, best, losses, Xb, Wt, Y, loss_partial, total;
   int64_t tiles;
 };
 
-Layout plan(int in_dtype, int64_t M, int64_t K, int64_t N, int n_grid, int num_sms) {
+Layout plan(int in_dtype, int64_t M, int64_t K, int64_t N, int n_grid) {
   Layout L;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -89,12 +88,10 @@ Layout plan(int in_dtype, int64_t M, int64_t K, int64_t N, int n_grid, int num_s
     off += align_up(bytes);
     return at;
   };
-  L.row_chunks = statistic_row_chunks(M, K, in_dtype, num_sms);
   const int64_t tiles_m = ceil_div(M, kTileM), tiles_n = ceil_div(N, kTileN);
   L.tiles = tiles_m * tiles_n;
   L.err = take(16 + static_cast<size_t>(L.tiles) * 4);  // status word, then the loss GEMM's per-tile flags
   L.a = take(static_cast<size_t>(K) * 4);
-  L.stat_partial = take(static_cast<size_t>(L.row_chunks) * K * 8);
   L.S = take(static_cast<size_t>(n_grid) * K * 4);
   L.best = take(16);
   L.losses = take(static_cast<size_t>(n_grid) * 4);
@@ -380,7 +377,7 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
       !is_device_memory(out_codes) || !is_device_memory(out_steps) || !is_device_memory(out_zeros) ||
       (out_losses && !is_device_memory(out_losses)) || (out_tile_sq_err && !is_device_memory(out_tile_sq_err)))
     return set_error(AWQ_ERR_INVALID_ARG, "inputs and outputs must be device memory (use awq_search_host for host buffers)");
-  const Layout L = plan(in_dtype, M, K, N, n_grid, num_sms);
+  const Layout L = plan(in_dtype, M, K, N, n_grid);
   if (out_tile_sq_err && tile_sq_err_len < static_cast<int64_t>(n_grid) * L.tiles)
     return set_error(AWQ_ERR_INVALID_ARG, "out_tile_sq_err holds fewer than n_grid * tiles values");
 
@@ -396,7 +393,6 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
   uint8_t* base = static_cast<uint8_t*>(ws);
   int* err = reinterpret_cast<int*>(base + L.err);
   float* a = reinterpret_cast<float*>(base + L.a);
-  double* stat_partial = reinterpret_cast<double*>(base + L.stat_partial);
   float* S = reinterpret_cast<float*>(base + L.S);
   int* best = reinterpret_cast<int*>(base + L.best);
   float* losses = reinterpret_cast<float*>(base + L.losses);
@@ -419,7 +415,7 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
     }
     if (feed && (e = cudaStreamWaitEvent(s, feed->x_ready, 0)) != cudaSuccess) { where = "waiting for X"; break; }
     ev.mark(kPhStatistic);
-    if ((e = launch_statistic(X, in_dtype, M, K, L.row_chunks, stat_partial, a, err, s, &launches)) != cudaSuccess) {
+    if ((e = launch_statistic(X, in_dtype, M, K, a, err, s, &launches)) != cudaSuccess) {
       where = "statistic kernel";
       break;
     }
@@ -846,19 +842,16 @@ int awq_activation_statistic(const void* X, int in_dtype, int64_t M, int64_t K, 
     return set_error(AWQ_ERR_INVALID_ARG, "X and out_a must be device memory");
   cudaMemPool_t pool;
   if ((st = get_pool(dev, &pool)) != AWQ_OK) return st;
-  const int R = statistic_row_chunks(M, K, in_dtype, num_sms);
-  const size_t bytes = 256 + align_up(static_cast<size_t>(R) * K * 8);
   void* ws = nullptr;
-  cudaError_t e = cudaMallocFromPoolAsync(&ws, bytes, pool, s);
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, 256, pool, s);  // the status word
   if (e != cudaSuccess || !ws) {
     cudaGetLastError();
     return set_error(AWQ_ERR_OOM, "statistic work space");
   }
   int* err = static_cast<int*>(ws);
-  double* partial = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + 256);
   int launches = 0, h_err = 0;
   if ((e = cudaMemsetAsync(err, 0, 16, s)) == cudaSuccess &&
-      (e = launch_statistic(X, in_dtype, M, K, R, partial, out_a, err, s, &launches)) == cudaSuccess)
+      (e = launch_statistic(X, in_dtype, M, K, out_a, err, s, &launches)) == cudaSuccess)
     e = cudaMemcpyAsync(&h_err, err, sizeof(int), cudaMemcpyDeviceToHost, s);
   cudaFreeAsync(ws, s);
   cudaError_t se = cudaStreamSynchronize(s);
@@ -1302,7 +1295,7 @@ int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_d
   const char* where = "";
   do {
     if ((e = cudaMemsetAsync(err, 0, 16, s)) != cudaSuccess) { where = "cudaMemsetAsync"; break; }
-    if ((e = launch_statistic(X, in_dtype, M, K, 1, nullptr, a, err, s, &launches)) != cudaSuccess) {
+    if ((e = launch_statistic(X, in_dtype, M, K, a, err, s, &launches)) != cudaSuccess) {
       where = "statistic kernel";
       break;
     }
@@ -1493,7 +1486,7 @@ int64_t awq_workspace_bytes(int in_dtype, int64_t M, int64_t K, int64_t N, int g
   static int dummy;
   if (validate(&dummy, &dummy, in_dtype, M, K, N, group, n_grid, &dummy, &dummy, &dummy, &dummy, false) != AWQ_OK)
     return 0;
-  return static_cast<int64_t>(plan(in_dtype, M, K, N, n_grid, 148).total);
+  return static_cast<int64_t>(plan(in_dtype, M, K, N, n_grid).total);
 }
 
 int awq_release_cached(void) {

@@ -15,10 +15,8 @@ constexpr int kTileN = 256;
 constexpr int kTileK = 64;
 
 // ---- statistic (AWQ-P1 §1) -------------------------------------------------------
-// Number of row chunks the first pass splits M into for a K of this size.
-int statistic_row_chunks(int64_t M, int64_t K, int in_dtype, int num_sms);
-cudaError_t launch_statistic(const void* X, int in_dtype, int64_t M, int64_t K, int row_chunks,
-                             double* partial, float* a, int* err, cudaStream_t s, int* launches);
+cudaError_t launch_statistic(const void* X, int in_dtype, int64_t M, int64_t K, float* a, int* err, cudaStream_t s,
+                             int* launches);
 
 // ---- candidate scales (AWQ-P1 §3-§4) ---------------------------------------------
 cudaError_t launch_scales(const float* a, int64_t K, int n_grid, float* S, cudaStream_t s,

@@ -116,7 +116,6 @@ extern "C" int awq_search_noalloc(const void* X, const void* W, int in_dtype, in
     return noalloc_fail(AWQ_ERR_INVALID_ARG, "inputs and outputs must be device memory");
 
   // carve the work space out of the fixed array (same pieces as the pooled entry points)
-  const int row_chunks = statistic_row_chunks(M, K, in_dtype, num_sms);
   const int64_t tiles = ceil_div(M, kTileM) * ceil_div(N, kTileN);
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -124,7 +123,7 @@ extern "C" int awq_search_noalloc(const void* X, const void* W, int in_dtype, in
     off += round256(bytes);
     return at;
   };
-  const size_t o_err = take(16), o_a = take(size_t(K) * 4), o_part = take(size_t(row_chunks) * K * 8),
+  const size_t o_err = take(16), o_a = take(size_t(K) * 4),
                o_S = take(size_t(n_grid) * K * 4), o_best = take(16), o_loss = take(size_t(n_grid) * 4),
                o_Xb = in_dtype == AWQ_DTYPE_F32 ? take(size_t(M) * K * 2) : 0,
                o_Wt = take(size_t(n_grid + 1) * N * K * 2), o_Y = take(size_t(tiles) * kTileM * kTileN * 4),
@@ -141,7 +140,6 @@ extern "C" int awq_search_noalloc(const void* X, const void* W, int in_dtype, in
   uint8_t* base = static_cast<uint8_t*>(scratch);
   int* err = reinterpret_cast<int*>(base + o_err);
   float* a = reinterpret_cast<float*>(base + o_a);
-  double* stat_partial = reinterpret_cast<double*>(base + o_part);
   float* S = reinterpret_cast<float*>(base + o_S);
   int* best = reinterpret_cast<int*>(base + o_best);
   float* losses = reinterpret_cast<float*>(base + o_loss);
@@ -155,7 +153,7 @@ extern "C" int awq_search_noalloc(const void* X, const void* W, int in_dtype, in
   const char* where = "";
   do {
     if ((e = cudaMemsetAsync(err, 0, 16, s)) != cudaSuccess) { where = "clearing the status word"; break; }
-    if ((e = launch_statistic(X, in_dtype, M, K, row_chunks, stat_partial, a, err, s, &launches)) != cudaSuccess) {
+    if ((e = launch_statistic(X, in_dtype, M, K, a, err, s, &launches)) != cudaSuccess) {
       where = "statistic kernel";
       break;
     }

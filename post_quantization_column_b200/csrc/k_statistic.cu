@@ -164,10 +164,8 @@ __global__ void to_bf16_kernel(const float4* __restrict__ x, int64_t n4, uint2* 
 
 }  // namespace
 
-int statistic_row_chunks(int64_t, int64_t, int, int) { return 1; }
-
-cudaError_t launch_statistic(const void* X, int in_dtype, int64_t M, int64_t K, int /*row_chunks*/,
-                             double* /*partial*/, float* a, int* err, cudaStream_t s, int* launches) {
+cudaError_t launch_statistic(const void* X, int in_dtype, int64_t M, int64_t K, float* a, int* err, cudaStream_t s,
+                             int* launches) {
   // Clusters of 8 column vectors (64 bf16 / 32 fp32 columns, 128-byte row segments) while
   // they fit in one wave of resident CTAs; wider clusters of 16 vectors (256-byte
   // segments) for larger K, which halves the CTAs and keeps the grid to about one wave.
