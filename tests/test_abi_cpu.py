@@ -105,3 +105,13 @@ def test_clip_search_validation_happens_on_the_host(lib):
     assert b"group" in lib.awq_last_error_message()
     assert lib.awq_clip_search(*args(quantizer=2)) == 1
     assert b"quantizer" in lib.awq_last_error_message()
+
+
+def test_plain_c_client_compiles_against_the_header(lib, tmp_path):
+    """tests/c/awq_client.c (C99, -Wall -Werror) builds against include/awq_search.h and
+    links with libawqsearch.so and the CUDA runtime: the boundary is usable from C."""
+    from tests import c_client
+    if not c_client.compiler() or not os.path.exists(os.path.join(c_client.CUDA, "include", "cuda_runtime_api.h")):
+        pytest.skip("no C compiler or CUDA headers")
+    exe = c_client.build(str(tmp_path))
+    assert os.path.exists(exe)
