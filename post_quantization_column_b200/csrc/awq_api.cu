@@ -180,6 +180,7 @@ struct Events {
   cudaStream_t s = nullptr;
   void create(bool enable, cudaStream_t stream) {
     s = stream;
+    t_last_ticket = -1;  // an unprofiled call has no ticket
     if (!enable) return;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return;

@@ -171,6 +171,20 @@ def test_async_searches_back_to_back_match_the_synchronous_call():
         assert all(v >= 0.0 for v in prof.values()) and prof["gemm_loss"] > 0.0
 
 
+def test_unprofiled_async_call_has_no_phase_times():
+    spec = custom_spec(128, 256, 264, seed=54)
+    X, W = (t.cuda() for t in generate(spec))
+    awq.profile_enable(True)
+    try:
+        awq.search_async(X, W).wait()
+    finally:
+        awq.profile_enable(False)
+    p = awq.search_async(X, W)
+    p.wait()
+    with pytest.raises(RuntimeError):
+        p.profile()
+
+
 def test_async_search_reports_kernel_errors_on_wait():
     spec = custom_spec(64, 128, 64, seed=3)
     X, W = generate(spec)
