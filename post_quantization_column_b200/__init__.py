@@ -275,7 +275,7 @@ class PendingSearch:
 
     def wait(self) -> SearchOutput:
         if not self._done:
-            (self._stream or torch.cuda.current_stream(self._device)).synchronize()
+            self._stream.synchronize()
             self._done = True
         _check(library().awq_search_status(int(self._status[0])))
         return self.out
@@ -309,6 +309,8 @@ def search_async(X: torch.Tensor, W: torch.Tensor, group: int = 128, n_grid: int
         raise ValueError("group must divide K and N must be a multiple of 8")
     scales, codes, steps, zeros, losses = _alloc_outputs(K, N, group, n_grid, X.device)
     status = torch.full((1,), -1, dtype=torch.int32, pin_memory=True)
+    if stream is None:  # the stream current now is the one wait() synchronizes later
+        stream = torch.cuda.current_stream(X.device)
     _check(lib.awq_search_async(_ptr(X), _ptr(W), _dtype_code(X), M, K, N, group, n_grid, _ptr(scales), _ptr(codes),
                                 _ptr(steps), _ptr(zeros), _ptr(losses), status.data_ptr(),
                                 _stream_handle(stream, X.device)))
