@@ -9,7 +9,8 @@ import numpy as np
 import pytest
 import torch
 
-from workloads import WORKLOADS, LayerSpec, as_f32_numpy, custom_spec, generate, generate_down, outlier_channels
+from workloads import (WORKLOADS, LayerSpec, as_f32_numpy, custom_spec, generate, generate_down, generate_qkv,
+                       outlier_channels)
 
 
 def test_the_five_layers():
@@ -89,3 +90,20 @@ def test_down_projection_is_drawn_from_its_own_substream():
     assert torch.equal(W.view(torch.int16), W2.view(torch.int16))
     with pytest.raises(ValueError):  # [gate | up] needs an even column count
         generate_down(LayerSpec("odd", 16, 256, 135, "bf16", "normal", 0.5, 20.0, 0.02), 96)
+
+
+def test_qkv_projections_extend_the_query_layer():
+    """An attention block's [W_q | W_k | W_v]: W_q is the layer's own W, W_k and W_v come from
+    their own substreams with the layer's weight spread, and X is unchanged."""
+    spec = custom_spec(32, 256, 256, seed=11)
+    X, W = generate(spec)
+    Wqkv = generate_qkv(spec)
+    assert Wqkv.shape == (256, 768) and Wqkv.dtype == torch.bfloat16
+    assert torch.equal(Wqkv[:, :256], W)
+    Wk, Wv = as_f32_numpy(Wqkv[:, 256:512]), as_f32_numpy(Wqkv[:, 512:])
+    for part in (Wk, Wv):
+        assert abs(float(part.std()) - spec.w_std) < 0.05 * spec.w_std
+    assert not np.array_equal(Wk, Wv) and not np.array_equal(Wk, as_f32_numpy(W))
+    assert torch.equal(generate(spec)[0], X)
+    with pytest.raises(ValueError):
+        generate_qkv(custom_spec(16, 256, 512, seed=1))

@@ -129,3 +129,21 @@ def generate_down(spec: LayerSpec, K_out: int, w_std: float = 0.015) -> torch.Te
     w *= np.float32(w_std)
     t = torch.from_numpy(w)
     return t.to(torch.bfloat16) if spec.dtype == "bf16" else t
+
+
+def generate_qkv(spec: LayerSpec) -> torch.Tensor:
+    """[W_q | W_k | W_v] (K x 3K) of an attention block whose query projection is
+    `generate(spec)`'s W (K x K): the key and value projections are drawn from their own
+    Philox substreams (the sixth and seventh of the layer's seed), N(0, w_std), so X and
+    W_q are unchanged. Same storage dtype as the layer."""
+    if spec.N != spec.K:
+        raise ValueError("the query projection of an attention block is square (K x K)")
+    _, W_q = generate(spec)
+    streams = _streams(spec.seed, 7)
+    parts = [W_q.float()]
+    for g in streams[5:7]:
+        w = g.standard_normal((spec.K, spec.K), dtype=np.float32)
+        w *= np.float32(spec.w_std)
+        parts.append(torch.from_numpy(w))
+    W = torch.cat(parts, dim=1).contiguous()
+    return W.to(torch.bfloat16) if spec.dtype == "bf16" else W
