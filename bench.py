@@ -4,6 +4,9 @@
 One step = one complete search of one synthetic layer (statistic, 20 candidate scale
 vectors, QDQ + fold-back of every candidate, the reference GEMM, 20 candidate GEMMs
 with the fused squared-error epilogue, argmin, packing) through the library's C ABI.
+The headline layer is the largest one, the Llama-70B-shaped gate+up projection
+(16384 x 8192 x 57344); the other four layers of the workload set are timed in the
+same run and reported as objects of the same line (``workloads``).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
@@ -33,14 +36,16 @@ import torch  # noqa: E402
 from workloads import WORKLOADS, LayerSpec, generate, as_f32_numpy  # noqa: E402
 
 METRIC = "AWQ search candidate-GEMM TFLOP/s & layers/s; % of BF16 tensor peak"
-DEFAULT_WORKLOAD = "llama7b_attn_proj_4096x4096x4096"
+DEFAULT_WORKLOAD = "llama70b_mlp_gate_up_16384x8192x57344"
+# the layer the clipping search, the W4A16 consumer and the kernel-level objects run on
+SIDE_WORKLOAD = "llama7b_attn_proj_4096x4096x4096"
 FLUSH_BYTES = 256 << 20   # > 126 MB L2
 
 
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
@@ -50,6 +55,12 @@ def parse_args(argv=None):
     ap.add_argument("--no-clip", action="store_true", help="skip the clipping-search measurement")
     ap.add_argument("--no-w4a16", action="store_true", help="skip the W4A16 consumer measurement")
     ap.add_argument("--no-mlp-block", action="store_true", help="skip the MLP-block objective measurement")
+    ap.add_argument("--no-attn-block", action="store_true", help="skip the attention-block objective measurement")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="time only the headline layer (skip the other layers' objects)")
+    ap.add_argument("--slice-columns", type=int, default=0,
+                    help="search a column slice of the layer instead: the first C columns of each half of a "
+                         "[gate | up] layer (2C columns), else the first C; full X. For sized profiling captures")
     return ap.parse_args(argv)
 
 
@@ -146,10 +157,11 @@ class ClockSampler:
                 "power_w_median": statistics.median(watts) if watts else None}
 
 
-def cpu_oracle_sample(spec: LayerSpec, target_s: float):
+def cpu_oracle_sample(spec: LayerSpec, target_s: float, X=None, W=None):
     """Time the oracle as it stands on a column slice of the layer (full X)."""
     import oracle as O
-    X, W = generate(spec)
+    if X is None:
+        X, W = generate(spec)
     X32, W32 = as_f32_numpy(X), as_f32_numpy(W)
 
     def run(ncols):
@@ -319,6 +331,67 @@ def measure_mlp_block(awq, stream, flush, steps: int, peaks, k_out: int = 4096):
                          "work": "(n_grid + 1) x (2 M K 2F + 2 M F K_out) flops over the whole call"}}
 
 
+ATTN_BLOCK = "llama7b_attn_proj_4096x4096x4096"  # the query projection; 8 sequences x 512 tokens, 32 heads
+
+
+def attn_flops_per_slot(M: int, D: int, T: int) -> float:
+    """Tensor-core flops of the causal attention of one slot: for every query block i of
+    128 rows, (i + 1) key tiles of 128 x 128 x 128 for the scores and as many for P V."""
+    nqt = T // 128
+    return 4.0 * 128 ** 3 * (nqt * (nqt + 1) / 2) * (M // T) * (D // 128)
+
+
+def measure_attn_block(awq, stream, flush, steps: int, peaks, seq_len: int = 512, n_heads: int = 32):
+    """The module-level objective on a Llama-7B attention block: the query, key and value
+    projections searched on their causal multi-head attention output. Device time of the
+    whole call (CUDA events) and of its phases (the library's events)."""
+    from workloads import generate_qkv
+    spec = WORKLOADS[ATTN_BLOCK]
+    X, _ = generate(spec)
+    W = generate_qkv(spec)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    Xd, Wd = X.to(dev), W.to(dev)
+    for _ in range(2):
+        out = awq.search_attn(Xd, Wd, n_heads, seq_len, spec.group, spec.n_grid, stream=stream)
+    s_ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    phases = []
+    for i in range(steps):
+        flush.zero_()
+        s_ev[i].record(stream)
+        out = awq.search_attn(Xd, Wd, n_heads, seq_len, spec.group, spec.n_grid, stream=stream)
+        e_ev[i].record(stream)
+        phases.append(awq.attn_profile_last())
+    torch.cuda.synchronize()
+    ms = statistics.mean(s.elapsed_time(e) for s, e in zip(s_ev, e_ev))
+    M, K, D = spec.M, spec.K, spec.K
+    slots = spec.n_grid + 1
+    gemm_flops = slots * 2.0 * M * K * 3 * D
+    attn_flops = slots * attn_flops_per_slot(M, D, seq_len)
+    ph = {k: statistics.mean(p[k] for p in phases) for k in phases[0]}
+    gemm_ms = ph["gemm_qk"] + ph["gemm_vt"]
+    att_ms = ph["attention_reference"] + ph["attention_loss"]
+    peak = float(peaks["bf16_tflops"])
+    gemm_tf = gemm_flops / (gemm_ms / 1e3) / 1e12
+    att_tf = attn_flops / (att_ms / 1e3) / 1e12
+    total_tf = (gemm_flops + attn_flops) / (ms / 1e3) / 1e12
+    del Xd, Wd
+    return {"workload": f"{ATTN_BLOCK} as W_q of [W_q | W_k | W_v] 4096x12288, {M // seq_len} sequences x "
+                        f"{seq_len} tokens, {n_heads} heads of 128",
+            "ms_per_search": ms, "steps": steps, "gpu_launches_per_search": awq.last_launch_count(),
+            "chosen_alpha_index": out.best, "TFLOP/s": total_tf, "phases_ms": ph,
+            "roofline": {"bound": "tensor", "kernel": "loss_gemm_kernel mode 5 (Q|K and V^T products of all slots)",
+                         "achieved": gemm_tf, "peak": peak, "unit": "TFLOP/s", "frac": gemm_tf / peak,
+                         "peak_source": "measured bf16_tflops (burst)",
+                         "work": "(n_grid + 1) x 2 M K 3D flops"},
+            "attention_roofline": {"bound": "tensor",
+                                   "kernel": "attn_loss_kernel (tcgen05 scores and P V, exact-max softmax, fused loss)",
+                                   "achieved": att_tf, "peak": peak, "unit": "TFLOP/s", "frac": att_tf / peak,
+                                   "peak_source": "measured bf16_tflops (burst)",
+                                   "work": "(n_grid + 1) x 4 x 128^3 x (causal key tiles) flops",
+                                   "ms": att_ms}}
+
+
 def cpu_clip_sample(spec: LayerSpec, target_s: float, n_shrink: int = 10):
     """The clipping oracle as it stands on a column slice (full X, same scales reading)."""
     import oracle as O
@@ -405,6 +478,173 @@ def run_reference(args, rank, world):
     return 0
 
 
+def time_searches(awq, spec: LayerSpec, Xd, Wd, stream, flush, steps: int, warmup: int, barrier=None,
+                  sample_clocks: int | None = None):
+    """Device time of `steps` searches of one resident layer, enqueued back to back through
+    the asynchronous entry point (a model's layers are searched this way). Each step's
+    events bracket its own kernels; the L2 flush before it stays outside them. Returns the
+    per-step times, the phase times of every step and the last search's output."""
+    for _ in range(warmup):
+        awq.search(Xd, Wd, spec.group, spec.n_grid, stream=stream)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    if barrier:
+        barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(sample_clocks) if sample_clocks is not None else None
+    pending = []
+    for i in range(steps):
+        flush.zero_()
+        starts[i].record(stream)
+        pending.append(awq.search_async(Xd, Wd, spec.group, spec.n_grid, stream=stream))
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    clock_info = clocks.stop() if clocks is not None else None
+    phases = []
+    out = None
+    for p in pending:
+        out = p.wait()
+        phases.append(p.profile())
+    if barrier:
+        barrier()
+    return {"step_ms": [s.elapsed_time(e) for s, e in zip(starts, ends)], "phases": phases, "out": out,
+            "launches": awq.last_launch_count() * steps, "clocks": clock_info}
+
+
+def search_object(awq, spec: LayerSpec, t: dict, peaks: dict, peak_kind: str, sustained: bool) -> dict:
+    """ms per search, layers/s, candidate-GEMM TFLOP/s and the rooflines of one layer."""
+    steps = len(t["step_ms"])
+    total_ms = float(sum(t["step_ms"]))
+    phases = t["phases"]
+    mean = lambda key: statistics.mean(p[key] for p in phases)  # noqa: E731
+    gemm_ms = statistics.mean(p["gemm_reference"] + p["gemm_loss"] for p in phases)
+    gemm_flops = spec.candidate_flops * (spec.n_grid + 1) / spec.n_grid
+    achieved = gemm_flops / (gemm_ms / 1e3) / 1e12
+    peak_key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+    peak = float(peaks[peak_key])
+    gemm_kernel = ("loss_gemm_pair_kernel" if awq.loss_gemm_variant(spec.M, spec.K, spec.N, spec.n_grid) == 2
+                   else "loss_gemm_kernel")
+    eb = 2 if spec.dtype == "bf16" else 4
+    hbm = float(peaks["hbm_gbs"])
+    qdq_bytes = (eb + 2 * (spec.n_grid + 1)) * spec.K * spec.N
+    stat_bytes = spec.M * spec.K * eb + 4 * spec.K
+    pack_bytes = spec.K * spec.N * (eb + 0.5) + 4 * (spec.K // spec.group) * spec.N + 4 * spec.K
+    phase_tot = {}
+    for p in phases:
+        for k, v in p.items():
+            phase_tot[k] = phase_tot.get(k, 0.0) + v
+
+    def hbm_obj(name, nbytes, ms, work):
+        gbs = nbytes / (ms / 1e3) / 1e9
+        return {"kernel": name, "ms": ms, "bytes": nbytes, "GB/s": gbs, "hbm_frac": gbs / hbm, "work": work}
+
+    roof = {"bound": "tensor",
+            "kernel": gemm_kernel + (" (reference output + candidate GEMMs + fused squared error, one launch)"
+                                     if gemm_kernel == "loss_gemm_kernel" else
+                                     " (candidate GEMMs + fused squared error; reference output in its own launch)"),
+            "work": "(n_grid + 1) x 2 M K N flops per search (the reference output and every candidate)",
+            "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "peak_source": f"{peak_kind} {peak_key} ({'sustained: the kernel runs for a long step' if sustained else 'burst'})",
+            "traffic": recorded_traffic(gemm_kernel, spec.name),
+            "traffic_unit": "DRAM bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
+            "ms_per_launch": gemm_ms}
+    return {
+        "workload": spec.name, "M": spec.M, "K": spec.K, "N": spec.N, "group": spec.group, "n_grid": spec.n_grid,
+        "input_dtype": spec.dtype, "steps": steps, "ms_per_step": total_ms / steps,
+        "layers_per_s": steps / (total_ms / 1e3),
+        "TFLOP/s": spec.candidate_flops * steps / (total_ms / 1e3) / 1e12,
+        "roofline": roof,
+        "other_kernels": {
+            "qdq": hbm_obj("qdq_kernel", qdq_bytes, mean("qdq"),
+                           "reads W once, writes n_grid + 1 bf16 operand slots"),
+            "statistic": hbm_obj("statistic_kernel", stat_bytes, mean("statistic"), "reads X once, writes a"),
+            "pack": hbm_obj("pack_kernel", pack_bytes, mean("pack"),
+                            "reads W once, writes the codes, steps, zeros and scales"),
+            "scales_ms": mean("scales"), "loss_reduce_ms": mean("loss_reduce"),
+        },
+        "phases_ms": {k: v / steps for k, v in phase_tot.items()},
+        "host_gap_ms": total_ms / steps - statistics.mean(sum(p.values()) for p in phases),
+        "gpu_launches_per_search": t["launches"] // steps,
+        "chosen_alpha_index": t["out"].best,
+    }
+
+
+def measure_e2e(awq, spec: LayerSpec, X, W, stream, flush, dev, steps: int, barrier):
+    """The same metric end to end through the host-buffer entry points: every step copies
+    its X and W from pinned host memory, searches, and copies its artifact back. The
+    batched call (the way a model's layers are quantized) overlaps step i + 1's upload and
+    step i - 1's download with step i's search; the one-layer call is reported beside it."""
+    Xh, Wh = X.pin_memory(), W.pin_memory()
+
+    def host_outputs():
+        return (torch.empty(spec.K, dtype=torch.float32, pin_memory=True),
+                torch.empty(spec.K, spec.N // 8, dtype=torch.int32, pin_memory=True),
+                torch.empty(spec.K // spec.group, spec.N, dtype=torch.float16, pin_memory=True),
+                torch.empty(spec.K // spec.group, spec.N, dtype=torch.float16, pin_memory=True),
+                torch.empty(spec.n_grid, dtype=torch.float32, pin_memory=True),
+                torch.empty(1, dtype=torch.int32, pin_memory=True))
+
+    # two output sets used in turn: layer i and i + 2 copy back on one stream, in order
+    sets = [host_outputs(), host_outputs()]
+    outs = [sets[i % 2] for i in range(steps)]
+    awq.search_host_batch([Xh, Xh], [Wh, Wh], spec.group, spec.n_grid, stream=stream, outs=sets, device=dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    flush.zero_()
+    b_s, b_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b_s.record(stream)
+    awq.search_host_batch([Xh] * steps, [Wh] * steps, spec.group, spec.n_grid, stream=stream, outs=outs, device=dev)
+    b_e.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = float(b_s.elapsed_time(b_e))
+    single_steps = 3
+    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(single_steps)]
+    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(single_steps)]
+    for i in range(single_steps):
+        flush.zero_()
+        e_s[i].record(stream)
+        awq.search_host(Xh, Wh, spec.group, spec.n_grid, stream=stream, out=sets[0], device=dev)
+        e_e[i].record(stream)
+    torch.cuda.synchronize(dev)
+    single_ms = float(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e))) / single_steps
+    h2d = X.numel() * X.element_size() + W.numel() * W.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in sets[0])
+    return e2e_ms, single_ms, h2d, d2h
+
+
+def other_workload(awq, name: str, stream, flush, steps: int, warmup: int, peaks, peak_kind):
+    """One of the other layers of the workload set, timed like the headline (its own
+    inputs resident in HBM, L2 flushed between steps). Its oracle sample is taken later,
+    once every GPU timing is done, so that no host thread competes with the enqueueing."""
+    spec = WORKLOADS[name]
+    X, W = generate(spec)
+    Xd, Wd = X.cuda(), W.cuda()
+    t = time_searches(awq, spec, Xd, Wd, stream, flush, steps, warmup)
+    obj = search_object(awq, spec, t, peaks, peak_kind, sustained=False)
+    if spec.M * spec.K * spec.N <= 128 * 256 * 256:
+        obj["bound"] = ("latency: 6 launches of a few microseconds each; the tensor and HBM "
+                        "fractions are not meaningful at this size")
+    del Xd, Wd
+    return obj, (spec, X, t["out"])
+
+
+def column_slice(spec: LayerSpec, W: torch.Tensor, cols: int):
+    """The layer restricted to a column slice of W (the same values as in the full layer):
+    for a joint [gate | up] layer the first `cols` columns of each half, else the first
+    `cols` columns."""
+    if cols <= 0 or cols % 8:
+        raise ValueError("--slice-columns takes a positive multiple of 8")
+    if "gate_up" in spec.name:
+        half = spec.N // 2
+        Ws = torch.cat([W[:, :min(cols, half)], W[:, half:half + min(cols, half)]], dim=1).contiguous()
+        tag = f"cols0-{min(cols, half)}+{half}-{half + min(cols, half)}"
+    else:
+        Ws = W[:, :min(cols, spec.N)].contiguous()
+        tag = f"cols0-{min(cols, spec.N)}"
+    return LayerSpec(**{**spec.as_dict(), "name": f"{spec.name}[{tag}]", "N": Ws.shape[1]}), Ws
+
+
 def run_ours(args, rank, world, local):
     import post_quantization_column_b200 as awq
     torch.cuda.set_device(local)
@@ -415,10 +655,16 @@ def run_ours(args, rank, world, local):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     spec = rank_spec(WORKLOADS[args.workload], rank)
     X, W = generate(spec)
+    if args.slice_columns:
+        spec, W = column_slice(spec, W, args.slice_columns)
     Xd, Wd = X.to(dev), W.to(dev)
     stream = torch.cuda.Stream(dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     awq.profile_enable(True)
+    peaks, peak_kind = measured_peaks()
+    # a step of the large layers runs its loss GEMM for tens to hundreds of milliseconds:
+    # the power-capped sustained peak is its ceiling; the small layers' steps are bursts
+    sustained = spec.candidate_flops >= 50e12
 
     def barrier():
         if world > 1:
@@ -426,105 +672,48 @@ def run_ours(args, rank, world, local):
             dist.barrier(device_ids=[local])
 
     with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            awq.search(Xd, Wd, spec.group, spec.n_grid, stream=stream)
-        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        gemm_ms, qdq_ms, stat_ms, pack_ms, phase_sums = [], [], [], [], []
-        phase_tot = {}
-        barrier()
-        torch.cuda.synchronize(dev)
-        clocks = ClockSampler(local)
-        # the steps are enqueued back to back through the asynchronous entry point (a
-        # model's layers are searched this way); each step's events bracket its own
-        # kernels, the L2 flush before it stays outside them
-        pending = []
-        for i in range(args.steps):
-            flush.zero_()
-            starts[i].record(stream)
-            pending.append(awq.search_async(Xd, Wd, spec.group, spec.n_grid, stream=stream))
-            ends[i].record(stream)
-        torch.cuda.synchronize(dev)
-        for p in pending:
-            out = p.wait()
-            prof = p.profile()
-            for k, v in prof.items():
-                phase_tot[k] = phase_tot.get(k, 0.0) + v
-            phase_sums.append(sum(prof.values()))
-            gemm_ms.append(prof["gemm_reference"] + prof["gemm_loss"])  # one launch (or two) for both
-            qdq_ms.append(prof["qdq"])
-            stat_ms.append(prof["statistic"])
-            pack_ms.append(prof["pack"])
-        torch.cuda.synchronize(dev)
-        barrier()
-        clock_info = clocks.stop()
-        launches = awq.last_launch_count() * args.steps
-        step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-        total_ms = float(sum(step_ms))
-
-        # end to end through the host-buffer entry points: every step copies its X and W
-        # from pinned host memory, searches, and copies its artifact back. The batched call
-        # (the way a model's layers are quantized) overlaps step i + 1's upload and step
-        # i - 1's download with step i's search; the one-layer call is reported beside it.
+        t = time_searches(awq, spec, Xd, Wd, stream, flush, args.steps, args.warmup, barrier, sample_clocks=local)
+        total_ms = float(sum(t["step_ms"]))
+        head = search_object(awq, spec, t, peaks, peak_kind, sustained)
+        out = t["out"]
+        del Xd, Wd
         e2e_steps = args.e2e_steps or max(3, min(args.steps, 20))
-        Xh, Wh = X.pin_memory(), W.pin_memory()
+        e2e_ms, single_ms, h2d, d2h = measure_e2e(awq, spec, X, W, stream, flush, dev, e2e_steps, barrier)
 
-        def host_outputs():
-            return (torch.empty(spec.K, dtype=torch.float32, pin_memory=True),
-                    torch.empty(spec.K, spec.N // 8, dtype=torch.int32, pin_memory=True),
-                    torch.empty(spec.K // spec.group, spec.N, dtype=torch.float16, pin_memory=True),
-                    torch.empty(spec.K // spec.group, spec.N, dtype=torch.float16, pin_memory=True),
-                    torch.empty(spec.n_grid, dtype=torch.float32, pin_memory=True))
+        # the other layers of the workload set (rank 0 of a single-GPU run only: under
+        # torchrun every rank runs the headline layer alone)
+        others = {}
+        side = None
+        if world == 1 and not args.no_other_workloads:
+            for name in WORKLOADS:
+                if name == spec.name:
+                    continue
+                obj, keep = other_workload(awq, name, stream, flush, max(3, min(args.steps, 20)), max(3, args.warmup),
+                                           peaks, peak_kind)
+                others[name] = obj
+                if name == SIDE_WORKLOAD:
+                    side = keep
+        if side is None and spec.name == SIDE_WORKLOAD:
+            side = (spec, X, out)
 
-        outs = [host_outputs() for _ in range(max(2, e2e_steps))]
-        awq.search_host_batch([Xh, Xh], [Wh, Wh], spec.group, spec.n_grid, stream=stream, outs=outs[:2], device=dev)
-        barrier()
-        torch.cuda.synchronize(dev)
-        flush.zero_()
-        b_s, b_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        b_s.record(stream)
-        awq.search_host_batch([Xh] * e2e_steps, [Wh] * e2e_steps, spec.group, spec.n_grid, stream=stream,
-                              outs=outs[:e2e_steps], device=dev)
-        b_e.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier()
-        e2e_ms = float(b_s.elapsed_time(b_e))
-        single_steps = max(3, min(e2e_steps, 10))
-        e_s = [torch.cuda.Event(enable_timing=True) for _ in range(single_steps)]
-        e_e = [torch.cuda.Event(enable_timing=True) for _ in range(single_steps)]
-        for i in range(single_steps):
-            flush.zero_()
-            e_s[i].record(stream)
-            awq.search_host(Xh, Wh, spec.group, spec.n_grid, stream=stream, out=outs[0], device=dev)
-            e_e[i].record(stream)
-        torch.cuda.synchronize(dev)
-        single_ms = float(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e))) / single_steps
-
-        # the next rows of the pipeline: clipping search with the chosen scales, and the
-        # artifact's W4A16 consumer
-        clip = None if args.no_clip else measure_clip(awq, spec, Xd, Wd, out.scales, stream, flush,
-                                                      max(3, min(args.steps, 10)))
-        w4a16 = None if args.no_w4a16 else measure_w4a16(awq, spec, X, out, stream, flush,
-                                                         max(5, min(args.steps, 20)), measured_peaks()[0])
-        mlp = None if args.no_mlp_block else measure_mlp_block(awq, stream, flush, 3, measured_peaks()[0])
+        # the next rows of the pipeline on the 4096^3 layer: clipping search with the
+        # chosen scales, the artifact's W4A16 consumer, and the MLP-block objective
+        clip = w4a16 = mlp = None
+        if side is not None:
+            s_spec, s_X, s_out = side
+            s_Xd, s_Wd = (t_.to(dev) for t_ in generate(s_spec))
+            clip = None if args.no_clip else measure_clip(awq, s_spec, s_Xd, s_Wd, s_out.scales, stream, flush,
+                                                          max(3, min(args.steps, 10)))
+            w4a16 = None if args.no_w4a16 else measure_w4a16(awq, s_spec, s_X, s_out, stream, flush,
+                                                             max(5, min(args.steps, 20)), peaks)
+            del s_Xd, s_Wd
+        mlp = None if args.no_mlp_block else measure_mlp_block(awq, stream, flush, 3, peaks)
+        attn = None if args.no_attn_block else measure_attn_block(awq, stream, flush, 3, peaks)
 
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
-
     flops = spec.candidate_flops
-    gemm_kernel = ("loss_gemm_pair_kernel" if awq.loss_gemm_variant(spec.M, spec.K, spec.N, spec.n_grid) == 2
-                   else "loss_gemm_kernel")
     value = weak_scaling_tflops(world, args.steps, flops, total_ms)
-    layers_per_s = world * args.steps / (total_ms / 1e3)
     e2e_value = weak_scaling_tflops(world, e2e_steps, flops, e2e_ms)
-    peaks, peak_kind = measured_peaks()
-    gemm_avg = statistics.mean(gemm_ms)
-    gemm_flops = flops * (spec.n_grid + 1) / spec.n_grid  # the candidates' GEMMs and the reference output's
-    achieved = gemm_flops / (gemm_avg / 1e3) / 1e12
-    peak = float(peaks["bf16_tflops"])
-    h2d = X.numel() * X.element_size() + W.numel() * W.element_size()
-    d2h = sum(t.numel() * t.element_size() for t in outs[0])
-    qdq_bytes = (W.element_size() + 2 * (spec.n_grid + 1)) * spec.K * spec.N
-    stat_bytes = X.numel() * X.element_size() + 4 * spec.K
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -532,47 +721,37 @@ def run_ours(args, rank, world, local):
         "config": {"workload": spec.name, "M": spec.M, "K": spec.K, "N": spec.N, "group": spec.group,
                    "n_grid": spec.n_grid, "input_dtype": spec.dtype, "parallelism": f"independent layers x{world}",
                    "l2": "flushed between steps (256 MiB device write outside the timed events)"},
-        "layers_per_s": layers_per_s,
-        "roofline": {"bound": "tensor",
-                     "kernel": gemm_kernel + (" (reference output + candidate GEMMs + fused squared error, one launch)"
-                                              if gemm_kernel == "loss_gemm_kernel" else
-                                              " (candidate GEMMs + fused squared error; reference output in its own launch)"),
-                     "work": "(n_grid + 1) x 2 M K N flops per search (the reference output and every candidate)",
-                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "peak_source": f"{peak_kind} bf16_tflops (burst)",
-                     "traffic": recorded_traffic(gemm_kernel, spec.name),
-                     "traffic_unit": "DRAM bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
-                     "ms_per_launch": gemm_avg},
-        "other_kernels": {
-            "qdq": {"ms": statistics.mean(qdq_ms),
-                    "GB/s": qdq_bytes / (statistics.mean(qdq_ms) / 1e3) / 1e9,
-                    "hbm_frac": qdq_bytes / (statistics.mean(qdq_ms) / 1e3) / 1e9 / float(peaks["hbm_gbs"])},
-            "statistic": {"ms": statistics.mean(stat_ms),
-                          "GB/s": stat_bytes / (statistics.mean(stat_ms) / 1e3) / 1e9,
-                          "hbm_frac": stat_bytes / (statistics.mean(stat_ms) / 1e3) / 1e9 / float(peaks["hbm_gbs"])},
-            "pack": {"ms": statistics.mean(pack_ms)},
-        },
-        "phases_ms": {k: v / args.steps for k, v in phase_tot.items()},
-        "host_gap_ms": total_ms / args.steps - statistics.mean(phase_sums),
+        "layers_per_s": world * args.steps / (total_ms / 1e3),
+        "roofline": head["roofline"],
+        "other_kernels": head["other_kernels"],
+        "phases_ms": head["phases_ms"],
+        "host_gap_ms": head["host_gap_ms"],
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms / e2e_steps, "steps": e2e_steps,
                 "api": "awq_search_host_batch over the steps (step i + 1 uploaded while step i runs)",
                 "single_call_ms": single_ms,
                 "single_call_value": flops / (single_ms / 1e3) / 1e12},
-        "gpu_launches": launches,
-        "clocks": clock_info,
+        "gpu_launches": t["launches"],
+        "clocks": t["clocks"],
         "chosen_alpha_index": out.best,
     }
+    if others:
+        line["workloads"] = others
     if clip is not None:
         line["clip_search"] = clip
     if w4a16 is not None:
         line["w4a16"] = w4a16
     if mlp is not None:
         line["mlp_block"] = mlp
+    if attn is not None:
+        line["attn_block"] = attn
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_oracle_sample(spec, args.cpu_seconds)
+        # the oracle samples, after every GPU timing
+        line["cpu_baseline"] = cpu_oracle_sample(spec, args.cpu_seconds, X, W)
+        for name, obj in others.items():
+            obj["cpu_baseline"] = cpu_oracle_sample(WORKLOADS[name], min(args.cpu_seconds, 5.0))
         if clip is not None:
-            clip["cpu_baseline"] = cpu_clip_sample(spec, min(args.cpu_seconds, 10.0))
+            clip["cpu_baseline"] = cpu_clip_sample(side[0], min(args.cpu_seconds, 10.0))
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

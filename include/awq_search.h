@@ -31,6 +31,8 @@
  *   out_steps  [K/group][N] fp16 step of each (group, column), in the scaled domain
  *   out_zeros  [K/group][N] fp16 zero point (an integer 0..15)
  *   out_losses [n_grid]   fp32   L_i (optional, may be NULL)
+ *   out_best   [1]        int32  i*, the index the library chose (the forms that take it;
+ *                                may be NULL): alpha* = i* / n_grid
  *   Dequantized weight: W[k][n] ~= step[g][n] * (q[k][n] - zero[g][n]) / s[k], g = k/group.
  *   4 bits + 32/group bits per weight: 4.25 at group 128 (AWQ-P1 §8).
  *
@@ -46,7 +48,9 @@
  *
  * Streams: all device work is enqueued on `stream` (NULL = the legacy default
  * stream); the call then synchronizes `stream`, so the status reflects errors the
- * kernels detected (non-finite input, a wait that ran out). Outputs are valid only
+ * kernels detected (non-finite input, a wait that ran out). Each call runs on the
+ * device that owns `stream` (or X, for the legacy default stream) and gives the
+ * calling thread's current device back unchanged when it returns. Outputs are valid only
  * when the status is AWQ_OK. The library is not reentrant across host threads
  * that share a device (one call at a time per process is the tested use).
  *
@@ -101,6 +105,10 @@ int awq_search_f32(const float* X, const float* W, int64_t M, int64_t K, int64_t
                    awq_stream_t stream);
 
 /* Full form: `in_dtype` is AWQ_DTYPE_BF16 or AWQ_DTYPE_F32 for both X and W.
+ * `out_best` (device, one int32, may be NULL) receives i*, the candidate the library
+ * chose and packed: the first minimum of the fp32 losses it computed (AWQ-P1 §3: the
+ * search keeps the first of equal losses), decided on the device by the kernel that
+ * emits the artifact.
  * `out_tile_sq_err` (may be NULL) receives the fp64 squared-error partial sums the
  * loss GEMM produced: [n_grid][tiles_m][tiles_n], tile (tm, tn) covering rows
  * tm*tile_m .. and columns tn*tile_n .. (awq_tile_shape); L_i equals the sum of row i
@@ -108,15 +116,15 @@ int awq_search_f32(const float* X, const float* W, int64_t M, int64_t K, int64_t
 int awq_search_ex(const void* X, const void* W, int in_dtype, int64_t M, int64_t K,
                   int64_t N, int group, int n_grid, float* out_scales,
                   int32_t* out_codes, void* out_steps, void* out_zeros,
-                  float* out_losses, double* out_tile_sq_err, int64_t tile_sq_err_len,
-                  awq_stream_t stream);
+                  float* out_losses, int32_t* out_best, double* out_tile_sq_err,
+                  int64_t tile_sq_err_len, awq_stream_t stream);
 
 /* The search with the candidates quantized by `quantizer` (AWQ_QUANT_ASYM gives
  * awq_search_ex without tile partials). */
 int awq_search_quant(const void* X, const void* W, int in_dtype, int64_t M, int64_t K,
                      int64_t N, int group, int n_grid, int quantizer, float* out_scales,
                      int32_t* out_codes, void* out_steps, void* out_zeros, float* out_losses,
-                     awq_stream_t stream);
+                     int32_t* out_best, awq_stream_t stream);
 
 /* Asynchronous form of awq_search_ex (no tile partials): enqueues the whole search on
  * `stream` and returns without waiting. Argument checks happen before anything is
@@ -130,20 +138,21 @@ int awq_search_quant(const void* X, const void* W, int in_dtype, int64_t M, int6
  * back to back, with no host round trip between them. */
 int awq_search_async(const void* X, const void* W, int in_dtype, int64_t M, int64_t K,
                      int64_t N, int group, int n_grid, float* out_scales, int32_t* out_codes,
-                     void* out_steps, void* out_zeros, float* out_losses, int32_t* status_word,
-                     awq_stream_t stream);
+                     void* out_steps, void* out_zeros, float* out_losses, int32_t* out_best,
+                     int32_t* status_word, awq_stream_t stream);
 int awq_search_status(int32_t status_word);
 
 /* End-to-end form with HOST buffers: copies X and W to the device on `stream`,
- * runs awq_search_ex, copies the outputs back (out_losses may be NULL). Pinned
- * host memory makes the copies asynchronous; pageable memory also works. */
+ * runs awq_search_ex, copies the outputs back (out_losses and out_best may be NULL;
+ * out_best receives the chosen index as one int32). Pinned host memory makes the
+ * copies asynchronous; pageable memory also works. */
 int awq_search_host(const void* X_host, const void* W_host, int in_dtype, int64_t M,
                     int64_t K, int64_t N, int group, int n_grid, float* out_scales_host,
                     int32_t* out_codes_host, void* out_steps_host, void* out_zeros_host,
-                    float* out_losses_host, awq_stream_t stream);
+                    float* out_losses_host, int32_t* out_best_host, awq_stream_t stream);
 /* The same for n_layers layers of one shape (X_hosts[i] M x K, W_hosts[i] K x N; the
- * output arrays hold one host pointer per layer, out_losses_host or its entries may be
- * NULL). Layer i + 1's inputs are copied to the device while layer i is searched (two
+ * output arrays hold one host pointer per layer, out_losses_host and out_best_host or
+ * their entries may be NULL). Layer i + 1's inputs are copied to the device while layer i is searched (two
  * device slots) and layer i's artifact is copied back while layer i + 1 runs, so with
  * pinned host memory the transfers hide behind the searches. The whole batch is enqueued
  * at once and the call returns when every output has landed. A layer whose kernels
@@ -154,7 +163,8 @@ int awq_search_host_batch(int n_layers, const void* const* X_hosts, const void* 
                           int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid,
                           float* const* out_scales_host, int32_t* const* out_codes_host,
                           void* const* out_steps_host, void* const* out_zeros_host,
-                          float* const* out_losses_host, awq_stream_t stream);
+                          float* const* out_losses_host, int32_t* const* out_best_host,
+                          awq_stream_t stream);
 
 /* ---- The steps one at a time (same kernels as awq_search; device pointers) ----
  * Step 1 (AWQ-P1 §1): out_a[K] = mean_m |X[m,j]| (fp64 sum, one rounding to fp32).
@@ -255,7 +265,8 @@ int awq_fp64_mma_peak(double* tflops, awq_stream_t stream);
  *   L_i = ||Y_i - Y_ref||_F^2 / (M K_out),  Y_ref the block with bf16(W_gu)
  * silu(x) = x / (1 + exp(-x)) in fp32; the GEMMs take bf16 operands and accumulate in
  * fp32. Steps 1-4 and 6 as awq_search (statistic and scales from X; QDQ, argmin and the
- * artifact of W_gu: out_codes [K][2F/8], out_steps/out_zeros [K/group][2F]).
+ * artifact of W_gu: out_codes [K][2F/8], out_steps/out_zeros [K/group][2F]; out_best,
+ * device, may be NULL: the chosen index).
  * Preconditions as awq_search with N = 2F, plus F and K_out multiples of 8; W_down has
  * the dtype of X and W_gu. When F % 128 == 0 the silu-mul runs in the first GEMM's
  * epilogue (gate and up columns interleaved by 128 in the candidate operand) and each
@@ -268,7 +279,40 @@ int awq_fp64_mma_peak(double* tflops, awq_stream_t stream);
 int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_dtype,
                    int64_t M, int64_t K, int64_t F, int64_t K_out, int group, int n_grid,
                    float* out_scales, int32_t* out_codes, void* out_steps, void* out_zeros,
-                   float* out_losses, awq_stream_t stream);
+                   float* out_losses, int32_t* out_best, awq_stream_t stream);
+
+/* ---- Module-level objective: an attention block ---------------------------------------
+ * [AWQ-P1] §4: the inspected module may be an attention block holding several
+ * projections. The query, key and value projections read the same input X (M x K) and
+ * are searched jointly with one scale vector, W_qkv = [W_q | W_k | W_v] (K x 3D, row-major,
+ * D = n_heads * 128); each candidate is scored on the causal multi-head attention output
+ * of the calibration sequences:
+ *   [Q | K | V]_i = bf16(X_b W_hat_i,b)  (fp32 accumulation, then bf16);
+ *   per sequence (seq_len consecutive rows of X) and head h (columns 128 h .. 128 h + 127
+ *   of each of Q, K, V), for query t and keys u <= t:
+ *     s_tu = q_t . k_u;  m_t = max_u s_tu;  e_tu = exp((s_tu - m_t) / sqrt(128));
+ *     o_t = (sum_u bf16(e_tu) v_u) / (sum_u e_tu)       (fp32; no position encoding,
+ *                                                        no output projection)
+ *   L_i = ||O_i - O_ref||_F^2 / (M D),  O_ref the module with bf16(W_qkv).
+ * Steps 1-4 and 6 as awq_search (statistic and scales from X; QDQ, first argmin and the
+ * artifact of W_qkv: out_codes [K][3D/8], out_steps / out_zeros [K/group][3D]; out_losses
+ * [n_grid] and out_best (one int32, the chosen index) device, may be NULL).
+ * Preconditions as awq_search with N = 3D, plus n_heads >= 1, D = n_heads * 128, seq_len
+ * in {128, 256, 384, 512} dividing M. The Q|K and V^T products run on the tensor cores for
+ * all candidates at once; the attention kernel forms each unit's weights from the exact
+ * row maximum (the scores of up to 512 keys are held in tensor memory) and reduces the
+ * squared error in its epilogue, so no candidate's output reaches device memory. Work
+ * space from the library's pool: (n_grid + 1) (3 D K + 3 D M) bf16 values, M D fp32 of
+ * reference output and n_grid (M / 128) n_heads fp64 partials. Synchronizes `stream`. */
+int awq_search_attn(const void* X, const void* W_qkv, int in_dtype, int64_t M, int64_t K,
+                    int64_t D, int n_heads, int64_t seq_len, int group, int n_grid,
+                    float* out_scales, int32_t* out_codes, void* out_steps, void* out_zeros,
+                    float* out_losses, int32_t* out_best, awq_stream_t stream);
+/* With profiling on (awq_profile_enable), device times (ms) of the last attention-block
+ * search's phases: [0] statistic, scales and QDQ, [1] the Q|K products, [2] the V^T
+ * products, [3] the reference attention, [4] the candidates' attention with the fused
+ * loss, [5] the loss reduction and the artifact. Returns 6. */
+int awq_attn_profile_last(float* ms, int n);
 
 /* ---- W4A16 consumer of the artifact ---------------------------------------------
  * [AWQ-P1] §7: the artifact feeds a W4A16 kernel, checked by decoding it and comparing
@@ -321,25 +365,31 @@ int awq_loss_gemm_variant(int64_t M, int64_t K, int64_t N, int n_grid);
  * awq_search_ex for callers that cannot call cudaMalloc — e.g. a plugin whose host
  * framework owns all device memory, a process whose memory budget was fixed at
  * start-up, or a loop that must not risk an allocation's synchronisation or
- * failure. Same arguments, same kernels and same results as awq_search_ex (without
- * the tile partials), but the work space comes from one array of
- * AWQ_NOALLOC_SCRATCH_BYTES compiled into the library, which every GPU that loads
- * the library holds until the process exits; nothing is allocated or freed.
- * Layers whose work space (awq_workspace_bytes) exceeds the array are rejected with
- * AWQ_ERR_SHAPE and a message giving both sizes — a 1024 x 1024 x 1024 bf16 layer
- * with 20 candidates fits, the Llama-shaped layers do not.
- * The first call on each device looks up the array's device address
+ * failure. Same arguments as awq_search_ex without the tile partials; it runs the
+ * same search (argument checks, kernels, launch sequence and work-space layout), so
+ * its results are bit-identical to awq_search_ex's. The work space comes from one
+ * array of AWQ_NOALLOC_SCRATCH_BYTES compiled into the library instead of the
+ * library's pool; nothing is allocated or freed, and the call synchronizes `stream`
+ * (its status word is read back into pageable host memory).
+ * The array belongs to the library's code module: CUDA materialises it on a GPU at
+ * the first call made there, which returns AWQ_ERR_CUDA if that GPU has no room left
+ * for it; from then on that GPU holds it until the process exits.
+ * Layers whose work space (awq_workspace_bytes, the same layout) exceeds the array
+ * are rejected with AWQ_ERR_SHAPE and a message giving both sizes — a
+ * 1024 x 1024 x 1024 bf16 layer with 20 candidates fits, the Llama-shaped layers do
+ * not; an fp32 layer also needs M*K*2 bytes for its bf16 copy of X.
+ * The first call on each device also looks up the array's device address
  * (cudaGetSymbolAddress, with that device current); make that first call before
  * any stream capture. All calls share the array and it keeps the last call's
- * contents (the status word is cleared at the start of each call, everything else
- * is overwritten before it is read): calls that overlap on the GPU — on different
- * streams or from different host threads on one device — race on it and must be
- * serialised by the caller. */
+ * contents (the status word and the per-tile flags are cleared at the start of each
+ * call, everything else is overwritten before it is read): calls that overlap on the
+ * GPU — on different streams or from different host threads on one device — race on
+ * it and must be serialised by the caller. */
 #define AWQ_NOALLOC_SCRATCH_BYTES (64ll << 20)
 int awq_search_noalloc(const void* X, const void* W, int in_dtype, int64_t M, int64_t K,
                        int64_t N, int group, int n_grid, float* out_scales,
                        int32_t* out_codes, void* out_steps, void* out_zeros,
-                       float* out_losses, awq_stream_t stream);
+                       float* out_losses, int32_t* out_best, awq_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -7,7 +7,7 @@ library is missing or cannot load, every call raises.
 
     import torch, post_quantization_column_b200 as awq
     out = awq.search(X, W, group=128, n_grid=20)   # X: (M, K) bf16/fp32 CUDA, W: (K, N)
-    out.scales, out.codes, out.steps, out.zeros, out.losses, out.best
+    out.scales, out.codes, out.steps, out.zeros, out.losses, out.best   # best: the library's chosen index
 """
 from __future__ import annotations
 
@@ -24,6 +24,7 @@ __all__ = [
     "last_launch_count", "debug_set_fault", "status_string", "exported_functions",
     "activation_statistic", "candidate_scales", "qdq_candidates", "ClipOutput", "clip_search",
     "clip_token_count", "clip_profile_last", "fp64_mma_peak", "w4a16_matmul", "w4a16_dequant", "w4a16_profile_last", "search_mlp", "QUANTIZERS", "w4a16_repack", "w4a16_matmul_packed", "loss_gemm_variant",
+    "search_attn", "attn_profile_last", "ATTN_HEAD_DIM",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -63,10 +64,12 @@ def library() -> ctypes.CDLL:
     vp, i64, i32, f32p, f64p = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p
     lib.awq_search.argtypes = [vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp]
     lib.awq_search_f32.argtypes = [vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp]
-    lib.awq_search_ex.argtypes = [vp, vp, i32, i64, i64, i64, i32, i32, vp, vp, vp, vp, f32p, f64p, i64, vp]
-    lib.awq_search_host.argtypes = [vp, vp, i32, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp]
-    lib.awq_search_host_batch.argtypes = [i32, vp, vp, i32, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp]
-    lib.awq_search_async.argtypes = [vp, vp, i32, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+    lib.awq_search_ex.argtypes = [vp, vp, i32, i64, i64, i64, i32, i32, vp, vp, vp, vp, f32p, vp, f64p, i64, vp]
+    lib.awq_search_host.argtypes = [vp, vp, i32, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+    lib.awq_search_host_batch.argtypes = [i32, vp, vp, i32, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+    lib.awq_search_async.argtypes = [vp, vp, i32, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.awq_search_noalloc.argtypes = [vp, vp, i32, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+    lib.awq_search_noalloc.restype = ctypes.c_int
     lib.awq_search_async.restype = ctypes.c_int
     lib.awq_search_status.argtypes = [ctypes.c_int32]
     lib.awq_search_status.restype = ctypes.c_int
@@ -96,8 +99,12 @@ def library() -> ctypes.CDLL:
     lib.awq_candidate_scales.argtypes = [vp, i64, i32, vp, vp]
     lib.awq_qdq_candidates.argtypes = [vp, i32, i64, i64, i32, i32, vp, vp, vp]
     lib.awq_clip_search.argtypes = [vp, vp, i32, vp, i64, i64, i64, i32, i32, i64, i32, vp, vp, vp, vp, vp, vp, vp]
-    lib.awq_search_quant.argtypes = [vp, vp, i32, i64, i64, i64, i32, i32, i32, vp, vp, vp, vp, vp, vp]
-    lib.awq_search_mlp.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp]
+    lib.awq_search_quant.argtypes = [vp, vp, i32, i64, i64, i64, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+    lib.awq_search_mlp.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+    lib.awq_search_attn.argtypes = [vp, vp, i32, i64, i64, i64, i32, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+    lib.awq_search_attn.restype = ctypes.c_int
+    lib.awq_attn_profile_last.argtypes = [ctypes.POINTER(ctypes.c_float), i32]
+    lib.awq_attn_profile_last.restype = ctypes.c_int
     lib.awq_clip_profile_last.argtypes = [ctypes.POINTER(ctypes.c_float), i32]
     lib.awq_clip_profile_last.restype = ctypes.c_int
     lib.awq_fp64_mma_peak.argtypes = [ctypes.POINTER(ctypes.c_double), vp]
@@ -143,8 +150,14 @@ def _ptr(t):
 
 
 def _stream_handle(stream, device) -> ctypes.c_void_p:
+    """The stream a call runs on (default: the current stream of ``device``). A stream
+    other than the current one first waits for the work already enqueued on the current
+    stream, which is where the inputs (and their contiguous copies) were produced."""
+    current = torch.cuda.current_stream(device)
     if stream is None:
-        stream = torch.cuda.current_stream(device)
+        stream = current
+    elif stream.cuda_stream != current.cuda_stream:
+        stream.wait_stream(current)
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -189,17 +202,13 @@ class SearchOutput:
     steps: torch.Tensor         # (K/group, N) fp16
     zeros: torch.Tensor         # (K/group, N) fp16
     losses: torch.Tensor        # (n_grid,) fp32
+    best_index: torch.Tensor    # (1,) int32: the index the library chose (out_best of the C ABI)
     tile_sq_err: torch.Tensor | None = None  # (n_grid, tiles_m, tiles_n) fp64
 
     @property
     def best(self) -> int:
-        """Index of the chosen alpha = first minimum of the losses."""
-        vals = self.losses.detach().cpu().tolist()
-        b = 0
-        for i, v in enumerate(vals):
-            if v < vals[b]:
-                b = i
-        return b
+        """Index of the chosen alpha (alpha = best / n_grid), as the library returned it."""
+        return int(self.best_index[0])
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -211,12 +220,19 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 
 def _alloc_outputs(K, N, group, n_grid, device, pin=False):
+    """scales, codes, steps, zeros, losses and the chosen index of one layer."""
     kw = dict(device=device) if not pin else dict(pin_memory=True)
     return (torch.empty(K, dtype=torch.float32, **kw),
             torch.empty(K, N // 8, dtype=torch.int32, **kw),
             torch.empty(K // group, N, dtype=torch.float16, **kw),
             torch.empty(K // group, N, dtype=torch.float16, **kw),
-            torch.empty(n_grid, dtype=torch.float32, **kw))
+            torch.empty(n_grid, dtype=torch.float32, **kw),
+            torch.full((1,), -1, dtype=torch.int32, **kw))
+
+
+def _with_best(out: tuple) -> tuple:
+    """A caller's 5-tuple of host outputs plus a pinned word for the chosen index."""
+    return tuple(out) if len(out) == 6 else tuple(out) + (torch.full((1,), -1, dtype=torch.int32, pin_memory=True),)
 
 
 QUANTIZERS = {"asym": 0, "sym": 1}
@@ -242,7 +258,7 @@ def search(X: torch.Tensor, W: torch.Tensor, group: int = 128, n_grid: int = 20,
     N = W.shape[1]
     if group <= 0 or K % group or N % 8:
         raise ValueError("group must divide K and N must be a multiple of 8")
-    scales, codes, steps, zeros, losses = _alloc_outputs(K, N, group, n_grid, X.device)
+    scales, codes, steps, zeros, losses, best = _alloc_outputs(K, N, group, n_grid, X.device)
     tiles = None
     if tile_sq_err:
         tm, tn = tile_shape()
@@ -253,15 +269,15 @@ def search(X: torch.Tensor, W: torch.Tensor, group: int = 128, n_grid: int = 20,
         if tile_sq_err:
             raise ValueError("tile partials are available for the asymmetric quantizer only")
         st = lib.awq_search_quant(_ptr(X), _ptr(W), _dtype_code(X), M, K, N, group, n_grid, QUANTIZERS[quantizer],
-                                  _ptr(scales), _ptr(codes), _ptr(steps), _ptr(zeros), _ptr(losses),
+                                  _ptr(scales), _ptr(codes), _ptr(steps), _ptr(zeros), _ptr(losses), _ptr(best),
                                   _stream_handle(stream, X.device))
         _check(st)
-        return SearchOutput(scales, codes, steps, zeros, losses, None)
+        return SearchOutput(scales, codes, steps, zeros, losses, best, None)
     st = lib.awq_search_ex(_ptr(X), _ptr(W), _dtype_code(X), M, K, N, group, n_grid, _ptr(scales), _ptr(codes),
-                           _ptr(steps), _ptr(zeros), _ptr(losses), _ptr(tiles),
+                           _ptr(steps), _ptr(zeros), _ptr(losses), _ptr(best), _ptr(tiles),
                            tiles.numel() if tiles is not None else 0, _stream_handle(stream, X.device))
     _check(st)
-    return SearchOutput(scales, codes, steps, zeros, losses, tiles)
+    return SearchOutput(scales, codes, steps, zeros, losses, best, tiles)
 
 
 class PendingSearch:
@@ -307,15 +323,20 @@ def search_async(X: torch.Tensor, W: torch.Tensor, group: int = 128, n_grid: int
     N = W.shape[1]
     if group <= 0 or K % group or N % 8:
         raise ValueError("group must divide K and N must be a multiple of 8")
-    scales, codes, steps, zeros, losses = _alloc_outputs(K, N, group, n_grid, X.device)
+    outs = _alloc_outputs(K, N, group, n_grid, X.device)
+    scales, codes, steps, zeros, losses, best = outs
     status = torch.full((1,), -1, dtype=torch.int32, pin_memory=True)
     if stream is None:  # the stream current now is the one wait() synchronizes later
         stream = torch.cuda.current_stream(X.device)
+    handle = _stream_handle(stream, X.device)   # a side stream waits for the current one
     _check(lib.awq_search_async(_ptr(X), _ptr(W), _dtype_code(X), M, K, N, group, n_grid, _ptr(scales), _ptr(codes),
-                                _ptr(steps), _ptr(zeros), _ptr(losses), status.data_ptr(),
-                                _stream_handle(stream, X.device)))
+                                _ptr(steps), _ptr(zeros), _ptr(losses), _ptr(best), status.data_ptr(), handle))
+    if stream.cuda_stream != torch.cuda.current_stream(X.device).cuda_stream:
+        # the caching allocator must not hand these blocks out again before `stream` is done
+        for t in (X, W) + outs:
+            t.record_stream(stream)
     ticket = int(lib.awq_profile_last_ticket())
-    out = SearchOutput(scales, codes, steps, zeros, losses, None)
+    out = SearchOutput(scales, codes, steps, zeros, losses, best, None)
     # keep the inputs alive until the stream has passed the call
     pending = PendingSearch(out, status, stream, X.device, ticket)
     pending._inputs = (X, W)
@@ -369,14 +390,13 @@ def search_host(X: torch.Tensor, W: torch.Tensor, group: int = 128, n_grid: int 
     W = W.contiguous()
     M, K = X.shape
     N = W.shape[1]
-    if out is None:
-        out = _alloc_outputs(K, N, group, n_grid, None, pin=True)
-    scales, codes, steps, zeros, losses = out
+    out = _alloc_outputs(K, N, group, n_grid, None, pin=True) if out is None else _with_best(out)
+    scales, codes, steps, zeros, losses, best = out
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     st = lib.awq_search_host(_ptr(X), _ptr(W), _dtype_code(X), M, K, N, group, n_grid, _ptr(scales), _ptr(codes),
-                             _ptr(steps), _ptr(zeros), _ptr(losses), _stream_handle(stream, dev))
+                             _ptr(steps), _ptr(zeros), _ptr(losses), _ptr(best), _stream_handle(stream, dev))
     _check(st)
-    return SearchOutput(scales, codes, steps, zeros, losses)
+    return SearchOutput(scales, codes, steps, zeros, losses, best)
 
 
 def search_host_batch(Xs: list, Ws: list, group: int = 128, n_grid: int = 20, *,
@@ -400,16 +420,17 @@ def search_host_batch(Xs: list, Ws: list, group: int = 128, n_grid: int = 20, *,
         outs = [_alloc_outputs(K, N, group, n_grid, None, pin=True) for _ in Xs]
     if len(outs) != len(Xs):
         raise ValueError("outs needs one output tuple per layer")
+    outs = [_with_best(o) for o in outs]
     n = len(Xs)
 
     def arr(ptrs):
         return (ctypes.c_void_p * n)(*ptrs)
 
     keep = [arr([_ptr(x) for x in Xs]), arr([_ptr(w) for w in Ws])] + [arr([_ptr(o[k]) for o in outs])
-                                                                        for k in range(5)]
+                                                                        for k in range(6)]
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     st = library().awq_search_host_batch(n, keep[0], keep[1], _dtype_code(X0), M, K, N, group, n_grid, keep[2],
-                                         keep[3], keep[4], keep[5], keep[6], _stream_handle(stream, dev))
+                                         keep[3], keep[4], keep[5], keep[6], keep[7], _stream_handle(stream, dev))
     _check(st)
     return [SearchOutput(*o) for o in outs]
 
@@ -537,11 +558,43 @@ def search_mlp(X: torch.Tensor, W_gu: torch.Tensor, W_down: torch.Tensor, group:
     F, K_out = W_down.shape
     if W_gu.shape[0] != K or N != 2 * F:
         raise ValueError("W_gu must be (K, 2F) and W_down (F, K_out)")
-    scales, codes, steps, zeros, losses = _alloc_outputs(K, N, group, n_grid, X.device)
+    scales, codes, steps, zeros, losses, best = _alloc_outputs(K, N, group, n_grid, X.device)
     _check(library().awq_search_mlp(_ptr(X), _ptr(W_gu), _ptr(W_down), _dtype_code(X), M, K, F, K_out, group, n_grid,
-                                    _ptr(scales), _ptr(codes), _ptr(steps), _ptr(zeros), _ptr(losses),
+                                    _ptr(scales), _ptr(codes), _ptr(steps), _ptr(zeros), _ptr(losses), _ptr(best),
                                     _stream_handle(stream, X.device)))
-    return SearchOutput(scales, codes, steps, zeros, losses)
+    return SearchOutput(scales, codes, steps, zeros, losses, best)
+
+
+ATTN_HEAD_DIM = 128   # head dimension of the attention-block objective
+
+
+def search_attn(X: torch.Tensor, W_qkv: torch.Tensor, n_heads: int, seq_len: int, group: int = 128,
+                n_grid: int = 20, *, stream: torch.cuda.Stream | None = None) -> SearchOutput:
+    """Scale search of the query, key and value projections W_qkv = [W_q | W_k | W_v]
+    (K, 3D), D = n_heads * 128, scored on the causal multi-head attention output of the
+    calibration sequences (seq_len consecutive rows of X (M, K) each)."""
+    if not (X.is_cuda and W_qkv.is_cuda):
+        raise ValueError("search_attn() takes CUDA tensors")
+    if X.dtype != W_qkv.dtype:
+        raise TypeError("X and W_qkv must share a dtype")
+    X, W_qkv = X.contiguous(), W_qkv.contiguous()
+    M, K = X.shape
+    N = W_qkv.shape[1]
+    if W_qkv.shape[0] != K or N % 3:
+        raise ValueError("W_qkv must be (K, 3D)")
+    scales, codes, steps, zeros, losses, best = _alloc_outputs(K, N, group, n_grid, X.device)
+    _check(library().awq_search_attn(_ptr(X), _ptr(W_qkv), _dtype_code(X), M, K, N // 3, n_heads, seq_len, group,
+                                     n_grid, _ptr(scales), _ptr(codes), _ptr(steps), _ptr(zeros), _ptr(losses),
+                                     _ptr(best), _stream_handle(stream, X.device)))
+    return SearchOutput(scales, codes, steps, zeros, losses, best)
+
+
+def attn_profile_last() -> dict:
+    """Device times (ms) of the last attention-block search's phases (profiling on)."""
+    ms = (ctypes.c_float * 6)()
+    n = library().awq_attn_profile_last(ms, 6)
+    names = ("qdq", "gemm_qk", "gemm_vt", "attention_reference", "attention_loss", "reduce_pack")
+    return {names[i]: float(ms[i]) for i in range(n)}
 
 
 def w4a16_repack(codes: torch.Tensor, *, stream=None) -> torch.Tensor:

@@ -358,38 +358,54 @@ int status_from_word(int h_err) {
   return AWQ_OK;
 }
 
+// The whole search of one layer on `s`. `out_best` (device, may be NULL) receives the
+// index the pack kernel chose. With `fixed` the work space is the caller's array
+// instead of a pool block and nothing is allocated.
 int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid,
                   float* out_scales, int32_t* out_codes, void* out_steps, void* out_zeros, float* out_losses,
-                  double* out_tile_sq_err, int64_t tile_sq_err_len, cudaStream_t s, const HostFeed* feed = nullptr,
-                  int quantizer = kQuantAsym, int* async_status = nullptr) {
+                  int32_t* out_best, double* out_tile_sq_err, int64_t tile_sq_err_len, cudaStream_t s,
+                  const HostFeed* feed = nullptr, int quantizer = kQuantAsym, int* async_status = nullptr,
+                  const FixedWorkspace* fixed = nullptr) {
   if (quantizer != kQuantAsym && quantizer != kQuantSym)
     return set_error(AWQ_ERR_INVALID_ARG, "quantizer must be AWQ_QUANT_ASYM or AWQ_QUANT_SYM");
   int st = validate(X, W, in_dtype, M, K, N, group, n_grid, out_scales, out_codes, out_steps, out_zeros, true);
   if (st != AWQ_OK) return st;
-  if (out_losses && !aligned16(out_losses)) {
-    // losses are written as plain floats; 4-byte alignment is enough
-    if (reinterpret_cast<uintptr_t>(out_losses) & 3u) return set_error(AWQ_ERR_INVALID_ARG, "out_losses misaligned");
-  }
+  // losses and the chosen index are written as plain 4-byte words
+  if (out_losses && (reinterpret_cast<uintptr_t>(out_losses) & 3u))
+    return set_error(AWQ_ERR_INVALID_ARG, "out_losses misaligned");
+  if (out_best && (reinterpret_cast<uintptr_t>(out_best) & 3u))
+    return set_error(AWQ_ERR_INVALID_ARG, "out_best misaligned");
+  DeviceRestore restore_device;
   bind_device(s, X);
   int dev = 0, num_sms = 0;
   st = check_device(&dev, &num_sms);
   if (st != AWQ_OK) return st;
   if (!is_device_memory(X) || !is_device_memory(W) || !is_device_memory(out_scales) ||
       !is_device_memory(out_codes) || !is_device_memory(out_steps) || !is_device_memory(out_zeros) ||
-      (out_losses && !is_device_memory(out_losses)) || (out_tile_sq_err && !is_device_memory(out_tile_sq_err)))
+      (out_losses && !is_device_memory(out_losses)) || (out_best && !is_device_memory(out_best)) ||
+      (out_tile_sq_err && !is_device_memory(out_tile_sq_err)))
     return set_error(AWQ_ERR_INVALID_ARG, "inputs and outputs must be device memory (use awq_search_host for host buffers)");
   const Layout L = plan(in_dtype, M, K, N, n_grid);
   if (out_tile_sq_err && tile_sq_err_len < static_cast<int64_t>(n_grid) * L.tiles)
     return set_error(AWQ_ERR_INVALID_ARG, "out_tile_sq_err holds fewer than n_grid * tiles values");
 
-  cudaMemPool_t pool;
-  st = get_pool(dev, &pool);
-  if (st != AWQ_OK) return st;
   void* ws = nullptr;
-  cudaError_t e = cudaMallocFromPoolAsync(&ws, L.total, pool, s);
-  if (e != cudaSuccess || !ws) {
-    cudaGetLastError();
-    return set_error(AWQ_ERR_OOM, "work space of " + std::to_string(L.total) + " bytes: " + cudaGetErrorString(e));
+  cudaError_t e = cudaSuccess;
+  if (fixed) {
+    if (L.total > fixed->bytes)
+      return set_error(AWQ_ERR_SHAPE, "this layer needs " + std::to_string(L.total) + " bytes of work space; the " +
+                                          "fixed array holds " + std::to_string(fixed->bytes) +
+                                          " (use awq_search for larger layers)");
+    if ((st = fixed->resolve(dev, &ws)) != AWQ_OK) return st;
+  } else {
+    cudaMemPool_t pool;
+    st = get_pool(dev, &pool);
+    if (st != AWQ_OK) return st;
+    e = cudaMallocFromPoolAsync(&ws, L.total, pool, s);
+    if (e != cudaSuccess || !ws) {
+      cudaGetLastError();
+      return set_error(AWQ_ERR_OOM, "work space of " + std::to_string(L.total) + " bytes: " + cudaGetErrorString(e));
+    }
   }
   uint8_t* base = static_cast<uint8_t*>(ws);
   int* err = reinterpret_cast<int*>(base + L.err);
@@ -405,7 +421,7 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
 
   int launches = 0;
   Events ev;
-  ev.create(g_profile, s);
+  ev.create(g_profile && !fixed, s);
   const char* where = "";
   int status = AWQ_OK;
   do {
@@ -497,6 +513,10 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
       where = "copy of the losses";
       break;
     }
+    if (out_best && (e = cudaMemcpyAsync(out_best, best, sizeof(int32_t), cudaMemcpyDeviceToDevice, s)) != cudaSuccess) {
+      where = "copy of the chosen index";
+      break;
+    }
     if (out_tile_sq_err &&
         (e = cudaMemcpyAsync(out_tile_sq_err, loss_partial, static_cast<size_t>(n_grid) * L.tiles * 8,
                              cudaMemcpyDeviceToDevice, s)) != cudaSuccess) {
@@ -512,19 +532,20 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
       if (e != cudaSuccess) where = "status read-back";
     }
     if (status == AWQ_OK && e != cudaSuccess) status = cuda_error(e, where);
-    cudaFreeAsync(ws, s);
+    if (!fixed) cudaFreeAsync(ws, s);
     g_last_launches = launches;
     return status;
   }
   int h_err = 0;
-  int* pinned = pinned_status_word(dev);
+  // a fixed work space's call reads its status into pageable memory (no pinned word)
+  int* pinned = fixed ? nullptr : pinned_status_word(dev);
   int* status_dst = pinned ? pinned : &h_err;
   if (status == AWQ_OK && e == cudaSuccess) {
     e = cudaMemcpyAsync(status_dst, err, sizeof(int), cudaMemcpyDeviceToHost, s);
     if (e != cudaSuccess) where = "status read-back";
   }
   if (status == AWQ_OK && e != cudaSuccess) status = cuda_error(e, where);
-  cudaFreeAsync(ws, s);
+  if (!fixed) cudaFreeAsync(ws, s);
   cudaError_t se = cudaStreamSynchronize(s);
   if (status == AWQ_OK && se != cudaSuccess) status = cuda_error(se, "stream synchronize");
   if (pinned) h_err = *pinned;
@@ -540,21 +561,29 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
 
 namespace awq {
 void record_error_message(const char* msg) { t_last_error = msg; }
+
+int search_in_workspace(const void* X, const void* W, int in_dtype, int64_t M, int64_t K, int64_t N, int group,
+                        int n_grid, float* out_scales, int32_t* out_codes, void* out_steps, void* out_zeros,
+                        float* out_losses, int32_t* out_best, cudaStream_t s, const FixedWorkspace& fixed) {
+  t_last_error.clear();
+  return search_device(X, W, in_dtype, M, K, N, group, n_grid, out_scales, out_codes, out_steps, out_zeros,
+                       out_losses, out_best, nullptr, 0, s, nullptr, kQuantAsym, nullptr, &fixed);
+}
 }  // namespace awq
 
 extern "C" {
 
 int awq_search_ex(const void* X, const void* W, int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid,
                   float* out_scales, int32_t* out_codes, void* out_steps, void* out_zeros, float* out_losses,
-                  double* out_tile_sq_err, int64_t tile_sq_err_len, awq_stream_t stream) {
+                  int32_t* out_best, double* out_tile_sq_err, int64_t tile_sq_err_len, awq_stream_t stream) {
   t_last_error.clear();
   return search_device(X, W, in_dtype, M, K, N, group, n_grid, out_scales, out_codes, out_steps, out_zeros,
-                       out_losses, out_tile_sq_err, tile_sq_err_len, reinterpret_cast<cudaStream_t>(stream));
+                       out_losses, out_best, out_tile_sq_err, tile_sq_err_len, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int awq_search_async(const void* X, const void* W, int in_dtype, int64_t M, int64_t K, int64_t N, int group,
                      int n_grid, float* out_scales, int32_t* out_codes, void* out_steps, void* out_zeros,
-                     float* out_losses, int32_t* status_word, awq_stream_t stream) {
+                     float* out_losses, int32_t* out_best, int32_t* status_word, awq_stream_t stream) {
   t_last_error.clear();
   if (!status_word) return set_error(AWQ_ERR_INVALID_ARG, "status_word is NULL");
   cudaPointerAttributes attr;
@@ -563,7 +592,7 @@ int awq_search_async(const void* X, const void* W, int in_dtype, int64_t M, int6
     return set_error(AWQ_ERR_INVALID_ARG, "status_word must be pinned host memory");
   }
   return search_device(X, W, in_dtype, M, K, N, group, n_grid, out_scales, out_codes, out_steps, out_zeros,
-                       out_losses, nullptr, 0, reinterpret_cast<cudaStream_t>(stream), nullptr, kQuantAsym,
+                       out_losses, out_best, nullptr, 0, reinterpret_cast<cudaStream_t>(stream), nullptr, kQuantAsym,
                        status_word);
 }
 
@@ -576,32 +605,33 @@ int awq_search(const void* X, const void* W, int64_t M, int64_t K, int64_t N, in
                float* out_scales, int32_t* out_codes, void* out_steps, void* out_zeros, float* out_losses,
                awq_stream_t stream) {
   return awq_search_ex(X, W, AWQ_DTYPE_BF16, M, K, N, group, n_grid, out_scales, out_codes, out_steps, out_zeros,
-                       out_losses, nullptr, 0, stream);
+                       out_losses, nullptr, nullptr, 0, stream);
 }
 
 int awq_search_f32(const float* X, const float* W, int64_t M, int64_t K, int64_t N, int group, int n_grid,
                    float* out_scales, int32_t* out_codes, void* out_steps, void* out_zeros, float* out_losses,
                    awq_stream_t stream) {
   return awq_search_ex(X, W, AWQ_DTYPE_F32, M, K, N, group, n_grid, out_scales, out_codes, out_steps, out_zeros,
-                       out_losses, nullptr, 0, stream);
+                       out_losses, nullptr, nullptr, 0, stream);
 }
 
 int awq_search_quant(const void* X, const void* W, int in_dtype, int64_t M, int64_t K, int64_t N, int group,
                      int n_grid, int quantizer, float* out_scales, int32_t* out_codes, void* out_steps,
-                     void* out_zeros, float* out_losses, awq_stream_t stream) {
+                     void* out_zeros, float* out_losses, int32_t* out_best, awq_stream_t stream) {
   t_last_error.clear();
   return search_device(X, W, in_dtype, M, K, N, group, n_grid, out_scales, out_codes, out_steps, out_zeros,
-                       out_losses, nullptr, 0, reinterpret_cast<cudaStream_t>(stream), nullptr, quantizer);
+                       out_losses, out_best, nullptr, 0, reinterpret_cast<cudaStream_t>(stream), nullptr, quantizer);
 }
 
 int awq_search_host(const void* X_host, const void* W_host, int in_dtype, int64_t M, int64_t K, int64_t N, int group,
                     int n_grid, float* out_scales_host, int32_t* out_codes_host, void* out_steps_host,
-                    void* out_zeros_host, float* out_losses_host, awq_stream_t stream) {
+                    void* out_zeros_host, float* out_losses_host, int32_t* out_best_host, awq_stream_t stream) {
   t_last_error.clear();
   int st = validate(X_host, W_host, in_dtype, M, K, N, group, n_grid, out_scales_host, out_codes_host,
                     out_steps_host, out_zeros_host, false);
   if (st != AWQ_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DeviceRestore restore_device;
   bind_device(s, nullptr);
   int dev = 0, num_sms = 0;
   st = check_device(&dev, &num_sms);
@@ -616,9 +646,9 @@ int awq_search_host(const void* X_host, const void* W_host, int in_dtype, int64_
   const size_t bx = static_cast<size_t>(M) * K * eb, bw = static_cast<size_t>(K) * N * eb;
   const size_t bs = static_cast<size_t>(K) * 4, bc = static_cast<size_t>(K) * (N / 8) * 4;
   const size_t bst = G * N * 2, bl = static_cast<size_t>(n_grid) * 4;
-  size_t off[7], total = 0;
-  const size_t sizes[7] = {bx, bw, bs, bc, bst, bst, bl};
-  for (int i = 0; i < 7; ++i) {
+  size_t off[8], total = 0;
+  const size_t sizes[8] = {bx, bw, bs, bc, bst, bst, bl, sizeof(int32_t)};
+  for (int i = 0; i < 8; ++i) {
     off[i] = total;
     total += align_up(sizes[i]);
   }
@@ -658,14 +688,17 @@ int awq_search_host(const void* X_host, const void* W_host, int in_dtype, int64_
   if (status == AWQ_OK)
     status = search_device(b + off[0], b + off[1], in_dtype, M, K, N, group, n_grid, reinterpret_cast<float*>(b + off[2]),
                            reinterpret_cast<int32_t*>(b + off[3]), b + off[4], b + off[5],
-                           reinterpret_cast<float*>(b + off[6]), nullptr, 0, s, &feed);
+                           reinterpret_cast<float*>(b + off[6]), reinterpret_cast<int32_t*>(b + off[7]), nullptr, 0, s,
+                           &feed);
   if (status == AWQ_OK) {
     if ((e = cudaMemcpyAsync(out_scales_host, b + off[2], bs, cudaMemcpyDeviceToHost, s)) != cudaSuccess ||
         (e = cudaMemcpyAsync(out_codes_host, b + off[3], bc, cudaMemcpyDeviceToHost, s)) != cudaSuccess ||
         (e = cudaMemcpyAsync(out_steps_host, b + off[4], bst, cudaMemcpyDeviceToHost, s)) != cudaSuccess ||
         (e = cudaMemcpyAsync(out_zeros_host, b + off[5], bst, cudaMemcpyDeviceToHost, s)) != cudaSuccess ||
         (out_losses_host &&
-         (e = cudaMemcpyAsync(out_losses_host, b + off[6], bl, cudaMemcpyDeviceToHost, s)) != cudaSuccess))
+         (e = cudaMemcpyAsync(out_losses_host, b + off[6], bl, cudaMemcpyDeviceToHost, s)) != cudaSuccess) ||
+        (out_best_host &&
+         (e = cudaMemcpyAsync(out_best_host, b + off[7], sizeof(int32_t), cudaMemcpyDeviceToHost, s)) != cudaSuccess))
       status = cuda_error(e, "device-to-host copy");
   }
   // the copy stream must be done with the buffers before they return to the pool
@@ -686,7 +719,7 @@ int awq_search_host(const void* X_host, const void* W_host, int in_dtype, int64_
 int awq_search_host_batch(int n_layers, const void* const* X_hosts, const void* const* W_hosts, int in_dtype,
                           int64_t M, int64_t K, int64_t N, int group, int n_grid, float* const* out_scales_host,
                           int32_t* const* out_codes_host, void* const* out_steps_host, void* const* out_zeros_host,
-                          float* const* out_losses_host, awq_stream_t stream) {
+                          float* const* out_losses_host, int32_t* const* out_best_host, awq_stream_t stream) {
   t_last_error.clear();
   if (n_layers < 1 || !X_hosts || !W_hosts || !out_scales_host || !out_codes_host || !out_steps_host ||
       !out_zeros_host)
@@ -697,6 +730,7 @@ int awq_search_host_batch(int n_layers, const void* const* X_hosts, const void* 
     if (st != AWQ_OK) return st;
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DeviceRestore restore_device;
   bind_device(s, nullptr);
   int dev = 0, num_sms = 0;
   int st = check_device(&dev, &num_sms);
@@ -708,10 +742,10 @@ int awq_search_host_batch(int n_layers, const void* const* X_hosts, const void* 
   const size_t bx = static_cast<size_t>(M) * K * eb, bw = static_cast<size_t>(K) * N * eb;
   const size_t bs = static_cast<size_t>(K) * 4, bc = static_cast<size_t>(K) * (N / 8) * 4;
   const size_t bst = G * N * 2, bl = static_cast<size_t>(n_grid) * 4;
-  // per slot: X, W, scales, codes, steps, zeros, losses
-  const size_t sizes[7] = {bx, bw, bs, bc, bst, bst, bl};
-  size_t off[7], slot_bytes = 0;
-  for (int k = 0; k < 7; ++k) {
+  // per slot: X, W, scales, codes, steps, zeros, losses, chosen index
+  const size_t sizes[8] = {bx, bw, bs, bc, bst, bst, bl, sizeof(int32_t)};
+  size_t off[8], slot_bytes = 0;
+  for (int k = 0; k < 8; ++k) {
     off[k] = slot_bytes;
     slot_bytes += align_up(sizes[k]);
   }
@@ -794,8 +828,9 @@ int awq_search_host_batch(int n_layers, const void* const* X_hosts, const void* 
     }
     status = search_device(slot_ptr(i, 0), slot_ptr(i, 1), in_dtype, M, K, N, group, n_grid,
                            reinterpret_cast<float*>(slot_ptr(i, 2)), reinterpret_cast<int32_t*>(slot_ptr(i, 3)),
-                           slot_ptr(i, 4), slot_ptr(i, 5), reinterpret_cast<float*>(slot_ptr(i, 6)), nullptr, 0, s,
-                           i == 0 ? &feed : nullptr, kQuantAsym, words + i);
+                           slot_ptr(i, 4), slot_ptr(i, 5), reinterpret_cast<float*>(slot_ptr(i, 6)),
+                           reinterpret_cast<int32_t*>(slot_ptr(i, 7)), nullptr, 0, s, i == 0 ? &feed : nullptr,
+                           kQuantAsym, words + i);
     if (status != AWQ_OK) break;
     if ((e = cudaEventRecord(sl.in_free, s)) != cudaSuccess || (e = cudaEventRecord(search_done, s)) != cudaSuccess ||
         (e = cudaStreamWaitEvent(d2h, search_done, 0)) != cudaSuccess ||
@@ -805,6 +840,9 @@ int awq_search_host_batch(int n_layers, const void* const* X_hosts, const void* 
         (e = cudaMemcpyAsync(out_zeros_host[i], slot_ptr(i, 5), bst, cudaMemcpyDeviceToHost, d2h)) != cudaSuccess ||
         (out_losses_host && out_losses_host[i] &&
          (e = cudaMemcpyAsync(out_losses_host[i], slot_ptr(i, 6), bl, cudaMemcpyDeviceToHost, d2h)) != cudaSuccess) ||
+        (out_best_host && out_best_host[i] &&
+         (e = cudaMemcpyAsync(out_best_host[i], slot_ptr(i, 7), sizeof(int32_t), cudaMemcpyDeviceToHost, d2h)) !=
+             cudaSuccess) ||
         (e = cudaEventRecord(sl.out_done, d2h)) != cudaSuccess) {
       status = cuda_error(e, "device-to-host copy");
       break;
@@ -836,6 +874,7 @@ int awq_activation_statistic(const void* X, int in_dtype, int64_t M, int64_t K, 
   if (!aligned16(X) || (reinterpret_cast<uintptr_t>(out_a) & 3u))
     return set_error(AWQ_ERR_INVALID_ARG, "X must be 16-byte aligned and out_a 4-byte aligned");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DeviceRestore restore_device;
   bind_device(s, X);
   int dev = 0, num_sms = 0;
   if ((st = check_device(&dev, &num_sms)) != AWQ_OK) return st;
@@ -869,6 +908,7 @@ int awq_candidate_scales(const float* a, int64_t K, int n_grid, float* out_S, aw
   if (K <= 0 || K >= (int64_t(1) << 31)) return set_error(AWQ_ERR_SHAPE, "K must be in 1 .. 2^31-1");
   if (n_grid < 1 || n_grid > kMaxGrid) return set_error(AWQ_ERR_INVALID_ARG, "n_grid must be in 1..64");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DeviceRestore restore_device;
   bind_device(s, a);
   int dev = 0, num_sms = 0, st;
   if ((st = check_device(&dev, &num_sms)) != AWQ_OK) return st;
@@ -892,6 +932,7 @@ int awq_qdq_candidates(const void* W, int in_dtype, int64_t K, int64_t N, int gr
   if (!aligned16(W) || !aligned16(out_wt) || (reinterpret_cast<uintptr_t>(S) & 3u))
     return set_error(AWQ_ERR_INVALID_ARG, "W and out_wt must be 16-byte aligned, S 4-byte aligned");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DeviceRestore restore_device;
   bind_device(s, W);
   int dev = 0, num_sms = 0;
   if ((st = check_device(&dev, &num_sms)) != AWQ_OK) return st;
@@ -938,6 +979,7 @@ int awq_clip_search(const void* X, const void* W, int in_dtype, const float* sca
       (reinterpret_cast<uintptr_t>(out_steps) & 1u) || (reinterpret_cast<uintptr_t>(out_zeros) & 1u))
     return set_error(AWQ_ERR_INVALID_ARG, "X and W must be 16-byte aligned, the other pointers aligned to their type");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DeviceRestore restore_device;
   bind_device(s, X);
   int dev = 0, num_sms = 0;
   if ((st = check_device(&dev, &num_sms)) != AWQ_OK) return st;
@@ -1024,6 +1066,7 @@ int awq_w4a16_matmul(const void* A, const int32_t* codes, const void* steps, con
   int st = validate_w4a16(A, codes, steps, zeros, M, K, N, group, Y);
   if (st != AWQ_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DeviceRestore restore_device;
   bind_device(s, codes);
   int dev = 0, num_sms = 0;
   if ((st = check_device(&dev, &num_sms)) != AWQ_OK) return st;
@@ -1128,6 +1171,7 @@ int awq_w4a16_repack(const int32_t* codes, int64_t K, int64_t N, int32_t* out_pa
   if (!aligned16(codes) || !aligned16(out_packed))
     return set_error(AWQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DeviceRestore restore_device;
   bind_device(s, codes);
   int dev = 0, num_sms = 0, st;
   if ((st = check_device(&dev, &num_sms)) != AWQ_OK) return st;
@@ -1150,6 +1194,7 @@ int awq_w4a16_matmul_packed(const void* A, const int32_t* packed, const void* st
   if (M > kW4A16GemvMaxM) return set_error(AWQ_ERR_SHAPE, "the repacked layout serves at most 16 tokens");
   if (N % 64) return set_error(AWQ_ERR_SHAPE, "the repacked layout needs N % 64 == 0");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DeviceRestore restore_device;
   bind_device(s, packed);
   int dev = 0, num_sms = 0;
   if ((st = check_device(&dev, &num_sms)) != AWQ_OK) return st;
@@ -1206,6 +1251,7 @@ int awq_w4a16_dequant(const int32_t* codes, const void* steps, const void* zeros
   int st = validate_w4a16(dummy, codes, steps, zeros, 1, K, N, group, out_wt);
   if (st != AWQ_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DeviceRestore restore_device;
   bind_device(s, codes);
   int dev = 0, num_sms = 0;
   if ((st = check_device(&dev, &num_sms)) != AWQ_OK) return st;
@@ -1224,7 +1270,7 @@ int awq_w4a16_dequant(const int32_t* codes, const void* steps, const void* zeros
 // ---- MLP-block objective --------------------------------------------------------------
 int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_dtype, int64_t M, int64_t K,
                    int64_t F, int64_t K_out, int group, int n_grid, float* out_scales, int32_t* out_codes,
-                   void* out_steps, void* out_zeros, float* out_losses, awq_stream_t stream) {
+                   void* out_steps, void* out_zeros, float* out_losses, int32_t* out_best, awq_stream_t stream) {
   t_last_error.clear();
   int st = validate(X, W_gu, in_dtype, M, K, 2 * F, group, n_grid, out_scales, out_codes, out_steps, out_zeros, true);
   if (st != AWQ_OK) return st;
@@ -1233,13 +1279,16 @@ int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_d
     return set_error(AWQ_ERR_SHAPE, "F and K_out must be positive multiples of 8");
   if (out_losses && (reinterpret_cast<uintptr_t>(out_losses) & 3u))
     return set_error(AWQ_ERR_INVALID_ARG, "out_losses misaligned");
+  if (out_best && (reinterpret_cast<uintptr_t>(out_best) & 3u))
+    return set_error(AWQ_ERR_INVALID_ARG, "out_best misaligned");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DeviceRestore restore_device;
   bind_device(s, X);
   int dev = 0, num_sms = 0;
   if ((st = check_device(&dev, &num_sms)) != AWQ_OK) return st;
   if (!is_device_memory(X) || !is_device_memory(W_gu) || !is_device_memory(W_down) || !is_device_memory(out_scales) ||
       !is_device_memory(out_codes) || !is_device_memory(out_steps) || !is_device_memory(out_zeros) ||
-      (out_losses && !is_device_memory(out_losses)))
+      (out_losses && !is_device_memory(out_losses)) || (out_best && !is_device_memory(out_best)))
     return set_error(AWQ_ERR_INVALID_ARG, "inputs and outputs must be device memory");
   const int64_t N = 2 * F;
   const int64_t tiles2 = ceil_div(M, kTileM) * ceil_div(K_out, kTileN);
@@ -1408,6 +1457,10 @@ int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_d
       where = "copy of the losses";
       break;
     }
+    if (out_best && (e = cudaMemcpyAsync(out_best, best, sizeof(int32_t), cudaMemcpyDeviceToDevice, s)) != cudaSuccess) {
+      where = "copy of the chosen index";
+      break;
+    }
   } while (false);
   int* pinned = pinned_status_word(dev);
   int* status_dst = pinned ? pinned : &h_err;
@@ -1432,6 +1485,230 @@ int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_d
   return status;
 }
 
+// ---- module-level objective: an attention block ----------------------------------------
+// Phase events of the last profiled attention-block search: QDQ, the Q|K GEMM, the V^T
+// GEMM, the reference attention, the candidates' attention with the fused loss, and the
+// loss reduction with the artifact.
+constexpr int kAttnPhases = 6;
+float g_attn_ms[kAttnPhases] = {0};
+cudaEvent_t* attn_events(int dev) {
+  static cudaEvent_t ev[64][kAttnPhases + 1];
+  static bool made[64] = {false};
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!made[dev]) {
+    for (auto& e : ev[dev])
+      if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    made[dev] = true;
+  }
+  return ev[dev];
+}
+
+int awq_search_attn(const void* X, const void* W_qkv, int in_dtype, int64_t M, int64_t K, int64_t D, int n_heads,
+                    int64_t seq_len, int group, int n_grid, float* out_scales, int32_t* out_codes, void* out_steps,
+                    void* out_zeros, float* out_losses, int32_t* out_best, awq_stream_t stream) {
+  t_last_error.clear();
+  int st = validate(X, W_qkv, in_dtype, M, K, 3 * D, group, n_grid, out_scales, out_codes, out_steps, out_zeros, true);
+  if (st != AWQ_OK) return st;
+  if (n_heads < 1 || D != static_cast<int64_t>(n_heads) * kAttnHeadDim)
+    return set_error(AWQ_ERR_SHAPE, "D must be n_heads * 128 (heads of dimension 128)");
+  if (seq_len < 128 || seq_len > kAttnMaxSeq || seq_len % 128 || M % seq_len)
+    return set_error(AWQ_ERR_SHAPE, "seq_len must be 128, 256, 384 or 512 and divide M");
+  if ((out_losses && (reinterpret_cast<uintptr_t>(out_losses) & 3u)) ||
+      (out_best && (reinterpret_cast<uintptr_t>(out_best) & 3u)))
+    return set_error(AWQ_ERR_INVALID_ARG, "out_losses / out_best misaligned");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DeviceRestore restore_device;
+  bind_device(s, X);
+  int dev = 0, num_sms = 0;
+  if ((st = check_device(&dev, &num_sms)) != AWQ_OK) return st;
+  if (!is_device_memory(X) || !is_device_memory(W_qkv) || !is_device_memory(out_scales) ||
+      !is_device_memory(out_codes) || !is_device_memory(out_steps) || !is_device_memory(out_zeros) ||
+      (out_losses && !is_device_memory(out_losses)) || (out_best && !is_device_memory(out_best)))
+    return set_error(AWQ_ERR_INVALID_ARG, "inputs and outputs must be device memory");
+  const int64_t N = 3 * D;
+  const int slots = n_grid + 1;  // slot 0: bf16(W), slot 1 + i: candidate i
+  const int64_t units = (M / seq_len) * n_heads * (seq_len / 128);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += align_up(bytes);
+    return at;
+  };
+  const size_t o_err = take(16), o_a = take(static_cast<size_t>(K) * 4), o_S = take(static_cast<size_t>(n_grid) * K * 4),
+               o_best = take(16), o_losses = take(static_cast<size_t>(n_grid) * 4),
+               o_Xb = in_dtype == AWQ_DTYPE_F32 ? take(static_cast<size_t>(M) * K * 2) : 0,
+               o_Wqk = take(static_cast<size_t>(slots) * 2 * D * K * 2),
+               o_Wv = take(static_cast<size_t>(slots) * D * K * 2),
+               o_QK = take(static_cast<size_t>(slots) * M * 2 * D * 2),
+               o_VT = take(static_cast<size_t>(slots) * D * M * 2),
+               o_O = take(static_cast<size_t>(M) * D * 4),
+               o_part = take(static_cast<size_t>(n_grid) * units * 8);
+  cudaMemPool_t pool;
+  if ((st = get_pool(dev, &pool)) != AWQ_OK) return st;
+  void* ws = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, off, pool, s);
+  if (e != cudaSuccess || !ws) {
+    cudaGetLastError();
+    return set_error(AWQ_ERR_OOM, "work space of " + std::to_string(off) + " bytes");
+  }
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  int* err = reinterpret_cast<int*>(b + o_err);
+  float* a = reinterpret_cast<float*>(b + o_a);
+  float* S = reinterpret_cast<float*>(b + o_S);
+  int* best = reinterpret_cast<int*>(b + o_best);
+  float* losses = reinterpret_cast<float*>(b + o_losses);
+  __nv_bfloat16* Wqk = reinterpret_cast<__nv_bfloat16*>(b + o_Wqk);
+  __nv_bfloat16* Wv = reinterpret_cast<__nv_bfloat16*>(b + o_Wv);
+  __nv_bfloat16* QK = reinterpret_cast<__nv_bfloat16*>(b + o_QK);
+  __nv_bfloat16* VT = reinterpret_cast<__nv_bfloat16*>(b + o_VT);
+  float* O_ref = reinterpret_cast<float*>(b + o_O);
+  double* part = reinterpret_cast<double*>(b + o_part);
+  const __nv_bfloat16* Xb = in_dtype == AWQ_DTYPE_F32 ? reinterpret_cast<__nv_bfloat16*>(b + o_Xb)
+                                                      : static_cast<const __nv_bfloat16*>(X);
+  const size_t eb = in_dtype == AWQ_DTYPE_F32 ? 4 : 2;
+  const void* W_v = static_cast<const uint8_t*>(W_qkv) + 2 * D * eb;  // columns 2D .. 3D - 1 of each row
+  cudaEvent_t* ev = g_profile ? attn_events(dev) : nullptr;
+  auto mark = [&](int i) {
+    if (ev) cudaEventRecord(ev[i], s);
+  };
+  int launches = 0, h_err = 0, status = AWQ_OK;
+  const char* where = "";
+  do {
+    if ((e = cudaMemsetAsync(err, 0, 16, s)) != cudaSuccess) { where = "cudaMemsetAsync"; break; }
+    mark(0);
+    if ((e = launch_statistic(X, in_dtype, M, K, a, err, s, &launches)) != cudaSuccess) {
+      where = "statistic kernel";
+      break;
+    }
+    if ((e = launch_scales(a, K, n_grid, S, s, &launches)) != cudaSuccess) { where = "scales kernel"; break; }
+    if (in_dtype == AWQ_DTYPE_F32 &&
+        (e = launch_to_bf16(static_cast<const float*>(X), M * K, const_cast<__nv_bfloat16*>(Xb), s, &launches)) !=
+            cudaSuccess) {
+      where = "bf16 operand kernel";
+      break;
+    }
+    // the query and key columns, then the value columns, each into a stack of K-major slots
+    if ((e = launch_qdq(W_qkv, in_dtype, K, 2 * D, group, n_grid, S, Wqk, err, s, &launches, kQuantAsym, 0, N)) !=
+            cudaSuccess ||
+        (e = launch_qdq(W_v, in_dtype, K, D, group, n_grid, S, Wv, err, s, &launches, kQuantAsym, 0, N)) !=
+            cudaSuccess) {
+      where = "qdq kernel";
+      break;
+    }
+    mark(1);
+    // [Q | K] of every slot: X_b [M][K] times the slot's [W_q | W_k] (mode 5, bf16 out)
+    LossGemmArgs g;
+    g.Xb = Xb;
+    g.Wt = Wqk;
+    g.M = M;
+    g.K = K;
+    g.N = 2 * D;
+    g.n_grid = n_grid;
+    g.Y = nullptr;
+    g.partial = nullptr;
+    g.err = err;
+    g.timeout_ns = g_timeout_ns;
+    g.fault_mode = 0;
+    g.num_sms = num_sms;
+    g.H = QK;
+    g.h_stride = M * 2 * D;
+    g.cands = slots;
+    g.slot_base = 0;
+    g.b_per_cand = 1;
+    // V^T of every slot: the slot's W_v^T [D][K] (a stack of A operands) times X_b
+    LossGemmArgs gv = g;
+    gv.Xb = Wv;
+    gv.a_slotted = 1;
+    gv.a_slots = slots;
+    gv.a_slot_base = 0;
+    gv.M = D;
+    gv.Wt = Xb;
+    gv.N = M;
+    gv.n_grid = 0;  // one B slot for the tensor map
+    gv.H = VT;
+    gv.h_stride = D * M;
+    gv.b_per_cand = 0;
+    CUtensorMap mA, mB, vA, vB;
+    const char* why = "";
+    if ((e = make_operand_maps(g, &mA, &mB, &why, kTileN)) != cudaSuccess ||
+        (e = make_operand_maps(gv, &vA, &vB, &why, kTileN)) != cudaSuccess) {
+      status = set_error(AWQ_ERR_CUDA, std::string("TMA descriptor: ") + why);
+      break;
+    }
+    if ((e = launch_loss_gemm(g, mA, mB, 5, s, &launches)) != cudaSuccess) { where = "Q|K GEMM"; break; }
+    mark(2);
+    if ((e = launch_loss_gemm(gv, vA, vB, 5, s, &launches)) != cudaSuccess) { where = "V^T GEMM"; break; }
+    mark(3);
+    AttnLossArgs at;
+    at.QK = QK;
+    at.VT = VT;
+    at.total_slots = slots;
+    at.M = M;
+    at.D = D;
+    at.T = seq_len;
+    at.n_heads = n_heads;
+    at.O_ref = O_ref;
+    at.partial = part;
+    at.err = err;
+    at.timeout_ns = g_timeout_ns;
+    at.num_sms = num_sms;
+    at.fault_mode = g_fault_mode;
+    at.slot0 = 0;
+    at.slots = 1;
+    if ((e = launch_attn_loss(at, 1, s, &launches)) != cudaSuccess) { where = "reference attention"; break; }
+    mark(4);
+    at.slot0 = 1;
+    at.slots = n_grid;
+    if ((e = launch_attn_loss(at, 0, s, &launches)) != cudaSuccess) { where = "candidate attention"; break; }
+    mark(5);
+    if ((e = launch_loss_reduce(part, units, n_grid, M, D, losses, s, &launches)) != cudaSuccess) {
+      where = "loss reduction kernel";
+      break;
+    }
+    if ((e = launch_pack(W_qkv, in_dtype, K, N, group, n_grid, S, losses, best, out_codes,
+                         static_cast<__half*>(out_steps), static_cast<__half*>(out_zeros), out_scales, s,
+                         &launches)) != cudaSuccess) {
+      where = "pack kernel";
+      break;
+    }
+    mark(6);
+    if (out_losses &&
+        (e = cudaMemcpyAsync(out_losses, losses, static_cast<size_t>(n_grid) * 4, cudaMemcpyDeviceToDevice, s)) !=
+            cudaSuccess) {
+      where = "copy of the losses";
+      break;
+    }
+    if (out_best && (e = cudaMemcpyAsync(out_best, best, sizeof(int32_t), cudaMemcpyDeviceToDevice, s)) != cudaSuccess) {
+      where = "copy of the chosen index";
+      break;
+    }
+  } while (false);
+  int* pinned = pinned_status_word(dev);
+  int* status_dst = pinned ? pinned : &h_err;
+  if (status == AWQ_OK && e == cudaSuccess) {
+    e = cudaMemcpyAsync(status_dst, err, sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) where = "status read-back";
+  }
+  if (status == AWQ_OK && e != cudaSuccess) status = cuda_error(e, where);
+  cudaFreeAsync(ws, s);
+  cudaError_t se = cudaStreamSynchronize(s);
+  if (status == AWQ_OK && se != cudaSuccess) status = cuda_error(se, "stream synchronize");
+  if (pinned) h_err = *pinned;
+  if (status == AWQ_OK) {
+    g_last_launches = launches;
+    if (ev)
+      for (int i = 0; i < kAttnPhases; ++i) cudaEventElapsedTime(&g_attn_ms[i], ev[i], ev[i + 1]);
+    status = status_from_word(h_err);
+  }
+  return status;
+}
+
+int awq_attn_profile_last(float* ms, int n) {
+  for (int i = 0; i < n && i < kAttnPhases; ++i) ms[i] = g_attn_ms[i];
+  return kAttnPhases;
+}
+
 int awq_clip_profile_last(float* ms, int n) {
   for (int i = 0; i < n && i < 2; ++i) ms[i] = g_clip_ms[i];
   return 2;
@@ -1441,6 +1718,7 @@ int awq_fp64_mma_peak(double* tflops, awq_stream_t stream) {
   t_last_error.clear();
   if (!tflops) return set_error(AWQ_ERR_INVALID_ARG, "tflops is NULL");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DeviceRestore restore_device;
   bind_device(s, nullptr);
   int dev = 0, num_sms = 0, st;
   if ((st = check_device(&dev, &num_sms)) != AWQ_OK) return st;

@@ -32,14 +32,16 @@ cudaError_t launch_to_bf16(const float* x, int64_t n, __nv_bfloat16* out, cudaSt
 // Writes Wt[0] = bf16(W)^T and Wt[1 + i] = bf16(W_hat_i)^T, each N x K (K contiguous).
 // `interleave` = F > 0 (N = 2F, F % 128 == 0) writes the columns of [W_gate | W_up] in the
 // order the fused MLP GEMM reads them: every 256 rows are 128 gate columns followed by the
-// 128 up columns of the same outputs.
+// 128 up columns of the same outputs. `ldw` > 0: W's rows are ldw elements apart (N columns
+// of a wider matrix, e.g. the key or value part of [W_q | W_k | W_v]); 0 means N.
 cudaError_t launch_qdq(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid,
                        const float* S, __nv_bfloat16* Wt, int* err, cudaStream_t s, int* launches,
-                       int quantizer = 0, int64_t interleave = 0);
+                       int quantizer = 0, int64_t interleave = 0, int64_t ldw = 0);
 // The same for the groups group0 .. group0 + groups - 1 only (rows group0*group ..).
 cudaError_t launch_qdq_groups(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid,
                               const float* S, __nv_bfloat16* Wt, int* err, int64_t group0, int64_t groups,
-                              cudaStream_t s, int* launches, int quantizer = 0, int64_t interleave = 0);
+                              cudaStream_t s, int* launches, int quantizer = 0, int64_t interleave = 0,
+                              int64_t ldw = 0);
 
 // ---- artifact of the chosen candidate (AWQ-P1 §7; QUANT-P4 §5.3) ------------------
 // The chosen candidate is the first minimum of `losses` (AWQ-P1 §3); its index is
@@ -64,10 +66,10 @@ struct LossGemmArgs {
   int variant = 1;           // 1 the one-SM kernel, 2 the two-SM kernel (modes 0 and 1, slot_base 1)
   int slot_base = 1;         // B slot of candidate 0 (mode 1; the search's slot 0 is bf16(W)) or the
                              // slot multiplied (modes 2, 3); values other than 1 run on the one-SM kernel
-  __nv_bfloat16* H = nullptr;  // mode 3: the MLP block's intermediate h, M x N/2 row-major bf16
-  int64_t h_stride = 0;        // mode 3: elements between successive candidates' h
-  int cands = 0;               // modes 1, 3: candidates this launch walks (0: n_grid for mode 1, 1 for mode 3)
-  int b_per_cand = 1;          // modes 1, 3: candidate c reads B slot slot_base + c (1) or slot_base (0)
+  __nv_bfloat16* H = nullptr;  // mode 3: the MLP block's intermediate h, M x N/2 row-major bf16; mode 5: the output
+  int64_t h_stride = 0;        // modes 3, 5: elements between successive candidates' outputs
+  int cands = 0;               // modes 1, 3, 5: candidates this launch walks (0: n_grid for mode 1, else 1)
+  int b_per_cand = 1;          // modes 1, 3, 5: candidate c reads B slot slot_base + c (1) or slot_base (0)
   int a_slotted = 0;           // A is a stack of a_slots operands [a_slots][M][K]; c reads a_slot_base + c
   int a_slot_base = 0;
   int a_slots = 1;
@@ -90,7 +92,10 @@ cudaError_t make_operand_maps(const LossGemmArgs& a, CUtensorMap* mapA, CUtensor
 // kernel only; the grid never exceeds the SMs, so every awaited flag belongs to a running CTA);
 // mode 3: the MLP block's first GEMM with the silu-mul fused in its epilogue: the B slot
 // holds [W_gate | W_up] interleaved by 128 columns (launch_qdq's `interleave`), and
-// h = bf16(fl32(silu(g) u)) is written row-major into a.H (M x N/2), one-SM kernel only.
+// h = bf16(fl32(silu(g) u)) is written row-major into a.H (M x N/2), one-SM kernel only;
+// mode 5: for each of a.cands candidates (B slot slot_base + c when b_per_cand, A slot
+// a_slot_base + c when a_slotted) the product rounded to bf16, row-major (pitch N) at
+// a.H + c * a.h_stride, one-SM kernel only.
 cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, const CUtensorMap& mapB,
                              int mode, cudaStream_t s, int* launches);
 
@@ -160,6 +165,29 @@ cudaError_t launch_silu_mul(const float* H, int64_t M, int64_t F, __nv_bfloat16*
 cudaError_t launch_transpose_bf16(const void* W, int in_dtype, int64_t rows, int64_t cols, __nv_bfloat16* Wt,
                                   cudaStream_t s, int* launches);
 
+// ---- attention-block objective (AWQ-P1 §4: the candidate scored on its module's output) --
+// Causal multi-head attention of Q, K, V = bf16(X_b W_hat) over sequences of T tokens
+// (T a multiple of 128, at most kAttnMaxSeq), heads kAttnHeadDim wide, with the loss
+// against the reference output fused into the epilogue.
+constexpr int kAttnHeadDim = 128;
+constexpr int kAttnMaxSeq = 512;
+struct AttnLossArgs {
+  const __nv_bfloat16* QK;  // [total_slots][M][2D]: Q in columns 0 .. D-1, K in D .. 2D-1
+  const __nv_bfloat16* VT;  // [total_slots][D][M]: V transposed
+  int total_slots;          // slots in both stacks
+  int slot0, slots;         // the slots this launch walks
+  int64_t M, D, T;          // tokens, model width (n_heads * kAttnHeadDim), tokens per sequence
+  int n_heads;
+  float* O_ref;             // [M][D] fp32: written by the reference launch, read by the others
+  double* partial;          // [slots][M / T * n_heads * T / 128] squared-error partials
+  int* err;
+  uint64_t timeout_ns;
+  int num_sms;
+  int fault_mode = 0;       // 1: the producer skips its first key tile (tests the bounded waits)
+};
+// ref = 1: O of slot slot0 stored into O_ref; ref = 0: per-unit squared error against it.
+cudaError_t launch_attn_loss(const AttnLossArgs& a, int ref, cudaStream_t s, int* launches);
+
 __host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Raise a kernel's dynamic shared-memory limit to `bytes` once per device (the first
@@ -178,5 +206,35 @@ cudaError_t set_smem_limit_once(Kernel kernel, int bytes, unsigned long long* do
 
 // Sets the text awq_last_error_message returns on the calling thread.
 void record_error_message(const char* msg);
+
+// Puts the calling thread's current device back when an entry point returns: the entry
+// points make the device of the caller's stream (or pointer) current for their own work.
+struct DeviceRestore {
+  int dev = -1;
+  DeviceRestore() {
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+      cudaGetLastError();
+      dev = -1;
+    }
+  }
+  ~DeviceRestore() {
+    if (dev >= 0) cudaSetDevice(dev);
+  }
+  DeviceRestore(const DeviceRestore&) = delete;
+  DeviceRestore& operator=(const DeviceRestore&) = delete;
+};
+
+// Work space the caller of the search provides instead of the library's pool: `bytes`
+// long, its device address resolved by `resolve` once the call's device is current.
+// A search given one allocates nothing (no pool block, no pinned status word, no
+// profiling events) and reads the status word back into pageable host memory.
+struct FixedWorkspace {
+  size_t bytes;
+  int (*resolve)(int dev, void** base);
+};
+// The search of awq_search_ex (plus the chosen index) in a fixed work space.
+int search_in_workspace(const void* X, const void* W, int in_dtype, int64_t M, int64_t K, int64_t N, int group,
+                        int n_grid, float* out_scales, int32_t* out_codes, void* out_steps, void* out_zeros,
+                        float* out_losses, int32_t* out_best, cudaStream_t s, const FixedWorkspace& fixed);
 
 }  // namespace awq

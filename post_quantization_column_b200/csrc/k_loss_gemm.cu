@@ -18,7 +18,9 @@
 //   mode 3: the MLP block's first GEMM, B = [W_gate | W_up] interleaved by 128 columns so
 //           that a 256-column tile holds the gate and up halves of 128 intermediate
 //           columns; the epilogue writes h = bf16(silu(g) u) row-major and never stores
-//           the fp32 halves.
+//           the fp32 halves;
+//   mode 5: a plain product per candidate, rounded to bf16 and written row-major (the
+//           attention block's Q, K and V^T operands), ragged rows and columns masked.
 //
 // Blackwell structure (sm_100a): 128 x 256 output tiles, K in 64-element (128-byte)
 // slices; a 4-stage TMA -> shared-memory ring (128-byte swizzle, no multicast); one
@@ -158,7 +160,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
-  const int64_t n_units = (p.mode == 1 || p.mode == 3 ? p.cands : (p.mode == 4 ? p.n_grid + 1 : 1)) * tiles;
+  const int64_t n_units =
+      (p.mode == 1 || p.mode == 3 || p.mode == 5 ? p.cands : (p.mode == 4 ? p.n_grid + 1 : 1)) * tiles;
   const uint64_t budget = p.timeout_ns;
 
   auto fail = [&]() {
@@ -179,7 +182,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         unit_coords(u, p, c, mt, nt);
         const int slot = p.mode == 0 ? 0
                          : p.mode == 4 ? c  // 0: bf16(W), then candidate c - 1 in slot c
-                                       : p.slot_base + ((p.mode == 1 || p.mode == 3) && p.b_per_cand ? c : 0);
+                                       : p.slot_base +
+                                             ((p.mode == 1 || p.mode == 3 || p.mode == 5) && p.b_per_cand ? c : 0);
         for (int kb = 0; kb < p.nk; ++kb) {
           if (!mbar_wait_bounded(empty + stage, phase ^ 1u, abort_flag, budget)) {
             ok = false;
@@ -295,6 +299,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const __nv_bfloat162 hv =
                     __floats2bfloat162_rn(silu_mul_f32(__uint_as_float(g[k]), __uint_as_float(up[k])),
                                           silu_mul_f32(__uint_as_float(g[k + 1]), __uint_as_float(up[k + 1])));
+                w[e] = *reinterpret_cast<const uint32_t*>(&hv);
+              }
+              orow[q] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(tempty + acc);
+        continue;
+      }
+      if (p.mode == 5) {
+        // the product of candidate c rounded to bf16, row-major with pitch ldo
+        const int64_t grow = static_cast<int64_t>(mt) * BM + row;
+#pragma unroll 1
+        for (int j0 = 0; j0 < BN; j0 += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(j0), v);
+          tmem_ld_wait();
+          const int64_t col0 = static_cast<int64_t>(nt) * BN + j0;
+          if (grow < p.M) {
+            uint4* orow = reinterpret_cast<uint4*>(p.H + static_cast<int64_t>(c) * p.h_stride + grow * p.ldo + col0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {  // N % 8 == 0: eight columns lie wholly inside or outside
+              if (col0 + 8 * q >= p.N) continue;
+              uint32_t w[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const __nv_bfloat162 hv = __floats2bfloat162_rn(__uint_as_float(v[8 * q + 2 * e]),
+                                                                __uint_as_float(v[8 * q + 2 * e + 1]));
                 w[e] = *reinterpret_cast<const uint32_t*>(&hv);
               }
               orow[q] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -823,7 +856,7 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
   p.timeout_ns = a.timeout_ns;
   p.fault_mode = a.fault_mode;
   const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
-  const int64_t units = (mode == 1 || mode == 3 ? p.cands : (mode == 4 ? a.n_grid + 1 : 1)) * tiles;
+  const int64_t units = (mode == 1 || mode == 3 || mode == 5 ? p.cands : (mode == 4 ? a.n_grid + 1 : 1)) * tiles;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(units, a.num_sms));
   loss_gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(mapA, mapB, p);
   *launches += 1;

@@ -86,11 +86,12 @@ __device__ __forceinline__ float round_small(float x) {
   return __fsub_rn(__fadd_rn(x, kRoundMagic), kRoundMagic);
 }
 
-// Stage a G x L::kCols tile of W transposed in shared memory (sWT[col][row]) from
-// coalesced 16-byte global loads; columns at or beyond N read as 0. Returns whether a
-// non-finite value was seen.
+// Stage a G x L::kCols tile of W (row pitch ldw elements) transposed in shared memory
+// (sWT[col][row]) from coalesced 16-byte global loads; columns at or beyond N read as 0.
+// Returns whether a non-finite value was seen.
 template <typename T, int G, typename L>
-__device__ __forceinline__ bool stage_tile(const T* __restrict__ W, int64_t N, int64_t k0, int64_t n0, float* sWT) {
+__device__ __forceinline__ bool stage_tile(const T* __restrict__ W, int64_t N, int64_t ldw, int64_t k0, int64_t n0,
+                                           float* sWT) {
   constexpr int VEC = 16 / sizeof(T);
   constexpr int VPR = L::kCols / VEC;
   bool bad = false;
@@ -99,7 +100,7 @@ __device__ __forceinline__ bool stage_tile(const T* __restrict__ W, int64_t N, i
     const int64_t col = n0 + static_cast<int64_t>(v) * VEC;
     float vals[VEC];
     if (col < N) {  // N % 8 == 0: a vector lies wholly inside or outside
-      const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(W + (k0 + r) * N + col));
+      const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(W + (k0 + r) * ldw + col));
       const T* e = reinterpret_cast<const T*>(&raw);
 #pragma unroll
       for (int i = 0; i < VEC; ++i) {
@@ -280,7 +281,8 @@ __device__ __noinline__ void exact_run(float2 w0, float2 w1, float2 w2, float2 w
 template <typename T, int G>
 __global__ void __launch_bounds__(Tile<G>::kThreads, Tile<G>::kBlocksPerSm)
     qdq_kernel(const T* __restrict__ W, int64_t K, int64_t N, int n_grid, const float* __restrict__ S,
-               __nv_bfloat16* __restrict__ Wt, int* err, int64_t group0, int quantizer, int64_t interleave) {
+               __nv_bfloat16* __restrict__ Wt, int* err, int64_t group0, int quantizer, int64_t interleave,
+               int64_t ldw) {
   using L = Tile<G>;
   extern __shared__ float smem[];
   float* sWT = smem;                                    // [64][kPitch]
@@ -296,7 +298,7 @@ __global__ void __launch_bounds__(Tile<G>::kThreads, Tile<G>::kBlocksPerSm)
 
   if (threadIdx.x < 2) sRowsExact[threadIdx.x] = 0u;
   __syncthreads();
-  if (stage_tile<T, G, L>(W, N, k0, n0, sWT)) atomicOr(err, kErrNonfiniteW);
+  if (stage_tile<T, G, L>(W, N, ldw, k0, n0, sWT)) atomicOr(err, kErrNonfiniteW);
   for (int idx = threadIdx.x; idx < n_grid * G; idx += L::kThreads) {
     const int c = idx / G, r = idx % G;
     const float s = S[static_cast<int64_t>(c) * K + k0 + r];
@@ -382,9 +384,11 @@ __global__ void __launch_bounds__(Tile<G>::kThreads, Tile<G>::kBlocksPerSm)
   __syncwarp();
 
   // Phase B: codes, reconstruction and fold-back of every candidate. A candidate for
-  // which one of the lane's runs holds a code decided only by the exact quotient, or
-  // lies outside the range guards, is recorded and redone after the pass (the thread
-  // rewrites its own stores), which keeps the rare paths out of the streaming loop.
+  // which one of the lane's runs holds a code decided only by the exact quotient, lies
+  // outside the range guards, or may clamp a code (a column whose zero point clips its
+  // range, or whose rounded zero sits half a step from the range's end) is recorded and
+  // redone after the pass (the thread rewrites its own stores), which keeps the rare
+  // paths out of the streaming loop: it runs one instruction stream for every lane.
   uint64_t redo = 0;
   for (int c = 0; c < n_grid; ++c) {
     float2 s2[4];
@@ -409,9 +413,8 @@ __global__ void __launch_bounds__(Tile<G>::kThreads, Tile<G>::kBlocksPerSm)
 #pragma unroll
       for (int i = 0; i < 4; ++i) wp[i] = __fmul2_rn(s2[i], w2[j][i]);
       uint32_t out[4];
-      flag |= (flags & 1) != 0;
-      flag |= (flags & 2) ? fold_back_pairs<false, false>(wp, s2, rs, cq, out)
-                          : fold_back_pairs<true, false>(wp, s2, rs, cq, out);
+      flag |= (flags & 3) != 2;  // outside the range guards, or a code may clamp
+      flag |= fold_back_pairs<false, false>(wp, s2, rs, cq, out);
       if (active) *reinterpret_cast<uint4*>(slot + (j ? dst1_off : 0)) = make_uint4(out[0], out[1], out[2], out[3]);
     }
     redo |= static_cast<uint64_t>(flag) << c;
@@ -696,7 +699,7 @@ __global__ void __launch_bounds__(PackShape<T, G>::kThreads, 4)
 template <typename T, int G>
 cudaError_t launch_qdq_t(const T* W, int64_t K, int64_t N, int n_grid, const float* S, __nv_bfloat16* Wt,
                          int* err, int64_t group0, int64_t groups, cudaStream_t s, int quantizer,
-                         int64_t interleave) {
+                         int64_t interleave, int64_t ldw) {
   using L = Tile<G>;
   auto bytes = [](int grid_points) {
     return (static_cast<size_t>(L::kCols) * L::kPitch + 2 * static_cast<size_t>(grid_points) * L::kSkewPitch +
@@ -708,7 +711,7 @@ cudaError_t launch_qdq_t(const T* W, int64_t K, int64_t N, int n_grid, const flo
   if (e != cudaSuccess) return e;
   dim3 grid(static_cast<unsigned>(ceil_div(N, static_cast<int64_t>(L::kCols))), static_cast<unsigned>(groups));
   qdq_kernel<T, G><<<grid, L::kThreads, bytes(n_grid), s>>>(W, K, N, n_grid, S, Wt, err, group0, quantizer,
-                                                            interleave);
+                                                            interleave, ldw > 0 ? ldw : N);
   return cudaGetLastError();
 }
 
@@ -728,28 +731,29 @@ cudaError_t launch_pack_t(const T* W, int64_t K, int64_t N, int n_grid, const fl
 
 cudaError_t launch_qdq_groups(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid,
                               const float* S, __nv_bfloat16* Wt, int* err, int64_t group0, int64_t groups,
-                              cudaStream_t s, int* launches, int quantizer, int64_t interleave) {
+                              cudaStream_t s, int* launches, int quantizer, int64_t interleave, int64_t ldw) {
   *launches += 1;
   if (in_dtype == 0) {
     const auto* w = static_cast<const __nv_bfloat16*>(W);
     switch (group) {
-      case 32: return launch_qdq_t<__nv_bfloat16, 32>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer, interleave);
-      case 64: return launch_qdq_t<__nv_bfloat16, 64>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer, interleave);
-      default: return launch_qdq_t<__nv_bfloat16, 128>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer, interleave);
+      case 32: return launch_qdq_t<__nv_bfloat16, 32>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer, interleave, ldw);
+      case 64: return launch_qdq_t<__nv_bfloat16, 64>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer, interleave, ldw);
+      default: return launch_qdq_t<__nv_bfloat16, 128>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer, interleave, ldw);
     }
   }
   const auto* w = static_cast<const float*>(W);
   switch (group) {
-    case 32: return launch_qdq_t<float, 32>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer, interleave);
-    case 64: return launch_qdq_t<float, 64>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer, interleave);
-    default: return launch_qdq_t<float, 128>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer, interleave);
+    case 32: return launch_qdq_t<float, 32>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer, interleave, ldw);
+    case 64: return launch_qdq_t<float, 64>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer, interleave, ldw);
+    default: return launch_qdq_t<float, 128>(w, K, N, n_grid, S, Wt, err, group0, groups, s, quantizer, interleave, ldw);
   }
 }
 
 cudaError_t launch_qdq(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid, const float* S,
-                       __nv_bfloat16* Wt, int* err, cudaStream_t s, int* launches, int quantizer, int64_t interleave) {
+                       __nv_bfloat16* Wt, int* err, cudaStream_t s, int* launches, int quantizer, int64_t interleave,
+                       int64_t ldw) {
   return launch_qdq_groups(W, in_dtype, K, N, group, n_grid, S, Wt, err, 0, K / group, s, launches, quantizer,
-                           interleave);
+                           interleave, ldw);
 }
 
 cudaError_t launch_pack(const void* W, int in_dtype, int64_t K, int64_t N, int group, int n_grid, const float* S,

@@ -10,7 +10,7 @@
  *
  * IN:  int64 M, K, N; int32 group, n_grid, dtype (0 bf16, 1 fp32); X (M x K), W (K x N).
  * OUT: three records, each: int32 status; scales [K] fp32; codes [K][N/8] int32;
- *      steps, zeros [K/group][N] fp16; losses [n_grid] fp32.
+ *      steps, zeros [K/group][N] fp16; losses [n_grid] fp32; best (the chosen index) int32.
  * Exit status 0 when every call returned AWQ_OK, 1 on a call error, 2 on I/O or CUDA
  * setup errors.
  */
@@ -21,14 +21,6 @@
 #include <cuda_runtime_api.h>
 
 #include "awq_search.h"
-
-struct Outputs {
-  float* scales;
-  int32_t* codes;
-  uint16_t* steps;
-  uint16_t* zeros;
-  float* losses;
-};
 
 static int read_all(FILE* f, void* p, size_t n) { return fread(p, 1, n, f) == n; }
 static int write_all(FILE* f, const void* p, size_t n) { return fwrite(p, 1, n, f) == n; }
@@ -52,11 +44,12 @@ int main(int argc, char** argv) {
   if (!hX || !hW || !read_all(in, hX, bx) || !read_all(in, hW, bw)) return 2;
   fclose(in);
 
-  const size_t nb[5] = {(size_t)K * 4, (size_t)K * (N / 8) * 4, (size_t)(K / group) * N * 2,
-                        (size_t)(K / group) * N * 2, (size_t)n_grid * 4};
-  void *dX, *dW, *dout[5], *hout[5];
+  /* scales, codes, steps, zeros, losses, chosen index */
+  const size_t nb[6] = {(size_t)K * 4, (size_t)K * (N / 8) * 4, (size_t)(K / group) * N * 2,
+                        (size_t)(K / group) * N * 2, (size_t)n_grid * 4, 4};
+  void *dX, *dW, *dout[6], *hout[6];
   if (cudaMalloc(&dX, bx) != cudaSuccess || cudaMalloc(&dW, bw) != cudaSuccess) return 2;
-  for (int i = 0; i < 5; ++i) {
+  for (int i = 0; i < 6; ++i) {
     if (cudaMalloc(&dout[i], nb[i]) != cudaSuccess) return 2;
     hout[i] = malloc(nb[i]);
     if (!hout[i]) return 2;
@@ -75,32 +68,32 @@ int main(int argc, char** argv) {
     int32_t st;
     if (call == 0) {
       st = awq_search_ex(dX, dW, dtype, M, K, N, group, n_grid, (float*)dout[0], (int32_t*)dout[1], dout[2], dout[3],
-                         (float*)dout[4], NULL, 0, (awq_stream_t)stream);
+                         (float*)dout[4], (int32_t*)dout[5], NULL, 0, (awq_stream_t)stream);
     } else if (call == 1) {
       *status_word = -1;
       st = awq_search_async(dX, dW, dtype, M, K, N, group, n_grid, (float*)dout[0], (int32_t*)dout[1], dout[2],
-                            dout[3], (float*)dout[4], status_word, (awq_stream_t)stream);
+                            dout[3], (float*)dout[4], (int32_t*)dout[5], status_word, (awq_stream_t)stream);
       if (st == AWQ_OK) {
         if (cudaStreamSynchronize(stream) != cudaSuccess) return 2;
         st = awq_search_status(*status_word);
       }
     } else {
       st = awq_search_host(hX, hW, dtype, M, K, N, group, n_grid, (float*)hout[0], (int32_t*)hout[1], hout[2],
-                           hout[3], (float*)hout[4], (awq_stream_t)stream);
+                           hout[3], (float*)hout[4], (int32_t*)hout[5], (awq_stream_t)stream);
     }
     if (st != AWQ_OK) {
       fprintf(stderr, "call %d: %s: %s\n", call, awq_status_string(st), awq_last_error_message());
       failed = 1;
     }
     if (call < 2)
-      for (int i = 0; i < 5; ++i)
+      for (int i = 0; i < 6; ++i)
         if (cudaMemcpy(hout[i], dout[i], nb[i], cudaMemcpyDeviceToHost) != cudaSuccess) return 2;
     if (!write_all(out, &st, 4)) return 2;
-    for (int i = 0; i < 5; ++i)
+    for (int i = 0; i < 6; ++i)
       if (!write_all(out, hout[i], nb[i])) return 2;
   }
   fclose(out);
-  for (int i = 0; i < 5; ++i) {
+  for (int i = 0; i < 6; ++i) {
     cudaFree(dout[i]);
     free(hout[i]);
   }

@@ -39,10 +39,10 @@ def write_input(path: str, X: np.ndarray, W: np.ndarray, group: int, n_grid: int
 
 
 def read_output(path: str, K: int, N: int, group: int, n_grid: int):
-    """Three records (status, scales, codes, steps, zeros, losses) of the client's calls."""
+    """Three records (status, scales, codes, steps, zeros, losses, best) of the client's calls."""
     sizes = [("scales", np.float32, (K,)), ("codes", np.int32, (K, N // 8)),
              ("steps", np.uint16, (K // group, N)), ("zeros", np.uint16, (K // group, N)),
-             ("losses", np.float32, (n_grid,))]
+             ("losses", np.float32, (n_grid,)), ("best", np.int32, (1,))]
     out = []
     with open(path, "rb") as f:
         for _ in range(3):

@@ -101,6 +101,9 @@ def full_parity(X: torch.Tensor, W: torch.Tensor, group: int, n_grid: int):
     X32, W32 = as_f32_numpy(X), as_f32_numpy(W)
     gpu = run_gpu(X, W, group, n_grid, tiles=True)
     orc = O.search(X32, W32, group=group, n_grid=n_grid)
+    # the index the library returned is the first minimum of the losses it returned
+    # (AWQ-P1 §3), and follows the oracle's choice up to near-ties
+    assert gpu["best"] == O.first_argmin(list(gpu["losses"])), "library index is not its losses' first minimum"
     check_alpha(gpu["best"], orc.losses)
     check_losses(gpu["losses"], orc.losses)
     check_artifact(gpu, W32, orc.S, group)

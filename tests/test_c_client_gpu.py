@@ -13,6 +13,7 @@ import torch
 import oracle as O
 import post_quantization_column_b200 as awq
 from tests import c_client
+from tests.parity import check_alpha
 from workloads import custom_spec, generate, as_f32_numpy
 
 pytestmark = pytest.mark.gpu
@@ -37,15 +38,21 @@ def test_c_client_matches_the_binding_and_the_oracle(dtype, group, tmp_path):
     ref = awq.search(X.cuda(), W.cuda(), group, spec.n_grid)
     want = {"scales": ref.scales.cpu().numpy(), "codes": ref.codes.cpu().numpy(),
             "steps": ref.steps.cpu().view(torch.int16).numpy().view(np.uint16),
-            "zeros": ref.zeros.cpu().view(torch.int16).numpy().view(np.uint16), "losses": ref.losses.cpu().numpy()}
+            "zeros": ref.zeros.cpu().view(torch.int16).numpy().view(np.uint16), "losses": ref.losses.cpu().numpy(),
+            "best": ref.best_index.cpu().numpy()}
     for call, rec in zip(("awq_search_ex", "awq_search_async", "awq_search_host"), recs):
         assert rec["status"] == 0, call
         for name, value in want.items():
             assert np.array_equal(rec[name].view(np.uint8), value.view(np.uint8)), (call, name)
 
-    # the artifact at the chosen alpha, against the oracle
+    # the index the library returned (out_best) follows the oracle's rule on the losses
+    # it returned (AWQ-P1 §3: the first minimum), and the artifact at that alpha is the
+    # oracle's
     X32, W32 = as_f32_numpy(X), as_f32_numpy(W)
-    best = ref.best
+    best = int(recs[0]["best"][0])
+    assert best == int(np.argmin(recs[0]["losses"]))
+    r = O.search(X32, W32, group=group, n_grid=spec.n_grid)
+    check_alpha(best, r.losses)
     s = O.candidate_scales(O.activation_statistic(X32), spec.n_grid)[best]
     assert np.array_equal(recs[0]["scales"].view(np.uint32), s.view(np.uint32))
     q, step, zero, _ = O.asym_qdq(O.scale_weights(W32, s), group)

@@ -62,3 +62,28 @@ def test_full_size_workload(name):
         orc = O.search(X32, W32, group=spec.group, n_grid=spec.n_grid)
         P.check_alpha(gpu["best"], orc.losses)
         P.check_losses(gpu["losses"], orc.losses)
+
+
+def test_llama70b_column_slice_against_the_complete_oracle():
+    """The 70B gate+up layer's full X (16384 x 8192, 64 groups) with 1024 columns from
+    each half of W (the first of the gate half and of the up half): the layer the
+    complete oracle can finish in about a minute on the host. Alpha rule, every loss,
+    the artifact over every column and sampled tiles, as for the small layers."""
+    spec = WORKLOADS["llama70b_mlp_gate_up_16384x8192x57344"]
+    X, W = generate(spec)
+    half = spec.N // 2
+    Ws = torch.cat([W[:, :1024], W[:, half:half + 1024]], dim=1).contiguous()
+    del W
+    gpu = P.run_gpu(X, Ws, spec.group, spec.n_grid, tiles=True)
+    torch.cuda.empty_cache()
+    X32, W32 = as_f32_numpy(X), as_f32_numpy(Ws)
+    del X, Ws
+    orc = O.search(X32, W32, group=spec.group, n_grid=spec.n_grid)
+    assert gpu["best"] == O.first_argmin(list(gpu["losses"]))
+    P.check_alpha(gpu["best"], orc.losses)
+    P.check_losses(gpu["losses"], orc.losses)
+    P.check_artifact(gpu, W32, orc.S, spec.group)
+    T = gpu["tiles"]
+    samples = [(c, mt, nt) for c in sorted({0, gpu["best"], spec.n_grid - 1})
+               for mt, nt in ((0, 0), (T.shape[1] - 1, T.shape[2] - 1), (T.shape[1] // 2, T.shape[2] // 2))]
+    P.check_tiles(gpu, X32, W32, orc.S, spec.group, samples)

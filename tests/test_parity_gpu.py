@@ -93,7 +93,7 @@ def test_results_are_deterministic():
     X, W = generate(spec)
     a = awq.search(X.cuda(), W.cuda(), tile_sq_err=True)
     b = awq.search(X.cuda(), W.cuda(), tile_sq_err=True)
-    for name in ("scales", "codes", "steps", "zeros", "losses", "tile_sq_err"):
+    for name in ("scales", "codes", "steps", "zeros", "losses", "best_index", "tile_sq_err"):
         assert torch.equal(getattr(a, name), getattr(b, name)), name
 
 
@@ -102,7 +102,7 @@ def test_host_entry_point_matches_device_entry_point():
     X, W = generate(spec)
     d = awq.search(X.cuda(), W.cuda())
     h = awq.search_host(X.pin_memory(), W.pin_memory())
-    for name in ("scales", "codes", "steps", "zeros", "losses"):
+    for name in ("scales", "codes", "steps", "zeros", "losses", "best_index"):
         assert torch.equal(getattr(d, name).cpu(), getattr(h, name)), name
 
 
@@ -115,7 +115,7 @@ def test_host_batch_matches_one_layer_at_a_time(dtype, group):
                                  group)
     for (X, W), o in zip(layers, outs):
         d = awq.search(X.cuda(), W.cuda(), group)
-        for name in ("scales", "codes", "steps", "zeros", "losses"):
+        for name in ("scales", "codes", "steps", "zeros", "losses", "best_index"):
             assert torch.equal(getattr(d, name).cpu(), getattr(o, name)), name
 
 
@@ -165,7 +165,7 @@ def test_async_searches_back_to_back_match_the_synchronous_call():
         awq.profile_enable(False)
     for s, (X, W), o, prof in zip(specs, layers, outs, profs):
         d = awq.search(X, W, s.group, s.n_grid)
-        for name in ("scales", "codes", "steps", "zeros", "losses"):
+        for name in ("scales", "codes", "steps", "zeros", "losses", "best_index"):
             assert torch.equal(getattr(d, name), getattr(o, name)), (s.name, name)
         assert set(prof) >= {"statistic", "qdq", "gemm_loss", "pack"}
         assert all(v >= 0.0 for v in prof.values()) and prof["gemm_loss"] > 0.0
@@ -208,7 +208,7 @@ def test_async_search_needs_a_pinned_status_word():
     word = (ctypes.c_int32 * 1)()  # pageable host memory
     p = lambda t: ctypes.c_void_p(t.data_ptr())
     st = lib.awq_search_async(p(X), p(W), 0, 16, 128, 64, 128, 20, p(outs[0]), p(outs[1]), p(outs[2]), p(outs[3]),
-                              p(outs[4]), ctypes.cast(word, ctypes.c_void_p),
+                              p(outs[4]), p(outs[5]), ctypes.cast(word, ctypes.c_void_p),
                               ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 1  # AWQ_ERR_INVALID_ARG
 
@@ -239,3 +239,45 @@ def test_launch_count_and_profile():
     assert awq.last_launch_count() == (6 if awq.loss_gemm_variant(256, 256, 512, 20) == 1 else 7)
     assert set(prof) >= {"statistic", "scales", "qdq", "gemm_reference", "gemm_loss", "loss_reduce", "pack"}
     assert all(v >= 0 for v in prof.values()) and prof["gemm_loss"] > 0
+
+
+def test_async_search_on_a_side_stream_with_a_non_contiguous_input():
+    """An explicit side stream first waits for the current stream, where the inputs and
+    their contiguous copies are produced: X is a transposed view whose contiguous copy is
+    made on the current stream just before the call. The result equals search()'s bit
+    for bit."""
+    spec = custom_spec(256, 384, 520, seed=71)
+    X, W = (t.cuda() for t in generate(spec))
+    ref = awq.search(X, W, spec.group, spec.n_grid)
+    Xt = X.t().contiguous()          # (K, M) storage; Xt.t() is X as a non-contiguous view
+    side = torch.cuda.Stream()
+    torch.cuda._sleep(2_000_000)     # keeps the current stream busy while the call is enqueued
+    Xv = Xt.t()
+    assert not Xv.is_contiguous()
+    out = awq.search_async(Xv, W, spec.group, spec.n_grid, stream=side).wait()
+    for name in ("scales", "codes", "steps", "zeros", "losses", "best_index"):
+        assert torch.equal(getattr(ref, name), getattr(out, name)), name
+
+
+def test_the_callers_current_device_is_given_back():
+    """A call on a stream of another device runs there and leaves the caller's current
+    device as it was."""
+    if torch.cuda.device_count() < 2:
+        pytest.skip("needs two GPUs")
+    spec = custom_spec(128, 256, 264, seed=72)
+    X, W = (t.to("cuda:1") for t in generate(spec))
+    torch.cuda.set_device(0)
+    out = awq.search(X, W, spec.group, spec.n_grid, stream=torch.cuda.Stream(device=1))
+    assert torch.cuda.current_device() == 0
+    assert out.codes.device == X.device
+
+
+def test_library_index_is_the_first_minimum_of_tied_losses():
+    """An all-zero layer ties every candidate at loss 0: the library keeps the first
+    index (AWQ-P1 §3)."""
+    K, N = 128, 64
+    X = torch.zeros(16, K, dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros(K, N, dtype=torch.bfloat16, device="cuda")
+    out = awq.search(X, W, 128, 20)
+    assert torch.all(out.losses == 0.0)
+    assert out.best == 0
