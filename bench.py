@@ -18,6 +18,7 @@ from __future__ import annotations
 
 import argparse
 import csv
+import gc
 import io
 import json
 import os
@@ -488,17 +489,27 @@ def time_searches(awq, spec: LayerSpec, Xd, Wd, stream, flush, steps: int, warmu
         awq.search(Xd, Wd, spec.group, spec.n_grid, stream=stream)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    # every step's outputs and status word exist before the timed region, so the host
+    # enqueues the steps without allocating (and without the garbage collector running)
+    outs = [awq.alloc_outputs(spec.K, spec.N, spec.group, spec.n_grid, Xd.device) for _ in range(steps)]
+    words = [torch.full((1,), -1, dtype=torch.int32, pin_memory=True) for _ in range(steps)]
     if barrier:
         barrier()
     torch.cuda.synchronize()
     clocks = ClockSampler(sample_clocks) if sample_clocks is not None else None
     pending = []
-    for i in range(steps):
-        flush.zero_()
-        starts[i].record(stream)
-        pending.append(awq.search_async(Xd, Wd, spec.group, spec.n_grid, stream=stream))
-        ends[i].record(stream)
-    torch.cuda.synchronize()
+    gc.collect()
+    gc.disable()
+    try:
+        for i in range(steps):
+            flush.zero_()
+            starts[i].record(stream)
+            pending.append(awq.search_async(Xd, Wd, spec.group, spec.n_grid, stream=stream, out=outs[i],
+                                            status=words[i]))
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    finally:
+        gc.enable()
     clock_info = clocks.stop() if clocks is not None else None
     phases = []
     out = None
@@ -551,6 +562,7 @@ def search_object(awq, spec: LayerSpec, t: dict, peaks: dict, peak_kind: str, su
     return {
         "workload": spec.name, "M": spec.M, "K": spec.K, "N": spec.N, "group": spec.group, "n_grid": spec.n_grid,
         "input_dtype": spec.dtype, "steps": steps, "ms_per_step": total_ms / steps,
+        "ms_per_step_min_max": [min(t["step_ms"]), max(t["step_ms"])],
         "layers_per_s": steps / (total_ms / 1e3),
         "TFLOP/s": spec.candidate_flops * steps / (total_ms / 1e3) / 1e12,
         "roofline": roof,

@@ -19,7 +19,7 @@ from dataclasses import dataclass
 import torch
 
 __all__ = [
-    "AwqError", "SearchOutput", "search", "search_async", "PendingSearch", "search_host", "search_host_batch", "library", "library_path", "header_path",
+    "AwqError", "SearchOutput", "search", "search_async", "alloc_outputs", "PendingSearch", "search_host", "search_host_batch", "library", "library_path", "header_path",
     "tile_shape", "workspace_bytes", "release_cached", "profile_enable", "profile_last",
     "last_launch_count", "debug_set_fault", "status_string", "exported_functions",
     "activation_statistic", "candidate_scales", "qdq_candidates", "ClipOutput", "clip_search",
@@ -230,6 +230,12 @@ def _alloc_outputs(K, N, group, n_grid, device, pin=False):
             torch.full((1,), -1, dtype=torch.int32, **kw))
 
 
+def alloc_outputs(K: int, N: int, group: int = 128, n_grid: int = 20, device=None, pin: bool = False) -> tuple:
+    """The six output tensors of one layer's search (scales, codes, steps, zeros, losses,
+    chosen index), on ``device`` or in pinned host memory."""
+    return _alloc_outputs(K, N, group, n_grid, device, pin)
+
+
 def _with_best(out: tuple) -> tuple:
     """A caller's 5-tuple of host outputs plus a pinned word for the chosen index."""
     return tuple(out) if len(out) == 6 else tuple(out) + (torch.full((1,), -1, dtype=torch.int32, pin_memory=True),)
@@ -306,10 +312,13 @@ class PendingSearch:
 
 
 def search_async(X: torch.Tensor, W: torch.Tensor, group: int = 128, n_grid: int = 20, *,
-                 stream: torch.cuda.Stream | None = None) -> PendingSearch:
+                 stream: torch.cuda.Stream | None = None, out: tuple | None = None,
+                 status: torch.Tensor | None = None) -> PendingSearch:
     """search() without waiting: the whole search is enqueued on ``stream`` and the call
     returns at once, so consecutive layers run back to back on the device. Argument
-    errors raise here; errors the kernels detect raise from ``wait()``."""
+    errors raise here; errors the kernels detect raise from ``wait()``. ``out`` (the six
+    device outputs of _alloc_outputs) and ``status`` (one pinned int32) may be given to
+    enqueue without allocating."""
     if X.dim() != 2 or W.dim() != 2 or X.shape[1] != W.shape[0]:
         raise ValueError("X must be (M, K) and W must be (K, N)")
     if X.dtype != W.dtype:
@@ -323,9 +332,12 @@ def search_async(X: torch.Tensor, W: torch.Tensor, group: int = 128, n_grid: int
     N = W.shape[1]
     if group <= 0 or K % group or N % 8:
         raise ValueError("group must divide K and N must be a multiple of 8")
-    outs = _alloc_outputs(K, N, group, n_grid, X.device)
+    outs = _alloc_outputs(K, N, group, n_grid, X.device) if out is None else tuple(out)
     scales, codes, steps, zeros, losses, best = outs
-    status = torch.full((1,), -1, dtype=torch.int32, pin_memory=True)
+    if status is None:
+        status = torch.full((1,), -1, dtype=torch.int32, pin_memory=True)
+    elif not status.is_pinned():
+        raise ValueError("status must be pinned host memory")
     if stream is None:  # the stream current now is the one wait() synchronizes later
         stream = torch.cuda.current_stream(X.device)
     handle = _stream_handle(stream, X.device)   # a side stream waits for the current one
