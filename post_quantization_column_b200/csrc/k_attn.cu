@@ -19,12 +19,15 @@
 //
 // Blackwell structure (sm_100a): one CTA per SM walks units (c, b, h, i), the longest
 // query blocks first. Warp 0 issues TMA loads (128-byte swizzle, no multicast): the query
-// tile, then the key tiles and the V^T tiles through a 2-stage ring. Warp 1 issues
+// tile, then the key tiles and the V^T tiles through a 4-stage ring. Warp 1 issues
 // tcgen05.mma (M = 128, N = 128, K = 16, bf16 -> fp32): the score tiles into tensor-memory
 // columns 128 j, then O += P_j V_j into columns 0 .. 127 (the first score tile's columns,
-// free once its weights are formed). Warps 4-7 (one query row per thread, warp w % 4 on
-// tensor-memory lanes 32 (w % 4) ..) read the scores with tcgen05.ld, form the weights
-// into shared memory in the swizzled K-major layout the MMA reads, and finish O. Every
+// free once its weights are formed). Warps 4-11 (two threads per query row, warp w on
+// tensor-memory lanes 32 (w % 4) .., one half of the key columns each) read the scores with
+// tcgen05.ld, 64 columns per wait, take the row max over the whole row, form the weights
+// (one FMA and one ex2 per score) into shared memory in the swizzled K-major layout the MMA
+// reads (two weight buffers, P_j in buffer j % 2 once the MMAs of tile j - 2 are done with
+// it), and finish O, with the reference row prefetched into L2 when the unit starts. Every
 // wait is bounded by the global timer; a wait that runs out sets the call's timeout bit,
 // raises a CTA-wide abort flag and the CTA drains its copies and MMAs before it exits.
 #include "awq_device.cuh"
@@ -38,14 +41,15 @@ namespace {
 
 constexpr int kHd = kAttnHeadDim;            // head dimension = rows of the V^T tile
 constexpr int kBlk = 128;                    // queries per unit, keys per key tile
-constexpr int kMaxKeyTiles = kAttnMaxSeq / kBlk;  // 4: the scores of a unit fill <= 512 TMEM columns
+static_assert(kAttnMaxSeq / kBlk * kBlk <= 512, "the scores of a unit fit the 512 tensor-memory columns");
 constexpr int kAtomBytes = kBlk * 128;       // one 64-column (128-byte) swizzle atom of 128 rows
 constexpr int kTileBytes = 2 * kAtomBytes;   // a 128 x 128 bf16 tile
-constexpr int kRing = 2;
-constexpr int kThreads = 256;
-constexpr int kEpi = 128;
+constexpr int kRing = 4;                     // key / V^T tiles in flight
+constexpr int kPBufs = 2;                    // weight tiles: P_j in buffer j % 2
+constexpr int kThreads = 384;               // warps 0-3 roles, warps 4-11 weights and epilogue
+constexpr int kEpi = 256;                   // two threads per query row, one per half of the key columns
 constexpr int kTmemCols = 512;
-constexpr int kSmemBytes = kTileBytes + kRing * kTileBytes + kMaxKeyTiles * kTileBytes + 512 + 1024;
+constexpr int kSmemBytes = kTileBytes + kRing * kTileBytes + kPBufs * kTileBytes + 512 + 1024 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 constexpr uint64_t kDrainNs = 200ull * 1000 * 1000;
 
@@ -96,9 +100,34 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x by the special-function unit (PTX ex2.approx.f32: subnormal results kept, 2^-inf = 0).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// 64 consecutive columns of this thread's tensor-memory row: two loads, one wait.
+__device__ __forceinline__ void load_row64(uint32_t taddr, uint32_t (&v)[2][32]) {
+  tmem_ld_32x32b_x32(taddr, v[0]);
+  tmem_ld_32x32b_x32(taddr + 32u, v[1]);
+  tmem_ld_wait_tied(v[0]);
+  tmem_ld_wait_tied(v[1]);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -108,19 +137,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                              // the query tile
   uint8_t* sRing = sQ + kTileBytes;                // key / V^T tiles
-  uint8_t* sP = sRing + kRing * kTileBytes;        // the weights of each key tile
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + kMaxKeyTiles * kTileBytes);
+  uint8_t* sP = sRing + kRing * kTileBytes;        // weight tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + kPBufs * kTileBytes);
   uint64_t* q_full = bars;              // the query tile landed
   uint64_t* q_empty = bars + 1;         // the score MMAs are done with it
   uint64_t* kv_full = bars + 2;         // [kRing]
-  uint64_t* kv_empty = bars + 4;        // [kRing]
-  uint64_t* s_full = bars + 6;          // every score tile of the unit is in tensor memory
-  uint64_t* p_ready = bars + 7;         // [kMaxKeyTiles] weights j written (128 arrivals)
-  uint64_t* o_full = bars + 11;         // O of the unit is in tensor memory
-  uint64_t* tmem_free = bars + 12;      // the epilogue has read O (128 arrivals)
-  uint64_t* drain = bars + 13;          // abort path: every issued MMA has completed
-  double* red = reinterpret_cast<double*>(bars + 14);  // [2][4]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red + 8);
+  uint64_t* kv_empty = bars + 6;        // [kRing]
+  uint64_t* s_full = bars + 10;         // every score tile of the unit is in tensor memory
+  uint64_t* p_ready = bars + 11;        // [kPBufs] a weight tile written (128 arrivals)
+  uint64_t* p_empty = bars + 13;        // [kPBufs] the P V MMAs are done with a weight tile
+  uint64_t* o_full = bars + 15;         // O of the unit is in tensor memory
+  uint64_t* tmem_free = bars + 16;      // the epilogue has read O (128 arrivals)
+  uint64_t* drain = bars + 17;          // abort path: every issued MMA has completed
+  double* red = reinterpret_cast<double*>(bars + 18);  // [2][8] per-warp loss partials
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red + 16);
+  float* xl = reinterpret_cast<float*>(sP + kPBufs * kTileBytes + 512);  // [2][128] half-row normalisers
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -132,7 +163,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(kv_empty + s, 1);
     }
     mbar_init(s_full, 1);
-    for (int j = 0; j < kMaxKeyTiles; ++j) mbar_init(p_ready + j, kEpi);
+    for (int j = 0; j < kPBufs; ++j) {
+      mbar_init(p_ready + j, kEpi);
+      mbar_init(p_empty + j, 1);
+    }
     mbar_init(o_full, 1);
     mbar_init(tmem_free, kEpi);
     mbar_init(drain, 1);
@@ -228,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(kBlk, kBlk);
       int stage = 0;
-      uint32_t phase = 0, pmask = 0;
+      uint32_t phase = 0, pready_parity = 0;  // bit j: parity of weight buffer j's next p_ready phase
       bool ok = true;
       int local = 0;
       for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, ++local) {
@@ -268,15 +302,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(q_empty);
         // O = sum_j P_j V_j into columns 0 .. 127, each P_j once its weights are written
         for (int j = 0; j <= i && ok; ++j) {
+          const int pb = j & 1;
           if (!mbar_wait_bounded(kv_full + stage, phase, abort_flag, budget) ||
-              !mbar_wait_bounded(p_ready + j, (pmask >> j) & 1u, abort_flag, budget)) {
+              !mbar_wait_bounded(p_ready + pb, (pready_parity >> pb) & 1u, abort_flag, budget)) {
             ok = false;
             break;
           }
-          pmask ^= 1u << j;
+          pready_parity ^= 1u << pb;
           tc_fence_after();
           const uint8_t* vt = sRing + stage * kTileBytes;
-          const uint8_t* pt = sP + j * kTileBytes;
+          const uint8_t* pt = sP + pb * kTileBytes;
           const uint64_t pdesc0 = smem_desc_k_sw128(smem_u32(pt)), pdesc1 = smem_desc_k_sw128(smem_u32(pt + kAtomBytes));
           const uint64_t vdesc0 = smem_desc_k_sw128(smem_u32(vt)), vdesc1 = smem_desc_k_sw128(smem_u32(vt + kAtomBytes));
 #pragma unroll
@@ -284,6 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_bf16_f32(tmem_base, (k < 4 ? pdesc0 : pdesc1) + 2 * (k & 3), (k < 4 ? vdesc0 : vdesc1) + 2 * (k & 3),
                           idesc, (j | k) != 0 ? 1u : 0u);
           umma_commit(kv_empty + stage);
+          umma_commit(p_empty + pb);
           if (++stage == kRing) {
             stage = 0;
             phase ^= 1u;
@@ -301,70 +337,112 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------- weights and epilogue
+    // Warps 4-11: warp w reads tensor-memory lanes 32 (w % 4) .. (its query rows) and takes
+    // the key columns 64 hf .. 64 hf + 63 of every key tile, hf = (w - 4) / 4, which is
+    // swizzle atom hf of the weight tile; the two threads of a row share its normaliser
+    // through shared memory.
     const int ew = warp - 4;
-    const int row = ew * 32 + lane;  // query row of the unit = tensor-memory lane
-    const uint32_t tl = tmem_base + (static_cast<uint32_t>(ew * 32) << 16);
+    const int quarter = ew & 3, hf = ew >> 2;
+    const int row = quarter * 32 + lane;  // query row of the unit = tensor-memory lane
+    const uint32_t tl = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
     const int64_t units_per_slot = static_cast<int64_t>(p.n_seq) * p.n_heads * p.nqt;
+    const float2 scale2 = make_float2(p.score_scale, p.score_scale);
+    uint32_t pc0 = 0u, pc1 = 0u;  // P V commits to weight buffers 0 and 1 so far (all units)
     int local = 0;
     for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, ++local) {
       int c, b, h, i;
       unit_coords(u, p, c, b, h, i);
       const uint32_t up = static_cast<uint32_t>(local & 1);
+      const int64_t grow = static_cast<int64_t>(b) * p.T + static_cast<int64_t>(i) * kBlk + row;
+      float* orow = p.O_ref + grow * p.D + static_cast<int64_t>(h) * kHd + 64 * hf;
+      if (!p.ref) {  // this thread's half of the reference row, read in the epilogue
+        prefetch_l2(orow);
+        prefetch_l2(orow + 32);
+      }
       bool ok = mbar_wait_bounded(s_full, up, abort_flag, budget);
       if (bar_or(1, kEpi, !ok)) {
         if (!ok) fail();
         break;
       }
       tc_fence_after();
-      // pass 1: the row max over the causal key range (keys <= this query)
-      float m = -INFINITY;
+      // pass 1: the row max over the causal key range (keys <= this query), every column
+      // of the row (four independent chains; max is exact in any order)
+      float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       for (int j = 0; j <= i; ++j) {
 #pragma unroll 1
-        for (int k0 = 0; k0 < kBlk; k0 += 32) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(tl + static_cast<uint32_t>(j * kBlk + k0), v);
-          tmem_ld_wait();
-          const int lim = j < i ? kBlk : row + 1;  // keys k0 + e < lim are in range
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t v[2][32];
+          load_row64(tl + static_cast<uint32_t>(j * kBlk + 64 * h2), v);
+          if (j < i) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (k0 + e < lim) m = fmaxf(m, __uint_as_float(v[e]));
+            for (int q = 0; q < 2; ++q)
+#pragma unroll
+              for (int e = 0; e < 32; e += 4)
+                mq[e / 8 % 4] = fmax3(mq[e / 8 % 4], fmaxf(__uint_as_float(v[q][e]), __uint_as_float(v[q][e + 1])),
+                                      fmaxf(__uint_as_float(v[q][e + 2]), __uint_as_float(v[q][e + 3])));
+          } else {
+            const int lim = row + 1 - 64 * h2;  // diagonal tile: keys <= row
+#pragma unroll
+            for (int q = 0; q < 2; ++q)
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (32 * q + e < lim) mq[e % 4] = fmaxf(mq[e % 4], __uint_as_float(v[q][e]));
+          }
         }
       }
-      // pass 2: e = exp2((s - m) * log2(e) / sqrt(d)), the normaliser, and P = bf16(e)
-      // stored row by row in the 128-byte-swizzled K-major layout (16-byte chunk q of a
-      // row at position q ^ (row % 8) of its 128-byte line)
-      float l = 0.0f;
+      const float m = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+      const float ms = __fmul_rn(m, p.score_scale);
+      const float2 nms2 = make_float2(-ms, -ms);
+      // pass 2: e = 2^(s log2(e) / sqrt(d) - m log2(e) / sqrt(d)) for this thread's half of
+      // each key tile, partial normalisers, and P = bf16(e) into atom hf of the weight tile
+      // (16-byte chunk q of a row at position q ^ (row % 8) of its 128-byte line), P_j in
+      // buffer j % 2 once the P V MMAs of tile j - 2 are done with it
+      float2 lq[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       for (int j = 0; j <= i; ++j) {
-        uint8_t* pt = sP + j * kTileBytes;
-#pragma unroll 1
-        for (int k0 = 0; k0 < kBlk; k0 += 32) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(tl + static_cast<uint32_t>(j * kBlk + k0), v);
-          tmem_ld_wait();
-          const int lim = j < i ? kBlk : row + 1;
+        const int pb = j & 1;
+        uint32_t v[2][32];
+        load_row64(tl + static_cast<uint32_t>(j * kBlk + 64 * hf), v);
+        if (j >= 2) {  // buffer pb free once the P V MMAs of tile j - 2 are done
+          const bool w = mbar_wait_bounded(p_empty + pb, ((pb ? pc1 : pc0) - 1u) & 1u, abort_flag, budget);
+          if (bar_or(1, kEpi, !w)) {
+            if (!w) fail();
+            ok = false;
+            break;
+          }
+        }
+        const int lim = j < i ? kBlk : row + 1 - 64 * hf;  // keys 64 hf + k, k < lim, are in range
+        uint8_t* line = sP + pb * kTileBytes + hf * kAtomBytes + row * 128;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
           uint32_t w[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float e0 = k0 + e < lim ? exp2f(__fmul_rn(__fsub_rn(__uint_as_float(v[e]), m), p.score_scale)) : 0.0f;
-            const float e1 =
-                k0 + e + 1 < lim ? exp2f(__fmul_rn(__fsub_rn(__uint_as_float(v[e + 1]), m), p.score_scale)) : 0.0f;
-            l = __fadd_rn(__fadd_rn(l, e0), e1);
-            w[e / 2] = pack_bf16x2(e0, e1);
+            float2 x = __ffma2_rn(make_float2(__uint_as_float(v[q][e]), __uint_as_float(v[q][e + 1])), scale2, nms2);
+            if (32 * q + e >= lim) x.x = -INFINITY;
+            if (32 * q + e + 1 >= lim) x.y = -INFINITY;
+            const float2 ev = make_float2(ex2(x.x), ex2(x.y));
+            lq[e / 2 % 4] = __fadd2_rn(lq[e / 2 % 4], ev);
+            w[e / 2] = pack_bf16x2(ev.x, ev.y);
           }
-          const int atom = k0 / 64;
-          uint8_t* line = pt + atom * kAtomBytes + row * 128;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int chunk = (k0 % 64) / 8 + q;  // 16-byte chunk of the 128-byte line
+          for (int r = 0; r < 4; ++r) {
+            const int chunk = q * 4 + r;  // 16-byte chunk of the 128-byte line
             *reinterpret_cast<uint4*>(line + ((chunk ^ (row & 7)) << 4)) =
-                make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+                make_uint4(w[4 * r], w[4 * r + 1], w[4 * r + 2], w[4 * r + 3]);
           }
         }
         fence_proxy_async_smem();  // the weights are read by the tensor cores
         tc_fence_before();         // and the score columns of tile j are no longer read
-        mbar_arrive(p_ready + j);
+        mbar_arrive(p_ready + pb);
+        if (pb) ++pc1; else ++pc0;  // P V_j commits to p_empty[pb]
       }
-      // epilogue: O / l, stored (reference) or compared with the reference
+      if (!ok) break;
+      // the row's normaliser: this half's partials in a fixed order, then half 0 + half 1
+      const float lh = ((lq[0].x + lq[0].y) + (lq[1].x + lq[1].y)) + ((lq[2].x + lq[2].y) + (lq[3].x + lq[3].y));
+      xl[hf * 128 + row] = lh;
+      named_barrier_sync(3, kEpi);
+      const float l = __fadd_rn(xl[row], xl[128 + row]);
+      // epilogue: O / l for this thread's 64 columns, stored (reference) or compared
       ok = mbar_wait_bounded(o_full, up, abort_flag, budget);
       if (bar_or(1, kEpi, !ok)) {
         if (!ok) fail();
@@ -372,29 +450,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const float inv_l = __frcp_rn(l);
-      const int64_t grow = static_cast<int64_t>(b) * p.T + static_cast<int64_t>(i) * kBlk + row;
-      float* orow = p.O_ref + grow * p.D + static_cast<int64_t>(h) * kHd;
       float sq = 0.0f;
-#pragma unroll 1
-      for (int k0 = 0; k0 < kHd; k0 += 32) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tl + static_cast<uint32_t>(k0), v);
-        tmem_ld_wait();
-        float4* o4 = reinterpret_cast<float4*>(orow + k0);
-        if (p.ref) {
+      {
+        float4 r[16];
+        if (!p.ref)
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            o4[q] = make_float4(__fmul_rn(__uint_as_float(v[4 * q]), inv_l), __fmul_rn(__uint_as_float(v[4 * q + 1]), inv_l),
-                                __fmul_rn(__uint_as_float(v[4 * q + 2]), inv_l),
-                                __fmul_rn(__uint_as_float(v[4 * q + 3]), inv_l));
-        } else {
+          for (int q = 0; q < 16; ++q) r[q] = __ldg(reinterpret_cast<const float4*>(orow) + q);
+        uint32_t v[2][32];
+        load_row64(tl + static_cast<uint32_t>(64 * hf), v);
+        float4* o4 = reinterpret_cast<float4*>(orow);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 r = __ldg(o4 + q);
-            const float d0 = __fmul_rn(__uint_as_float(v[4 * q]), inv_l) - r.x;
-            const float d1 = __fmul_rn(__uint_as_float(v[4 * q + 1]), inv_l) - r.y;
-            const float d2 = __fmul_rn(__uint_as_float(v[4 * q + 2]), inv_l) - r.z;
-            const float d3 = __fmul_rn(__uint_as_float(v[4 * q + 3]), inv_l) - r.w;
+        for (int q = 0; q < 16; ++q) {
+          const uint32_t* x = &v[q / 8][4 * (q % 8)];
+          const float4 o = make_float4(__fmul_rn(__uint_as_float(x[0]), inv_l), __fmul_rn(__uint_as_float(x[1]), inv_l),
+                                       __fmul_rn(__uint_as_float(x[2]), inv_l), __fmul_rn(__uint_as_float(x[3]), inv_l));
+          if (p.ref) {
+            o4[q] = o;
+          } else {
+            const float d0 = o.x - r[q].x, d1 = o.y - r[q].y, d2 = o.z - r[q].z, d3 = o.w - r[q].w;
             sq = fmaf(d0, d0, sq);
             sq = fmaf(d1, d1, sq);
             sq = fmaf(d2, d2, sq);
@@ -408,11 +481,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         double ds = static_cast<double>(sq);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
-        if (lane == 0) red[up * 4 + ew] = ds;
+        if (lane == 0) red[up * 8 + ew] = ds;
         named_barrier_sync(2, kEpi);
-        if (ew == 0 && lane == 0)
-          p.partial[static_cast<int64_t>(c) * units_per_slot + (static_cast<int64_t>(b) * p.n_heads + h) * p.nqt + i] =
-              ((red[up * 4 + 0] + red[up * 4 + 1]) + red[up * 4 + 2]) + red[up * 4 + 3];
+        if (ew == 0 && lane == 0) {
+          double t = 0.0;
+          for (int k = 0; k < 8; ++k) t += red[up * 8 + k];
+          p.partial[static_cast<int64_t>(c) * units_per_slot + (static_cast<int64_t>(b) * p.n_heads + h) * p.nqt + i] = t;
+        }
       }
     }
     tc_fence_before();
