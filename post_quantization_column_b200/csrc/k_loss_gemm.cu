@@ -56,12 +56,15 @@ constexpr int kEpiThreads = 128;
 constexpr int kBarrierBytes = 256;
 constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;  // + alignment slack
 // Row tiles per raster group (the host picks one per launch): 32 when a group's rows of A
-// take at most 64 MB (K <= 8192), which keeps them and the group's W_hat column blocks in
-// L2 (measured 3.8 % faster than 16 on the 4096^3 layer, 1.4 % on the 70B gate+up layer),
-// else 16 (the MLP block's second GEMM, K = 11008, ran 2 % slower with 32).
+// take at most 32 MB (K <= 4096), which keeps them and the group's W_hat column blocks in
+// L2 (measured 3.8 % faster than 16 on the 4096^3 layer), else 16. On the 70B gate+up layer
+// (K = 8192; one B200, 15 searches each, interleaved) 16 row tiles took 259.2 ms per launch,
+// 32 took 266.3 ms (their 64 MB of rows of X do not stay in L2 while a candidate's column
+// tiles are swept: 440 GB of DRAM reads per launch) and 8 took 267.5 ms; the MLP block's
+// second GEMM (K = 11008) ran 2 % slower with 32.
 constexpr int kGroupMLarge = 32, kGroupMSmall = 16;
 inline int raster_group_m(int64_t K) {
-  return static_cast<int64_t>(kGroupMLarge) * kTileM * K * 2 <= (int64_t(64) << 20) ? kGroupMLarge : kGroupMSmall;
+  return static_cast<int64_t>(kGroupMLarge) * kTileM * K * 2 <= (int64_t(32) << 20) ? kGroupMLarge : kGroupMSmall;
 }
 constexpr uint64_t kDrainNs = 200ull * 1000 * 1000;  // bound on the waits of the abort path
 
