@@ -535,6 +535,7 @@ def search_object(awq, spec: LayerSpec, t: dict, peaks: dict, peak_kind: str, su
     peak = float(peaks[peak_key])
     gemm_kernel = ("loss_gemm_pair_kernel" if awq.loss_gemm_variant(spec.M, spec.K, spec.N, spec.n_grid) == 2
                    else "loss_gemm_kernel")
+    gemm_launches = awq.loss_gemm_launches(spec.M, spec.K, spec.N, spec.n_grid)
     eb = 2 if spec.dtype == "bf16" else 4
     hbm = float(peaks["hbm_gbs"])
     qdq_bytes = (eb + 2 * (spec.n_grid + 1)) * spec.K * spec.N
@@ -549,16 +550,22 @@ def search_object(awq, spec: LayerSpec, t: dict, peaks: dict, peak_kind: str, su
         gbs = nbytes / (ms / 1e3) / 1e9
         return {"kernel": name, "ms": ms, "bytes": nbytes, "GB/s": gbs, "hbm_frac": gbs / hbm, "work": work}
 
+    if gemm_launches == 1:
+        what = " (reference output + candidate GEMMs + fused squared error, one launch)"
+    elif gemm_kernel == "loss_gemm_kernel":
+        what = (" (reference output in its own launch, then the candidate GEMMs + fused squared error, every"
+                " candidate of a column tile before the next; per launch = averaged over the two launches)")
+    else:
+        what = " (candidate GEMMs + fused squared error; reference output in its own launch)"
     roof = {"bound": "tensor",
-            "kernel": gemm_kernel + (" (reference output + candidate GEMMs + fused squared error, one launch)"
-                                     if gemm_kernel == "loss_gemm_kernel" else
-                                     " (candidate GEMMs + fused squared error; reference output in its own launch)"),
+            "kernel": gemm_kernel + what,
+            "launches_per_search": gemm_launches,
             "work": "(n_grid + 1) x 2 M K N flops per search (the reference output and every candidate)",
             "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
             "peak_source": f"{peak_kind} {peak_key} ({'sustained: the kernel runs for a long step' if sustained else 'burst'})",
             "traffic": recorded_traffic(gemm_kernel, spec.name),
             "traffic_unit": "DRAM bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
-            "ms_per_launch": gemm_ms}
+            "ms_per_launch": gemm_ms / gemm_launches}
     return {
         "workload": spec.name, "M": spec.M, "K": spec.K, "N": spec.N, "group": spec.group, "n_grid": spec.n_grid,
         "input_dtype": spec.dtype, "steps": steps, "ms_per_step": total_ms / steps,

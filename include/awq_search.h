@@ -360,6 +360,16 @@ int awq_version(void);
  * the environment. */
 int awq_loss_gemm_variant(int64_t M, int64_t K, int64_t N, int n_grid);
 
+/* How many loss-GEMM launches a search of this size runs on the current device: 1 when
+ * the reference output Y (M x N fp32) fits in the device's L2 cache (one launch computes
+ * the reference tiles and then the candidates, each candidate tile waiting for its
+ * reference tile), 2 otherwise (the reference output in its own launch, then a launch
+ * that scores every candidate of a column tile before the next column tile, so each tile
+ * of Y is read from DRAM once) and always with the two-SM kernel. AWQ_REFERENCE_LAUNCH=own
+ * or =fused in the environment selects a form at every size. Both forms give bit-identical
+ * results. Returns the count, or minus an AWQ_ERR_* status when the device cannot be queried. */
+int awq_loss_gemm_launches(int64_t M, int64_t K, int64_t N, int n_grid);
+
 /* ---- Searching without allocating -------------------------------------------
  * No counterpart in the paper or the pages: this is a deployment variant of
  * awq_search_ex for callers that cannot call cudaMalloc — e.g. a plugin whose host

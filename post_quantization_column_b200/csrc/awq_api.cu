@@ -485,11 +485,23 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
       break;
     }
     ev.mark(kPhGemmY);
-    if (ga.variant == 1) {
+    int l2_bytes = 0;
+    if ((e = cudaDeviceGetAttribute(&l2_bytes, cudaDevAttrL2CacheSize, dev)) != cudaSuccess) {
+      where = "querying the L2 cache size";
+      break;
+    }
+    if (ga.variant == 1 && !reference_in_own_launch(M, N, l2_bytes)) {
       // one launch: the reference tiles first, each candidate tile waits for its tile of Y
       ga.ready = err + 4;
       ev.mark(kPhGemmLoss);
       if ((e = launch_loss_gemm(ga, mapA, mapB, 4, s, &launches)) != cudaSuccess) { where = "loss GEMM"; break; }
+    } else if (ga.variant == 1) {
+      // Y larger than L2: the reference in its own launch, then every candidate of a column
+      // tile while that tile of Y is in L2
+      if ((e = launch_loss_gemm(ga, mapA, mapB, 0, s, &launches)) != cudaSuccess) { where = "reference GEMM"; break; }
+      ev.mark(kPhGemmLoss);
+      ga.cand_inner = 1;
+      if ((e = launch_loss_gemm(ga, mapA, mapB, 1, s, &launches)) != cudaSuccess) { where = "loss GEMM"; break; }
     } else {
       if ((e = launch_loss_gemm(ga, mapA, mapB, 0, s, &launches)) != cudaSuccess) { where = "reference GEMM"; break; }
       ev.mark(kPhGemmLoss);
@@ -1830,5 +1842,14 @@ int awq_debug_set_fault(int mode, int64_t timeout_ns) {
 int awq_version(void) { return kVersion; }
 
 int awq_loss_gemm_variant(int64_t M, int64_t K, int64_t N, int n_grid) { return gemm_variant(M, K, N, n_grid); }
+
+int awq_loss_gemm_launches(int64_t M, int64_t K, int64_t N, int n_grid) {
+  if (gemm_variant(M, K, N, n_grid) == 2) return 2;
+  int dev = 0, l2_bytes = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&l2_bytes, cudaDevAttrL2CacheSize, dev);
+  if (e != cudaSuccess) return -cuda_error(e, "querying the L2 cache size");
+  return reference_in_own_launch(M, N, l2_bytes) ? 2 : 1;
+}
 
 }  // extern "C"

@@ -74,7 +74,15 @@ struct LossGemmArgs {
   int a_slot_base = 0;
   int a_slots = 1;
   int* ready = nullptr;        // mode 4: per-tile flags (tiles_m * tiles_n ints), zero at launch
+  int cand_inner = 0;          // mode 1: walk raster group -> column tile -> candidate -> row tile, so
+                               // that every candidate reads a tile of Y while it is still in L2
 };
+// Whether a search scores its candidates in two launches (mode 0, then mode 1 with
+// cand_inner) rather than one mode-4 launch: when the reference output Y (M x N fp32) is
+// larger than the L2 cache, so that a walk with the candidate outermost would read all of Y
+// from DRAM once per candidate. AWQ_REFERENCE_LAUNCH=own or =fused in the environment
+// selects a form at every size (both give bit-identical results).
+bool reference_in_own_launch(int64_t M, int64_t N, int l2_bytes);
 // Which loss GEMM runs for a search of this size: 1 = the one-SM kernel (every size; it
 // measured as fast or faster than the pair kernel on every workload), 2 = the two-SM
 // (cta_group::2) kernel, selected with AWQ_GEMM_VARIANT=2 in the environment.
@@ -85,7 +93,8 @@ inline int operand_b_box_rows(int variant) { return variant == 2 ? kTileN / 2 : 
 // Builds the TMA descriptors (driver entry point) for the two operands.
 cudaError_t make_operand_maps(const LossGemmArgs& a, CUtensorMap* mapA, CUtensorMap* mapB,
                               const char** why, int b_box_rows);
-// mode 0: Y = X_b W_b into the tiled buffer; mode 1: per-tile sum of (X_b W_hat_i - Y)^2;
+// mode 0: Y = X_b W_b into the tiled buffer; mode 1: per-tile sum of (X_b W_hat_i - Y)^2
+// (candidate outermost, or innermost but one with a.cand_inner);
 // mode 2: Y = X_b Wt[0]^T written row-major fp32 into a.Y (M x N, pitch N), always on
 // the one-SM kernel (make the maps with b_box_rows = kTileN);
 // mode 4: modes 0 and 1 in one launch (reference tiles first, flags in a.ready; one-SM

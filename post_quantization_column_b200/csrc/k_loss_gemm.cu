@@ -6,7 +6,10 @@
 //   mode 0: Y = X_b W_b, written once to HBM in a tile-major layout;
 //   mode 1: for every (candidate i, output tile): acc = X_b W_hat_i,b on the tensor
 //           cores, and the epilogue adds (acc - Y)^2 over the tile and writes one fp64
-//           partial sum. The candidate output Y_hat is never written to HBM;
+//           partial sum. The candidate output Y_hat is never written to HBM. With
+//           cand_inner the walk visits, for each column tile of a raster group, every
+//           candidate before the next column tile, so each tile of Y is read from DRAM once
+//           and by the other candidates from L2 (used when Y is larger than L2);
 //   mode 2: a plain product A B^T (B stored K-major), written row-major in fp32 with
 //           the ragged rows and columns masked (the packed artifact's consumer);
 //   mode 4: modes 0 and 1 in one launch: units 0 .. tiles - 1 are the reference tiles
@@ -40,6 +43,7 @@
 
 #include <cudaTypedefs.h>
 #include <cstdlib>
+#include <cstring>
 #include <cstdio>
 
 namespace awq {
@@ -89,9 +93,23 @@ struct GemmParams {
   int* err;
   uint64_t timeout_ns;
   int fault_mode;
+  int cand_inner;     // mode 1: raster group -> column tile -> candidate -> row tile
 };
 
 __device__ __forceinline__ void unit_coords(int64_t u, const GemmParams& p, int& c, int& mt, int& nt) {
+  if (p.cand_inner) {
+    const int64_t group_units = static_cast<int64_t>(p.group_m) * p.tiles_n * p.cands;  // a full group
+    const int64_t gi = u / group_units;
+    const int first_m = static_cast<int>(gi * p.group_m);
+    const int gm = min(p.group_m, p.tiles_m - first_m);
+    const int64_t r = u - gi * group_units;
+    const int64_t per_column = static_cast<int64_t>(gm) * p.cands;
+    nt = static_cast<int>(r / per_column);
+    const int rc = static_cast<int>(r - nt * per_column);
+    c = rc / gm;
+    mt = first_m + rc % gm;
+    return;
+  }
   const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
   c = static_cast<int>(u / tiles);
   const int64_t t = u - static_cast<int64_t>(c) * tiles;
@@ -783,6 +801,23 @@ int gemm_variant(int64_t M, int64_t K, int64_t N, int n_grid) {
   return (v && v[0] == '2') ? 2 : 1;
 }
 
+// Measured on one B200 (the candidate-GEMM phases, reference launch included, median of 15
+// searches per form, interleaved): on the 70B gate+up layer (Y 3.76 GB) the two launches
+// with the candidate-inner walk took 249.6 ms against 257.8 ms for the one mode-4 launch
+// (its candidates read Y from DRAM once each, 75 GB per search); on the 7B gate+up layer
+// (Y 361 MB) 11.37 against 11.56 ms; on the 4096^3 layer (Y 67 MB, held in L2 by the
+// mode-4 walk) 2.047 against 2.033 ms, so mode 4 stays below the L2 size. The candidate-
+// inner walk inside the one mode-4 launch lost instead: its candidate tiles then wait for
+// reference tiles computed in the same wave, and the static tile-to-CTA assignment lets
+// CTAs drift apart by many tiles over a launch.
+// AWQ_REFERENCE_LAUNCH=own or =fused in the environment selects a form at every size.
+bool reference_in_own_launch(int64_t M, int64_t N, int l2_bytes) {
+  const char* f = getenv("AWQ_REFERENCE_LAUNCH");
+  if (f && !strcmp(f, "own")) return true;
+  if (f && !strcmp(f, "fused")) return false;
+  return M * N * 4 > static_cast<int64_t>(l2_bytes);
+}
+
 cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, const CUtensorMap& mapB, int mode,
                              cudaStream_t s, int* launches) {
   const int tiles_m = static_cast<int>(ceil_div(a.M, BM));
@@ -858,6 +893,7 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
   p.err = a.err;
   p.timeout_ns = a.timeout_ns;
   p.fault_mode = a.fault_mode;
+  p.cand_inner = mode == 1 ? a.cand_inner : 0;
   const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
   const int64_t units = (mode == 1 || mode == 3 || mode == 5 ? p.cands : (mode == 4 ? a.n_grid + 1 : 1)) * tiles;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(units, a.num_sms));

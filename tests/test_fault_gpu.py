@@ -16,11 +16,12 @@ from workloads import custom_spec, generate
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("variant", ["1", "2"])
-def test_wait_that_runs_out_returns_timeout_and_the_context_survives(variant, monkeypatch):
+@pytest.mark.parametrize("variant,form", [("1", "fused"), ("1", "own"), ("2", "own")])
+def test_wait_that_runs_out_returns_timeout_and_the_context_survives(variant, form, monkeypatch):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     monkeypatch.setenv("AWQ_GEMM_VARIANT", variant)
+    monkeypatch.setenv("AWQ_REFERENCE_LAUNCH", form)
     spec = custom_spec(520, 512, 776, seed=31)
     X, W = (t.cuda() for t in generate(spec))
     ref = awq.search(X, W)

@@ -59,6 +59,24 @@ def test_both_gemm_variants(M, K, N, group, dtype, variant, monkeypatch):
     P.full_parity(X, W, group, 20)
 
 
+@pytest.mark.parametrize("M,K,N,group,n_grid,dtype", [(300, 384, 520, 128, 20, "bf16"), (129, 320, 776, 64, 7, "f32"),
+                                                      (520, 256, 264, 32, 20, "bf16"), (64, 160, 136, 32, 64, "bf16")])
+def test_reference_launch_forms(M, K, N, group, n_grid, dtype, monkeypatch):
+    # The one-SM GEMM scores the candidates either in one launch with the reference tiles
+    # (Y within L2) or after a reference launch, walking every candidate of a column tile
+    # before the next (Y larger than L2); the environment forces each form at this size.
+    # Both match the oracle, and each tile's squared error is the same bits in both.
+    spec = custom_spec(M, K, N, dtype=dtype, group=group, n_grid=n_grid, seed=M * 3 + K + N)
+    X, W = generate(spec)
+    outs = {}
+    for form in ("fused", "own"):
+        monkeypatch.setenv("AWQ_REFERENCE_LAUNCH", form)
+        P.full_parity(X, W, group, n_grid)
+        outs[form] = awq.search(X.cuda(), W.cuda(), group, n_grid, tile_sq_err=True)
+    for name in ("scales", "codes", "steps", "zeros", "losses", "best_index", "tile_sq_err"):
+        assert torch.equal(getattr(outs["fused"], name), getattr(outs["own"], name)), name
+
+
 def test_weights_on_the_grid_give_zero_loss():
     # every (group, column) spans all 16 levels with step 1/16 and zero 7: alpha = 0
     # reproduces W exactly (AWQ-P1 §7 reconstruction), so L_0 = 0 and alpha 0 wins
@@ -235,8 +253,8 @@ def test_launch_count_and_profile():
     finally:
         awq.profile_enable(False)
     # statistic + scales + qdq + one GEMM launch for the reference output and the candidates
-    # (two with the two-SM variant) + reduce + pack
-    assert awq.last_launch_count() == (6 if awq.loss_gemm_variant(256, 256, 512, 20) == 1 else 7)
+    # (two when the reference has its own launch) + reduce + pack
+    assert awq.last_launch_count() == 5 + awq.loss_gemm_launches(256, 256, 512, 20)
     assert set(prof) >= {"statistic", "scales", "qdq", "gemm_reference", "gemm_loss", "loss_reduce", "pack"}
     assert all(v >= 0 for v in prof.values()) and prof["gemm_loss"] > 0
 
