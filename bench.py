@@ -535,7 +535,9 @@ def search_object(awq, spec: LayerSpec, t: dict, peaks: dict, peak_kind: str, su
     peak = float(peaks[peak_key])
     gemm_kernel = ("loss_gemm_pair_kernel" if awq.loss_gemm_variant(spec.M, spec.K, spec.N, spec.n_grid) == 2
                    else "loss_gemm_kernel")
-    gemm_launches = awq.loss_gemm_launches(spec.M, spec.K, spec.N, spec.n_grid)
+    tdt = torch.bfloat16 if spec.dtype == "bf16" else torch.float32
+    gemm_launches = awq.loss_gemm_launches(spec.M, spec.K, spec.N, spec.n_grid, spec.group, tdt)
+    qdq_warps = awq.qdq_in_loss_gemm(spec.M, spec.K, spec.N, spec.n_grid, spec.group, tdt)
     eb = 2 if spec.dtype == "bf16" else 4
     hbm = float(peaks["hbm_gbs"])
     qdq_bytes = (eb + 2 * (spec.n_grid + 1)) * spec.K * spec.N
@@ -557,6 +559,8 @@ def search_object(awq, spec: LayerSpec, t: dict, peaks: dict, peak_kind: str, su
                 " candidate of a column tile before the next; per launch = averaged over the two launches)")
     else:
         what = " (candidate GEMMs + fused squared error; reference output in its own launch)"
+    if qdq_warps:
+        what += "; its QDQ warps make the candidate operands (QDQ) inside the same launches"
     roof = {"bound": "tensor",
             "kernel": gemm_kernel + what,
             "launches_per_search": gemm_launches,
@@ -574,8 +578,10 @@ def search_object(awq, spec: LayerSpec, t: dict, peaks: dict, peak_kind: str, su
         "TFLOP/s": spec.candidate_flops * steps / (total_ms / 1e3) / 1e12,
         "roofline": roof,
         "other_kernels": {
-            "qdq": hbm_obj("qdq_kernel", qdq_bytes, mean("qdq"),
-                           "reads W once, writes n_grid + 1 bf16 operand slots"),
+            "qdq": (hbm_obj("qdq_kernel (the reference operand alone)", (eb + 2) * spec.K * spec.N, mean("qdq"),
+                            "reads W once, writes the bf16 reference operand; the n_grid candidate operands "
+                            "are made by the loss GEMM's QDQ warps inside its two launches") if qdq_warps else
+                    hbm_obj("qdq_kernel", qdq_bytes, mean("qdq"), "reads W once, writes n_grid + 1 bf16 operand slots")),
             "statistic": hbm_obj("statistic_kernel", stat_bytes, mean("statistic"), "reads X once, writes a"),
             "pack": hbm_obj("pack_kernel", pack_bytes, mean("pack"),
                             "reads W once, writes the codes, steps, zeros and scales"),

@@ -212,8 +212,10 @@ int awq_last_launch_count(void);
 
 /* Testing hook for the bounded waits: mode 1 makes the loss GEMM's producer skip
  * one stage's loads and arrive, so its consumer's wait runs out and the call
- * returns AWQ_ERR_TIMEOUT; `timeout_ns` bounds every wait (0 = the default 2 s).
- * Mode 0 restores normal operation. */
+ * returns AWQ_ERR_TIMEOUT; mode 3 makes the loss GEMM's QDQ warps (bf16 W, group
+ * 128) withhold one finished tile's count, so the producer's wait for that column
+ * tile runs out, with the same result; `timeout_ns` bounds every wait (0 = the
+ * default 2 s). Mode 0 restores normal operation. */
 int awq_debug_set_fault(int mode, int64_t timeout_ns);
 
 /* ---- Clipping search after the scaling ----------------------------------------
@@ -360,15 +362,25 @@ int awq_version(void);
  * the environment. */
 int awq_loss_gemm_variant(int64_t M, int64_t K, int64_t N, int n_grid);
 
-/* How many loss-GEMM launches a search of this size runs on the current device: 1 when
- * the reference output Y (M x N fp32) fits in the device's L2 cache (one launch computes
- * the reference tiles and then the candidates, each candidate tile waiting for its
- * reference tile), 2 otherwise (the reference output in its own launch, then a launch
- * that scores every candidate of a column tile before the next column tile, so each tile
- * of Y is read from DRAM once) and always with the two-SM kernel. AWQ_REFERENCE_LAUNCH=own
- * or =fused in the environment selects a form at every size. Both forms give bit-identical
- * results. Returns the count, or minus an AWQ_ERR_* status when the device cannot be queried. */
-int awq_loss_gemm_launches(int64_t M, int64_t K, int64_t N, int n_grid);
+/* Whether a search of this form makes its candidate operands with the loss GEMM's own
+ * QDQ warps (1) or with a QDQ kernel launched before it (0): 1 for bf16 inputs with
+ * group 128 on the one-SM GEMM kernel, unless AWQ_QDQ=standalone is set in the
+ * environment. Eight more warps per GEMM CTA then quantize W while the tensor cores
+ * run; a load of a column tile of a candidate operand waits (bounded) for that tile.
+ * Both forms give bit-identical results. */
+int awq_qdq_in_loss_gemm(int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid);
+
+/* How many loss-GEMM launches a search of this form runs on the current device: 2 when
+ * the QDQ warps make the operands (the reference output's launch makes the reference
+ * operand and the first candidate tiles), when the reference output Y (M x N fp32) is
+ * larger than the device's L2 cache, or with the two-SM kernel: the reference output in
+ * its own launch, then a launch that scores every candidate of a column tile before the
+ * next column tile, so each tile of Y is read from DRAM once; 1 otherwise (one launch
+ * computes the reference tiles and then the candidates, each candidate tile waiting for
+ * its reference tile). Without the QDQ warps, AWQ_REFERENCE_LAUNCH=own or =fused in the
+ * environment selects a form at every size. All forms give bit-identical results.
+ * Returns the count, or minus an AWQ_ERR_* status when the device cannot be queried. */
+int awq_loss_gemm_launches(int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid);
 
 /* ---- Searching without allocating -------------------------------------------
  * No counterpart in the paper or the pages: this is a deployment variant of

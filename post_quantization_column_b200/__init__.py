@@ -23,7 +23,7 @@ __all__ = [
     "tile_shape", "workspace_bytes", "release_cached", "profile_enable", "profile_last",
     "last_launch_count", "debug_set_fault", "status_string", "exported_functions",
     "activation_statistic", "candidate_scales", "qdq_candidates", "ClipOutput", "clip_search",
-    "clip_token_count", "clip_profile_last", "fp64_mma_peak", "w4a16_matmul", "w4a16_dequant", "w4a16_profile_last", "search_mlp", "QUANTIZERS", "w4a16_repack", "w4a16_matmul_packed", "loss_gemm_variant", "loss_gemm_launches",
+    "clip_token_count", "clip_profile_last", "fp64_mma_peak", "w4a16_matmul", "w4a16_dequant", "w4a16_profile_last", "search_mlp", "QUANTIZERS", "w4a16_repack", "w4a16_matmul_packed", "loss_gemm_variant", "loss_gemm_launches", "qdq_in_loss_gemm",
     "search_attn", "attn_profile_last", "ATTN_HEAD_DIM",
 ]
 
@@ -117,8 +117,10 @@ def library() -> ctypes.CDLL:
     lib.awq_w4a16_profile_last.restype = ctypes.c_float
     lib.awq_loss_gemm_variant.argtypes = [i64, i64, i64, i32]
     lib.awq_loss_gemm_variant.restype = ctypes.c_int
-    lib.awq_loss_gemm_launches.argtypes = [i64, i64, i64, i32]
+    lib.awq_loss_gemm_launches.argtypes = [i32, i64, i64, i64, i32, i32]
     lib.awq_loss_gemm_launches.restype = ctypes.c_int
+    lib.awq_qdq_in_loss_gemm.argtypes = [i32, i64, i64, i64, i32, i32]
+    lib.awq_qdq_in_loss_gemm.restype = ctypes.c_int
     lib.awq_clip_token_count.argtypes = [i64, i64]
     lib.awq_clip_token_count.restype = ctypes.c_int64
     for name in ("awq_activation_statistic", "awq_candidate_scales", "awq_qdq_candidates", "awq_clip_search",
@@ -640,11 +642,18 @@ def loss_gemm_variant(M: int, K: int, N: int, n_grid: int = 20) -> int:
     return int(library().awq_loss_gemm_variant(M, K, N, n_grid))
 
 
-def loss_gemm_launches(M: int, K: int, N: int, n_grid: int = 20) -> int:
-    """How many loss-GEMM launches a search of this size runs on the current device: 1
-    (reference and candidates in one launch, Y within L2) or 2 (the reference output in
-    its own launch)."""
-    n = int(library().awq_loss_gemm_launches(M, K, N, n_grid))
+def loss_gemm_launches(M: int, K: int, N: int, n_grid: int = 20, group: int = 128,
+                       dtype: torch.dtype = torch.bfloat16) -> int:
+    """How many loss-GEMM launches a search of this form runs on the current device: 1
+    (reference and candidates in one launch) or 2 (the reference output in its own launch)."""
+    n = int(library().awq_loss_gemm_launches(_dtype_code(torch.empty(0, dtype=dtype)), M, K, N, group, n_grid))
     if n < 0:
         _check(-n)
     return n
+
+
+def qdq_in_loss_gemm(M: int, K: int, N: int, n_grid: int = 20, group: int = 128,
+                     dtype: torch.dtype = torch.bfloat16) -> bool:
+    """Whether a search of this form makes its candidate operands with the loss GEMM's own
+    QDQ warps (else a QDQ kernel runs before the GEMM)."""
+    return bool(library().awq_qdq_in_loss_gemm(_dtype_code(torch.empty(0, dtype=dtype)), M, K, N, group, n_grid))

@@ -77,7 +77,8 @@ int get_pool(int dev, cudaMemPool_t* out) {
 
 struct Layout {
   size_t err, a, S, best, losses, Xb, Wt, Y, loss_partial, total;
-  int64_t tiles;
+  int64_t tiles, tiles_n;
+  size_t flag_bytes;  // the status word, the per-tile flags and the QDQ counters, zeroed per call
 };
 
 Layout plan(int in_dtype, int64_t M, int64_t K, int64_t N, int n_grid) {
@@ -90,7 +91,11 @@ Layout plan(int in_dtype, int64_t M, int64_t K, int64_t N, int n_grid) {
   };
   const int64_t tiles_m = ceil_div(M, kTileM), tiles_n = ceil_div(N, kTileN);
   L.tiles = tiles_m * tiles_n;
-  L.err = take(16 + static_cast<size_t>(L.tiles) * 4);  // status word, then the loss GEMM's per-tile flags
+  L.tiles_n = tiles_n;
+  // status word, then the loss GEMM's per-tile flags, then its QDQ warps' counters and
+  // their claim counter
+  L.flag_bytes = 16 + static_cast<size_t>(L.tiles + tiles_n + 1) * 4;
+  L.err = take(L.flag_bytes);
   L.a = take(static_cast<size_t>(K) * 4);
   L.S = take(static_cast<size_t>(n_grid) * K * 4);
   L.best = take(16);
@@ -425,8 +430,8 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
   const char* where = "";
   int status = AWQ_OK;
   do {
-    // the status word and the loss GEMM's per-tile flags
-    if ((e = cudaMemsetAsync(err, 0, 16 + static_cast<size_t>(L.tiles) * 4, s)) != cudaSuccess) {
+    // the status word, the loss GEMM's per-tile flags and its QDQ counters
+    if ((e = cudaMemsetAsync(err, 0, L.flag_bytes, s)) != cudaSuccess) {
       where = "cudaMemsetAsync";
       break;
     }
@@ -446,8 +451,14 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
         break;
       }
     }
+    const int variant = gemm_variant(M, K, N, n_grid);
+    // bf16 W, group 128: the candidate operands are made inside the loss GEMM's launches
+    const bool qdq_in_gemm = !feed && qdq_in_loss_gemm(in_dtype, group, variant);
     ev.mark(kPhQdq);
-    if (feed) {
+    if (qdq_in_gemm) {
+      // the reference operand only: the loss GEMM's QDQ warps make the candidates'
+      e = launch_qdq(W, in_dtype, K, N, group, 0, S, Wt, err, s, &launches, quantizer);
+    } else if (feed) {
       // quantize each chunk of row groups as soon as it has arrived
       const int64_t groups = K / group;
       for (int c = 0; c < feed->chunks && e == cudaSuccess; ++c) {
@@ -477,7 +488,13 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
     ga.timeout_ns = g_timeout_ns;
     ga.fault_mode = g_fault_mode;
     ga.num_sms = num_sms;
-    ga.variant = gemm_variant(M, K, N, n_grid);
+    ga.variant = variant;
+    if (qdq_in_gemm) {
+      ga.qdq_W = static_cast<const __nv_bfloat16*>(W);
+      ga.qdq_S = S;
+      ga.qdq_ready = err + 4 + L.tiles;
+      ga.qdq_quantizer = quantizer;
+    }
     CUtensorMap mapA, mapB;
     const char* why = "";
     if ((e = make_operand_maps(ga, &mapA, &mapB, &why, operand_b_box_rows(ga.variant))) != cudaSuccess) {
@@ -490,17 +507,21 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
       where = "querying the L2 cache size";
       break;
     }
-    if (ga.variant == 1 && !reference_in_own_launch(M, N, l2_bytes)) {
+    if (ga.variant == 1 && !qdq_in_gemm && !reference_in_own_launch(M, N, l2_bytes)) {
       // one launch: the reference tiles first, each candidate tile waits for its tile of Y
       ga.ready = err + 4;
       ev.mark(kPhGemmLoss);
       if ((e = launch_loss_gemm(ga, mapA, mapB, 4, s, &launches)) != cudaSuccess) { where = "loss GEMM"; break; }
     } else if (ga.variant == 1) {
-      // Y larger than L2: the reference in its own launch, then every candidate of a column
-      // tile while that tile of Y is in L2
+      // the reference in its own launch (its QDQ warps make candidate tiles while its GEMM
+      // runs), then every candidate of a column tile while that tile of Y is in L2 (the
+      // QDQ warps make the remaining candidate tiles, column tiles in the order the GEMM
+      // reads them)
+      ga.qdq_cands = 2;
       if ((e = launch_loss_gemm(ga, mapA, mapB, 0, s, &launches)) != cudaSuccess) { where = "reference GEMM"; break; }
       ev.mark(kPhGemmLoss);
       ga.cand_inner = 1;
+      ga.qdq_cands = 1;
       if ((e = launch_loss_gemm(ga, mapA, mapB, 1, s, &launches)) != cudaSuccess) { where = "loss GEMM"; break; }
     } else {
       if ((e = launch_loss_gemm(ga, mapA, mapB, 0, s, &launches)) != cudaSuccess) { where = "reference GEMM"; break; }
@@ -1833,7 +1854,7 @@ const char* awq_profile_phase_name(int phase) {
 int awq_last_launch_count(void) { return g_last_launches; }
 
 int awq_debug_set_fault(int mode, int64_t timeout_ns) {
-  if (mode != 0 && mode != 1) return set_error(AWQ_ERR_INVALID_ARG, "fault mode must be 0 or 1");
+  if (mode != 0 && mode != 1 && mode != 3) return set_error(AWQ_ERR_INVALID_ARG, "fault mode must be 0, 1 or 3");
   g_fault_mode = mode;
   g_timeout_ns = timeout_ns > 0 ? static_cast<uint64_t>(timeout_ns) : kDefaultTimeoutNs;
   return AWQ_OK;
@@ -1843,13 +1864,18 @@ int awq_version(void) { return kVersion; }
 
 int awq_loss_gemm_variant(int64_t M, int64_t K, int64_t N, int n_grid) { return gemm_variant(M, K, N, n_grid); }
 
-int awq_loss_gemm_launches(int64_t M, int64_t K, int64_t N, int n_grid) {
-  if (gemm_variant(M, K, N, n_grid) == 2) return 2;
+int awq_loss_gemm_launches(int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid) {
+  const int variant = gemm_variant(M, K, N, n_grid);
+  if (variant == 2 || qdq_in_loss_gemm(in_dtype, group, variant)) return 2;
   int dev = 0, l2_bytes = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&l2_bytes, cudaDevAttrL2CacheSize, dev);
   if (e != cudaSuccess) return -cuda_error(e, "querying the L2 cache size");
   return reference_in_own_launch(M, N, l2_bytes) ? 2 : 1;
+}
+
+int awq_qdq_in_loss_gemm(int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid) {
+  return qdq_in_loss_gemm(in_dtype, group, gemm_variant(M, K, N, n_grid)) ? 1 : 0;
 }
 
 }  // extern "C"

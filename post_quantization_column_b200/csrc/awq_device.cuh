@@ -182,6 +182,32 @@ __device__ __forceinline__ bool flag_wait_bounded(const int* flag, volatile int*
   }
 }
 
+// A counter other CTAs of the same grid raise (red.release.gpu after the data each
+// increment guards); waits until it reaches `target`, with the same bounds.
+__device__ __forceinline__ void red_release_add_gpu(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ bool counter_wait_bounded(const int* counter, int target, volatile int* abort,
+                                                     uint64_t budget_ns) {
+  if (ld_acquire_gpu(counter) >= target) return true;
+  const uint64_t t0 = global_timer_ns();
+  uint32_t spins = 0;
+  while (true) {
+    __nanosleep(128);
+    if (ld_acquire_gpu(counter) >= target) return true;
+    if (++spins % 16u == 0u) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > budget_ns) return false;
+    }
+  }
+}
+// Orders this thread's generic-proxy view of global memory with its later async-proxy
+// (TMA) accesses: data another CTA stored with st.global and published through a
+// counter, read here by cp.async.bulk.tensor after the counter's acquire.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------------
 // TMA (no multicast anywhere in this library)
 // ---------------------------------------------------------------------------------

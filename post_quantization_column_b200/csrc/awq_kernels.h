@@ -76,6 +76,19 @@ struct LossGemmArgs {
   int* ready = nullptr;        // mode 4: per-tile flags (tiles_m * tiles_n ints), zero at launch
   int cand_inner = 0;          // mode 1: walk raster group -> column tile -> candidate -> row tile, so
                                // that every candidate reads a tile of Y while it is still in L2
+  // Modes 0 and 1 on the one-SM kernel with bf16 W and group 128: when qdq_W is set,
+  // eight more warps per CTA make the candidate operand slots (the QDQ of the candidate
+  // loop, slots 1 .. n_grid; slot 0 comes from launch_qdq with n_grid = 0) while the
+  // tensor cores run, claiming 128 x 32 tiles of W from a counter that spans the search's
+  // launches (qdq_cands 2: while this CTA's GEMM runs, the reference launch; 1: until
+  // none is left, the candidate launch); every mode-1 load of a column tile of B waits
+  // (bounded) until that tile is complete. qdq_ready: tiles_n + 1 ints, zero before the
+  // first of the launches.
+  const __nv_bfloat16* qdq_W = nullptr;  // [K][N]
+  const float* qdq_S = nullptr;          // [n_grid][K]
+  int* qdq_ready = nullptr;
+  int qdq_cands = 0;
+  int qdq_quantizer = 0;
 };
 // Whether a search scores its candidates in two launches (mode 0, then mode 1 with
 // cand_inner) rather than one mode-4 launch: when the reference output Y (M x N fp32) is
@@ -83,6 +96,10 @@ struct LossGemmArgs {
 // from DRAM once per candidate. AWQ_REFERENCE_LAUNCH=own or =fused in the environment
 // selects a form at every size (both give bit-identical results).
 bool reference_in_own_launch(int64_t M, int64_t N, int l2_bytes);
+// Whether a search makes its candidate operands with the loss GEMM's QDQ warps (bf16 W,
+// group 128, the one-SM kernel) rather than with qdq_kernel before it. AWQ_QDQ=standalone
+// in the environment selects qdq_kernel at every size (both give bit-identical operands).
+bool qdq_in_loss_gemm(int in_dtype, int group, int variant);
 // Which loss GEMM runs for a search of this size: 1 = the one-SM kernel (every size; it
 // measured as fast or faster than the pair kernel on every workload), 2 = the two-SM
 // (cta_group::2) kernel, selected with AWQ_GEMM_VARIANT=2 in the environment.

@@ -40,6 +40,7 @@
 // flight, the MMA thread waits for its issued MMAs, and tensor memory is freed.
 #include "awq_device.cuh"
 #include "awq_kernels.h"
+#include "qdq_tile.cuh"
 
 #include <cudaTypedefs.h>
 #include <cstdlib>
@@ -94,6 +95,43 @@ struct GemmParams {
   uint64_t timeout_ns;
   int fault_mode;
   int cand_inner;     // mode 1: raster group -> column tile -> candidate -> row tile
+  // QDQ warps (loss_gemm_kernel<true>, modes 0 and 1): the candidate operand slots are
+  // made by warps 8 .. 15 of the same CTAs while the tensor cores run. qdq_ready[nt]
+  // counts the finished 128 x 32 tiles of W (all candidates) of 256-column tile nt; a
+  // mode-1 B load waits for its column tile's count. qdq_ready[tiles_n] is the claim
+  // counter of the tiles, which spans the search's two launches.
+  const __nv_bfloat16* qdq_W;  // [K][N] bf16
+  const float* qdq_S;          // [n_grid][K] candidate scales
+  __nv_bfloat16* qdq_Wt;       // [n_grid + 1][N][K]
+  int* qdq_ready;
+  int qdq_cands;               // claim tiles: 1 until none is left, 2 while this CTA's GEMM runs
+  int qdq_quantizer;
+  int64_t K;
+};
+
+// QDQ warps: group 128, tiles of 128 rows x 32 columns (8 warps of 16 row-lanes x 2
+// column-lanes, each lane 8 rows of 2 columns), up to kQdqChunk candidates staged per
+// pass over a tile.
+using QdqTile = Tile<128, 32>;
+constexpr int kQdqTileCols = QdqTile::kCols;
+constexpr int kQdqThreads = QdqTile::kThreads;  // 256
+constexpr int kQdqChunk = 10;
+constexpr int kQdqSmemBytes = kQdqTileCols * QdqTile::kPitch * 4 + 2 * kQdqChunk * QdqTile::kSkewPitch * 4 +
+                              kQdqChunk * kQdqTileCols * 16 + 16;
+static_assert(kQdqThreads == 256, "QDQ warps 8 .. 15");
+static_assert((kQdqTileCols * QdqTile::kPitch * 4) % 16 == 0 && (QdqTile::kSkewPitch * 4 * 2) % 16 == 0,
+              "16-byte aligned parameter sets");
+constexpr int kQdqColsPerTileN = kTileN / kQdqTileCols;  // 8 QDQ column blocks per GEMM column tile
+
+// Finished QDQ tiles a 256-column tile needs: its 32-column blocks (the last tile may be
+// ragged) times the groups of K.
+__device__ __forceinline__ int qdq_target(const GemmParams& p, int nt) {
+  const int64_t cols = min(static_cast<int64_t>(kTileN), p.N - static_cast<int64_t>(nt) * kTileN);
+  return static_cast<int>(ceil_div(cols, static_cast<int64_t>(kQdqTileCols)) * (p.K / 128));
+}
+
+struct QdqWarpsSync {
+  __device__ __forceinline__ void operator()() const { asm volatile("bar.sync 5, 256;" ::: "memory"); }
 };
 
 __device__ __forceinline__ void unit_coords(int64_t u, const GemmParams& p, int& c, int& mt, int& nt) {
@@ -135,7 +173,8 @@ __device__ __forceinline__ int named_barrier_or(uint32_t id, uint32_t nthreads, 
   return static_cast<int>(r);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+template <bool kQdq>
+__global__ void __launch_bounds__(kQdq ? kThreads + kQdqThreads : kThreads, 1)
     loss_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                      const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -151,6 +190,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   double* red = reinterpret_cast<double*>(bars + 2 * kStages + 5);  // [2][4]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 13);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* gemm_done = reinterpret_cast<volatile int*>(bars + 2 * kStages + 14);  // the epilogue's last unit is done
+  volatile int* qdq_claim = gemm_done + 1;  // the QDQ warps' current candidate tile
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
@@ -165,6 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
+    *gemm_done = 0;
     fence_mbarrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -198,9 +240,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t issued = 0, last_parity = 0;  // per-stage bits
       bool ok = true;
       bool fault_pending = p.fault_mode == 1;
+      int confirmed = -1;  // the last column tile whose candidate operands were seen complete
+      (void)confirmed;
       for (int64_t u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         int c, mt, nt;
         unit_coords(u, p, c, mt, nt);
+        if constexpr (kQdq) {
+          // a candidate operand: its column tile must be complete
+          if (p.mode == 1 && confirmed != nt) {
+            if (!counter_wait_bounded(p.qdq_ready + nt, qdq_target(p, nt), abort_flag, budget)) {
+              ok = false;
+              break;
+            }
+            fence_proxy_async_global();
+            confirmed = nt;
+          }
+        }
         const int slot = p.mode == 0 ? 0
                          : p.mode == 4 ? c  // 0: bf16(W), then candidate c - 1 in slot c
                                        : p.slot_base +
@@ -281,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------- epilogue
     const int ew = warp - 4;  // == warp % 4: TMEM lanes 32*ew .. 32*ew+31
     const int row = ew * 32 + lane;
@@ -431,7 +486,50 @@ __global__ void __launch_bounds__(kThreads, 1)
               ((red[acc * 4 + 0] + red[acc * 4 + 1]) + red[acc * 4 + 2]) + red[acc * 4 + 3];
       }
     }
+    if (kQdq && ew == 0 && lane == 0) *gemm_done = 1;
     tc_fence_before();
+  } else if constexpr (kQdq) {
+    if (warp >= 8) {
+      // --------------------------------------------------------------- QDQ warps
+      // The 128 x 32 tiles of W, claimed one at a time in column-major order (the column
+      // tiles the GEMM reads first are finished first) from a counter that spans the
+      // search's launches: the reference launch claims tiles while its own GEMM runs,
+      // the candidate launch until none is left. Each tile's stores, for every candidate,
+      // are published by its column tile's count.
+      const int tid = static_cast<int>(threadIdx.x) - kThreads;
+      uint8_t* qs = smem + kSmemBytes - 1024;  // past the ring, the barriers and their slack
+      float* sWT = reinterpret_cast<float*>(qs);
+      float* sS = sWT + kQdqTileCols * QdqTile::kPitch;
+      float* sR = sS + kQdqChunk * QdqTile::kSkewPitch;
+      float4* sPar = reinterpret_cast<float4*>(sR + kQdqChunk * QdqTile::kSkewPitch);
+      uint32_t* sRowsExact = reinterpret_cast<uint32_t*>(sPar + kQdqChunk * kQdqTileCols);
+      const int64_t groups = p.K / 128;
+      const int64_t qtiles = ceil_div(p.N, static_cast<int64_t>(kQdqTileCols)) * groups;
+      int* const next = p.qdq_ready + p.tiles_n;
+      bool skip_publish = p.fault_mode == 3 && blockIdx.x == 0;  // fault injection: one count never arrives
+      while (p.qdq_cands) {
+        if (tid == 0) *qdq_claim = (p.qdq_cands == 2 && *gemm_done) ? -1 : atomicAdd(next, 1);
+        QdqWarpsSync{}();
+        const int64_t t = *qdq_claim;
+        if (t < 0 || t >= qtiles) break;
+        const int64_t cb = t / groups, k0 = (t - cb * groups) * 128;
+        for (int c0 = 0; c0 < p.n_grid; c0 += kQdqChunk)
+          qdq_tile<__nv_bfloat16, 128, QdqTile>(p.qdq_W, p.K, p.N, p.N, k0, cb * kQdqTileCols, p.qdq_S, c0,
+                                                min(c0 + kQdqChunk, p.n_grid), c0 == 0, false, p.qdq_Wt, p.err,
+                                                p.qdq_quantizer, 0, sWT, sS, sR, sPar, sRowsExact, tid,
+                                                QdqWarpsSync{});
+        // publish: every thread's stores, then the column tile's count
+        fence_proxy_async_global();
+        __threadfence();
+        QdqWarpsSync{}();
+        if (tid == 0) {
+          if (skip_publish)
+            skip_publish = false;
+          else
+            red_release_add_gpu(p.qdq_ready + cb / kQdqColsPerTileN, 1);
+        }
+      }
+    }
   }
 
   __syncthreads();
@@ -818,6 +916,12 @@ bool reference_in_own_launch(int64_t M, int64_t N, int l2_bytes) {
   return M * N * 4 > static_cast<int64_t>(l2_bytes);
 }
 
+bool qdq_in_loss_gemm(int in_dtype, int group, int variant) {
+  const char* f = getenv("AWQ_QDQ");
+  if (f && !strcmp(f, "standalone")) return false;
+  return in_dtype == 0 /* bf16 */ && group == 128 && variant == 1;
+}
+
 cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, const CUtensorMap& mapB, int mode,
                              cudaStream_t s, int* launches) {
   const int tiles_m = static_cast<int>(ceil_div(a.M, BM));
@@ -866,8 +970,13 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
     *launches += 1;
     return e != cudaSuccess ? e : cudaGetLastError();
   }
-  static unsigned long long attr_done = 0;
-  cudaError_t e = set_smem_limit_once(loss_gemm_kernel, kSmemBytes, &attr_done);
+  const bool qdq = a.qdq_W != nullptr;
+  if (qdq && ((mode != 0 && mode != 1) || !a.qdq_ready || !a.qdq_S || a.slot_base != 1 || a.a_slotted ||
+              !a.b_per_cand || a.K % 128 || ceil_div(a.N, static_cast<int64_t>(kQdqTileCols)) * (a.K / 128) >= (int64_t(1) << 30)))
+    return cudaErrorInvalidValue;
+  static unsigned long long attr_done = 0, attr_done_qdq = 0;
+  cudaError_t e = qdq ? set_smem_limit_once(loss_gemm_kernel<true>, kSmemBytes + kQdqSmemBytes, &attr_done_qdq)
+                      : set_smem_limit_once(loss_gemm_kernel<false>, kSmemBytes, &attr_done);
   if (e != cudaSuccess) return e;
   GemmParams p;
   p.mode = mode;
@@ -894,10 +1003,20 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
   p.timeout_ns = a.timeout_ns;
   p.fault_mode = a.fault_mode;
   p.cand_inner = mode == 1 ? a.cand_inner : 0;
+  p.qdq_W = a.qdq_W;
+  p.qdq_S = a.qdq_S;
+  p.qdq_Wt = const_cast<__nv_bfloat16*>(a.Wt);
+  p.qdq_ready = a.qdq_ready;
+  p.qdq_cands = a.qdq_cands;
+  p.qdq_quantizer = a.qdq_quantizer;
+  p.K = a.K;
   const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
   const int64_t units = (mode == 1 || mode == 3 || mode == 5 ? p.cands : (mode == 4 ? a.n_grid + 1 : 1)) * tiles;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(units, a.num_sms));
-  loss_gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(mapA, mapB, p);
+  if (qdq)
+    loss_gemm_kernel<true><<<grid, kThreads + kQdqThreads, kSmemBytes + kQdqSmemBytes, s>>>(mapA, mapB, p);
+  else
+    loss_gemm_kernel<false><<<grid, kThreads, kSmemBytes, s>>>(mapA, mapB, p);
   *launches += 1;
   return cudaGetLastError();
 }

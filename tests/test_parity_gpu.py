@@ -68,6 +68,7 @@ def test_reference_launch_forms(M, K, N, group, n_grid, dtype, monkeypatch):
     # Both match the oracle, and each tile's squared error is the same bits in both.
     spec = custom_spec(M, K, N, dtype=dtype, group=group, n_grid=n_grid, seed=M * 3 + K + N)
     X, W = generate(spec)
+    monkeypatch.setenv("AWQ_QDQ", "standalone")
     outs = {}
     for form in ("fused", "own"):
         monkeypatch.setenv("AWQ_REFERENCE_LAUNCH", form)
@@ -75,6 +76,32 @@ def test_reference_launch_forms(M, K, N, group, n_grid, dtype, monkeypatch):
         outs[form] = awq.search(X.cuda(), W.cuda(), group, n_grid, tile_sq_err=True)
     for name in ("scales", "codes", "steps", "zeros", "losses", "best_index", "tile_sq_err"):
         assert torch.equal(getattr(outs["fused"], name), getattr(outs["own"], name)), name
+
+
+@pytest.mark.parametrize("M,K,N,n_grid,quantizer", [(300, 384, 520, 20, "asym"), (129, 256, 776, 64, "asym"),
+                                                     (520, 512, 264, 11, "sym"), (1, 128, 8, 20, "asym"),
+                                                     (1000, 1024, 2056, 20, "asym")])
+def test_qdq_warps_match_the_qdq_kernel(M, K, N, n_grid, quantizer, monkeypatch):
+    # bf16 W with group 128: the candidate operands are made by the loss GEMM's own QDQ
+    # warps while its tensor cores run (the reference launch makes the reference operand
+    # and claims candidate tiles while its GEMM runs, the candidate launch the rest);
+    # AWQ_QDQ=standalone makes them with qdq_kernel first. Both match the oracle and give
+    # the same bits everywhere, tile errors included.
+    assert awq.qdq_in_loss_gemm(M, K, N, n_grid) == (awq.loss_gemm_variant(M, K, N, n_grid) == 1)
+    spec = custom_spec(M, K, N, group=128, n_grid=n_grid, seed=M + 5 * K + N)
+    X, W = generate(spec)
+    outs = {}
+    for qdq in ("standalone", "warps"):
+        if qdq == "standalone":
+            monkeypatch.setenv("AWQ_QDQ", "standalone")
+        else:
+            monkeypatch.delenv("AWQ_QDQ", raising=False)
+        if quantizer == "asym":
+            P.full_parity(X, W, 128, n_grid)
+        outs[qdq] = awq.search(X.cuda(), W.cuda(), 128, n_grid, tile_sq_err=quantizer == "asym", quantizer=quantizer)
+    for name in ("scales", "codes", "steps", "zeros", "losses", "best_index") + (("tile_sq_err",) if quantizer == "asym"
+                                                                               else ()):
+        assert torch.equal(getattr(outs["standalone"], name), getattr(outs["warps"], name)), name
 
 
 def test_weights_on_the_grid_give_zero_loss():
@@ -243,8 +270,13 @@ def test_host_pointer_is_rejected_by_the_device_entry_point():
     assert st == 1
 
 
-def test_launch_count_and_profile():
-    spec = custom_spec(256, 256, 512, seed=2)
+@pytest.mark.parametrize("qdq", ["warps", "standalone"])
+def test_launch_count_and_profile(qdq, monkeypatch):
+    if qdq == "standalone":
+        monkeypatch.setenv("AWQ_QDQ", "standalone")
+    else:
+        monkeypatch.delenv("AWQ_QDQ", raising=False)
+    spec = custom_spec(256, 256, 512, seed=2)   # bf16, group 128
     X, W = generate(spec)
     awq.profile_enable(True)
     try:
@@ -252,9 +284,14 @@ def test_launch_count_and_profile():
         prof = awq.profile_last()
     finally:
         awq.profile_enable(False)
-    # statistic + scales + qdq + one GEMM launch for the reference output and the candidates
-    # (two when the reference has its own launch) + reduce + pack
-    assert awq.last_launch_count() == 5 + awq.loss_gemm_launches(256, 256, 512, 20)
+    # statistic + scales + qdq (the reference operand alone when the loss GEMM's QDQ warps
+    # make the candidates') + one GEMM launch for the reference output and the candidates
+    # (two when the reference has its own launch, always with the QDQ warps) + reduce + pack
+    gemm = awq.loss_gemm_launches(256, 256, 512, 20)
+    qdq_warps = awq.qdq_in_loss_gemm(256, 256, 512, 20)
+    assert qdq_warps == (qdq == "warps" and awq.loss_gemm_variant(256, 256, 512, 20) == 1)
+    assert gemm == 2 or not qdq_warps
+    assert awq.last_launch_count() == 5 + gemm
     assert set(prof) >= {"statistic", "scales", "qdq", "gemm_reference", "gemm_loss", "loss_reduce", "pack"}
     assert all(v >= 0 for v in prof.values()) and prof["gemm_loss"] > 0
 
