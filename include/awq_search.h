@@ -364,10 +364,11 @@ int awq_loss_gemm_variant(int64_t M, int64_t K, int64_t N, int n_grid);
 
 /* Whether a search of this form makes its candidate operands with the loss GEMM's own
  * QDQ warps (1) or with a QDQ kernel launched before it (0): 1 for bf16 inputs with
- * group 128 on the one-SM GEMM kernel, unless AWQ_QDQ=standalone is set in the
- * environment. Eight more warps per GEMM CTA then quantize W while the tensor cores
- * run; a load of a column tile of a candidate operand waits (bounded) for that tile.
- * Both forms give bit-identical results. */
+ * group 128 on the one-SM GEMM kernel below 100 TFLOP of candidate GEMM work
+ * (2 M K N n_grid); AWQ_QDQ=standalone or =warps in the environment selects a form at
+ * every size. Eight more warps per GEMM CTA then quantize W while the tensor cores run;
+ * a load of a column tile of a candidate operand waits (bounded) for that tile. Both
+ * forms give bit-identical results. */
 int awq_qdq_in_loss_gemm(int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid);
 
 /* How many loss-GEMM launches a search of this form runs on the current device: 2 when

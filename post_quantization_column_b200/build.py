@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libawqsearch.so")
-SOURCES = ["awq_api.cu", "k_statistic.cu", "k_qdq.cu", "k_loss_gemm.cu", "k_clip.cu", "k_w4a16.cu", "k_module.cu", "k_attn.cu", "awq_noalloc.cu"]
+SOURCES = ["awq_api.cu", "k_statistic.cu", "k_qdq.cu", "k_loss_gemm.cu", "k_clip.cu", "k_w4a16.cu", "k_module.cu", "k_attn.cu", "awq_noalloc.cu", "gemm_policy.cu"]
 HEADERS = ["awq_device.cuh", "awq_kernels.h", "qdq_tile.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

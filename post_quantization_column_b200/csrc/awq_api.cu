@@ -453,7 +453,7 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
     }
     const int variant = gemm_variant(M, K, N, n_grid);
     // bf16 W, group 128: the candidate operands are made inside the loss GEMM's launches
-    const bool qdq_in_gemm = !feed && qdq_in_loss_gemm(in_dtype, group, variant);
+    const bool qdq_in_gemm = !feed && qdq_in_loss_gemm(in_dtype, group, variant, M, K, N, n_grid);
     ev.mark(kPhQdq);
     if (qdq_in_gemm) {
       // the reference operand only: the loss GEMM's QDQ warps make the candidates'
@@ -1866,7 +1866,7 @@ int awq_loss_gemm_variant(int64_t M, int64_t K, int64_t N, int n_grid) { return 
 
 int awq_loss_gemm_launches(int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid) {
   const int variant = gemm_variant(M, K, N, n_grid);
-  if (variant == 2 || qdq_in_loss_gemm(in_dtype, group, variant)) return 2;
+  if (variant == 2 || qdq_in_loss_gemm(in_dtype, group, variant, M, K, N, n_grid)) return 2;
   int dev = 0, l2_bytes = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&l2_bytes, cudaDevAttrL2CacheSize, dev);
@@ -1875,7 +1875,7 @@ int awq_loss_gemm_launches(int in_dtype, int64_t M, int64_t K, int64_t N, int gr
 }
 
 int awq_qdq_in_loss_gemm(int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid) {
-  return qdq_in_loss_gemm(in_dtype, group, gemm_variant(M, K, N, n_grid)) ? 1 : 0;
+  return qdq_in_loss_gemm(in_dtype, group, gemm_variant(M, K, N, n_grid), M, K, N, n_grid) ? 1 : 0;
 }
 
 }  // extern "C"

@@ -97,9 +97,10 @@ struct LossGemmArgs {
 // selects a form at every size (both give bit-identical results).
 bool reference_in_own_launch(int64_t M, int64_t N, int l2_bytes);
 // Whether a search makes its candidate operands with the loss GEMM's QDQ warps (bf16 W,
-// group 128, the one-SM kernel) rather than with qdq_kernel before it. AWQ_QDQ=standalone
-// in the environment selects qdq_kernel at every size (both give bit-identical operands).
-bool qdq_in_loss_gemm(int in_dtype, int group, int variant);
+// group 128, the one-SM kernel, below 100 TFLOP of candidate GEMM work) rather than with
+// qdq_kernel before it. AWQ_QDQ=standalone or =warps in the environment selects a form
+// at every size (both give bit-identical operands).
+bool qdq_in_loss_gemm(int in_dtype, int group, int variant, int64_t M, int64_t K, int64_t N, int n_grid);
 // Which loss GEMM runs for a search of this size: 1 = the one-SM kernel (every size; it
 // measured as fast or faster than the pair kernel on every workload), 2 = the two-SM
 // (cta_group::2) kernel, selected with AWQ_GEMM_VARIANT=2 in the environment.
