@@ -122,11 +122,12 @@ static_assert((kQdqTileCols * QdqTile::kPitch * 4) % 16 == 0 && (QdqTile::kSkewP
               "16-byte aligned parameter sets");
 constexpr int kQdqColsPerTileN = kTileN / kQdqTileCols;  // 8 QDQ column blocks per GEMM column tile
 
-// Finished QDQ tiles a 256-column tile needs: its 32-column blocks (the last tile may be
-// ragged) times the groups of K.
+// Finished QDQ claims a 256-column tile needs: its 32-column blocks (the last tile may be
+// ragged) times the groups of K times the candidate chunks.
 __device__ __forceinline__ int qdq_target(const GemmParams& p, int nt) {
   const int64_t cols = min(static_cast<int64_t>(kTileN), p.N - static_cast<int64_t>(nt) * kTileN);
-  return static_cast<int>(ceil_div(cols, static_cast<int64_t>(kQdqTileCols)) * (p.K / 128));
+  return static_cast<int>(ceil_div(cols, static_cast<int64_t>(kQdqTileCols)) * (p.K / 128) *
+                          ceil_div(p.n_grid, kQdqChunk));
 }
 
 struct QdqWarpsSync {
@@ -490,11 +491,12 @@ __global__ void __launch_bounds__(kQdq ? kThreads + kQdqThreads : kThreads, 1)
   } else if constexpr (kQdq) {
     if (warp >= 8) {
       // --------------------------------------------------------------- QDQ warps
-      // The 128 x 32 tiles of W, claimed one at a time in column-major order (the column
-      // tiles the GEMM reads first are finished first) from a counter that spans the
-      // search's launches: the reference launch claims tiles while its own GEMM runs,
-      // the candidate launch until none is left. Each tile's stores, for every candidate,
-      // are published by its column tile's count.
+      // (128 x 32 tile of W, chunk of up to kQdqChunk candidates) pieces, claimed one at a
+      // time in column-major order (the column tiles the GEMM reads first are finished
+      // first) from a counter that spans the search's launches: the reference launch
+      // claims while its own GEMM runs (a claim takes a few microseconds, so the launch
+      // outlasts its GEMM by at most that), the candidate launch until none is left. Each
+      // piece's stores are published by its column tile's count.
       const int tid = static_cast<int>(threadIdx.x) - kThreads;
       uint8_t* qs = smem + kSmemBytes - 1024;  // past the ring, the barriers and their slack
       float* sWT = reinterpret_cast<float*>(qs);
@@ -503,20 +505,20 @@ __global__ void __launch_bounds__(kQdq ? kThreads + kQdqThreads : kThreads, 1)
       float4* sPar = reinterpret_cast<float4*>(sR + kQdqChunk * QdqTile::kSkewPitch);
       uint32_t* sRowsExact = reinterpret_cast<uint32_t*>(sPar + kQdqChunk * kQdqTileCols);
       const int64_t groups = p.K / 128;
-      const int64_t qtiles = ceil_div(p.N, static_cast<int64_t>(kQdqTileCols)) * groups;
+      const int64_t chunks = ceil_div(p.n_grid, kQdqChunk);
+      const int64_t pieces = ceil_div(p.N, static_cast<int64_t>(kQdqTileCols)) * groups * chunks;
       int* const next = p.qdq_ready + p.tiles_n;
       bool skip_publish = p.fault_mode == 3 && blockIdx.x == 0;  // fault injection: one count never arrives
       while (p.qdq_cands) {
         if (tid == 0) *qdq_claim = (p.qdq_cands == 2 && *gemm_done) ? -1 : atomicAdd(next, 1);
         QdqWarpsSync{}();
-        const int64_t t = *qdq_claim;
-        if (t < 0 || t >= qtiles) break;
-        const int64_t cb = t / groups, k0 = (t - cb * groups) * 128;
-        for (int c0 = 0; c0 < p.n_grid; c0 += kQdqChunk)
-          qdq_tile<__nv_bfloat16, 128, QdqTile>(p.qdq_W, p.K, p.N, p.N, k0, cb * kQdqTileCols, p.qdq_S, c0,
-                                                min(c0 + kQdqChunk, p.n_grid), c0 == 0, false, p.qdq_Wt, p.err,
-                                                p.qdq_quantizer, 0, sWT, sS, sR, sPar, sRowsExact, tid,
-                                                QdqWarpsSync{});
+        const int64_t q = *qdq_claim;
+        if (q < 0 || q >= pieces) break;
+        const int64_t t = q / chunks, cb = t / groups, k0 = (t - cb * groups) * 128;
+        const int c0 = static_cast<int>(q - t * chunks) * kQdqChunk;
+        qdq_tile<__nv_bfloat16, 128, QdqTile>(p.qdq_W, p.K, p.N, p.N, k0, cb * kQdqTileCols, p.qdq_S, c0,
+                                              min(c0 + kQdqChunk, p.n_grid), true, false, p.qdq_Wt, p.err,
+                                              p.qdq_quantizer, 0, sWT, sS, sR, sPar, sRowsExact, tid, QdqWarpsSync{});
         // publish: every thread's stores, then the column tile's count
         fence_proxy_async_global();
         __threadfence();
@@ -933,7 +935,9 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
   }
   const bool qdq = a.qdq_W != nullptr;
   if (qdq && ((mode != 0 && mode != 1) || !a.qdq_ready || !a.qdq_S || a.slot_base != 1 || a.a_slotted ||
-              !a.b_per_cand || a.K % 128 || ceil_div(a.N, static_cast<int64_t>(kQdqTileCols)) * (a.K / 128) >= (int64_t(1) << 30)))
+              !a.b_per_cand || a.K % 128 ||
+              ceil_div(a.N, static_cast<int64_t>(kQdqTileCols)) * (a.K / 128) * ceil_div(a.n_grid, kQdqChunk) >=
+                  (int64_t(1) << 30)))
     return cudaErrorInvalidValue;
   static unsigned long long attr_done = 0, attr_done_qdq = 0;
   cudaError_t e = qdq ? set_smem_limit_once(loss_gemm_kernel<true>, kSmemBytes + kQdqSmemBytes, &attr_done_qdq)
