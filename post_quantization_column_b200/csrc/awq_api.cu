@@ -492,8 +492,12 @@ int search_device(const void* X, const void* W, int in_dtype, int64_t M, int64_t
     if (qdq_in_gemm) {
       ga.qdq_W = static_cast<const __nv_bfloat16*>(W);
       ga.qdq_S = S;
+      ga.qdq_Wt = Wt;
       ga.qdq_ready = err + 4 + L.tiles;
       ga.qdq_quantizer = quantizer;
+      ga.qdq_K = K;
+      ga.qdq_N = N;
+      ga.qdq_grid = n_grid;
     }
     CUtensorMap mapA, mapB;
     const char* why = "";
@@ -1343,7 +1347,12 @@ int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_d
     off += align_up(bytes);
     return at;
   };
-  const size_t o_err = take(16), o_a = take(static_cast<size_t>(K) * 4), o_S = take(static_cast<size_t>(n_grid) * K * 4),
+  // bf16 W with group 128: the candidate operands of [W_gate | W_up] are made by the
+  // first GEMM's QDQ warps while the reference block runs and then while the candidates'
+  // first GEMM walks every candidate of an operand tile before the next
+  const bool qdq_warps = fused && qdq_in_loss_gemm(in_dtype, group, 1, M, K, N, n_grid);
+  const size_t flag_bytes = 16 + static_cast<size_t>(ceil_div(N, kTileN) + 1) * 4;  // status word, QDQ counters
+  const size_t o_err = take(flag_bytes), o_a = take(static_cast<size_t>(K) * 4), o_S = take(static_cast<size_t>(n_grid) * K * 4),
                o_best = take(16), o_losses = take(static_cast<size_t>(n_grid) * 4),
                o_Xb = in_dtype == AWQ_DTYPE_F32 ? take(static_cast<size_t>(M) * K * 2) : 0,
                o_Wt = take(static_cast<size_t>(n_grid + 1) * N * K * 2),
@@ -1377,7 +1386,7 @@ int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_d
   int launches = 0, h_err = 0, status = AWQ_OK;
   const char* where = "";
   do {
-    if ((e = cudaMemsetAsync(err, 0, 16, s)) != cudaSuccess) { where = "cudaMemsetAsync"; break; }
+    if ((e = cudaMemsetAsync(err, 0, flag_bytes, s)) != cudaSuccess) { where = "cudaMemsetAsync"; break; }
     if ((e = launch_statistic(X, in_dtype, M, K, a, err, s, &launches)) != cudaSuccess) {
       where = "statistic kernel";
       break;
@@ -1389,8 +1398,9 @@ int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_d
       where = "bf16 operand kernel";
       break;
     }
-    if ((e = launch_qdq(W_gu, in_dtype, K, N, group, n_grid, S, Wt, err, s, &launches, 0, fused ? F : 0)) !=
-        cudaSuccess) {
+    // every operand slot, or (QDQ warps) the reference slot alone
+    if ((e = launch_qdq(W_gu, in_dtype, K, N, group, qdq_warps ? 0 : n_grid, S, Wt, err, s, &launches, 0,
+                        fused ? F : 0)) != cudaSuccess) {
       where = "qdq kernel";
       break;
     }
@@ -1415,6 +1425,16 @@ int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_d
     g1.timeout_ns = g_timeout_ns;
     g1.fault_mode = 0;
     g1.num_sms = num_sms;
+    if (qdq_warps) {
+      g1.qdq_W = static_cast<const __nv_bfloat16*>(W_gu);
+      g1.qdq_S = S;
+      g1.qdq_Wt = Wt;
+      g1.qdq_ready = err + 4;
+      g1.qdq_K = K;
+      g1.qdq_N = N;
+      g1.qdq_interleave = F;
+      g1.qdq_grid = n_grid;
+    }
     // GEMM 2: h W_down^T; mode 0 writes the reference block output (tiled), mode 1 the
     // per-tile squared error of one candidate against it
     LossGemmArgs g2 = g1;
@@ -1430,6 +1450,7 @@ int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_d
     const char* why = "";
     // the batched second GEMM: A = the stack of intermediates [1 + h_batch][M][F]
     LossGemmArgs g2b = g2;
+    g2b.qdq_W = nullptr;  // the batched second GEMM reads no candidate operand
     g2b.a_slotted = 1;
     g2b.a_slots = 1 + h_batch;
     if ((e = make_operand_maps(g1, &a1, &b1, &why, kTileN)) != cudaSuccess ||
@@ -1443,9 +1464,12 @@ int awq_search_mlp(const void* X, const void* W_gu, const void* W_down, int in_d
       // reference block: h_0 = block intermediate with bf16(W), then Y = h_0 W_down^T
       g1.slot_base = 0;
       g1.cands = 1;
+      g1.qdq_cands = g2.qdq_cands = 2;  // the QDQ warps claim candidate pieces while these run
       if ((e = launch_loss_gemm(g1, a1, b1, 3, s, &launches)) != cudaSuccess) { where = "block GEMM 1"; break; }
       g2.partial = part;
       if ((e = launch_loss_gemm(g2, a2, b2, 0, s, &launches)) != cudaSuccess) { where = "block GEMM 2"; break; }
+      g1.qdq_cands = 1;   // ... and the rest during the candidates' first GEMM, which then walks
+      g1.cand_inner = qdq_warps ? 1 : 0;  // every candidate of an operand tile before the next
       for (int c0 = 0; c0 < n_grid && e == cudaSuccess; c0 += h_batch) {
         const int nb = std::min(h_batch, n_grid - c0);
         g1.slot_base = 1 + c0;  // candidate c0 + i in B slot 1 + c0 + i ...

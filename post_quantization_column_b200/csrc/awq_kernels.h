@@ -76,19 +76,24 @@ struct LossGemmArgs {
   int* ready = nullptr;        // mode 4: per-tile flags (tiles_m * tiles_n ints), zero at launch
   int cand_inner = 0;          // mode 1: walk raster group -> column tile -> candidate -> row tile, so
                                // that every candidate reads a tile of Y while it is still in L2
-  // Modes 0 and 1 on the one-SM kernel with bf16 W and group 128: when qdq_W is set,
-  // eight more warps per CTA make the candidate operand slots (the QDQ of the candidate
-  // loop, slots 1 .. n_grid; slot 0 comes from launch_qdq with n_grid = 0) while the
-  // tensor cores run, claiming 128 x 32 tiles of W from a counter that spans the search's
-  // launches (qdq_cands 2: while this CTA's GEMM runs, the reference launch; 1: until
-  // none is left, the candidate launch); every mode-1 load of a column tile of B waits
-  // (bounded) until that tile is complete. qdq_ready: tiles_n + 1 ints, zero before the
-  // first of the launches.
-  const __nv_bfloat16* qdq_W = nullptr;  // [K][N]
-  const float* qdq_S = nullptr;          // [n_grid][K]
+  // The one-SM kernel with bf16 W and group 128: when qdq_W is set, eight more warps per
+  // CTA make candidate operand slots (the QDQ of the candidate loop; slot 0 comes from
+  // launch_qdq with n_grid = 0) while the tensor cores run, claiming pieces (a 128 x 32
+  // tile of W, a chunk of candidates) column-major from a counter that spans a search's
+  // launches (qdq_cands 2: while this CTA's GEMM runs; 1: until none is left). A load of a
+  // candidate slot's 256-row tile (mode 1, or mode 3 past slot 0; those launches read
+  // qdq_Wt with the QDQ's K and N) waits (bounded) until that tile is complete for every
+  // candidate. Mode 0 may host the warps for another GEMM (the MLP block's reference down
+  // projection). qdq_interleave = F for the MLP block's [W_gate | W_up]. qdq_ready:
+  // ceil(qdq_N / 256) + 1 ints, zero before the first launch.
+  const __nv_bfloat16* qdq_W = nullptr;  // [qdq_K][qdq_N]
+  const float* qdq_S = nullptr;          // [qdq_grid][qdq_K]
+  __nv_bfloat16* qdq_Wt = nullptr;       // [qdq_grid + 1][qdq_N][qdq_K]
   int* qdq_ready = nullptr;
   int qdq_cands = 0;
   int qdq_quantizer = 0;
+  int64_t qdq_K = 0, qdq_N = 0, qdq_interleave = 0;
+  int qdq_grid = 0;
 };
 // Whether a search scores its candidates in two launches (mode 0, then mode 1 with
 // cand_inner) rather than one mode-4 launch: when the reference output Y (M x N fp32) is

@@ -94,18 +94,22 @@ struct GemmParams {
   uint64_t timeout_ns;
   int fault_mode;
   int cand_inner;     // mode 1: raster group -> column tile -> candidate -> row tile
-  // QDQ warps (loss_gemm_kernel<true>, modes 0 and 1): the candidate operand slots are
-  // made by warps 8 .. 15 of the same CTAs while the tensor cores run. qdq_ready[nt]
-  // counts the finished 128 x 32 tiles of W (all candidates) of 256-column tile nt; a
-  // mode-1 B load waits for its column tile's count. qdq_ready[tiles_n] is the claim
-  // counter of the tiles, which spans the search's two launches.
-  const __nv_bfloat16* qdq_W;  // [K][N] bf16
-  const float* qdq_S;          // [n_grid][K] candidate scales
-  __nv_bfloat16* qdq_Wt;       // [n_grid + 1][N][K]
-  int* qdq_ready;
-  int qdq_cands;               // claim tiles: 1 until none is left, 2 while this CTA's GEMM runs
-  int qdq_quantizer;
   int64_t K;
+  // QDQ warps (loss_gemm_kernel<true>): the candidate operand slots of a K x N bf16 W are
+  // made by warps 8 .. 15 of the same CTAs while the tensor cores run, in pieces claimed
+  // column-major from a counter that spans the launches of one search: a piece is a
+  // 128 x 32 tile of W for a chunk of up to kQdqChunk candidates, qdq_ready[nt] counts the
+  // finished pieces of the operand's 256-row tile nt, and a load of a candidate slot's
+  // tile nt (mode 1, or mode 3 past slot 0) waits for that count. qdq_ready[ceil(qdq_N /
+  // 256)] is the claim counter.
+  const __nv_bfloat16* qdq_W;  // [qdq_K][qdq_N]
+  const float* qdq_S;          // [qdq_grid][qdq_K] candidate scales
+  __nv_bfloat16* qdq_Wt;       // [qdq_grid + 1][qdq_N][qdq_K]
+  int* qdq_ready;
+  int qdq_cands;               // claim pieces: 1 until none is left, 2 while this CTA's GEMM runs
+  int qdq_quantizer;
+  int64_t qdq_K, qdq_N, qdq_interleave;
+  int qdq_grid;
 };
 
 // QDQ warps: group 128, tiles of 128 rows x 32 columns (8 warps of 16 row-lanes x 2
@@ -122,12 +126,22 @@ static_assert((kQdqTileCols * QdqTile::kPitch * 4) % 16 == 0 && (QdqTile::kSkewP
               "16-byte aligned parameter sets");
 constexpr int kQdqColsPerTileN = kTileN / kQdqTileCols;  // 8 QDQ column blocks per GEMM column tile
 
-// Finished QDQ claims a 256-column tile needs: its 32-column blocks (the last tile may be
-// ragged) times the groups of K times the candidate chunks.
+// Finished QDQ pieces a 256-row tile of the operand needs: its 32-column blocks of W (the
+// last tile may be ragged; with the gate/up interleave every tile holds four of each
+// half) times the groups of K times the candidate chunks.
 __device__ __forceinline__ int qdq_target(const GemmParams& p, int nt) {
-  const int64_t cols = min(static_cast<int64_t>(kTileN), p.N - static_cast<int64_t>(nt) * kTileN);
-  return static_cast<int>(ceil_div(cols, static_cast<int64_t>(kQdqTileCols)) * (p.K / 128) *
-                          ceil_div(p.n_grid, kQdqChunk));
+  const int64_t cols = min(static_cast<int64_t>(kTileN), p.qdq_N - static_cast<int64_t>(nt) * kTileN);
+  return static_cast<int>(ceil_div(cols, static_cast<int64_t>(kQdqTileCols)) * (p.qdq_K / 128) *
+                          ceil_div(p.qdq_grid, kQdqChunk));
+}
+
+// The column of W held by row `row` of the K-major candidate operand (the inverse of the
+// QDQ tile's interleaved_column): with the MLP block's interleave F > 0 every 256 rows
+// hold 128 gate columns, then the 128 up columns of the same outputs.
+__device__ __forceinline__ int64_t qdq_w_column(int64_t row, int64_t interleave) {
+  if (interleave <= 0) return row;
+  const int64_t nt = row / kTileN, j = row - nt * kTileN;
+  return j < kTileN / 2 ? nt * (kTileN / 2) + j : interleave + nt * (kTileN / 2) + (j - kTileN / 2);
 }
 
 struct QdqWarpsSync {
@@ -240,14 +254,15 @@ __global__ void __launch_bounds__(kQdq ? kThreads + kQdqThreads : kThreads, 1)
       uint32_t issued = 0, last_parity = 0;  // per-stage bits
       bool ok = true;
       bool fault_pending = p.fault_mode == 1;
-      int confirmed = -1;  // the last column tile whose candidate operands were seen complete
+      int confirmed = -1;  // the last operand tile whose candidate slots were seen complete
       (void)confirmed;
       for (int64_t u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         int c, mt, nt;
         unit_coords(u, p, c, mt, nt);
         if constexpr (kQdq) {
-          // a candidate operand: its column tile must be complete
-          if (p.mode == 1 && confirmed != nt) {
+          // a candidate operand: its tile nt must be complete for every candidate
+          const bool cand = p.mode == 1 || (p.mode == 3 && p.slot_base + c >= 1);
+          if (cand && confirmed != nt) {
             if (!counter_wait_bounded(p.qdq_ready + nt, qdq_target(p, nt), abort_flag, budget)) {
               ok = false;
               break;
@@ -504,22 +519,28 @@ __global__ void __launch_bounds__(kQdq ? kThreads + kQdqThreads : kThreads, 1)
       float* sR = sS + kQdqChunk * QdqTile::kSkewPitch;
       float4* sPar = reinterpret_cast<float4*>(sR + kQdqChunk * QdqTile::kSkewPitch);
       uint32_t* sRowsExact = reinterpret_cast<uint32_t*>(sPar + kQdqChunk * kQdqTileCols);
-      const int64_t groups = p.K / 128;
-      const int64_t chunks = ceil_div(p.n_grid, kQdqChunk);
-      const int64_t pieces = ceil_div(p.N, static_cast<int64_t>(kQdqTileCols)) * groups * chunks;
-      int* const next = p.qdq_ready + p.tiles_n;
+      const int64_t groups = p.qdq_K / 128;
+      const int64_t qtiles = ceil_div(p.qdq_N, static_cast<int64_t>(kQdqTileCols)) * groups;
+      const int64_t chunks = ceil_div(p.qdq_grid, kQdqChunk);
+      const int64_t pieces = qtiles * chunks;
+      int* const next = p.qdq_ready + ceil_div(p.qdq_N, static_cast<int64_t>(kTileN));
       bool skip_publish = p.fault_mode == 3 && blockIdx.x == 0;  // fault injection: one count never arrives
       while (p.qdq_cands) {
         if (tid == 0) *qdq_claim = (p.qdq_cands == 2 && *gemm_done) ? -1 : atomicAdd(next, 1);
         QdqWarpsSync{}();
         const int64_t q = *qdq_claim;
         if (q < 0 || q >= pieces) break;
-        const int64_t t = q / chunks, cb = t / groups, k0 = (t - cb * groups) * 128;
+        // q = (tile, chunk), chunk fastest; tiles in the order of the operand rows they
+        // fill (32 rows = 32 columns of W, never straddling a 128-column block), rows major
+        const int64_t t = q / chunks;
+        const int64_t rb = t / groups, k0 = (t - rb * groups) * 128;
         const int c0 = static_cast<int>(q - t * chunks) * kQdqChunk;
-        qdq_tile<__nv_bfloat16, 128, QdqTile>(p.qdq_W, p.K, p.N, p.N, k0, cb * kQdqTileCols, p.qdq_S, c0,
-                                              min(c0 + kQdqChunk, p.n_grid), true, false, p.qdq_Wt, p.err,
-                                              p.qdq_quantizer, 0, sWT, sS, sR, sPar, sRowsExact, tid, QdqWarpsSync{});
-        // publish: every thread's stores, then the column tile's count
+        const int c1 = min(c0 + kQdqChunk, p.qdq_grid);
+        const int64_t n0 = qdq_w_column(rb * kQdqTileCols, p.qdq_interleave);
+        qdq_tile<__nv_bfloat16, 128, QdqTile>(p.qdq_W, p.qdq_K, p.qdq_N, p.qdq_N, k0, n0, p.qdq_S, c0,
+                                              c1, true, false, p.qdq_Wt, p.err, p.qdq_quantizer, p.qdq_interleave,
+                                              sWT, sS, sR, sPar, sRowsExact, tid, QdqWarpsSync{});
+        // publish: every thread's stores, then the count of the operand tile the rows are in
         fence_proxy_async_global();
         __threadfence();
         QdqWarpsSync{}();
@@ -527,7 +548,7 @@ __global__ void __launch_bounds__(kQdq ? kThreads + kQdqThreads : kThreads, 1)
           if (skip_publish)
             skip_publish = false;
           else
-            red_release_add_gpu(p.qdq_ready + cb / kQdqColsPerTileN, 1);
+            red_release_add_gpu(p.qdq_ready + rb / kQdqColsPerTileN, 1);
         }
       }
     }
@@ -934,9 +955,12 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
     return e != cudaSuccess ? e : cudaGetLastError();
   }
   const bool qdq = a.qdq_W != nullptr;
-  if (qdq && ((mode != 0 && mode != 1) || !a.qdq_ready || !a.qdq_S || a.slot_base != 1 || a.a_slotted ||
-              !a.b_per_cand || a.K % 128 ||
-              ceil_div(a.N, static_cast<int64_t>(kQdqTileCols)) * (a.K / 128) * ceil_div(a.n_grid, kQdqChunk) >=
+  // the launches that read candidate slots (mode 1, mode 3) must read the operand the QDQ
+  // warps make, one B slot per candidate
+  if (qdq && ((mode != 0 && mode != 1 && mode != 3) || !a.qdq_ready || !a.qdq_S || !a.qdq_Wt || a.qdq_K % 128 ||
+              a.qdq_N % 8 || a.qdq_grid < 1 || (a.qdq_interleave && (a.qdq_interleave % 128 || a.qdq_N != 2 * a.qdq_interleave)) ||
+              (mode != 0 && (a.qdq_N != a.N || a.qdq_K != a.K || a.qdq_Wt != a.Wt || a.a_slotted || !a.b_per_cand)) ||
+              ceil_div(a.qdq_N, static_cast<int64_t>(kQdqTileCols)) * (a.qdq_K / 128) * ceil_div(a.qdq_grid, kQdqChunk) >=
                   (int64_t(1) << 30)))
     return cudaErrorInvalidValue;
   static unsigned long long attr_done = 0, attr_done_qdq = 0;
@@ -967,13 +991,17 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
   p.err = a.err;
   p.timeout_ns = a.timeout_ns;
   p.fault_mode = a.fault_mode;
-  p.cand_inner = mode == 1 ? a.cand_inner : 0;
+  p.cand_inner = (mode == 1 || mode == 3) ? a.cand_inner : 0;
   p.qdq_W = a.qdq_W;
   p.qdq_S = a.qdq_S;
-  p.qdq_Wt = const_cast<__nv_bfloat16*>(a.Wt);
+  p.qdq_Wt = const_cast<__nv_bfloat16*>(a.qdq_Wt);
   p.qdq_ready = a.qdq_ready;
   p.qdq_cands = a.qdq_cands;
   p.qdq_quantizer = a.qdq_quantizer;
+  p.qdq_K = a.qdq_K;
+  p.qdq_N = a.qdq_N;
+  p.qdq_interleave = a.qdq_interleave;
+  p.qdq_grid = a.qdq_grid;
   p.K = a.K;
   const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
   const int64_t units = (mode == 1 || mode == 3 || mode == 5 ? p.cands : (mode == 4 ? a.n_grid + 1 : 1)) * tiles;

@@ -95,3 +95,22 @@ def test_fused_epilogue_matches_separate_elementwise_kernel(monkeypatch):
     plain = awq.search_mlp(X, W_gu, W_down, 128, 20)
     for name in ("scales", "codes", "steps", "zeros", "losses"):
         assert torch.equal(getattr(fused, name), getattr(plain, name)), name
+
+
+@pytest.mark.parametrize("M,K,F,Ko,n_grid", [(300, 384, 256, 264, 20), (129, 256, 384, 136, 7), (64, 512, 128, 64, 64)])
+def test_qdq_warps_match_the_qdq_kernel_in_the_mlp_block(M, K, F, Ko, n_grid, monkeypatch):
+    """bf16 W with group 128 and F % 128 == 0: the first GEMM's QDQ warps make the candidate
+    operands of [W_gate | W_up] candidate by candidate (claimed while the reference block
+    runs, the rest during the candidates' first GEMM, each candidate's loads waiting for its
+    slot); AWQ_QDQ=standalone makes them with qdq_kernel first. Both match the oracle and
+    give the same bits."""
+    out, r, Wgu32 = _run(M, K, F, Ko, 128, "bf16", seed=M + 2 * K + F, n_grid=n_grid)
+    _check(out, r, Wgu32, 128)
+    spec = custom_spec(M, K, 2 * F, dtype="bf16", group=128, seed=M + 2 * K + F)
+    X, W_gu = (t.cuda() for t in generate(spec))
+    W_down = generate_down(spec, Ko).cuda()
+    warps = awq.search_mlp(X, W_gu, W_down, 128, n_grid)
+    monkeypatch.setenv("AWQ_QDQ", "standalone")
+    plain = awq.search_mlp(X, W_gu, W_down, 128, n_grid)
+    for name in ("scales", "codes", "steps", "zeros", "losses"):
+        assert torch.equal(getattr(warps, name), getattr(plain, name)), name
