@@ -1592,7 +1592,12 @@ int awq_search_attn(const void* X, const void* W_qkv, int in_dtype, int64_t M, i
     off += align_up(bytes);
     return at;
   };
-  const size_t o_err = take(16), o_a = take(static_cast<size_t>(K) * 4), o_S = take(static_cast<size_t>(n_grid) * K * 4),
+  // bf16 W with group 128: the Q|K GEMM's QDQ warps make the candidate operands of
+  // [W_q | W_k] (while that GEMM walks every slot of an operand tile before the next) and
+  // then of W_v (which the V^T GEMM, the next launch, reads)
+  const bool qdq_warps = qdq_in_loss_gemm(in_dtype, group, 1, M, K, N, n_grid);
+  const size_t flag_bytes = 16 + static_cast<size_t>(ceil_div(2 * D, kTileN) + 1) * 4;  // status word, QDQ counters
+  const size_t o_err = take(flag_bytes), o_a = take(static_cast<size_t>(K) * 4), o_S = take(static_cast<size_t>(n_grid) * K * 4),
                o_best = take(16), o_losses = take(static_cast<size_t>(n_grid) * 4),
                o_Xb = in_dtype == AWQ_DTYPE_F32 ? take(static_cast<size_t>(M) * K * 2) : 0,
                o_Wqk = take(static_cast<size_t>(slots) * 2 * D * K * 2),
@@ -1632,7 +1637,7 @@ int awq_search_attn(const void* X, const void* W_qkv, int in_dtype, int64_t M, i
   int launches = 0, h_err = 0, status = AWQ_OK;
   const char* where = "";
   do {
-    if ((e = cudaMemsetAsync(err, 0, 16, s)) != cudaSuccess) { where = "cudaMemsetAsync"; break; }
+    if ((e = cudaMemsetAsync(err, 0, flag_bytes, s)) != cudaSuccess) { where = "cudaMemsetAsync"; break; }
     mark(0);
     if ((e = launch_statistic(X, in_dtype, M, K, a, err, s, &launches)) != cudaSuccess) {
       where = "statistic kernel";
@@ -1646,9 +1651,11 @@ int awq_search_attn(const void* X, const void* W_qkv, int in_dtype, int64_t M, i
       break;
     }
     // the query and key columns, then the value columns, each into a stack of K-major slots
-    if ((e = launch_qdq(W_qkv, in_dtype, K, 2 * D, group, n_grid, S, Wqk, err, s, &launches, kQuantAsym, 0, N)) !=
+    // (with the QDQ warps, the reference slot alone)
+    const int qdq_slots = qdq_warps ? 0 : n_grid;
+    if ((e = launch_qdq(W_qkv, in_dtype, K, 2 * D, group, qdq_slots, S, Wqk, err, s, &launches, kQuantAsym, 0, N)) !=
             cudaSuccess ||
-        (e = launch_qdq(W_v, in_dtype, K, D, group, n_grid, S, Wv, err, s, &launches, kQuantAsym, 0, N)) !=
+        (e = launch_qdq(W_v, in_dtype, K, D, group, qdq_slots, S, Wv, err, s, &launches, kQuantAsym, 0, N)) !=
             cudaSuccess) {
       where = "qdq kernel";
       break;
@@ -1673,8 +1680,26 @@ int awq_search_attn(const void* X, const void* W_qkv, int in_dtype, int64_t M, i
     g.cands = slots;
     g.slot_base = 0;
     g.b_per_cand = 1;
+    if (qdq_warps) {
+      g.qdq_W = static_cast<const __nv_bfloat16*>(W_qkv);
+      g.qdq_S = S;
+      g.qdq_Wt = Wqk;
+      g.qdq_ready = err + 4;
+      g.qdq_cands = 1;
+      g.qdq_K = K;
+      g.qdq_N = 2 * D;
+      g.qdq_ldw = N;
+      g.qdq_grid = n_grid;
+      g.qdq_W2 = static_cast<const __nv_bfloat16*>(W_v);
+      g.qdq_Wt2 = Wv;
+      g.qdq_N2 = D;
+      g.cand_inner = 1;  // every slot of an operand tile before the next
+    }
     // V^T of every slot: the slot's W_v^T [D][K] (a stack of A operands) times X_b
     LossGemmArgs gv = g;
+    gv.qdq_W = nullptr;  // W_v's slots are complete when this launch starts
+    gv.qdq_W2 = nullptr;
+    gv.cand_inner = 0;
     gv.Xb = Wv;
     gv.a_slotted = 1;
     gv.a_slots = slots;

@@ -81,19 +81,25 @@ struct LossGemmArgs {
   // launch_qdq with n_grid = 0) while the tensor cores run, claiming pieces (a 128 x 32
   // tile of W, a chunk of candidates) column-major from a counter that spans a search's
   // launches (qdq_cands 2: while this CTA's GEMM runs; 1: until none is left). A load of a
-  // candidate slot's 256-row tile (mode 1, or mode 3 past slot 0; those launches read
+  // candidate slot's 256-row tile (mode 1, or modes 3 and 5 past slot 0; those launches read
   // qdq_Wt with the QDQ's K and N) waits (bounded) until that tile is complete for every
   // candidate. Mode 0 may host the warps for another GEMM (the MLP block's reference down
   // projection). qdq_interleave = F for the MLP block's [W_gate | W_up]. qdq_ready:
   // ceil(qdq_N / 256) + 1 ints, zero before the first launch.
-  const __nv_bfloat16* qdq_W = nullptr;  // [qdq_K][qdq_N]
+  // The attention block's Q|K launch (mode 5) also makes W_v's slots: qdq_W2 (columns of
+  // the same rows, pitch qdq_ldw) into qdq_Wt2, after the first operand, without counters
+  // (only the next launch reads them).
+  const __nv_bfloat16* qdq_W = nullptr;  // [qdq_K][qdq_N], row pitch qdq_ldw (0: qdq_N)
   const float* qdq_S = nullptr;          // [qdq_grid][qdq_K]
   __nv_bfloat16* qdq_Wt = nullptr;       // [qdq_grid + 1][qdq_N][qdq_K]
   int* qdq_ready = nullptr;
   int qdq_cands = 0;
   int qdq_quantizer = 0;
-  int64_t qdq_K = 0, qdq_N = 0, qdq_interleave = 0;
+  int64_t qdq_K = 0, qdq_N = 0, qdq_interleave = 0, qdq_ldw = 0;
   int qdq_grid = 0;
+  const __nv_bfloat16* qdq_W2 = nullptr;  // [qdq_K][qdq_N2], row pitch qdq_ldw
+  __nv_bfloat16* qdq_Wt2 = nullptr;       // [qdq_grid + 1][qdq_N2][qdq_K]
+  int64_t qdq_N2 = 0;
 };
 // Whether a search scores its candidates in two launches (mode 0, then mode 1 with
 // cand_inner) rather than one mode-4 launch: when the reference output Y (M x N fp32) is

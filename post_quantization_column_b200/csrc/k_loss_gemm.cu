@@ -100,16 +100,21 @@ struct GemmParams {
   // column-major from a counter that spans the launches of one search: a piece is a
   // 128 x 32 tile of W for a chunk of up to kQdqChunk candidates, qdq_ready[nt] counts the
   // finished pieces of the operand's 256-row tile nt, and a load of a candidate slot's
-  // tile nt (mode 1, or mode 3 past slot 0) waits for that count. qdq_ready[ceil(qdq_N /
-  // 256)] is the claim counter.
-  const __nv_bfloat16* qdq_W;  // [qdq_K][qdq_N]
+  // tile nt (mode 1, or modes 3 and 5 past slot 0) waits for that count. A second
+  // operand (qdq_W2: another column range, no counters; the attention block's W_v) is
+  // made after the first by the same claims. qdq_ready[ceil(qdq_N / 256)] is the claim
+  // counter.
+  const __nv_bfloat16* qdq_W;  // [qdq_K][qdq_N], row pitch qdq_ldw
   const float* qdq_S;          // [qdq_grid][qdq_K] candidate scales
   __nv_bfloat16* qdq_Wt;       // [qdq_grid + 1][qdq_N][qdq_K]
   int* qdq_ready;
   int qdq_cands;               // claim pieces: 1 until none is left, 2 while this CTA's GEMM runs
   int qdq_quantizer;
-  int64_t qdq_K, qdq_N, qdq_interleave;
+  int64_t qdq_K, qdq_N, qdq_interleave, qdq_ldw;
   int qdq_grid;
+  const __nv_bfloat16* qdq_W2;  // [qdq_K][qdq_N2], row pitch qdq_ldw, or null
+  __nv_bfloat16* qdq_Wt2;       // [qdq_grid + 1][qdq_N2][qdq_K]
+  int64_t qdq_N2;
 };
 
 // QDQ warps: group 128, tiles of 128 rows x 32 columns (8 warps of 16 row-lanes x 2
@@ -261,7 +266,7 @@ __global__ void __launch_bounds__(kQdq ? kThreads + kQdqThreads : kThreads, 1)
         unit_coords(u, p, c, mt, nt);
         if constexpr (kQdq) {
           // a candidate operand: its tile nt must be complete for every candidate
-          const bool cand = p.mode == 1 || (p.mode == 3 && p.slot_base + c >= 1);
+          const bool cand = p.mode == 1 || ((p.mode == 3 || p.mode == 5) && p.slot_base + c >= 1);
           if (cand && confirmed != nt) {
             if (!counter_wait_bounded(p.qdq_ready + nt, qdq_target(p, nt), abort_flag, budget)) {
               ok = false;
@@ -520,31 +525,40 @@ __global__ void __launch_bounds__(kQdq ? kThreads + kQdqThreads : kThreads, 1)
       float4* sPar = reinterpret_cast<float4*>(sR + kQdqChunk * QdqTile::kSkewPitch);
       uint32_t* sRowsExact = reinterpret_cast<uint32_t*>(sPar + kQdqChunk * kQdqTileCols);
       const int64_t groups = p.qdq_K / 128;
-      const int64_t qtiles = ceil_div(p.qdq_N, static_cast<int64_t>(kQdqTileCols)) * groups;
       const int64_t chunks = ceil_div(p.qdq_grid, kQdqChunk);
-      const int64_t pieces = qtiles * chunks;
+      const int64_t pieces1 = ceil_div(p.qdq_N, static_cast<int64_t>(kQdqTileCols)) * groups * chunks;
+      const int64_t pieces = pieces1 + (p.qdq_W2 ? ceil_div(p.qdq_N2, static_cast<int64_t>(kQdqTileCols)) * groups * chunks : 0);
       int* const next = p.qdq_ready + ceil_div(p.qdq_N, static_cast<int64_t>(kTileN));
       bool skip_publish = p.fault_mode == 3 && blockIdx.x == 0;  // fault injection: one count never arrives
       while (p.qdq_cands) {
         if (tid == 0) *qdq_claim = (p.qdq_cands == 2 && *gemm_done) ? -1 : atomicAdd(next, 1);
         QdqWarpsSync{}();
-        const int64_t q = *qdq_claim;
-        if (q < 0 || q >= pieces) break;
+        const int64_t qq = *qdq_claim;
+        if (qq < 0 || qq >= pieces) break;
         // q = (tile, chunk), chunk fastest; tiles in the order of the operand rows they
         // fill (32 rows = 32 columns of W, never straddling a 128-column block), rows major
+        const bool first = qq < pieces1;
+        const int64_t q = first ? qq : qq - pieces1;
         const int64_t t = q / chunks;
         const int64_t rb = t / groups, k0 = (t - rb * groups) * 128;
         const int c0 = static_cast<int>(q - t * chunks) * kQdqChunk;
         const int c1 = min(c0 + kQdqChunk, p.qdq_grid);
-        const int64_t n0 = qdq_w_column(rb * kQdqTileCols, p.qdq_interleave);
-        qdq_tile<__nv_bfloat16, 128, QdqTile>(p.qdq_W, p.qdq_K, p.qdq_N, p.qdq_N, k0, n0, p.qdq_S, c0,
-                                              c1, true, false, p.qdq_Wt, p.err, p.qdq_quantizer, p.qdq_interleave,
-                                              sWT, sS, sR, sPar, sRowsExact, tid, QdqWarpsSync{});
-        // publish: every thread's stores, then the count of the operand tile the rows are in
+        const int64_t ldw = p.qdq_ldw > 0 ? p.qdq_ldw : p.qdq_N;
+        if (first)
+          qdq_tile<__nv_bfloat16, 128, QdqTile>(p.qdq_W, p.qdq_K, p.qdq_N, ldw, k0,
+                                                qdq_w_column(rb * kQdqTileCols, p.qdq_interleave), p.qdq_S, c0, c1, true,
+                                                false, p.qdq_Wt, p.err, p.qdq_quantizer, p.qdq_interleave, sWT, sS, sR,
+                                                sPar, sRowsExact, tid, QdqWarpsSync{});
+        else
+          qdq_tile<__nv_bfloat16, 128, QdqTile>(p.qdq_W2, p.qdq_K, p.qdq_N2, ldw, k0, rb * kQdqTileCols, p.qdq_S, c0, c1,
+                                                true, false, p.qdq_Wt2, p.err, p.qdq_quantizer, 0, sWT, sS, sR, sPar,
+                                                sRowsExact, tid, QdqWarpsSync{});
+        // publish: every thread's stores, then (first operand) the count of the operand
+        // tile the rows are in; the second operand is read only by a later launch
         fence_proxy_async_global();
         __threadfence();
         QdqWarpsSync{}();
-        if (tid == 0) {
+        if (tid == 0 && first) {
           if (skip_publish)
             skip_publish = false;
           else
@@ -957,7 +971,9 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
   const bool qdq = a.qdq_W != nullptr;
   // the launches that read candidate slots (mode 1, mode 3) must read the operand the QDQ
   // warps make, one B slot per candidate
-  if (qdq && ((mode != 0 && mode != 1 && mode != 3) || !a.qdq_ready || !a.qdq_S || !a.qdq_Wt || a.qdq_K % 128 ||
+  if (qdq && ((mode != 0 && mode != 1 && mode != 3 && mode != 5) || !a.qdq_ready || !a.qdq_S || !a.qdq_Wt || a.qdq_K % 128 ||
+              (a.qdq_W2 && (!a.qdq_Wt2 || a.qdq_N2 % 8 || a.qdq_interleave)) ||
+              (a.qdq_ldw && a.qdq_ldw < a.qdq_N + (a.qdq_W2 ? a.qdq_N2 : 0)) ||
               a.qdq_N % 8 || a.qdq_grid < 1 || (a.qdq_interleave && (a.qdq_interleave % 128 || a.qdq_N != 2 * a.qdq_interleave)) ||
               (mode != 0 && (a.qdq_N != a.N || a.qdq_K != a.K || a.qdq_Wt != a.Wt || a.a_slotted || !a.b_per_cand)) ||
               ceil_div(a.qdq_N, static_cast<int64_t>(kQdqTileCols)) * (a.qdq_K / 128) * ceil_div(a.qdq_grid, kQdqChunk) >=
@@ -991,7 +1007,7 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
   p.err = a.err;
   p.timeout_ns = a.timeout_ns;
   p.fault_mode = a.fault_mode;
-  p.cand_inner = (mode == 1 || mode == 3) ? a.cand_inner : 0;
+  p.cand_inner = (mode == 1 || mode == 3 || mode == 5) ? a.cand_inner : 0;
   p.qdq_W = a.qdq_W;
   p.qdq_S = a.qdq_S;
   p.qdq_Wt = const_cast<__nv_bfloat16*>(a.qdq_Wt);
@@ -1002,6 +1018,10 @@ cudaError_t launch_loss_gemm(const LossGemmArgs& a, const CUtensorMap& mapA, con
   p.qdq_N = a.qdq_N;
   p.qdq_interleave = a.qdq_interleave;
   p.qdq_grid = a.qdq_grid;
+  p.qdq_ldw = a.qdq_ldw;
+  p.qdq_W2 = a.qdq_W2;
+  p.qdq_Wt2 = a.qdq_Wt2;
+  p.qdq_N2 = a.qdq_N2;
   p.K = a.K;
   const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
   const int64_t units = (mode == 1 || mode == 3 || mode == 5 ? p.cands : (mode == 4 ? a.n_grid + 1 : 1)) * tiles;

@@ -124,3 +124,20 @@ def test_attention_wait_that_runs_out_returns_timeout():
     again = awq.search_attn(Xd, Wd, 1, 128)
     for name in ("scales", "codes", "steps", "zeros", "losses"):
         assert torch.equal(getattr(again, name), getattr(ref, name)), name
+
+
+@pytest.mark.parametrize("M,K,n_heads,seq_len,n_grid", [(256, 256, 1, 128, 20), (1024, 384, 2, 512, 7),
+                                                         (512, 512, 2, 256, 64)])
+def test_qdq_warps_match_the_qdq_kernel_in_the_attention_block(M, K, n_heads, seq_len, n_grid, monkeypatch):
+    """bf16 W with group 128: the Q|K GEMM's QDQ warps make the candidate operands of
+    [W_q | W_k] (its loads of a slot's tile waiting for that tile) and then of W_v (read by
+    the next launch); AWQ_QDQ=standalone makes them with qdq_kernel first. Both give the
+    same bits, and the warps' form matches the oracle."""
+    X, W = _layer(M, K, n_heads * awq.ATTN_HEAD_DIM, "bf16", 128, seed=M + 3 * K)
+    monkeypatch.delenv("AWQ_QDQ", raising=False)
+    out, r, W32 = _run(X, W, n_heads, seq_len, 128, n_grid)
+    _check(out, r, W32, 128)
+    monkeypatch.setenv("AWQ_QDQ", "standalone")
+    plain = awq.search_attn(X.cuda(), W.cuda(), n_heads, seq_len, 128, n_grid)
+    for name in ("scales", "codes", "steps", "zeros", "losses", "best_index"):
+        assert torch.equal(getattr(out, name), getattr(plain, name)), name
