@@ -215,12 +215,16 @@ class SearchOutput:
         return int(self.best_index[0])
 
 
-def _dtype_code(t: torch.Tensor) -> int:
-    if t.dtype == torch.bfloat16:
+def _dtype_code_of(dtype: torch.dtype) -> int:
+    if dtype == torch.bfloat16:
         return DTYPE_BF16
-    if t.dtype == torch.float32:
+    if dtype == torch.float32:
         return DTYPE_F32
-    raise TypeError(f"X and W must be bfloat16 or float32, got {t.dtype}")
+    raise TypeError(f"X and W must be bfloat16 or float32, got {dtype}")
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    return _dtype_code_of(t.dtype)
 
 
 def _alloc_outputs(K, N, group, n_grid, device, pin=False):
@@ -646,7 +650,7 @@ def loss_gemm_launches(M: int, K: int, N: int, n_grid: int = 20, group: int = 12
                        dtype: torch.dtype = torch.bfloat16) -> int:
     """How many loss-GEMM launches a search of this form runs on the current device: 1
     (reference and candidates in one launch) or 2 (the reference output in its own launch)."""
-    n = int(library().awq_loss_gemm_launches(_dtype_code(torch.empty(0, dtype=dtype)), M, K, N, group, n_grid))
+    n = int(library().awq_loss_gemm_launches(_dtype_code_of(dtype), M, K, N, group, n_grid))
     if n < 0:
         _check(-n)
     return n
@@ -656,4 +660,4 @@ def qdq_in_loss_gemm(M: int, K: int, N: int, n_grid: int = 20, group: int = 128,
                      dtype: torch.dtype = torch.bfloat16) -> bool:
     """Whether a search of this form makes its candidate operands with the loss GEMM's own
     QDQ warps (else a QDQ kernel runs before the GEMM)."""
-    return bool(library().awq_qdq_in_loss_gemm(_dtype_code(torch.empty(0, dtype=dtype)), M, K, N, group, n_grid))
+    return bool(library().awq_qdq_in_loss_gemm(_dtype_code_of(dtype), M, K, N, group, n_grid))
