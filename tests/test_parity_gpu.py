@@ -80,7 +80,8 @@ def test_reference_launch_forms(M, K, N, group, n_grid, dtype, monkeypatch):
 
 @pytest.mark.parametrize("M,K,N,n_grid,quantizer", [(300, 384, 520, 20, "asym"), (129, 256, 776, 64, "asym"),
                                                      (520, 512, 264, 11, "sym"), (1, 128, 8, 20, "asym"),
-                                                     (1000, 1024, 2056, 20, "asym")])
+                                                     (1000, 1024, 2056, 20, "asym"), (64, 256, 256, 1, "asym"),
+                                                     (2, 640, 4104, 10, "asym")])
 def test_qdq_warps_match_the_qdq_kernel(M, K, N, n_grid, quantizer, monkeypatch):
     # bf16 W with group 128: the candidate operands are made by the loss GEMM's own QDQ
     # warps while its tensor cores run (the reference launch makes the reference operand
