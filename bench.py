@@ -645,10 +645,11 @@ def other_workload(awq, name: str, stream, flush, steps: int, warmup: int, peaks
     spec = WORKLOADS[name]
     X, W = generate(spec)
     Xd, Wd = X.cuda(), W.cuda()
-    t = time_searches(awq, spec, Xd, Wd, stream, flush, steps, warmup)
+    t = time_searches(awq, spec, Xd, Wd, stream, flush, steps, warmup, sample_clocks=Xd.device.index)
     obj = search_object(awq, spec, t, peaks, peak_kind, sustained=False)
+    obj["clocks"] = t["clocks"]  # sampled during this layer's timed region
     if spec.M * spec.K * spec.N <= 128 * 256 * 256:
-        obj["bound"] = ("latency: 6 launches of a few microseconds each; the tensor and HBM "
+        obj["bound"] = ("latency: 7 launches of a few microseconds each; the tensor and HBM "
                         "fractions are not meaningful at this size")
     del Xd, Wd
     return obj, (spec, X, t["out"])
