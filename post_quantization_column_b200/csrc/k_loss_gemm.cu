@@ -2,7 +2,7 @@
 // Activation" §4: every candidate is scored by the mean squared difference between the
 // original output and the candidate output, the difference cast to FP32).
 //
-// One persistent kernel, three modes:
+// One persistent kernel, six modes:
 //   mode 0: Y = X_b W_b, written once to HBM in a tile-major layout;
 //   mode 1: for every (candidate i, output tile): acc = X_b W_hat_i,b on the tensor
 //           cores, and the epilogue adds (acc - Y)^2 over the tile and writes one fp64
@@ -31,9 +31,12 @@
 // two 256-column tensor-memory accumulators, so the epilogue of tile t overlaps the
 // main loop of tile t+1; four epilogue warps read the accumulator with tcgen05.ld
 // (warp w % 4 owns TMEM lanes 32(w%4)..+31 = tile rows). Warp roles: 0 TMA producer,
-// 1 MMA issuer, 2 TMEM allocator, 4-7 epilogue. Units (candidate, tile) are walked in
-// a grouped raster (group_m row tiles at a time) so the X row block and the W_hat
-// column block of neighbouring CTAs stay in L2.
+// 1 MMA issuer, 2 TMEM allocator, 4-7 epilogue, and in loss_gemm_kernel<true> 8-15 the
+// QDQ warps, which make the candidate operands (the tile routine of qdq_tile.cuh) while
+// the tensor cores run, publishing each finished piece through a per-tile counter that
+// the producer waits for. Units (candidate, tile) are walked in a grouped raster
+// (group_m row tiles at a time) so the X row block and the W_hat column block of
+// neighbouring CTAs stay in L2.
 //
 // Every wait is bounded (global timer); a wait that runs out sets the call's
 // timeout bit, raises a CTA-wide abort flag, the producer waits for its own copies in
