@@ -372,8 +372,8 @@ int awq_loss_gemm_variant(int64_t M, int64_t K, int64_t N, int n_grid);
 int awq_qdq_in_loss_gemm(int in_dtype, int64_t M, int64_t K, int64_t N, int group, int n_grid);
 
 /* How many loss-GEMM launches a search of this form runs on the current device: 2 when
- * the QDQ warps make the operands (the reference output's launch makes the reference
- * operand and the first candidate tiles), when the reference output Y (M x N fp32) is
+ * the QDQ warps make the operands (they claim candidate pieces during the reference
+ * output's launch and make the rest during the candidates'), when the reference output Y (M x N fp32) is
  * larger than the device's L2 cache, or with the two-SM kernel: the reference output in
  * its own launch, then a launch that scores every candidate of a column tile before the
  * next column tile, so each tile of Y is read from DRAM once; 1 otherwise (one launch
